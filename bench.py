@@ -1,0 +1,411 @@
+"""Benchmark of the frame-sparse attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = the whole hot path over one batch of the LVSA workload at a
+Wan-2.1-1.3B-like shape (T=41 latent frames, P=1560 tokens/frame, H=12, d=128,
+budget C=21, window W=9, anchor period T_per=4, denoising step s=0): the attended
+frame sets are built on the GPU (sfa_build_sets), then frame-sparse attention runs
+over them (sfa_forward), all through the C ABI of libsfa.so.
+
+Metric: effective attended TFLOP/s = 4 d sum_{b,h,t} P * P |A(h,t)| / time, i.e. only
+the QK^T and PV flops of attended, unpadded (query, key) pairs count.
+
+With N > 1 (torchrun, one process per GPU) every rank runs its own batch of the
+same workload (weak scaling; heads and batches are independent, so there is no
+data-path collective); timing is the max over ranks.
+
+--impl reference times the CPU oracle (float64, the repository's plain reference
+implementation of the same computation) on the host cores, on a bounded sample of
+query rows of the same workload per step; rank 0 alone runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sfa_workloads import WORKLOADS, workload_qkv  # noqa: E402
+
+METRIC = "effective attended TFLOP/s (and % of BF16 tensor peak); ms per sparse-attn call"
+WORKLOAD = WORKLOADS["lvsa41"]
+STEP_S = 0
+WORKLOAD_DESC = ("LVSA frame-sparse attention, Wan-2.1-1.3B-like shape: T=41 frames, P=1560 "
+                 "tokens/frame, H=12, d=128, B=1, C=21, W=9, T_per=4, step s=0")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        p["source"] = "measured"
+        return p
+    p = dict(FALLBACK_PEAKS)
+    p["source"] = "fallback"
+    return p
+
+
+def attended_flops(counts: np.ndarray, w) -> float:
+    """4 d sum_{b,h,t} P * P |A(h,t)| (QK^T + PV, attended pairs only)."""
+    return 4.0 * w.d * w.B * float(counts.sum()) * w.P * w.P
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            import tempfile
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for name, val in zip(names, parts[5:9]):
+                    if val.lower() == "active":
+                        reasons.add(name)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    import frame_sparse_attention_b200 as sfa
+    sfa.load()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = WORKLOAD
+    kinds = [hs.kind for hs in w.heads]
+    params = sfa.set_params(T_kv=w.Tkv, Tq=w.Tq, q_off=w.q_off, C=w.C, W=w.W, T_per=w.T_per,
+                            step=STEP_S, n_sink=w.n_sink, n_prev=w.n_prev, chunk_len=w.chunk_len)
+    Amax = sfa.set_max_count(params, kinds)
+
+    q_h, k_h, v_h = workload_qkv(w, seed=rank)
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    frames = torch.empty((w.H, w.Tq, Amax), dtype=torch.int32, device=dev)
+    counts = torch.empty((w.H, w.Tq), dtype=torch.int32, device=dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.Lq), dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)  # 256 MB > L2
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        sfa.build_sets(params, kinds, None, Amax, frames, counts, stream=stream)
+        sfa.forward(q, k, v, frames, counts, w.P, out=out, lse=lse, dev_status=status, stream=stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    if status.item() != 0:
+        raise RuntimeError(f"device status {sfa.error_string(status.item())}")
+    flops = attended_flops(counts.cpu().numpy(), w)
+
+    # timed region: K steps, per-step events (the L2 flush between steps is outside them)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clocks = ClockSampler(local_rank)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    time.sleep(0.3)
+    for i in range(args.steps):
+        flush.zero_()
+        e0, e1, e2 = ev[i]
+        e0.record(stream)
+        sfa.build_sets(params, kinds, None, Amax, frames, counts, stream=stream)
+        e1.record(stream)
+        sfa.forward(q, k, v, frames, counts, w.P, out=out, lse=lse, dev_status=status, stream=stream)
+        e2.record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    if world > 1:
+        torch.distributed.barrier()
+    step_ms = [e0.elapsed_time(e2) for e0, _, e2 in ev]
+    fwd_ms = [e1.elapsed_time(e2) for _, e1, e2 in ev]
+    sets_ms = [e0.elapsed_time(e1) for e0, e1, _ in ev]
+    if status.item() != 0:
+        raise RuntimeError(f"device status {sfa.error_string(status.item())}")
+    total_ms = float(sum(step_ms))
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    # end to end through the public API with host buffers: H2D of Q, K, V from pinned
+    # memory, sets + attention, D2H of O and LSE into pinned memory, every step
+    q_p, k_p, v_p = (x.pin_memory() for x in (q_h, k_h, v_h))
+    o_p = torch.empty(q_h.shape, dtype=torch.bfloat16).pin_memory()
+    lse_p = torch.empty((w.B, w.H, w.Lq), dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        q.copy_(q_p, non_blocking=True)
+        k.copy_(k_p, non_blocking=True)
+        v.copy_(v_p, non_blocking=True)
+        step()
+        o_p.copy_(out, non_blocking=True)
+        lse_p.copy_(lse, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    n_e2e = max(3, min(args.steps, 10))
+    if world > 1:
+        torch.distributed.barrier()
+    s0 = torch.cuda.Event(enable_timing=True)
+    s1 = torch.cuda.Event(enable_timing=True)
+    s0.record(stream)
+    for _ in range(n_e2e):
+        e2e_step()
+    s1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = s0.elapsed_time(s1) / n_e2e
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = sum(x.numel() * x.element_size() for x in (q_h, k_h, v_h))
+    d2h = o_p.numel() * o_p.element_size() + lse_p.numel() * lse_p.element_size()
+
+    merge = bench_merge(sfa, dev, stream, flush) if rank == 0 else None
+
+    if rank != 0:
+        return None
+    peaks = measured_peaks()
+    ms_per_step = total_ms / args.steps
+    value = flops * world / (total_ms / args.steps) / 1e9  # TFLOP/s, whole job
+    fwd_avg = float(np.mean(fwd_ms))
+    achieved = flops / (fwd_avg * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    rec = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic: Q, K, V ~ N(0,1) fp32 rounded to bf16, seeded per rank",
+        "config": {"workload": WORKLOAD_DESC, "B": w.B, "H": w.H, "T": w.Tq, "P": w.P, "d": w.d,
+                   "C": w.C, "W": w.W, "T_per": w.T_per, "step_s": STEP_S,
+                   "attended_tflop_per_step": round(flops / 1e12, 4),
+                   "parallelism": f"replica x{world} (independent batch per GPU)",
+                   "l2": "flushed (256 MB write) between timed steps, outside the timed events"},
+        "roofline": {"bound": "tensor", "kernel": "sfa_forward_kernel<128>",
+                     "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4),
+                     "peak_source": f"{peaks['source']} bf16_tflops (burst)",
+                     "frac_of_sustained": round(achieved / float(peaks["bf16_tflops_sustained"]), 4),
+                     "traffic": None,
+                     "forward_ms": round(fwd_avg, 4), "set_build_ms": round(float(np.mean(sets_ms)), 4)},
+        "e2e": {"value": round(flops * world / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk,
+        "merge": merge,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        rec["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
+    return rec
+
+
+def bench_merge(sfa, dev, stream, flush, reps=20):
+    """LSE merge of the ISPA dual-stream shape (1560 rows x 12 heads, d=128)."""
+    w = WORKLOADS["lsemerge_local"]
+    rows = w.B * w.H * w.Lq
+    g = torch.Generator("cpu").manual_seed(7)
+    o1 = torch.randn(rows, w.d, generator=g).to(torch.bfloat16).to(dev)
+    o2 = torch.randn(rows, w.d, generator=g).to(torch.bfloat16).to(dev)
+    l1 = torch.randn(rows, generator=g).to(dev)
+    l2 = torch.randn(rows, generator=g).to(dev)
+    o = torch.empty_like(o1)
+    lse = torch.empty_like(l1)
+    for _ in range(3):
+        sfa.lse_merge(o1, l1, o2, l2, out=o, lse=lse, stream=stream)
+    times = []
+    for _ in range(reps):
+        flush.zero_()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        sfa.lse_merge(o1, l1, o2, l2, out=o, lse=lse, stream=stream)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        times.append(a.elapsed_time(b))
+    ms = float(np.median(times))
+    nbytes = rows * (3 * 2 * w.d + 3 * 4)
+    peaks = measured_peaks()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"kernel": "lse_merge_kernel<128>", "rows": rows, "bytes": nbytes, "us": round(ms * 1e3, 2),
+            "achieved_gbs": round(gbs, 1), "peak_gbs": float(peaks["hbm_gbs"]), "bound": "hbm",
+            "frac": round(gbs / float(peaks["hbm_gbs"]), 4)}
+
+
+# ----------------------------------------------------------------------------- oracle timing
+def cpu_baseline(seconds: float = 15.0, inputs=None):
+    """Time the float64 oracle on host cores for about `seconds` on sampled query rows."""
+    import oracle
+    from oracle import sets as S
+    from sfa_workloads import sample_rows
+    w = WORKLOAD
+    q, k, v = inputs if inputs is not None else workload_qkv(w, seed=0)
+    frames, counts = S.workload_sets(w, step=STEP_S)
+    cores = os.cpu_count() or 1
+    scale = 1.0 / math.sqrt(w.d)
+
+    def run(n_per_head, seed):
+        rows = sample_rows(w, n_per_head, seed=seed)
+        t0 = time.perf_counter()
+        oracle.attention(q, k, v, frames, counts, w.P, scale, rows=rows, n_threads=cores)
+        dt = time.perf_counter() - t0
+        h = (rows // w.Lq) % w.H
+        t = (rows % w.Lq) // w.P
+        fl = 4.0 * w.d * w.P * counts[h, t].astype(np.float64).sum()
+        return rows.size, fl, dt
+
+    n, fl, dt = run(max(1, cores // w.H + 1), seed=100)    # calibration
+    per_row = dt / max(n, 1)
+    n_per_head = max(1, int(seconds / per_row / w.H))
+    n, fl, dt = run(n_per_head, seed=101)
+    return {"value": round(fl / dt / 1e12, 8), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} sampled query rows of the LVSA workload (float64 C oracle, "
+                      f"{cores} threads, {dt:.1f} s)", "seconds": round(dt, 2)}
+
+
+def run_reference(args, rank):
+    """Reference arm: the oracle on host cores, a bounded sample of rows per step."""
+    if rank != 0:
+        return None
+    import oracle
+    from oracle import sets as S
+    from sfa_workloads import sample_rows
+    w = WORKLOAD
+    q, k, v = workload_qkv(w, seed=0)
+    frames, counts = S.workload_sets(w, step=STEP_S)
+    cores = os.cpu_count() or 1
+    scale = 1.0 / math.sqrt(w.d)
+    # rows per step sized so that warmup + steps end within a few minutes
+    probe = sample_rows(w, max(1, cores // w.H + 1), seed=999)
+    t0 = time.perf_counter()
+    oracle.attention(q, k, v, frames, counts, w.P, scale, rows=probe, n_threads=cores)
+    per_row = (time.perf_counter() - t0) / probe.size
+    budget_s = 120.0 / max(1, args.steps + args.warmup)
+    n_per_head = max(1, int(budget_s / per_row / w.H))
+    step_times, step_flops = [], []
+    for i in range(args.warmup + args.steps):
+        rows = sample_rows(w, n_per_head, seed=i)
+        h = (rows // w.Lq) % w.H
+        t = (rows % w.Lq) // w.P
+        fl = 4.0 * w.d * w.P * counts[h, t].astype(np.float64).sum()
+        t0 = time.perf_counter()
+        oracle.attention(q, k, v, frames, counts, w.P, scale, rows=rows, n_threads=cores)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            step_times.append(dt)
+            step_flops.append(fl)
+    total = sum(step_times)
+    value = sum(step_flops) / total / 1e12
+    sample = (f"{rows.size} sampled query rows per step of the LVSA workload, float64 C oracle "
+              f"on {cores} host threads")
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 8), "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(total / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD_DESC, "B": w.B, "H": w.H, "T": w.Tq, "P": w.P, "d": w.d,
+                   "C": w.C, "W": w.W, "T_per": w.T_per, "step_s": STEP_S},
+        "cpu_baseline": {"value": round(value, 8), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 8), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        rec = run_reference(args, rank)
+        if rec is not None:
+            print(json.dumps(rec), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        rec = run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+    if rec is not None:
+        print(json.dumps(rec), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,206 @@
+"""ctypes binding of libsfa.so (the C ABI declared in include/sfa.h).
+
+Argument marshalling only: every step of the computation runs in the library's
+CUDA kernels.  PyTorch supplies device memory and the current stream.  If the
+shared library is missing this module raises; there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libsfa.so")
+
+# sfa_status
+SFA_OK = 0
+SFA_ERR_INVALID_ARG = 1
+SFA_ERR_UNSUPPORTED = 2
+SFA_ERR_CUDA = 3
+SFA_ERR_TIMEOUT = 4
+SFA_ERR_BAD_SET = 5
+
+# sfa_set_kind
+SET_KINDS = {"dense": 0, "lvsa": 1, "local": 2, "anchor": 3, "memory": 4, "explicit": 5}
+SFA_MAX_HEADS = 1024
+SFA_DEBUG_STALL_SOFTMAX = 1
+
+
+class SfaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {error_string(status)} (status {status})")
+
+
+class SetParams(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in
+                ("T_kv", "Tq", "q_off", "C", "W", "T_per", "step", "n_sink", "n_prev", "chunk_len")]
+
+
+class AttnDesc(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("Tq", ctypes.c_int32),
+                ("T_kv", ctypes.c_int32), ("P", ctypes.c_int32), ("d", ctypes.c_int32),
+                ("scale", ctypes.c_float), ("Amax", ctypes.c_int32),
+                ("q_stride", ctypes.c_int64 * 3), ("k_stride", ctypes.c_int64 * 3),
+                ("v_stride", ctypes.c_int64 * 3), ("o_stride", ctypes.c_int64 * 3),
+                ("timeout_us", ctypes.c_uint32), ("debug_flags", ctypes.c_uint32)]
+
+
+_lib = None
+EXPORTS = ("sfa_error_string", "sfa_version", "sfa_set_max_count", "sfa_build_sets", "sfa_forward",
+           "sfa_lse_merge")
+
+
+def load():
+    """Load libsfa.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m frame_sparse_attention_b200.build` (needs nvcc)")
+    lib = ctypes.CDLL(LIB_PATH)
+    i32, i64, vp, st = ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int
+    lib.sfa_error_string.restype = ctypes.c_char_p
+    lib.sfa_error_string.argtypes = [st]
+    lib.sfa_version.restype = i32
+    lib.sfa_version.argtypes = []
+    lib.sfa_set_max_count.restype = st
+    lib.sfa_set_max_count.argtypes = [ctypes.POINTER(SetParams), i32, ctypes.POINTER(i32), i32,
+                                      ctypes.POINTER(i32)]
+    lib.sfa_build_sets.restype = st
+    lib.sfa_build_sets.argtypes = [ctypes.POINTER(SetParams), i32, ctypes.POINTER(i32), vp, i32, vp, vp,
+                                   i32, vp]
+    lib.sfa_forward.restype = st
+    lib.sfa_forward.argtypes = [ctypes.POINTER(AttnDesc), vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.sfa_lse_merge.restype = st
+    lib.sfa_lse_merge.argtypes = [i64, i32, vp, vp, vp, vp, vp, vp, vp]
+    _lib = lib
+    return lib
+
+
+def error_string(status: int) -> str:
+    return load().sfa_error_string(status).decode()
+
+
+def version() -> int:
+    return load().sfa_version()
+
+
+def _check(status: int, what: str):
+    if status != SFA_OK:
+        raise SfaError(status, what)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _kinds(kinds):
+    arr = (ctypes.c_int32 * len(kinds))()
+    for i, k in enumerate(kinds):
+        arr[i] = SET_KINDS[k] if isinstance(k, str) else int(k)
+    return arr
+
+
+def set_params(*, T_kv, Tq, q_off=0, C=1, W=1, T_per=1, step=0, n_sink=0, n_prev=0, chunk_len=1):
+    return SetParams(T_kv, Tq, q_off, C, W, T_per, step, n_sink, n_prev, chunk_len)
+
+
+def set_max_count(params: SetParams, kinds, n_extra: int = 0) -> int:
+    out = ctypes.c_int32(0)
+    _check(load().sfa_set_max_count(ctypes.byref(params), len(kinds), _kinds(kinds), n_extra,
+                                    ctypes.byref(out)), "sfa_set_max_count")
+    return out.value
+
+
+def build_sets(params: SetParams, kinds, extra: torch.Tensor | None = None, Amax: int | None = None,
+               frames: torch.Tensor | None = None, counts: torch.Tensor | None = None, stream=None):
+    """Attended frame lists on the device: frames int32 [H, Tq, Amax], counts int32 [H, Tq]."""
+    H = len(kinds)
+    n_extra = 0 if extra is None else int(extra.shape[1])
+    if Amax is None:
+        Amax = max(1, set_max_count(params, kinds, n_extra))
+    dev = torch.device("cuda", torch.cuda.current_device()) if extra is None else extra.device
+    if frames is None:
+        frames = torch.empty((H, params.Tq, Amax), dtype=torch.int32, device=dev)
+    if counts is None:
+        counts = torch.empty((H, params.Tq), dtype=torch.int32, device=dev)
+    if extra is not None:
+        assert extra.dtype == torch.int32 and extra.is_cuda and extra.is_contiguous()
+        assert extra.shape[0] == H
+    assert frames.is_contiguous() and counts.is_contiguous()
+    _check(load().sfa_build_sets(ctypes.byref(params), H, _kinds(kinds), _ptr(extra), n_extra,
+                                 frames.data_ptr(), counts.data_ptr(), Amax, _stream(stream)),
+           "sfa_build_sets")
+    return frames, counts
+
+
+def attn_desc(q, k, v, o, P: int, Amax: int, scale: float | None = None, timeout_us: int = 0,
+              debug_flags: int = 0) -> AttnDesc:
+    B, H, Lq, d = q.shape
+    Lkv = k.shape[2]
+    if Lq % P or Lkv % P:
+        raise ValueError(f"sequence lengths {Lq}, {Lkv} are not multiples of P = {P}")
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
+        if t.dtype != torch.bfloat16 or not t.is_cuda:
+            raise ValueError(f"{name} must be a bf16 CUDA tensor")
+        if t.dim() != 4 or t.stride(3) != 1:
+            raise ValueError(f"{name} must be [B, H, L, d] with d contiguous")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    desc = AttnDesc()
+    desc.B, desc.H, desc.Tq, desc.T_kv, desc.P, desc.d = B, H, Lq // P, Lkv // P, P, d
+    desc.scale, desc.Amax = float(scale), int(Amax)
+    for field, t in (("q_stride", q), ("k_stride", k), ("v_stride", v), ("o_stride", o)):
+        arr = getattr(desc, field)
+        arr[0], arr[1], arr[2] = t.stride(0), t.stride(1), t.stride(2)
+    desc.timeout_us = timeout_us
+    desc.debug_flags = debug_flags
+    return desc
+
+
+def forward(q, k, v, frames, counts, P: int, scale: float | None = None, out=None, lse=None,
+            dev_status=None, stream=None, timeout_us: int = 0, debug_flags: int = 0):
+    """Frame-sparse attention: (O bf16 like q, LSE fp32 [B, H, Tq*P])."""
+    B, H, Lq, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, Lq), dtype=torch.float32, device=q.device)
+    assert lse.is_contiguous() and lse.dtype == torch.float32
+    assert frames.dtype == torch.int32 and counts.dtype == torch.int32
+    assert frames.is_contiguous() and counts.is_contiguous()
+    desc = attn_desc(q, k, v, out, P, frames.shape[2], scale, timeout_us, debug_flags)
+    assert tuple(frames.shape[:2]) == (H, desc.Tq) and tuple(counts.shape) == (H, desc.Tq)
+    _check(load().sfa_forward(ctypes.byref(desc), q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                              frames.data_ptr(), counts.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                              _ptr(dev_status), _stream(stream)), "sfa_forward")
+    return out, lse
+
+
+def lse_merge(o1, lse1, o2, lse2, out=None, lse=None, stream=None):
+    """Merge two partial attentions by LSE: returns (O bf16, LSE fp32) shaped like o1 / lse1."""
+    d = o1.shape[-1]
+    rows = lse1.numel()
+    for t in (o1, o2, lse1, lse2):
+        assert t.is_cuda and t.is_contiguous()
+    assert o1.dtype == torch.bfloat16 and o2.dtype == torch.bfloat16
+    assert lse1.dtype == torch.float32 and lse2.dtype == torch.float32
+    assert o1.numel() == rows * d and o2.shape == o1.shape and lse2.shape == lse1.shape
+    if out is None:
+        out = torch.empty_like(o1)
+    if lse is None:
+        lse = torch.empty_like(lse1)
+    _check(load().sfa_lse_merge(rows, d, o1.data_ptr(), lse1.data_ptr(), o2.data_ptr(), lse2.data_ptr(),
+                                out.data_ptr(), lse.data_ptr(), _stream(stream)), "sfa_lse_merge")
+    return out, lse

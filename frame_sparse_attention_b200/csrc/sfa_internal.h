@@ -1,0 +1,23 @@
+// Host-side helpers shared by the libsfa translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "sfa.h"
+
+namespace sfa {
+
+inline sfa_status cuda_status(cudaError_t e)
+{
+    return e == cudaSuccess ? SFA_OK : SFA_ERR_CUDA;
+}
+
+// launch errors (bad configuration, missing kernel image) surface here
+inline sfa_status launch_status()
+{
+    return cuda_status(cudaGetLastError());
+}
+
+inline cudaStream_t as_cuda(sfa_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+}  // namespace sfa

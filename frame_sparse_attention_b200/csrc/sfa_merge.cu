@@ -1,0 +1,104 @@
+// LSE merge of two partial attentions over disjoint key sets.
+//
+// "ISPA" (Absorción Paramétrica Específica de Instancia), §2.1 Dual-Stream Warmup and
+// contribution 2: the per-row log-sum-exp kept by attention kernels lets attention be
+// split into a local and a history branch and fused afterwards.  Per row, with
+// M = max(L1, L2):  L = M + ln(e^{L1-M} + e^{L2-M}),  O = e^{L1-L} O1 + e^{L2-L} O2.
+//
+// Memory-bound: each row reads 2 x (d bf16 + 1 fp32) and writes d bf16 + 1 fp32.
+// A group of d/8 threads owns a row, every thread moves 16 bytes of each O.
+#include <cstdint>
+
+#include "sfa.h"
+#include "sfa_internal.h"
+
+namespace sfa {
+namespace {
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ uint32_t to_bf16x2(float lo, float hi)
+{
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) lse_merge_kernel(int64_t rows, const uint4 *__restrict__ o1,
+                                                        const float *__restrict__ lse1,
+                                                        const uint4 *__restrict__ o2,
+                                                        const float *__restrict__ lse2, uint4 *o, float *lse)
+{
+    constexpr int G = D / 8;  // threads per row
+    const int64_t gtid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int sub = threadIdx.x % G;
+    const int64_t row_stride = (int64_t)gridDim.x * blockDim.x / G;
+    for (int64_t r = gtid / G; r < rows; r += row_stride) {
+        // the row's first lane reads both LSEs and hands them to its group, so an
+        // in-place lse write below cannot overtake another lane's read
+        const unsigned group = ((1u << G) - 1u) << ((threadIdx.x % 32) & ~(G - 1));
+        float l1 = 0.f, l2 = 0.f;
+        if (sub == 0) {
+            l1 = lse1[r];
+            l2 = lse2[r];
+        }
+        l1 = __shfl_sync(group, l1, 0, G);
+        l2 = __shfl_sync(group, l2, 0, G);
+        const uint4 a = o1[r * G + sub];
+        const uint4 b = o2[r * G + sub];
+        const float m = fmaxf(l1, l2);
+        float w1 = 0.f, w2 = 0.f, L = -INFINITY;
+        if (m != -INFINITY) {
+            const float e1 = l1 == -INFINITY ? 0.f : expf(l1 - m);
+            const float e2 = l2 == -INFINITY ? 0.f : expf(l2 - m);
+            const float s = e1 + e2;
+            L = m + logf(s);
+            w1 = e1 / s;
+            w2 = e2 / s;
+        }
+        const uint32_t av[4] = {a.x, a.y, a.z, a.w};
+        const uint32_t bv[4] = {b.x, b.y, b.z, b.w};
+        uint32_t ov[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float lo = w1 * bf16_lo(av[i]) + w2 * bf16_lo(bv[i]);
+            const float hi = w1 * bf16_hi(av[i]) + w2 * bf16_hi(bv[i]);
+            ov[i] = to_bf16x2(lo, hi);
+        }
+        o[r * G + sub] = make_uint4(ov[0], ov[1], ov[2], ov[3]);
+        if (sub == 0) lse[r] = L;
+    }
+}
+
+}  // namespace
+}  // namespace sfa
+
+using namespace sfa;
+
+extern "C" sfa_status sfa_lse_merge(int64_t rows, int32_t d, const void *o1, const float *lse1,
+                                    const void *o2, const float *lse2, void *o, float *lse,
+                                    sfa_stream_t stream)
+{
+    if (rows < 0) return SFA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return SFA_ERR_UNSUPPORTED;
+    if (rows == 0) return SFA_OK;
+    if (!o1 || !o2 || !o || !lse1 || !lse2 || !lse) return SFA_ERR_INVALID_ARG;
+    for (const void *p : {o1, o2, (const void *)o})
+        if (reinterpret_cast<uintptr_t>(p) % 16) return SFA_ERR_INVALID_ARG;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int threads = 256;
+    const int64_t need = (rows * (d / 8) + threads - 1) / threads;
+    const int64_t cap = (int64_t)sms * 8;  // 8 resident blocks of 256 threads per SM
+    const int blocks = (int)(need < cap ? need : cap);
+    cudaStream_t s = as_cuda(stream);
+    if (d == 128)
+        lse_merge_kernel<128><<<blocks, threads, 0, s>>>(rows, (const uint4 *)o1, lse1, (const uint4 *)o2,
+                                                         lse2, (uint4 *)o, lse);
+    else
+        lse_merge_kernel<64><<<blocks, threads, 0, s>>>(rows, (const uint4 *)o1, lse1, (const uint4 *)o2,
+                                                        lse2, (uint4 *)o, lse);
+    return launch_status();
+}

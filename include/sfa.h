@@ -1,0 +1,198 @@
+/*
+ * sfa.h - frame-sparse attention for video diffusion transformers on B200 (sm_100a).
+ *
+ * C ABI of libsfa.so.  Three operations, all asynchronous on the caller's CUDA
+ * stream, all on device buffers that the caller owns:
+ *
+ *   sfa_build_sets  attended frame sets A(h, t), one sorted list per (head, query frame)
+ *   sfa_forward     softmax attention of every query frame over the tokens of A(h, t)
+ *                   only, writing O (bf16) and the per-row log-sum-exp (fp32)
+ *   sfa_lse_merge   merge of two partial attentions (e.g. local + history branch)
+ *
+ * Conventions
+ *   - A video has T latent frames of P tokens each; token i belongs to frame i / P.
+ *     Query frame t (0 <= t < Tq) sits at frame t + q_off of the key/value timeline
+ *     (0 <= frame < T_kv).  Frame lists hold absolute key/value frame indices.
+ *   - Device pointers are plain CUDA device addresses (cudaMalloc / torch memory).
+ *     The library never allocates device memory and keeps no state between calls,
+ *     apart from a per-process cache of the CUDA driver entry point it uses to
+ *     encode TMA descriptors.
+ *   - Every call validates its arguments on the host first and returns a status;
+ *     nothing is printed and nothing throws across the ABI.  Launch errors come
+ *     back as SFA_ERR_CUDA.  Errors that only the GPU can see (a malformed frame
+ *     list, a wait that ran out) are written to an optional device status word.
+ *   - sfa_stream_t is a cudaStream_t (0 = legacy default stream).
+ */
+#ifndef SFA_H_
+#define SFA_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *sfa_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    SFA_OK = 0,
+    SFA_ERR_INVALID_ARG = 1,  /* a size, pointer, stride or parameter is out of range   */
+    SFA_ERR_UNSUPPORTED = 2,  /* valid, but outside what this build implements (e.g. d) */
+    SFA_ERR_CUDA = 3,         /* a CUDA runtime / driver call or kernel launch failed   */
+    SFA_ERR_TIMEOUT = 4,      /* device: a pipeline wait hit its time limit             */
+    SFA_ERR_BAD_SET = 5       /* device: a frame list is unsorted, repeated or out of range,
+                                 or a count is outside [0, Amax]                        */
+} sfa_status;
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char *sfa_error_string(sfa_status s);
+
+/* Library version as 10000*major + 100*minor + patch. */
+int32_t sfa_version(void);
+
+/* ------------------------------------------------------------------------------------
+ * Attended frame sets
+ * ------------------------------------------------------------------------------------
+ * Kinds, for query frame t at timeline frame c = t + q_off:
+ *
+ *   SFA_SET_DENSE     A = {0 .. T_kv-1}: full attention (the set LVSA replaces;
+ *                     "LVSA: Atención Dispersa Libre de Entrenamiento para Difusión de
+ *                     Video Largo", §2 Mecanismo Central).
+ *   SFA_SET_LVSA      A = G_s ∪ W(c) (same page, §2.1 and §2.2):
+ *                       G_s  = { f : f mod T_per == step mod T_per }, rotating global
+ *                              anchors, each frame an anchor once per T_per steps;
+ *                       W(c) = window of W frames centred on c (an even W puts the extra
+ *                              frame after c), shifted inside [0, T_kv), then grown one
+ *                              frame at a time, alternating after/before c (after first,
+ *                              a side at the end of the video hands its turn over), until
+ *                              |A| = min(C, T_kv).  The window never shrinks: if G_s ∪ W
+ *                              already exceeds C, A is larger than C.
+ *   SFA_SET_LOCAL     A = current chunk ∪ the n_prev frames before it, where the chunk of
+ *                     c is [c0, c0 + chunk_len), c0 = c - c mod chunk_len ("Head Forcing",
+ *                     §2: local heads keep the current block and its nearest frames).
+ *   SFA_SET_ANCHOR    A = {0 .. n_sink-1} ∪ LOCAL (same page: anchor heads add the first
+ *                     latent frames; "ISPA", §2.1: local branch = current + sink).
+ *   SFA_SET_MEMORY    A = ANCHOR ∪ extra[h] (same page: memory heads add selected
+ *                     history frames; the selection itself is the caller's).
+ *   SFA_SET_EXPLICIT  A = extra[h] (any caller-chosen list, e.g. a history branch).
+ *
+ * Every list is clipped to [0, T_kv), sorted ascending and free of repeats.
+ */
+typedef enum {
+    SFA_SET_DENSE = 0,
+    SFA_SET_LVSA = 1,
+    SFA_SET_LOCAL = 2,
+    SFA_SET_ANCHOR = 3,
+    SFA_SET_MEMORY = 4,
+    SFA_SET_EXPLICIT = 5
+} sfa_set_kind;
+
+#define SFA_MAX_HEADS 1024
+
+typedef struct {
+    int32_t T_kv;      /* key/value frames, >= 1                                       */
+    int32_t Tq;        /* query frames, >= 1, with q_off + Tq <= T_kv                   */
+    int32_t q_off;     /* timeline frame of query frame 0, >= 0                          */
+    int32_t C;         /* LVSA budget, >= 1                                              */
+    int32_t W;         /* LVSA base window, >= 1                                         */
+    int32_t T_per;     /* LVSA anchor period, >= 1                                       */
+    int32_t step;      /* LVSA denoising step s, >= 0                                    */
+    int32_t n_sink;    /* ANCHOR/MEMORY: leading sink frames, >= 0                      */
+    int32_t n_prev;    /* LOCAL/ANCHOR/MEMORY: frames kept before the chunk, >= 0        */
+    int32_t chunk_len; /* LOCAL/ANCHOR/MEMORY: frames per chunk, >= 1                    */
+} sfa_set_params;
+
+/*
+ * Upper bound on |A(h, t)| over all heads and query frames for these parameters:
+ * the smallest Amax that sfa_build_sets accepts.  head_kind: host array [H].
+ * Returns SFA_ERR_INVALID_ARG for bad parameters or kinds.
+ */
+sfa_status sfa_set_max_count(const sfa_set_params *p, int32_t H, const int32_t *head_kind,
+                             int32_t n_extra, int32_t *amax_out);
+
+/*
+ * Build A(h, t) for every head h < H and query frame t < Tq.
+ *   p          host pointer to the parameters above.
+ *   head_kind  host array [H] of sfa_set_kind, 1 <= H <= SFA_MAX_HEADS.
+ *   extra      device int32 [H][n_extra], entries outside [0, T_kv) ignored (use -1 as
+ *              padding); may be NULL when n_extra == 0.  Read by MEMORY/EXPLICIT heads.
+ *   frames     device int32 [H][Tq][Amax], written: the sorted list, then -1 padding.
+ *   counts     device int32 [H][Tq], written: |A(h, t)|.
+ *   Amax       must be >= sfa_set_max_count(...), else SFA_ERR_INVALID_ARG.
+ * One thread per (h, t); output is bit-identical whatever the launch.
+ */
+sfa_status sfa_build_sets(const sfa_set_params *p, int32_t H, const int32_t *head_kind,
+                          const int32_t *extra, int32_t n_extra, int32_t *frames,
+                          int32_t *counts, int32_t Amax, sfa_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
+ * Frame-sparse attention forward
+ * ------------------------------------------------------------------------------------
+ * For each batch b, head h and query row i of query frame t = i / P, with the key set
+ *   K(h, t) = ∪_{f in A(h,t)} [f*P, (f+1)*P):
+ *     s_j = scale * q_i . k_j,  O_i = sum_j softmax(s)_j v_j,  LSE_i = ln sum_j exp(s_j)
+ * ("LVSA", §2 Mecanismo Central: attention restricted to A(t); §Complejidad: cost
+ *  O(|A(t)| P d) per query; "ISPA", §2.1: the per-row LSE kept by the kernel is what
+ *  makes two partial attentions mergeable).  An empty set gives O_i = 0, LSE_i = -inf.
+ * Attention is bidirectional inside every attended frame; nothing is token-causal.
+ *
+ * Layout: q [B][H][Tq*P][d], k and v [B][H][T_kv*P][d], o like q, all bf16, addressed
+ * as base + b*stride[0] + h*stride[1] + token*stride[2] + e (strides in elements; the
+ * d elements of a token are contiguous).  BHLD and BLHD layouts both fit.  Base
+ * addresses must be 16-byte aligned and strides multiples of 8 elements (TMA rule).
+ * lse is fp32 [B][H][Tq*P], contiguous.
+ * frames / counts as written by sfa_build_sets ([H][Tq][Amax], [H][Tq]; shared by all
+ * batch entries); each list must be strictly increasing inside [0, T_kv).
+ * Supported: d in {64, 128}, any P >= 1, any scale > 0 (the usual is 1/sqrt(d)).
+ * dev_status: optional device int32 (may be NULL), which the caller sets to 0; a
+ * device-side error stores its sfa_status there (first error wins) and the affected
+ * query tile's outputs are then unspecified.
+ * timeout_us: time limit of every pipeline wait inside the kernel (0 = 2 s).  When a wait
+ * runs out, its CTA stores SFA_ERR_TIMEOUT, drains its copies and tensor-core work, frees
+ * its tensor memory and exits; CTAs that start after that see the status and skip their
+ * work, so a broken pipeline costs about one time limit, not one per CTA.
+ */
+typedef struct {
+    int32_t B, H, Tq, T_kv, P, d;
+    float scale;
+    int32_t Amax;
+    int64_t q_stride[3]; /* batch, head, token */
+    int64_t k_stride[3];
+    int64_t v_stride[3];
+    int64_t o_stride[3];
+    uint32_t timeout_us;   /* limit of every pipeline wait in the kernel, microseconds;
+                              0 = 2 s (a healthy wait lasts microseconds) */
+    uint32_t debug_flags;  /* SFA_DEBUG_* below; 0 in normal use */
+} sfa_attn_desc;
+
+/* Test hook: the softmax warps never publish their first probability tile, so the
+ * tensor-core warp's wait for it runs out; the call must then report SFA_ERR_TIMEOUT
+ * through dev_status and still return cleanly. */
+#define SFA_DEBUG_STALL_SOFTMAX 1u
+
+sfa_status sfa_forward(const sfa_attn_desc *desc, const void *q, const void *k, const void *v,
+                       const int32_t *frames, const int32_t *counts, void *o, float *lse,
+                       int32_t *dev_status, sfa_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
+ * LSE merge
+ * ------------------------------------------------------------------------------------
+ * ("ISPA", §2.1 Dual-Stream Warmup and contribution 2: local and history branches of
+ *  attention, fused after the fact through their log-sum-exp.)  Per row r, with
+ *  M = max(L1, L2):
+ *     L = M + ln(exp(L1 - M) + exp(L2 - M)),  O = exp(L1 - L) O1 + exp(L2 - L) O2.
+ * A branch with L = -inf contributes nothing; both -inf gives O = 0, L = -inf.
+ * If the two branches cover disjoint key sets, (O, L) is attention over their union.
+ *   o1, o2, o: device bf16 [rows][d], contiguous rows; lse1, lse2, lse: device fp32
+ *   [rows].  o / lse may alias o1 / lse1 (in-place).  d in {64, 128}; rows >= 0.
+ * Math in fp32; O rounded to bf16 once.
+ */
+sfa_status sfa_lse_merge(int64_t rows, int32_t d, const void *o1, const float *lse1,
+                         const void *o2, const float *lse2, void *o, float *lse,
+                         sfa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SFA_H_ */

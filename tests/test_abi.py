@@ -1,0 +1,136 @@
+"""C-ABI checks that need no GPU: libsfa.so loads, exports every function that
+include/sfa.h declares, and rejects bad arguments on the host before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def sfa():
+    import frame_sparse_attention_b200 as sfa
+    from frame_sparse_attention_b200 import build
+    if not os.path.exists(build.LIB):
+        build.build()
+    sfa.load()
+    return sfa
+
+
+def _declared_functions():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"^\s*(?:const\s+)?\w+\s*\**\s*(sfa_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(sfa):
+    declared = _declared_functions()
+    assert {"sfa_build_sets", "sfa_forward", "sfa_lse_merge", "sfa_error_string"} <= set(declared)
+    lib = ctypes.CDLL(sfa._lib.LIB_PATH)
+    for name in declared:
+        assert hasattr(lib, name), f"{name} declared in include/ but not exported"
+    assert set(sfa._lib.EXPORTS) == set(declared)
+
+
+def test_error_strings_and_version(sfa):
+    for code in range(6):
+        assert sfa.error_string(code).startswith("SFA_")
+    assert "unknown" in sfa.error_string(99)
+    assert sfa.version() >= 100
+
+
+def test_set_max_count(sfa):
+    P = sfa.set_params
+    assert sfa.set_max_count(P(T_kv=41, Tq=41, C=21, W=9, T_per=4, step=0), ["lvsa"] * 12) == 21
+    assert sfa.set_max_count(P(T_kv=121, Tq=121, C=21, W=13, T_per=6), ["lvsa"] * 12) == 34
+    stream = P(T_kv=24, Tq=3, q_off=21, n_sink=1, n_prev=3, chunk_len=3)
+    kinds = ["local"] * 4 + ["anchor"] * 4 + ["memory"] * 4
+    assert sfa.set_max_count(stream, kinds, n_extra=6) == 13
+    assert sfa.set_max_count(P(T_kv=4, Tq=4, n_sink=1, n_prev=1, chunk_len=1), ["anchor"] * 2) == 3
+    assert sfa.set_max_count(P(T_kv=14, Tq=1, q_off=13), ["dense"]) == 14
+    assert sfa.set_max_count(P(T_kv=14, Tq=1, q_off=13), ["explicit"], n_extra=20) == 14
+
+
+@pytest.mark.parametrize("kw,kinds", [
+    (dict(T_kv=0, Tq=1), ["dense"]),
+    (dict(T_kv=4, Tq=3, q_off=2), ["dense"]),
+    (dict(T_kv=4, Tq=4, C=0, W=1, T_per=1), ["lvsa"]),
+    (dict(T_kv=4, Tq=4, C=2, W=1, T_per=0), ["lvsa"]),
+    (dict(T_kv=4, Tq=4, chunk_len=0), ["local"]),
+    (dict(T_kv=4, Tq=4), [7]),
+])
+def test_set_params_rejected(sfa, kw, kinds):
+    with pytest.raises(sfa.SfaError) as e:
+        sfa.set_max_count(sfa.set_params(**kw), kinds)
+    assert e.value.status == sfa.SFA_ERR_INVALID_ARG
+
+
+def test_build_sets_rejects_small_amax_without_launch(sfa):
+    lib = sfa.load()
+    p = sfa.set_params(T_kv=41, Tq=41, C=21, W=9, T_per=4)
+    kinds = (ctypes.c_int32 * 1)(1)
+    # Amax below the bound: refused on the host, the (bogus) device pointers are never used
+    assert lib.sfa_build_sets(ctypes.byref(p), 1, kinds, None, 0, 16, 16, 20, None) == sfa.SFA_ERR_INVALID_ARG
+    assert lib.sfa_build_sets(ctypes.byref(p), 1, kinds, None, 0, None, 16, 21, None) == sfa.SFA_ERR_INVALID_ARG
+    assert lib.sfa_build_sets(ctypes.byref(p), 0, kinds, None, 0, 16, 16, 21, None) == sfa.SFA_ERR_INVALID_ARG
+
+
+def _desc(sfa, **over):
+    d = sfa.AttnDesc()
+    d.B, d.H, d.Tq, d.T_kv, d.P, d.d, d.scale, d.Amax = 1, 2, 4, 4, 64, 64, 0.125, 4
+    for f in ("q_stride", "k_stride", "v_stride", "o_stride"):
+        arr = getattr(d, f)
+        arr[0], arr[1], arr[2] = 2 * 256 * 64, 256 * 64, 64
+    for k, v in over.items():
+        setattr(d, k, v)
+    return d
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(d=96), 2), (dict(d=32), 2), (dict(H=0), 1), (dict(P=0), 1), (dict(Amax=0), 1),
+    (dict(scale=0.0), 1), (dict(scale=float("nan")), 1), (dict(B=-1), 1),
+])
+def test_forward_rejects_bad_desc(sfa, over, code):
+    lib = sfa.load()
+    d = _desc(sfa, **over)
+    good = 1 << 20
+    assert lib.sfa_forward(ctypes.byref(d), good, good, good, good, good, good, good, None, None) == code
+
+
+def test_forward_rejects_bad_pointers_and_strides(sfa):
+    lib = sfa.load()
+    good = 1 << 20
+    d = _desc(sfa)
+    assert lib.sfa_forward(None, good, good, good, good, good, good, good, None, None) == 1
+    assert lib.sfa_forward(ctypes.byref(d), good + 2, good, good, good, good, good, good, None, None) == 1
+    assert lib.sfa_forward(ctypes.byref(d), good, good, good, None, good, good, good, None, None) == 1
+    d.k_stride[2] = 36  # token stride not a multiple of 8 elements (16 bytes)
+    assert lib.sfa_forward(ctypes.byref(d), good, good, good, good, good, good, good, None, None) == 1
+    d = _desc(sfa)
+    d.B = 0  # nothing to do
+    assert lib.sfa_forward(ctypes.byref(d), good, good, good, good, good, good, good, None, None) == 0
+
+
+def test_merge_rejects_bad_args(sfa):
+    lib = sfa.load()
+    good = 1 << 20
+    assert lib.sfa_lse_merge(-1, 128, good, good, good, good, good, good, None) == 1
+    assert lib.sfa_lse_merge(10, 96, good, good, good, good, good, good, None) == 2
+    assert lib.sfa_lse_merge(0, 128, None, None, None, None, None, None, None) == 0
+    assert lib.sfa_lse_merge(10, 128, good + 8, good, good, good, good, good, None) == 1
+
+
+def test_no_oracle_in_product_path():
+    # the product package and its C sources never reach for the oracle
+    pkg = os.path.join(ROOT, "frame_sparse_attention_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, fn)).read()
+                assert "oracle" not in text.lower(), f"{fn} mentions the oracle"
