@@ -80,7 +80,7 @@ class ClockSampler:
             os.close(fd)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
@@ -122,6 +122,9 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     w = WORKLOAD
+    if args.heads:
+        from dataclasses import replace
+        w = replace(w, H=args.heads, heads=w.heads[:1] * args.heads)
     kinds = [hs.kind for hs in w.heads]
     params = sfa.set_params(T_kv=w.Tkv, Tq=w.Tq, q_off=w.q_off, C=w.C, W=w.W, T_per=w.T_per,
                             step=STEP_S, n_sink=w.n_sink, n_prev=w.n_prev, chunk_len=w.chunk_len)
@@ -180,6 +183,13 @@ def run_ours(args, rank, world, local_rank):
         t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         total_ms = float(t.item())
+
+    if args.skip_extras:
+        return None if rank != 0 else {
+            "metric": METRIC, "value": round(flops * world / (total_ms / args.steps) / 1e9, 2),
+            "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(total_ms / args.steps, 4), "heads": w.H,
+            "forward_ms": round(float(np.mean(fwd_ms)), 4), "note": "device step only (--skip-extras)"}
 
     # end to end through the public API with host buffers: H2D of Q, K, V from pinned
     # memory, sets + attention, D2H of O and LSE into pinned memory, every step
@@ -380,6 +390,10 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--heads", type=int, default=0,
+                    help="run the workload with this many heads instead of 12 (smaller profiling case)")
+    ap.add_argument("--skip-extras", action="store_true",
+                    help="time the device step only: no end-to-end, merge or CPU-baseline legs")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

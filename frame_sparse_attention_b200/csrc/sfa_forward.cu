@@ -13,13 +13,15 @@
 //   * warp 4 (one thread) streams Q once and K/V tiles through a 3-stage (d = 128) or
 //     4-stage (d = 64) shared-memory ring with TMA, 128-byte swizzled;
 //   * warp 5 (one thread) issues tcgen05.mma: S = Q K^T into one of two TMEM S buffers
-//     while the softmax works on the other, then O += P V with P read from TMEM;
-//     a partial last tile uses an MMA N (for S) and K (for P V) rounded up to 16 only;
+//     (two tiles ahead of the softmax), then O += P V with P read from shared memory
+//     (both operands in shared memory: the tensor-memory-A form of this MMA runs at
+//     ~0.6x the rate on sm_100); a partial last tile uses an MMA N (for S) and K (for
+//     P V) rounded up to 16 only;
 //   * warps 0-3 (one thread per query row = TMEM lane) run the online softmax in fp32
 //     (exp2 with the scale folded into one FMA; O is rescaled only when a row's running
 //     max grows by more than 2^8, otherwise the stale max is kept), write P as bf16 into
-//     TMEM, and finally normalise O, stage it in shared memory and TMA-store it, clipped
-//     to the frame, plus the fp32 LSE.
+//     a 128-byte-swizzled shared-memory tile, and finally normalise O, stage it in shared
+//     memory and TMA-store it, clipped to the frame, plus the fp32 LSE.
 // Every mbarrier wait is bounded; a wait that runs out records SFA_ERR_TIMEOUT, the CTA
 // drains its in-flight copies and MMAs, frees its TMEM and returns.
 #include <cuda.h>
@@ -33,33 +35,66 @@
 #include "sfa_internal.h"
 #include "sfa_ptx.cuh"
 
+// K / V shared-memory ring depths (tiles); d = 64 tiles are half the size
+#ifndef SFA_RING_K
+#define SFA_RING_K (D == 128 ? 2 : 4)
+#endif
+#ifndef SFA_RING_V
+#define SFA_RING_V (D == 128 ? 2 : 4)
+#endif
+
 namespace sfa {
 namespace {
 
 constexpr int BM = 128;                 // query rows per tile = MMA M = TMEM lanes
 constexpr int BN = 128;                 // keys per K/V tile (largest MMA N used)
-constexpr int NUM_THREADS = 192;        // warps 0-3 softmax, 4 TMA producer, 5 MMA issuer
-constexpr int PRODUCER_WARP = 4;
+constexpr int NUM_THREADS = 224;        // warps 0-3 softmax, 4 Q+K loader, 5 MMA issuer, 6 V loader
+constexpr int K_LOAD_WARP = 4;
 constexpr int MMA_WARP = 5;
+constexpr int V_LOAD_WARP = 6;
 constexpr float RESCALE_LOG2 = 8.0f;    // keep a stale row max while the new one is < 2^8 above
 constexpr uint32_t DEFAULT_TIMEOUT_US = 2000000;  // 2 s; a healthy wait lasts microseconds
 constexpr uint32_t DRAIN_TIMEOUT_US = 2000000;
 constexpr uint32_t MAX_SPINS = 1u << 30;           // backstop should the timer not advance
 
-// tensor-memory columns (512 allocated: 2 x S fp32, O fp32, 2 x P bf16)
-constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_O = 256, TM_P0 = 384, TM_P1 = 448, TM_COLS = 512;
+// tensor-memory columns (512 allocated: 2 x S fp32, O fp32)
+constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_O = 256, TM_COLS = 512;
 
 template <int D>
 struct Cfg {
     static constexpr int KBOX = D / 64;                 // 128-byte swizzle boxes per row
     static constexpr int BOX_BYTES = 128 * 128;         // 128 rows x 64 bf16
     static constexpr int TILE_BYTES = BM * D * 2;       // one Q / K / V / O tile
-    static constexpr int NS = D == 128 ? 3 : 4;         // K/V ring depth
+    // separate K and V rings: a K slot frees once S of its tile is computed, a V slot
+    // once P V is; K therefore runs further ahead of the tensor cores than V
+    static constexpr int NSK = SFA_RING_K;
+    static constexpr int NSV = SFA_RING_V;
+    static constexpr int P_BYTES = BM * BN * 2;          // one bf16 probability tile
     static constexpr int SMEM_Q = 0;
-    static constexpr int SMEM_K = TILE_BYTES;
-    static constexpr int SMEM_V = SMEM_K + NS * TILE_BYTES;
-    static constexpr int SMEM_BAR = SMEM_V + NS * TILE_BYTES;
+    static constexpr int SMEM_P = TILE_BYTES;             // two P tiles (double buffer)
+    static constexpr int SMEM_K = SMEM_P + 2 * P_BYTES;
+    static constexpr int SMEM_V = SMEM_K + NSK * TILE_BYTES;
+    static constexpr int SMEM_BAR = SMEM_V + NSV * TILE_BYTES;
     static constexpr int SMEM_BYTES = SMEM_BAR + 256 + 1024;  // + barriers, + alignment slack
+    static_assert(2 * (NSK + NSV) + 9 <= 28, "mbarriers must fit in 224 bytes");
+    static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+};
+
+// mbarrier slots (8 bytes each) at SMEM_BAR
+template <int D>
+struct Bars {
+    uint32_t base;
+    __device__ uint32_t k_full(int s) const { return base + 8 * s; }
+    __device__ uint32_t k_empty(int s) const { return base + 8 * (Cfg<D>::NSK + s); }
+    __device__ uint32_t v_full(int s) const { return base + 8 * (2 * Cfg<D>::NSK + s); }
+    __device__ uint32_t v_empty(int s) const { return base + 8 * (2 * Cfg<D>::NSK + Cfg<D>::NSV + s); }
+    __device__ uint32_t q_full() const { return base + 8 * (2 * Cfg<D>::NSK + 2 * Cfg<D>::NSV); }
+    __device__ uint32_t s_full(int b) const { return q_full() + 8 + 8 * b; }   // S of a tile in TMEM
+    __device__ uint32_t p_full(int b) const { return q_full() + 24 + 8 * b; }  // P of a tile in TMEM
+    __device__ uint32_t p_free(int b) const { return q_full() + 40 + 8 * b; }  // P V done with a P buffer
+    __device__ uint32_t drain() const { return q_full() + 56; }
+    __device__ uint32_t o_final() const { return q_full() + 64; }              // after the last P V
+    static constexpr int COUNT = 2 * (Cfg<D>::NSK + Cfg<D>::NSV) + 9;
 };
 
 struct FwdArgs {
@@ -180,74 +215,76 @@ struct KvIter {
 __device__ __forceinline__ uint32_t mma_n(int nvalid) { return (uint32_t)((nvalid + 15) & ~15); }
 
 // ----------------------------------------------------------------- roles
-template <int D>
-__device__ void producer_role(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const CUtensorMap *tm_v,
-                              const FwdArgs &a, uint32_t sbase, int b, int h, int t, int qt, const int32_t *fl,
-                              int cnt, int n_tiles, const Ctl &ctl)
+// Streams the K tiles (IS_K, plus the Q tile first) or the V tiles of the attended
+// frames into their ring, one elected thread.
+template <int D, bool IS_K>
+__device__ void loader_role(const CUtensorMap *tm_q, const CUtensorMap *tm_kv, const FwdArgs &a, uint32_t sbase,
+                            int b, int h, int t, int qt, const int32_t *fl, int cnt, int n_tiles, const Ctl &ctl)
 {
     using C = Cfg<D>;
-    const uint32_t bars = sbase + C::SMEM_BAR;
-    const uint32_t q_full = bars + 8 * (3 * C::NS);
+    constexpr int NSR = IS_K ? C::NSK : C::NSV;
+    const Bars<D> bar{sbase + C::SMEM_BAR};
+    const uint32_t ring = sbase + (IS_K ? C::SMEM_K : C::SMEM_V);
     if (n_tiles <= 0) return;
-    mbar_arrive_expect_tx(q_full, C::TILE_BYTES);
+    if (IS_K) {
+        mbar_arrive_expect_tx(bar.q_full(), C::TILE_BYTES);
 #pragma unroll
-    for (int kb = 0; kb < C::KBOX; ++kb)
-        tma_load_5d(sbase + C::SMEM_Q + kb * C::BOX_BYTES, tm_q, q_full, kb * 64, qt * BM, t, h, b);
-
+        for (int kb = 0; kb < C::KBOX; ++kb)
+            tma_load_5d(sbase + C::SMEM_Q + kb * C::BOX_BYTES, tm_q, bar.q_full(), kb * 64, qt * BM, t, h, b);
+    }
     // K/V of one (h, t) are re-read by every query tile of the frame: keep them in L2
     const uint64_t policy = l2_policy_evict_last();
     KvIter it;
     it.init(fl, cnt, a.P);
     int j = 0;
     for (; j < n_tiles; ++j) {
-        const int s = j % C::NS;
-        const uint32_t k_full = bars + 8 * s, v_full = bars + 8 * (C::NS + s);
-        const uint32_t kv_empty = bars + 8 * (2 * C::NS + s);
-        if (j >= C::NS && !wait_bar(kv_empty, ((j / C::NS) - 1) & 1, ctl)) break;
+        const int s = j % NSR;
+        const uint32_t full = IS_K ? bar.k_full(s) : bar.v_full(s);
+        const uint32_t empty = IS_K ? bar.k_empty(s) : bar.v_empty(s);
+        if (j >= NSR && !wait_bar(empty, ((j / NSR) - 1) & 1, ctl)) break;
         int start, nv;
         it.next(start, nv);
-        mbar_arrive_expect_tx(k_full, C::TILE_BYTES);
+        mbar_arrive_expect_tx(full, C::TILE_BYTES);
 #pragma unroll
         for (int kb = 0; kb < C::KBOX; ++kb)
-            tma_load_4d(sbase + C::SMEM_K + s * C::TILE_BYTES + kb * C::BOX_BYTES, tm_k, k_full, kb * 64, start,
-                        h, b, policy);
-        mbar_arrive_expect_tx(v_full, C::TILE_BYTES);
-#pragma unroll
-        for (int kb = 0; kb < C::KBOX; ++kb)
-            tma_load_4d(sbase + C::SMEM_V + s * C::TILE_BYTES + kb * C::BOX_BYTES, tm_v, v_full, kb * 64, start,
-                        h, b, policy);
+            tma_load_4d(ring + s * C::TILE_BYTES + kb * C::BOX_BYTES, tm_kv, full, kb * 64, start, h, b, policy);
     }
     if (*ctl.abort) {  // let the copies still in flight land before the CTA exits
-        wait_drain(q_full, 0);
-        for (int jj = (j > C::NS ? j - C::NS : 0); jj < j; ++jj) {
-            const int s = jj % C::NS;
-            wait_drain(bars + 8 * s, (jj / C::NS) & 1);
-            wait_drain(bars + 8 * (C::NS + s), (jj / C::NS) & 1);
-        }
+        if (IS_K) wait_drain(bar.q_full(), 0);
+        for (int jj = (j > NSR ? j - NSR : 0); jj < j; ++jj)
+            wait_drain(IS_K ? bar.k_full(jj % NSR) : bar.v_full(jj % NSR), (jj / NSR) & 1);
     }
 }
 
+// Smem descriptors are built once per CTA; an operand at byte offset `off` from a
+// descriptor's base is that descriptor plus off >> 4 (the start address is the low 14
+// bits, in 16-byte units; every operand here lies below 256 KB, so nothing carries).
+__device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t off_bytes) { return desc + (off_bytes >> 4); }
+
 template <int D>
-__device__ __forceinline__ void issue_s(uint32_t t_s, uint32_t s_q, uint32_t s_k, uint32_t n)
+__device__ __forceinline__ void issue_s(uint32_t t_s, uint64_t dq, uint64_t dk, uint32_t idesc)
 {
-    // S[128 x n] = Q[128 x D] K[n x D]^T, both K-major; one MMA per 16 elements of D.
-    const uint32_t idesc = idesc_bf16_f32(BM, n, false);
+    // S[128 x n] = Q[128 x D] K[n x D]^T, both K-major; one MMA per 16 elements of D:
+    // +32 bytes inside a 128-byte swizzle row, the next 64 columns one box further on
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
         const uint32_t off = (kk >> 2) * Cfg<D>::BOX_BYTES + (kk & 3) * 32;
-        mma_ss(t_s, sdesc_sw128(s_q + off, 16, 1024), sdesc_sw128(s_k + off, 16, 1024), idesc, kk > 0);
+        mma_ss(t_s, desc_add(dq, off), desc_add(dk, off), idesc, kk > 0);
     }
 }
 
 template <int D>
-__device__ __forceinline__ void issue_pv(uint32_t t_o, uint32_t t_p, uint32_t s_v, uint32_t n, bool accumulate)
+__device__ __forceinline__ void issue_pv(uint32_t t_o, uint64_t dp, uint64_t dv, uint32_t n, bool accumulate)
 {
-    // O[128 x D] += P[128 x n] V[n x D]; P (bf16, 2 per column) from TMEM, V MN-major
-    // (D contiguous): 8-key groups 1024 B apart, 64-wide D blocks one box apart.
-    const uint32_t idesc = idesc_bf16_f32(BM, D, true);
-    for (uint32_t kk = 0; kk < n / 16; ++kk)
-        mma_ts(t_o, t_p + kk * 8, sdesc_sw128(s_v + kk * 2048, Cfg<D>::BOX_BYTES, 1024), idesc,
-               (accumulate || kk > 0) ? 1u : 0u);
+    // O[128 x D] += P[128 x n] V[n x D]; P K-major in shared memory (like Q), V MN-major
+    // (D contiguous): 8-key groups 1024 B apart, 64-wide D blocks one box apart
+    constexpr uint32_t idesc = idesc_bf16_f32(BM, D, true);
+    const uint32_t steps = n >> 4;
+#pragma unroll
+    for (uint32_t kk = 0; kk < 8; ++kk)
+        if (kk < steps)
+            mma_ss(t_o, desc_add(dp, (kk >> 2) * Cfg<D>::BOX_BYTES + (kk & 3) * 32), desc_add(dv, kk * 2048), idesc,
+                   (accumulate || kk > 0) ? 1u : 0u);
 }
 
 template <int D>
@@ -255,50 +292,214 @@ __device__ void mma_role(const FwdArgs &a, uint32_t sbase, uint32_t tmem, const 
                          int n_tiles, const Ctl &ctl)
 {
     using C = Cfg<D>;
-    const uint32_t bars = sbase + C::SMEM_BAR;
-    const uint32_t q_full = bars + 8 * (3 * C::NS);
-    const uint32_t s_full0 = q_full + 8, p_full0 = q_full + 24, o_done = q_full + 40, drain = q_full + 48;
-    const uint32_t o_final = q_full + 56;
-    const uint32_t s_q = sbase + C::SMEM_Q;
+    const Bars<D> bar{sbase + C::SMEM_BAR};
     if (n_tiles <= 0) return;
+    const uint64_t dq = sdesc_sw128(sbase + C::SMEM_Q, 16, 1024);
+    const uint64_t dk = sdesc_sw128(sbase + C::SMEM_K, 16, 1024);
+    const uint64_t dv = sdesc_sw128(sbase + C::SMEM_V, C::BOX_BYTES, 1024);
+    const uint64_t dp = sdesc_sw128(sbase + C::SMEM_P, 16, 1024);
     bool issued = false;
     KvIter it;
     it.init(fl, cnt, a.P);
-    int st, nv_cur, nv_next = 0;
-    it.next(st, nv_cur);
-    if (wait_bar(q_full, 0, ctl) && wait_bar(bars, 0, ctl)) {
+    // valid keys of tiles j, j+1, j+2 (S runs two tiles ahead of P V)
+    int st, nv0 = 0, nv1 = 0, nv2 = 0;
+    it.next(st, nv0);
+    if (n_tiles > 1) it.next(st, nv1);
+    if (!wait_bar(bar.q_full(), 0, ctl)) goto done;
+    // S of the first two tiles into the two S buffers
+    for (int j = 0; j < 2 && j < n_tiles; ++j) {
+        if (!wait_bar(bar.k_full(j), 0, ctl)) goto done;
         tc_fence_after();
-        issue_s<D>(tmem + TM_S0, s_q, sbase + C::SMEM_K, mma_n(nv_cur));
-        tc_commit(s_full0);
+        issue_s<D>(tmem + (j ? TM_S1 : TM_S0), dq, desc_add(dk, j * C::TILE_BYTES),
+                   idesc_bf16_f32(BM, mma_n(j ? nv1 : nv0), false));
+        tc_commit(bar.s_full(j));
+        tc_commit(bar.k_empty(j));
         issued = true;
-        for (int j = 0; j < n_tiles; ++j) {
-            if (j + 1 < n_tiles) {  // S for the next tile overlaps the softmax of this one
-                it.next(st, nv_next);
-                const int s1 = (j + 1) % C::NS;
-                if (!wait_bar(bars + 8 * s1, ((j + 1) / C::NS) & 1, ctl)) break;
-                tc_fence_after();
-                issue_s<D>(tmem + ((j + 1) & 1 ? TM_S1 : TM_S0), s_q, sbase + C::SMEM_K + s1 * C::TILE_BYTES,
-                           mma_n(nv_next));
-                tc_commit(s_full0 + 8 * ((j + 1) & 1));
-            }
-            const int s = j % C::NS;
-            if (!wait_bar(p_full0 + 8 * (j & 1), (j >> 1) & 1, ctl)) break;
-            if (!wait_bar(bars + 8 * (C::NS + s), (j / C::NS) & 1, ctl)) break;
+    }
+    for (int j = 0; j < n_tiles; ++j) {
+        // P of tile j published: its S buffer is free again, so S of tile j+2 goes to the
+        // tensor cores first (the softmax waits for it), P V of tile j after it
+        if (!wait_bar(bar.p_full(j & 1), (j >> 1) & 1, ctl)) break;
+        if (j + 2 < n_tiles) {
+            it.next(st, nv2);
+            const int sk = (j + 2) % C::NSK;
+            if (!wait_bar(bar.k_full(sk), ((j + 2) / C::NSK) & 1, ctl)) break;
             tc_fence_after();
-            issue_pv<D>(tmem + TM_O, tmem + ((j & 1) ? TM_P1 : TM_P0), sbase + C::SMEM_V + s * C::TILE_BYTES,
-                        mma_n(nv_cur), j > 0);
-            tc_commit(bars + 8 * (2 * C::NS + s));  // K/V stage free
-            tc_commit(o_done);                      // O holds tiles 0..j
-            nv_cur = nv_next;
-            // single-phase signal for the epilogue: with parity waits alone, the P V of the
-            // last two tiles can both be pending and would be indistinguishable
-            if (j == n_tiles - 1) tc_commit(o_final);
+            issue_s<D>(tmem + ((j & 1) ? TM_S1 : TM_S0), dq, desc_add(dk, sk * C::TILE_BYTES),
+                       idesc_bf16_f32(BM, mma_n(nv2), false));
+            tc_commit(bar.s_full(j & 1));
+            tc_commit(bar.k_empty(sk));  // K slot free once this S is computed
+        }
+        const int sv = j % C::NSV;
+        if (!wait_bar(bar.v_full(sv), (j / C::NSV) & 1, ctl)) break;
+        tc_fence_after();
+        issue_pv<D>(tmem + TM_O, desc_add(dp, (j & 1) * C::P_BYTES), desc_add(dv, sv * C::TILE_BYTES), mma_n(nv0),
+                    j > 0);
+        tc_commit(bar.v_empty(sv));    // V slot free
+        tc_commit(bar.p_free(j & 1));  // P buffer free, O holds tiles 0..j
+        // single-phase signal for the epilogue: with parity waits alone, the P V of the
+        // last two tiles can both be pending and would be indistinguishable
+        if (j == n_tiles - 1) tc_commit(bar.o_final());
+        nv0 = nv1;
+        nv1 = nv2;
+    }
+done:
+    if (*ctl.abort && issued) {  // wait for the tensor cores before TMEM is released
+        tc_commit(bar.drain());
+        wait_drain(bar.drain(), 0);
+    }
+}
+
+// Max of 32 values with 3-input max in a tree (depth 4).
+__device__ __forceinline__ float max32(const uint32_t (&r)[32])
+{
+    float t[11];
+#pragma unroll
+    for (int k = 0; k < 10; ++k)
+        t[k] = fmax3(__uint_as_float(r[3 * k]), __uint_as_float(r[3 * k + 1]), __uint_as_float(r[3 * k + 2]));
+    t[10] = fmaxf(__uint_as_float(r[30]), __uint_as_float(r[31]));
+    const float u0 = fmax3(t[0], t[1], t[2]), u1 = fmax3(t[3], t[4], t[5]), u2 = fmax3(t[6], t[7], t[8]);
+    return fmax3(fmax3(u0, u1, u2), t[9], t[10]);
+}
+
+// Columns at or past nv (partial tile) of a loaded 32-column chunk -> -inf.
+template <bool FULL>
+__device__ __forceinline__ void mask_chunk(int c, int nv, uint32_t (&r)[32])
+{
+    if (!FULL && (c + 1) * 32 > nv) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            if (c * 32 + i >= nv) r[i] = __float_as_uint(-INFINITY);
+    }
+}
+
+// Load 32 columns of this thread's S row; columns at or past nv (partial tile) -> -inf.
+template <bool FULL>
+__device__ __forceinline__ void load_s_chunk(uint32_t taddr, int c, int nv, uint32_t (&r)[32])
+{
+    tmem_ld32(taddr + c * 32, r);
+    tmem_wait_ld_regs(r);
+    if (!FULL && (c + 1) * 32 > nv) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            if (c * 32 + i >= nv) r[i] = __float_as_uint(-INFINITY);
+    }
+}
+
+// exp2(s * sl2 - m) of columns 32c..32c+31 -> bf16, stored into this thread's row of the
+// P tile in shared memory (K-major, 128-byte swizzle: 64 keys per 16 KB box, 16-byte
+// chunk k of row r at chunk position k ^ (r & 7)); row sum into acc
+__device__ __forceinline__ void exp_store_chunk(const uint32_t (&r)[32], float sl2, float neg_m, uint32_t p_row,
+                                                int row, int c, float (&acc)[8])
+{
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        uint32_t pk[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int e = q * 8 + 2 * i;
+            const float p0 = ex2_approx(fmaf(__uint_as_float(r[e]), sl2, neg_m));
+            const float p1 = ex2_approx(fmaf(__uint_as_float(r[e + 1]), sl2, neg_m));
+            acc[(2 * i) & 7] += p0;
+            acc[(2 * i + 1) & 7] += p1;
+            pk[i] = pack_bf16x2(p0, p1);
+        }
+        const uint32_t chunk = (uint32_t)((c & 1) * 4 + q);
+        st_shared_v4(p_row + (c >> 1) * 16384 + ((chunk ^ (uint32_t)(row & 7)) << 4), pk);
+    }
+}
+
+__device__ __forceinline__ float sum8(const float (&acc)[8])
+{
+    return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+}
+
+// One K/V tile of the online softmax for this thread's query row (thread = TMEM lane):
+// S (fp32, TMEM) -> P = exp2(S * scale * log2e - m) as bf16 into TMEM, running max m and
+// sum l.  A row keeps a stale max m until a tile's max exceeds it by 2^RESCALE_LOG2, so
+// the common case streams S through registers 32 columns at a time against the current
+// max.  The first tile, and a tile on which any lane of the warp finds a larger max,
+// take the exact two-pass path: row max first, then P (S is re-read from TMEM; P has
+// its own columns), and O is rescaled in place.  FULL: all 128 keys valid.
+// Returns false if a wait was abandoned.
+template <int D, bool FULL>
+__device__ __forceinline__ bool softmax_tile(uint32_t t_s, uint32_t p_row, int row, uint32_t t_o, int nv, float sl2,
+                                          float &m_used, float &l, int j, uint32_t p_free0, const Ctl &ctl)
+{
+    const int nch = FULL ? 4 : (nv + 31) >> 5;
+    // P of tile j goes to the buffer that P V of tile j-2 read: wait until it is done (S of
+    // tile j was committed after P V of tile j-3, so that is the only pending use)
+    if (j >= 2) {
+        const bool done = wait_bar(p_free0 + 8 * (j & 1), ((j >> 1) - 1) & 1, ctl);
+        if (!__all_sync(0xffffffffu, done)) return false;
+    }
+    if (j > 0) {  // streaming pass against the current max
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        bool grow = false;
+        const float neg_m = -m_used;
+        // two register buffers: the load of chunk c+1 is in flight while chunk c is used
+        uint32_t ra[32], rb[32];
+        tmem_ld32(t_s, ra);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            if (FULL || c < nch) {
+                uint32_t(&cur)[32] = (c & 1) ? rb : ra;
+                uint32_t(&nxt)[32] = (c & 1) ? ra : rb;
+                tmem_wait_ld_regs(cur);
+                if (c + 1 < 4 && (FULL || c + 1 < nch)) tmem_ld32(t_s + (c + 1) * 32, nxt);
+                mask_chunk<FULL>(c, nv, cur);
+                grow |= max32(cur) * sl2 > m_used + RESCALE_LOG2;
+                exp_store_chunk(cur, sl2, neg_m, p_row, row, c, acc);
+            }
+        }
+        if (!__any_sync(0xffffffffu, grow)) {
+            l += sum8(acc);
+            return true;
         }
     }
-    if (*ctl.abort && issued) {  // wait for the tensor cores before TMEM is released
-        tc_commit(drain);
-        wait_drain(drain, 0);
+    // exact pass: row max over the tile, then P against the new max
+    float mx = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        if (FULL || c < nch) {
+            uint32_t r[32];
+            load_s_chunk<FULL>(t_s, c, nv, r);
+            mx = fmaxf(mx, max32(r));
+        }
     }
+    const float m_cand = mx * sl2;
+    const bool resc = m_cand > m_used + RESCALE_LOG2;
+    const float m_new = resc ? m_cand : m_used;
+    const float alpha = ex2_approx(m_used - m_new);  // 0 on the first tile, 1 if unchanged
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        if (FULL || c < nch) {
+            uint32_t r[32];
+            load_s_chunk<FULL>(t_s, c, nv, r);
+            exp_store_chunk(r, sl2, -m_new, p_row, row, c, acc);
+        }
+    }
+    // O must be rescaled before P V of this tile accumulates into it; the warp does it
+    // together (tcgen05.ld/st are warp-wide) once P V of tile j-1 (and so every earlier
+    // one) is done.  Tile j-1's P buffer has no other pending use, so the parity is exact.
+    if (j > 0 && __any_sync(0xffffffffu, resc)) {
+        const bool done = wait_bar(p_free0 + 8 * ((j - 1) & 1), ((j - 1) >> 1) & 1, ctl);
+        if (!__all_sync(0xffffffffu, done)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(t_o + c * 32, o);
+            tmem_wait_ld_regs(o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(t_o + c * 32, o);
+        }
+    }
+    l = l * alpha + sum8(acc);
+    m_used = m_new;
+    return true;
 }
 
 template <int D>
@@ -307,10 +508,9 @@ __device__ void softmax_role(const CUtensorMap *tm_o, const FwdArgs &a, uint8_t 
                              bool bad_set, const Ctl &ctl)
 {
     using C = Cfg<D>;
-    const uint32_t bars = sbase + C::SMEM_BAR;
-    const uint32_t q_full = bars + 8 * (3 * C::NS);
-    const uint32_t s_full0 = q_full + 8, p_full0 = q_full + 24, o_done = q_full + 40;
-    const uint32_t o_final = q_full + 56;
+    const Bars<D> bar{sbase + C::SMEM_BAR};
+    const uint32_t s_full0 = bar.s_full(0), p_full0 = bar.p_full(0), p_free0 = bar.p_free(0);
+    const uint32_t o_final = bar.o_final();
     volatile int32_t *epi_ok = reinterpret_cast<volatile int32_t *>(smem + C::SMEM_BAR + 224);
     const int row = threadIdx.x;  // query row inside the tile == TMEM lane
     const int warp = row >> 5;
@@ -332,73 +532,16 @@ __device__ void softmax_role(const CUtensorMap *tm_o, const FwdArgs &a, uint8_t 
         }
         tc_fence_after();
         const uint32_t t_s = lane_base + ((j & 1) ? TM_S1 : TM_S0);
-        uint32_t sr[4][32];
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-            if (c * 32 < nv) tmem_ld32(t_s + c * 32, sr[c]);
-        tmem_wait_ld();
-
-        float mx = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            if (c * 32 < nv) {
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    if (nv < BN && c * 32 + i >= nv) sr[c][i] = __float_as_uint(-INFINITY);
-                    mx = fmaxf(mx, __uint_as_float(sr[c][i]));
-                }
-            }
+        const uint32_t p_row = sbase + C::SMEM_P + (j & 1) * C::P_BYTES + row * 128;
+        const bool ok = nv >= BN
+                            ? softmax_tile<D, true>(t_s, p_row, row, lane_base + TM_O, nv, sl2, m_used, l, j, p_free0, ctl)
+                            : softmax_tile<D, false>(t_s, p_row, row, lane_base + TM_O, nv, sl2, m_used, l, j, p_free0, ctl);
+        if (!ok) {
+            alive = false;
+            break;
         }
-        const float m_cand = mx * sl2;
-        const bool resc = m_cand > m_used + RESCALE_LOG2;
-        const float m_new = resc ? m_cand : m_used;
-        const float alpha = ex2_approx(m_used - m_new);  // 0 on the first tile, 1 if unchanged
-        const float neg_m = -m_new;
-
-        // P = exp2(s * scale * log2e - m) as bf16 pairs, stored to TMEM chunk by chunk
-        const uint32_t t_p = lane_base + ((j & 1) ? TM_P1 : TM_P0);
-        float rs0 = 0.f, rs1 = 0.f;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            if (c * 32 < nv) {
-                uint32_t pk[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c][2 * i]), sl2, neg_m));
-                    const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c][2 * i + 1]), sl2, neg_m));
-                    rs0 += p0;
-                    rs1 += p1;
-                    pk[i] = pack_bf16x2(p0, p1);
-                }
-                tmem_st16(t_p + c * 16, pk);
-            }
-        }
-
-        // O must be rescaled before P V of this tile accumulates into it; the warp
-        // does it together (tcgen05.ld/st are warp-wide) after P V of tile j-1 is done.
-        // The parity wait is unambiguous here: S of tile j was committed after P V of
-        // tile j-2, so only P V of tile j-1 can still be pending.
-        if (j > 0 && __any_sync(0xffffffffu, resc)) {
-            const bool done = wait_bar(o_done, (j - 1) & 1, ctl);
-            if (!__all_sync(0xffffffffu, done)) {
-                alive = false;
-                break;
-            }
-            tc_fence_after();
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t o[32];
-                tmem_ld32(lane_base + TM_O + c * 32, o);
-                tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                tmem_st32(lane_base + TM_O + c * 32, o);
-            }
-        }
-        l = l * alpha + (rs0 + rs1);
-        m_used = m_new;
-
-        tmem_wait_st();
+        tmem_wait_st();            // O rescale stores, if any
+        fence_proxy_async_smem();  // P written with st.shared is read by the tensor cores
         tc_fence_before();
         if (!((a.debug_flags & SFA_DEBUG_STALL_SOFTMAX) && j == 0)) mbar_arrive(p_full0 + 8 * (j & 1));
     }
@@ -421,7 +564,7 @@ __device__ void softmax_role(const CUtensorMap *tm_o, const FwdArgs &a, uint8_t 
             uint32_t o[32];
             if (n_tiles > 0) {
                 tmem_ld32(lane_base + TM_O + c * 32, o);
-                tmem_wait_ld();
+                tmem_wait_ld_regs(o);
             } else {
 #pragma unroll
                 for (int i = 0; i < 32; ++i) o[i] = 0u;
@@ -491,23 +634,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     volatile int32_t *skip = reinterpret_cast<volatile int32_t *>(smem + C::SMEM_BAR + 248);
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < 3 * C::NS; ++i) mbar_init(bars + 8 * i, 1);  // K full, V full, K/V empty
-        const uint32_t q_full = bars + 8 * (3 * C::NS);
-        mbar_init(q_full, 1);
-        mbar_init(q_full + 8, 1);        // S full x2 (tcgen05.commit)
-        mbar_init(q_full + 16, 1);
-        mbar_init(q_full + 24, BM);      // P full x2 (every softmax thread)
-        mbar_init(q_full + 32, BM);
-        mbar_init(q_full + 40, 1);       // O done (P V committed)
-        mbar_init(q_full + 48, 1);       // drain
-        mbar_init(q_full + 56, 1);       // O final (after the last P V)
+        const Bars<D> bar{bars};
+        for (int i = 0; i < Bars<D>::COUNT; ++i) mbar_init(bars + 8 * i, 1);
+        mbar_init(bar.p_full(0), BM);    // P full: every softmax thread arrives
+        mbar_init(bar.p_full(1), BM);
         *abort_flag = 0;
         // once a CTA has timed out, the ones that start later skip their work
         *skip = (a.status && *reinterpret_cast<volatile int32_t *>(a.status) == SFA_ERR_TIMEOUT) ? 1 : 0;
         fence_mbar_init();
         if (bad_set) report(a.status, SFA_ERR_BAD_SET);
     }
-    if (warp == PRODUCER_WARP && lane == 0) {
+    if (warp == K_LOAD_WARP && lane == 0) {
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
@@ -525,8 +662,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const bool skipped = *skip != 0;
     if (skipped) n_tiles = 0;
 
-    if (warp == PRODUCER_WARP) {
-        if (lane == 0) producer_role<D>(&tm_q, &tm_k, &tm_v, a, sbase, b, h, t, qt, fl, cnt, n_tiles, ctl);
+    if (warp == K_LOAD_WARP) {
+        if (lane == 0) loader_role<D, true>(&tm_q, &tm_k, a, sbase, b, h, t, qt, fl, cnt, n_tiles, ctl);
+    } else if (warp == V_LOAD_WARP) {
+        if (lane == 0) loader_role<D, false>(&tm_q, &tm_v, a, sbase, b, h, t, qt, fl, cnt, n_tiles, ctl);
     } else if (warp == MMA_WARP) {
         if (lane == 0) mma_role<D>(a, sbase, tmem, fl, cnt, n_tiles, ctl);
         __syncwarp();
