@@ -35,13 +35,6 @@
 #include "sfa_internal.h"
 #include "sfa_ptx.cuh"
 
-// K / V shared-memory ring depths (tiles); d = 64 tiles are half the size
-#ifndef SFA_RING_K
-#define SFA_RING_K (D == 128 ? 2 : 4)
-#endif
-#ifndef SFA_RING_V
-#define SFA_RING_V (D == 128 ? 2 : 4)
-#endif
 
 namespace sfa {
 namespace {
@@ -65,10 +58,11 @@ struct Cfg {
     static constexpr int KBOX = D / 64;                 // 128-byte swizzle boxes per row
     static constexpr int BOX_BYTES = 128 * 128;         // 128 rows x 64 bf16
     static constexpr int TILE_BYTES = BM * D * 2;       // one Q / K / V / O tile
-    // separate K and V rings: a K slot frees once S of its tile is computed, a V slot
-    // once P V is; K therefore runs further ahead of the tensor cores than V
-    static constexpr int NSK = SFA_RING_K;
-    static constexpr int NSV = SFA_RING_V;
+    // separate two-slot K and V rings: a K slot frees once S of its tile is computed (the
+    // loader waits on that S's own barrier), a V slot once P V is (it waits on the P
+    // buffer's release), so no extra tensor-core commits are needed for the rings
+    static constexpr int NSK = 2;
+    static constexpr int NSV = 2;
     static constexpr int P_BYTES = BM * BN * 2;          // one bf16 probability tile
     static constexpr int SMEM_Q = 0;
     static constexpr int SMEM_P = TILE_BYTES;             // two P tiles (double buffer)
@@ -76,7 +70,7 @@ struct Cfg {
     static constexpr int SMEM_V = SMEM_K + NSK * TILE_BYTES;
     static constexpr int SMEM_BAR = SMEM_V + NSV * TILE_BYTES;
     static constexpr int SMEM_BYTES = SMEM_BAR + 256 + 1024;  // + barriers, + alignment slack
-    static_assert(2 * (NSK + NSV) + 9 <= 28, "mbarriers must fit in 224 bytes");
+    static_assert(NSK + NSV + 9 <= 28, "mbarriers must fit in 224 bytes");
     static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 };
 
@@ -85,16 +79,14 @@ template <int D>
 struct Bars {
     uint32_t base;
     __device__ uint32_t k_full(int s) const { return base + 8 * s; }
-    __device__ uint32_t k_empty(int s) const { return base + 8 * (Cfg<D>::NSK + s); }
-    __device__ uint32_t v_full(int s) const { return base + 8 * (2 * Cfg<D>::NSK + s); }
-    __device__ uint32_t v_empty(int s) const { return base + 8 * (2 * Cfg<D>::NSK + Cfg<D>::NSV + s); }
-    __device__ uint32_t q_full() const { return base + 8 * (2 * Cfg<D>::NSK + 2 * Cfg<D>::NSV); }
+    __device__ uint32_t v_full(int s) const { return base + 8 * (Cfg<D>::NSK + s); }
+    __device__ uint32_t q_full() const { return base + 8 * (Cfg<D>::NSK + Cfg<D>::NSV); }
     __device__ uint32_t s_full(int b) const { return q_full() + 8 + 8 * b; }   // S of a tile in TMEM
     __device__ uint32_t p_full(int b) const { return q_full() + 24 + 8 * b; }  // P of a tile in TMEM
     __device__ uint32_t p_free(int b) const { return q_full() + 40 + 8 * b; }  // P V done with a P buffer
     __device__ uint32_t drain() const { return q_full() + 56; }
     __device__ uint32_t o_final() const { return q_full() + 64; }              // after the last P V
-    static constexpr int COUNT = 2 * (Cfg<D>::NSK + Cfg<D>::NSV) + 9;
+    static constexpr int COUNT = Cfg<D>::NSK + Cfg<D>::NSV + 9;
 };
 
 struct FwdArgs {
@@ -216,7 +208,8 @@ __device__ __forceinline__ uint32_t mma_n(int nvalid) { return (uint32_t)((nvali
 
 // ----------------------------------------------------------------- roles
 // Streams the K tiles (IS_K, plus the Q tile first) or the V tiles of the attended
-// frames into their ring, one elected thread.
+// frames into their ring.  The whole warp runs the loop (its state stays warp-uniform);
+// one elected lane issues each copy.
 template <int D, bool IS_K>
 __device__ void loader_role(const CUtensorMap *tm_q, const CUtensorMap *tm_kv, const FwdArgs &a, uint32_t sbase,
                             int b, int h, int t, int qt, const int32_t *fl, int cnt, int n_tiles, const Ctl &ctl)
@@ -226,12 +219,13 @@ __device__ void loader_role(const CUtensorMap *tm_q, const CUtensorMap *tm_kv, c
     const Bars<D> bar{sbase + C::SMEM_BAR};
     const uint32_t ring = sbase + (IS_K ? C::SMEM_K : C::SMEM_V);
     if (n_tiles <= 0) return;
-    if (IS_K) {
+    if (IS_K && elect_one()) {
         mbar_arrive_expect_tx(bar.q_full(), C::TILE_BYTES);
 #pragma unroll
         for (int kb = 0; kb < C::KBOX; ++kb)
             tma_load_5d(sbase + C::SMEM_Q + kb * C::BOX_BYTES, tm_q, bar.q_full(), kb * 64, qt * BM, t, h, b);
     }
+    __syncwarp();
     // K/V of one (h, t) are re-read by every query tile of the frame: keep them in L2
     const uint64_t policy = l2_policy_evict_last();
     KvIter it;
@@ -240,20 +234,31 @@ __device__ void loader_role(const CUtensorMap *tm_q, const CUtensorMap *tm_kv, c
     for (; j < n_tiles; ++j) {
         const int s = j % NSR;
         const uint32_t full = IS_K ? bar.k_full(s) : bar.v_full(s);
-        const uint32_t empty = IS_K ? bar.k_empty(s) : bar.v_empty(s);
-        if (j >= NSR && !wait_bar(empty, ((j / NSR) - 1) & 1, ctl)) break;
+        // slot s last held tile j-2: wait for its S (K ring) or P V (V ring).  Both
+        // barriers belong to buffer (j-2) & 1 and have exactly one pending phase here,
+        // because tile j's S or P V cannot run before this very load.
+        static_assert(NSR == 2, "the release waits below assume two-slot rings");
+        if (j >= 2) {
+            const int jj = j - 2;
+            const uint32_t rel = IS_K ? bar.s_full(jj & 1) : bar.p_free(jj & 1);
+            if (!__all_sync(0xffffffffu, wait_bar(rel, (jj >> 1) & 1, ctl))) break;
+        }
         int start, nv;
         it.next(start, nv);
-        mbar_arrive_expect_tx(full, C::TILE_BYTES);
+        if (elect_one()) {
+            mbar_arrive_expect_tx(full, C::TILE_BYTES);
 #pragma unroll
-        for (int kb = 0; kb < C::KBOX; ++kb)
-            tma_load_4d(ring + s * C::TILE_BYTES + kb * C::BOX_BYTES, tm_kv, full, kb * 64, start, h, b, policy);
+            for (int kb = 0; kb < C::KBOX; ++kb)
+                tma_load_4d(ring + s * C::TILE_BYTES + kb * C::BOX_BYTES, tm_kv, full, kb * 64, start, h, b, policy);
+        }
+        __syncwarp();
     }
     if (*ctl.abort) {  // let the copies still in flight land before the CTA exits
         if (IS_K) wait_drain(bar.q_full(), 0);
         for (int jj = (j > NSR ? j - NSR : 0); jj < j; ++jj)
             wait_drain(IS_K ? bar.k_full(jj % NSR) : bar.v_full(jj % NSR), (jj / NSR) & 1);
     }
+    __syncwarp();
 }
 
 // Smem descriptors are built once per CTA; an operand at byte offset `off` from a
@@ -266,11 +271,14 @@ __device__ __forceinline__ void issue_s(uint32_t t_s, uint64_t dq, uint64_t dk, 
 {
     // S[128 x n] = Q[128 x D] K[n x D]^T, both K-major; one MMA per 16 elements of D:
     // +32 bytes inside a 128-byte swizzle row, the next 64 columns one box further on
+    if (elect_one()) {
 #pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * Cfg<D>::BOX_BYTES + (kk & 3) * 32;
-        mma_ss(t_s, desc_add(dq, off), desc_add(dk, off), idesc, kk > 0);
+        for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * Cfg<D>::BOX_BYTES + (kk & 3) * 32;
+            mma_ss(t_s, desc_add(dq, off), desc_add(dk, off), idesc, kk > 0);
+        }
     }
+    __syncwarp();
 }
 
 template <int D>
@@ -280,11 +288,21 @@ __device__ __forceinline__ void issue_pv(uint32_t t_o, uint64_t dp, uint64_t dv,
     // (D contiguous): 8-key groups 1024 B apart, 64-wide D blocks one box apart
     constexpr uint32_t idesc = idesc_bf16_f32(BM, D, true);
     const uint32_t steps = n >> 4;
+    if (elect_one()) {
 #pragma unroll
-    for (uint32_t kk = 0; kk < 8; ++kk)
-        if (kk < steps)
-            mma_ss(t_o, desc_add(dp, (kk >> 2) * Cfg<D>::BOX_BYTES + (kk & 3) * 32), desc_add(dv, kk * 2048), idesc,
-                   (accumulate || kk > 0) ? 1u : 0u);
+        for (uint32_t kk = 0; kk < 8; ++kk)
+            if (kk < steps)
+                mma_ss(t_o, desc_add(dp, (kk >> 2) * Cfg<D>::BOX_BYTES + (kk & 3) * 32), desc_add(dv, kk * 2048),
+                       idesc, (accumulate || kk > 0) ? 1u : 0u);
+    }
+    __syncwarp();
+}
+
+// tcgen05.commit from one elected lane of the (converged) MMA warp
+__device__ __forceinline__ void commit_one(uint32_t bar)
+{
+    if (elect_one()) tc_commit(bar);
+    __syncwarp();
 }
 
 template <int D>
@@ -305,49 +323,48 @@ __device__ void mma_role(const FwdArgs &a, uint32_t sbase, uint32_t tmem, const 
     int st, nv0 = 0, nv1 = 0, nv2 = 0;
     it.next(st, nv0);
     if (n_tiles > 1) it.next(st, nv1);
-    if (!wait_bar(bar.q_full(), 0, ctl)) goto done;
+    if (!__all_sync(0xffffffffu, wait_bar(bar.q_full(), 0, ctl))) goto done;
     // S of the first two tiles into the two S buffers
     for (int j = 0; j < 2 && j < n_tiles; ++j) {
-        if (!wait_bar(bar.k_full(j), 0, ctl)) goto done;
+        if (!__all_sync(0xffffffffu, wait_bar(bar.k_full(j), 0, ctl))) goto done;
         tc_fence_after();
         issue_s<D>(tmem + (j ? TM_S1 : TM_S0), dq, desc_add(dk, j * C::TILE_BYTES),
                    idesc_bf16_f32(BM, mma_n(j ? nv1 : nv0), false));
-        tc_commit(bar.s_full(j));
-        tc_commit(bar.k_empty(j));
+        commit_one(bar.s_full(j));
         issued = true;
     }
     for (int j = 0; j < n_tiles; ++j) {
         // P of tile j published: its S buffer is free again, so S of tile j+2 goes to the
         // tensor cores first (the softmax waits for it), P V of tile j after it
-        if (!wait_bar(bar.p_full(j & 1), (j >> 1) & 1, ctl)) break;
+        if (!__all_sync(0xffffffffu, wait_bar(bar.p_full(j & 1), (j >> 1) & 1, ctl))) break;
         if (j + 2 < n_tiles) {
             it.next(st, nv2);
             const int sk = (j + 2) % C::NSK;
-            if (!wait_bar(bar.k_full(sk), ((j + 2) / C::NSK) & 1, ctl)) break;
+            if (!__all_sync(0xffffffffu, wait_bar(bar.k_full(sk), ((j + 2) / C::NSK) & 1, ctl))) break;
             tc_fence_after();
             issue_s<D>(tmem + ((j & 1) ? TM_S1 : TM_S0), dq, desc_add(dk, sk * C::TILE_BYTES),
                        idesc_bf16_f32(BM, mma_n(nv2), false));
-            tc_commit(bar.s_full(j & 1));
-            tc_commit(bar.k_empty(sk));  // K slot free once this S is computed
+            commit_one(bar.s_full(j & 1));  // S ready; also frees its K slot
         }
         const int sv = j % C::NSV;
-        if (!wait_bar(bar.v_full(sv), (j / C::NSV) & 1, ctl)) break;
+        if (!__all_sync(0xffffffffu, wait_bar(bar.v_full(sv), (j / C::NSV) & 1, ctl))) break;
         tc_fence_after();
         issue_pv<D>(tmem + TM_O, desc_add(dp, (j & 1) * C::P_BYTES), desc_add(dv, sv * C::TILE_BYTES), mma_n(nv0),
                     j > 0);
-        tc_commit(bar.v_empty(sv));    // V slot free
-        tc_commit(bar.p_free(j & 1));  // P buffer free, O holds tiles 0..j
+        commit_one(bar.p_free(j & 1));  // P buffer and V slot free, O holds tiles 0..j
         // single-phase signal for the epilogue: with parity waits alone, the P V of the
         // last two tiles can both be pending and would be indistinguishable
-        if (j == n_tiles - 1) tc_commit(bar.o_final());
+        if (j == n_tiles - 1) commit_one(bar.o_final());
         nv0 = nv1;
         nv1 = nv2;
     }
 done:
-    if (*ctl.abort && issued) {  // wait for the tensor cores before TMEM is released
-        tc_commit(bar.drain());
+    // (warp-uniform decision: the drain commit below is issued by an elected lane)
+    if (__any_sync(0xffffffffu, *ctl.abort != 0) && issued) {  // wait for the tensor cores before TMEM is released
+        commit_one(bar.drain());
         wait_drain(bar.drain(), 0);
     }
+    __syncwarp();
 }
 
 // Max of 32 values with 3-input max in a tree (depth 4).
@@ -663,12 +680,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (skipped) n_tiles = 0;
 
     if (warp == K_LOAD_WARP) {
-        if (lane == 0) loader_role<D, true>(&tm_q, &tm_k, a, sbase, b, h, t, qt, fl, cnt, n_tiles, ctl);
+        loader_role<D, true>(&tm_q, &tm_k, a, sbase, b, h, t, qt, fl, cnt, n_tiles, ctl);
     } else if (warp == V_LOAD_WARP) {
-        if (lane == 0) loader_role<D, false>(&tm_q, &tm_v, a, sbase, b, h, t, qt, fl, cnt, n_tiles, ctl);
+        loader_role<D, false>(&tm_q, &tm_v, a, sbase, b, h, t, qt, fl, cnt, n_tiles, ctl);
     } else if (warp == MMA_WARP) {
-        if (lane == 0) mma_role<D>(a, sbase, tmem, fl, cnt, n_tiles, ctl);
-        __syncwarp();
+        mma_role<D>(a, sbase, tmem, fl, cnt, n_tiles, ctl);
     } else {
         if (!skipped) softmax_role<D>(&tm_o, a, smem, sbase, tmem, b, h, t, qt, fl, cnt, n_tiles, bad_set, ctl);
     }
