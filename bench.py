@@ -57,6 +57,27 @@ def measured_peaks():
     return p
 
 
+# DRAM bytes (read + write) of one forward launch on this workload: one ncu capture of the
+# same kernel on the 4-head version of the workload (196.77 MB read + 52.34 MB written),
+# scaled by 3 to 12 heads (the traffic is per (head, frame, query tile) unit).  Must be
+# re-measured whenever the forward kernel changes.
+NCU_TRAFFIC_BYTES = 3 * (196_768_512 + 52_340_736)
+
+
+def max_over_ranks(x: float, device) -> float:
+    """Max of a per-rank scalar over all ranks (identity without a process group)."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate_tflops(flops_per_rank: float, world: int, ms_per_step: float) -> float:
+    """Whole-job rate: every rank does flops_per_rank per step; time is the slowest rank's."""
+    return flops_per_rank * world / (ms_per_step * 1e-3) / 1e12
+
+
 def attended_flops(counts: np.ndarray, w) -> float:
     """4 d sum_{b,h,t} P * P |A(h,t)| (QK^T + PV, attended pairs only)."""
     return 4.0 * w.d * w.B * float(counts.sum()) * w.P * w.P
@@ -178,15 +199,11 @@ def run_ours(args, rank, world, local_rank):
     sets_ms = [e0.elapsed_time(e1) for e0, e1, _ in ev]
     if status.item() != 0:
         raise RuntimeError(f"device status {sfa.error_string(status.item())}")
-    total_ms = float(sum(step_ms))
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(float(sum(step_ms)), dev)
 
     if args.skip_extras:
         return None if rank != 0 else {
-            "metric": METRIC, "value": round(flops * world / (total_ms / args.steps) / 1e9, 2),
+            "metric": METRIC, "value": round(job_rate_tflops(flops, world, total_ms / args.steps), 2),
             "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(total_ms / args.steps, 4), "heads": w.H,
             "forward_ms": round(float(np.mean(fwd_ms)), 4), "note": "device step only (--skip-extras)"}
@@ -217,11 +234,7 @@ def run_ours(args, rank, world, local_rank):
         e2e_step()
     s1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = s0.elapsed_time(s1) / n_e2e
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(s0.elapsed_time(s1) / n_e2e, dev)
     h2d = sum(x.numel() * x.element_size() for x in (q_h, k_h, v_h))
     d2h = o_p.numel() * o_p.element_size() + lse_p.numel() * lse_p.element_size()
 
@@ -231,7 +244,7 @@ def run_ours(args, rank, world, local_rank):
         return None
     peaks = measured_peaks()
     ms_per_step = total_ms / args.steps
-    value = flops * world / (total_ms / args.steps) / 1e9  # TFLOP/s, whole job
+    value = job_rate_tflops(flops, world, ms_per_step)  # whole job
     fwd_avg = float(np.mean(fwd_ms))
     achieved = flops / (fwd_avg * 1e-3) / 1e12
     peak = float(peaks["bf16_tflops"])
@@ -258,9 +271,10 @@ def run_ours(args, rank, world, local_rank):
                      "frac": round(achieved / peak, 4),
                      "peak_source": f"{peaks['source']} bf16_tflops (burst)",
                      "frac_of_sustained": round(achieved / float(peaks["bf16_tflops_sustained"]), 4),
-                     "traffic": None,
+                     "traffic": NCU_TRAFFIC_BYTES if w.H == 12 else None,
+                     "traffic_note": "DRAM read+write bytes per launch, ncu capture of the 4-head case x 3",
                      "forward_ms": round(fwd_avg, 4), "set_build_ms": round(float(np.mean(sets_ms)), 4)},
-        "e2e": {"value": round(flops * world / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+        "e2e": {"value": round(job_rate_tflops(flops, world, e2e_ms), 2), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": 2 * args.steps,
         "clocks": clk,
@@ -382,6 +396,68 @@ def run_reference(args, rank):
     }
 
 
+def run_other_workload(args):
+    """Device time of one step of another workload (set build + forward per branch; the
+    LSE-decomposed workload adds the merge of its local and history branches)."""
+    import frame_sparse_attention_b200 as sfa
+    sfa.load()
+    dev = torch.device("cuda", 0)
+    names = {"long121": ["long121"], "stream": ["stream"],
+             "lsemerge": ["lsemerge_local", "lsemerge_hist"]}[args.workload]
+    ws = [WORKLOADS[n] for n in names]
+    q_h, k_h, v_h = workload_qkv(ws[0], seed=0)
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    branches = []
+    for w in ws:
+        kinds = [hs.kind for hs in w.heads]
+        n_extra = max((len(hs.extra) for hs in w.heads), default=0)
+        extra = None
+        if n_extra:
+            ex = torch.full((w.H, n_extra), -1, dtype=torch.int32)
+            for h, hs in enumerate(w.heads):
+                ex[h, :len(hs.extra)] = torch.tensor(hs.extra, dtype=torch.int32)
+            extra = ex.to(dev)
+        params = sfa.set_params(T_kv=w.Tkv, Tq=w.Tq, q_off=w.q_off, C=max(w.C, 1), W=max(w.W, 1),
+                                T_per=w.T_per, step=0, n_sink=w.n_sink, n_prev=w.n_prev,
+                                chunk_len=w.chunk_len)
+        Amax = max(1, sfa.set_max_count(params, kinds, n_extra))
+        fr = torch.empty((w.H, w.Tq, Amax), dtype=torch.int32, device=dev)
+        cn = torch.empty((w.H, w.Tq), dtype=torch.int32, device=dev)
+        branches.append((w, params, kinds, extra, Amax, fr, cn, torch.empty_like(q),
+                         torch.empty((w.B, w.H, w.Lq), dtype=torch.float32, device=dev)))
+    merged = (torch.empty_like(q), torch.empty((ws[0].B, ws[0].H, ws[0].Lq), dtype=torch.float32, device=dev))
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        for (w, params, kinds, extra, Amax, fr, cn, o, lse) in branches:
+            sfa.build_sets(params, kinds, extra, Amax, fr, cn, stream=stream)
+            sfa.forward(q, k, v, fr, cn, w.P, out=o, lse=lse, stream=stream)
+        if len(branches) == 2:
+            sfa.lse_merge(branches[0][7], branches[0][8], branches[1][7], branches[1][8],
+                          out=merged[0], lse=merged[1], stream=stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    flops = sum(attended_flops(b[6].cpu().numpy(), b[0]) for b in branches)
+    times = []
+    for _ in range(args.steps):
+        flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        times.append(e0.elapsed_time(e1))
+    ms = float(np.median(times))
+    return {"workload": args.workload, "branches": names, "attended_tflop_per_step": round(flops / 1e12, 4),
+            "ms_per_step": round(ms, 4), "tflops": round(flops / (ms * 1e-3) / 1e12, 1),
+            "steps": args.steps, "warmup": args.warmup, "note": "device time, median, L2 flushed between steps"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -394,6 +470,8 @@ def main():
                     help="run the workload with this many heads instead of 12 (smaller profiling case)")
     ap.add_argument("--skip-extras", action="store_true",
                     help="time the device step only: no end-to-end, merge or CPU-baseline legs")
+    ap.add_argument("--workload", choices=["lvsa41", "long121", "stream", "lsemerge"], default="lvsa41",
+                    help="other workloads are timed on the device only (one JSON line, not the bench line)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -401,6 +479,11 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.workload != "lvsa41":
+        if rank == 0:
+            print(json.dumps(run_other_workload(args)), flush=True)
+        return
 
     if args.impl == "reference":
         rec = run_reference(args, rank)
