@@ -423,16 +423,23 @@ def run_other_workload(args):
         Amax = max(1, sfa.set_max_count(params, kinds, n_extra))
         fr = torch.empty((w.H, w.Tq, Amax), dtype=torch.int32, device=dev)
         cn = torch.empty((w.H, w.Tq), dtype=torch.int32, device=dev)
-        branches.append((w, params, kinds, extra, Amax, fr, cn, torch.empty_like(q),
-                         torch.empty((w.B, w.H, w.Lq), dtype=torch.float32, device=dev)))
+        o_b = torch.empty_like(q)
+        desc = sfa.attn_desc(q, k, v, o_b, w.P, Amax)
+        ws_bytes = sfa.split_workspace_bytes(desc, args.split)
+        wsp = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+        branches.append((w, params, kinds, extra, Amax, fr, cn, o_b,
+                         torch.empty((w.B, w.H, w.Lq), dtype=torch.float32, device=dev), wsp))
     merged = (torch.empty_like(q), torch.empty((ws[0].B, ws[0].H, ws[0].Lq), dtype=torch.float32, device=dev))
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        for (w, params, kinds, extra, Amax, fr, cn, o, lse) in branches:
+        for (w, params, kinds, extra, Amax, fr, cn, o, lse, wsp) in branches:
             sfa.build_sets(params, kinds, extra, Amax, fr, cn, stream=stream)
-            sfa.forward(q, k, v, fr, cn, w.P, out=o, lse=lse, stream=stream)
+            if args.split > 1:
+                sfa.forward_split(q, k, v, fr, cn, w.P, args.split, out=o, lse=lse, workspace=wsp, stream=stream)
+            else:
+                sfa.forward(q, k, v, fr, cn, w.P, out=o, lse=lse, stream=stream)
         if len(branches) == 2:
             sfa.lse_merge(branches[0][7], branches[0][8], branches[1][7], branches[1][8],
                           out=merged[0], lse=merged[1], stream=stream)
@@ -453,7 +460,7 @@ def run_other_workload(args):
         torch.cuda.synchronize(dev)
         times.append(e0.elapsed_time(e1))
     ms = float(np.median(times))
-    return {"workload": args.workload, "branches": names, "attended_tflop_per_step": round(flops / 1e12, 4),
+    return {"workload": args.workload, "branches": names, "split": args.split, "attended_tflop_per_step": round(flops / 1e12, 4),
             "ms_per_step": round(ms, 4), "tflops": round(flops / (ms * 1e-3) / 1e12, 1),
             "steps": args.steps, "warmup": args.warmup, "note": "device time, median, L2 flushed between steps"}
 
@@ -472,6 +479,8 @@ def main():
                     help="time the device step only: no end-to-end, merge or CPU-baseline legs")
     ap.add_argument("--workload", choices=["lvsa41", "long121", "stream", "lsemerge"], default="lvsa41",
                     help="other workloads are timed on the device only (one JSON line, not the bench line)")
+    ap.add_argument("--split", type=int, default=1,
+                    help="split-KV ranges per unit for --workload other than lvsa41 (sfa_forward_split)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -5,16 +5,18 @@ Python face of libsfa.so (C ABI in include/sfa.h):
 * ``build_sets``  - attended frame sets A(h, t) (LVSA anchors + window, sink/local/memory
                     caches, explicit lists), built on the GPU
 * ``forward``     - softmax attention over the tokens of A(h, t) only, O bf16 + LSE fp32
+* ``forward_split`` - the same with each unit's key tiles split over several CTAs and the
+                    partials merged by LSE (short or uneven grids)
 * ``lse_merge``   - merge of two partial attentions (local + history branch) by LSE
 
 Tensors are PyTorch CUDA tensors; calls run on the current CUDA stream.
 """
 from ._lib import (SET_KINDS, SFA_DEBUG_STALL_SOFTMAX, SFA_ERR_BAD_SET, SFA_ERR_CUDA,
                    SFA_ERR_INVALID_ARG, SFA_ERR_TIMEOUT, SFA_ERR_UNSUPPORTED, SFA_OK, AttnDesc,
-                   SetParams, SfaError, attn_desc, build_sets, error_string, forward, load,
-                   lse_merge, set_max_count, set_params, version)
+                   SetParams, SfaError, attn_desc, build_sets, error_string, forward, forward_split,
+                   load, lse_merge, set_max_count, set_params, split_workspace_bytes, version)
 
 __all__ = ["SET_KINDS", "SFA_DEBUG_STALL_SOFTMAX", "SFA_ERR_BAD_SET", "SFA_ERR_CUDA",
            "SFA_ERR_INVALID_ARG", "SFA_ERR_TIMEOUT", "SFA_ERR_UNSUPPORTED", "SFA_OK", "AttnDesc",
-           "SetParams", "SfaError", "attn_desc", "build_sets", "error_string", "forward", "load",
-           "lse_merge", "set_max_count", "set_params", "version"]
+           "SetParams", "SfaError", "attn_desc", "build_sets", "error_string", "forward", "forward_split",
+           "load", "lse_merge", "set_max_count", "set_params", "split_workspace_bytes", "version"]

@@ -51,7 +51,7 @@ class AttnDesc(ctypes.Structure):
 
 _lib = None
 EXPORTS = ("sfa_error_string", "sfa_version", "sfa_set_max_count", "sfa_build_sets", "sfa_forward",
-           "sfa_lse_merge")
+           "sfa_forward_split_workspace", "sfa_forward_split", "sfa_lse_merge")
 
 
 def load():
@@ -76,6 +76,11 @@ def load():
                                    i32, vp]
     lib.sfa_forward.restype = st
     lib.sfa_forward.argtypes = [ctypes.POINTER(AttnDesc), vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.sfa_forward_split_workspace.restype = st
+    lib.sfa_forward_split_workspace.argtypes = [ctypes.POINTER(AttnDesc), i32, ctypes.POINTER(ctypes.c_size_t)]
+    lib.sfa_forward_split.restype = st
+    lib.sfa_forward_split.argtypes = [ctypes.POINTER(AttnDesc), vp, vp, vp, vp, vp, vp, vp, i32, vp,
+                                      ctypes.c_size_t, vp, vp]
     lib.sfa_lse_merge.restype = st
     lib.sfa_lse_merge.argtypes = [i64, i32, vp, vp, vp, vp, vp, vp, vp]
     _lib = lib
@@ -185,6 +190,36 @@ def forward(q, k, v, frames, counts, P: int, scale: float | None = None, out=Non
     _check(load().sfa_forward(ctypes.byref(desc), q.data_ptr(), k.data_ptr(), v.data_ptr(),
                               frames.data_ptr(), counts.data_ptr(), out.data_ptr(), lse.data_ptr(),
                               _ptr(dev_status), _stream(stream)), "sfa_forward")
+    return out, lse
+
+
+def split_workspace_bytes(desc: AttnDesc, n_split: int) -> int:
+    out = ctypes.c_size_t(0)
+    _check(load().sfa_forward_split_workspace(ctypes.byref(desc), n_split, ctypes.byref(out)),
+           "sfa_forward_split_workspace")
+    return out.value
+
+
+def forward_split(q, k, v, frames, counts, P: int, n_split: int, scale: float | None = None, out=None,
+                  lse=None, workspace=None, dev_status=None, stream=None, timeout_us: int = 0):
+    """Split-KV frame-sparse attention (same result as forward); workspace is allocated
+    here with torch when not given."""
+    B, H, Lq, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, Lq), dtype=torch.float32, device=q.device)
+    assert frames.dtype == torch.int32 and counts.dtype == torch.int32
+    assert frames.is_contiguous() and counts.is_contiguous() and lse.is_contiguous()
+    desc = attn_desc(q, k, v, out, P, frames.shape[2], scale, timeout_us)
+    need = split_workspace_bytes(desc, n_split)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load().sfa_forward_split(ctypes.byref(desc), q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                    frames.data_ptr(), counts.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                    n_split, _ptr(workspace), ws_bytes, _ptr(dev_status), _stream(stream)),
+           "sfa_forward_split")
     return out, lse
 
 

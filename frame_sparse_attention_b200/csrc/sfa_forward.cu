@@ -185,22 +185,39 @@ struct KvIter {
         pos = 0;
         end = 0;
     }
+    __device__ void open_run()
+    {
+        const int f0 = __ldg(fl + a);
+        int f1 = f0;
+        ++a;
+        while (a < n && __ldg(fl + a) == f1 + 1) {
+            ++f1;
+            ++a;
+        }
+        pos = f0 * P;
+        end = (f1 + 1) * P;
+    }
     __device__ void next(int &start, int &nvalid)
     {
-        if (pos >= end) {
-            const int f0 = __ldg(fl + a);
-            int f1 = f0;
-            ++a;
-            while (a < n && __ldg(fl + a) == f1 + 1) {
-                ++f1;
-                ++a;
-            }
-            pos = f0 * P;
-            end = (f1 + 1) * P;
-        }
+        if (pos >= end) open_run();
         start = pos;
         nvalid = min(BN, end - pos);
         pos += BN;
+    }
+    // skip the first k tiles (whole runs at a time)
+    __device__ void skip(int k)
+    {
+        while (k > 0) {
+            if (pos >= end) open_run();
+            const int left = (end - pos + BN - 1) / BN;
+            if (k >= left) {
+                k -= left;
+                pos = end;
+            } else {
+                pos += k * BN;
+                k = 0;
+            }
+        }
     }
 };
 
@@ -212,7 +229,8 @@ __device__ __forceinline__ uint32_t mma_n(int nvalid) { return (uint32_t)((nvali
 // one elected lane issues each copy.
 template <int D, bool IS_K>
 __device__ void loader_role(const CUtensorMap *tm_q, const CUtensorMap *tm_kv, const FwdArgs &a, uint32_t sbase,
-                            int b, int h, int t, int qt, const int32_t *fl, int cnt, int n_tiles, const Ctl &ctl)
+                            int b, int h, int t, int qt, const int32_t *fl, int cnt, int t_off, int n_tiles,
+                            const Ctl &ctl)
 {
     using C = Cfg<D>;
     constexpr int NSR = IS_K ? C::NSK : C::NSV;
@@ -230,6 +248,7 @@ __device__ void loader_role(const CUtensorMap *tm_q, const CUtensorMap *tm_kv, c
     const uint64_t policy = l2_policy_evict_last();
     KvIter it;
     it.init(fl, cnt, a.P);
+    it.skip(t_off);
     int j = 0;
     for (; j < n_tiles; ++j) {
         const int s = j % NSR;
@@ -306,7 +325,7 @@ __device__ __forceinline__ void commit_one(uint32_t bar)
 }
 
 template <int D>
-__device__ void mma_role(const FwdArgs &a, uint32_t sbase, uint32_t tmem, const int32_t *fl, int cnt,
+__device__ void mma_role(const FwdArgs &a, uint32_t sbase, uint32_t tmem, const int32_t *fl, int cnt, int t_off,
                          int n_tiles, const Ctl &ctl)
 {
     using C = Cfg<D>;
@@ -319,6 +338,7 @@ __device__ void mma_role(const FwdArgs &a, uint32_t sbase, uint32_t tmem, const 
     bool issued = false;
     KvIter it;
     it.init(fl, cnt, a.P);
+    it.skip(t_off);
     // valid keys of tiles j, j+1, j+2 (S runs two tiles ahead of P V)
     int st, nv0 = 0, nv1 = 0, nv2 = 0;
     it.next(st, nv0);
@@ -521,8 +541,8 @@ __device__ __forceinline__ bool softmax_tile(uint32_t t_s, uint32_t p_row, int r
 
 template <int D>
 __device__ void softmax_role(const CUtensorMap *tm_o, const FwdArgs &a, uint8_t *smem, uint32_t sbase,
-                             uint32_t tmem, int b, int h, int t, int qt, const int32_t *fl, int cnt, int n_tiles,
-                             bool bad_set, const Ctl &ctl)
+                             uint32_t tmem, int b, int b_out, int h, int t, int qt, const int32_t *fl, int cnt,
+                             int t_off, int n_tiles, bool bad_set, const Ctl &ctl)
 {
     using C = Cfg<D>;
     const Bars<D> bar{sbase + C::SMEM_BAR};
@@ -539,6 +559,7 @@ __device__ void softmax_role(const CUtensorMap *tm_o, const FwdArgs &a, uint8_t 
     bool alive = true;
     KvIter it;
     it.init(fl, cnt, a.P);
+    it.skip(t_off);
     for (int j = 0; j < n_tiles; ++j) {
         int st, nv;
         it.next(st, nv);
@@ -604,7 +625,7 @@ __device__ void softmax_role(const CUtensorMap *tm_o, const FwdArgs &a, uint8_t 
     if (write && row == 0) {
 #pragma unroll
         for (int kb = 0; kb < C::KBOX; ++kb)
-            tma_store_5d(tm_o, sbase + C::SMEM_Q + kb * C::BOX_BYTES, kb * 64, qt * BM, t, h, b);
+            tma_store_5d(tm_o, sbase + C::SMEM_Q + kb * C::BOX_BYTES, kb * 64, qt * BM, t, h, b_out);
         tma_store_commit();
         tma_store_wait_read_all();
     }
@@ -614,7 +635,7 @@ __device__ void softmax_role(const CUtensorMap *tm_o, const FwdArgs &a, uint8_t 
         if (bad_set) lse = __int_as_float(0x7fc00000);  // NaN marks a rejected frame list
         else if (n_tiles == 0) lse = -INFINITY;
         else lse = (m_used + log2f(l)) * 0.69314718055994530942f;
-        a.lse[((int64_t)(b * a.H + h) * a.Tq + t) * a.P + p] = lse;
+        a.lse[((int64_t)(b_out * a.H + h) * a.Tq + t) * a.P + p] = lse;
     }
 }
 
@@ -645,9 +666,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int b = x / a.H;
     const int32_t *fl = a.frames + ((int64_t)h * a.Tq + t) * a.Amax;
     const int cnt = __ldg(a.counts + h * a.Tq + t);
-    int n_tiles = (cnt >= 0 && cnt <= a.Amax) ? count_tiles(fl, cnt, a.T_kv, a.P) : -1;
-    const bool bad_set = n_tiles < 0;
-    if (bad_set) n_tiles = 0;
+    int n_all = (cnt >= 0 && cnt <= a.Amax) ? count_tiles(fl, cnt, a.T_kv, a.P) : -1;
+    const bool bad_set = n_all < 0;
+    if (bad_set) n_all = 0;
+    // split-KV: CTA (unit, split) takes the unit's key tiles [t_off, t_off + n_tiles) and
+    // writes a partial result into slice `split` of the output (batch index b_out)
+    const int split = blockIdx.y, n_split = gridDim.y;
+    const int t_off = (int)(((int64_t)n_all * split) / n_split);
+    int n_tiles = (int)(((int64_t)n_all * (split + 1)) / n_split) - t_off;
+    const int b_out = split * a.B + b;
     volatile int32_t *skip = reinterpret_cast<volatile int32_t *>(smem + C::SMEM_BAR + 248);
 
     if (threadIdx.x == 0) {
@@ -659,7 +686,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // once a CTA has timed out, the ones that start later skip their work
         *skip = (a.status && *reinterpret_cast<volatile int32_t *>(a.status) == SFA_ERR_TIMEOUT) ? 1 : 0;
         fence_mbar_init();
-        if (bad_set) report(a.status, SFA_ERR_BAD_SET);
+        if (bad_set && split == 0) report(a.status, SFA_ERR_BAD_SET);
     }
     if (warp == K_LOAD_WARP && lane == 0) {
         tma_prefetch_desc(&tm_q);
@@ -680,13 +707,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (skipped) n_tiles = 0;
 
     if (warp == K_LOAD_WARP) {
-        loader_role<D, true>(&tm_q, &tm_k, a, sbase, b, h, t, qt, fl, cnt, n_tiles, ctl);
+        loader_role<D, true>(&tm_q, &tm_k, a, sbase, b, h, t, qt, fl, cnt, t_off, n_tiles, ctl);
     } else if (warp == V_LOAD_WARP) {
-        loader_role<D, false>(&tm_q, &tm_v, a, sbase, b, h, t, qt, fl, cnt, n_tiles, ctl);
+        loader_role<D, false>(&tm_q, &tm_v, a, sbase, b, h, t, qt, fl, cnt, t_off, n_tiles, ctl);
     } else if (warp == MMA_WARP) {
-        mma_role<D>(a, sbase, tmem, fl, cnt, n_tiles, ctl);
+        mma_role<D>(a, sbase, tmem, fl, cnt, t_off, n_tiles, ctl);
     } else {
-        if (!skipped) softmax_role<D>(&tm_o, a, smem, sbase, tmem, b, h, t, qt, fl, cnt, n_tiles, bad_set, ctl);
+        if (!skipped)
+            softmax_role<D>(&tm_o, a, smem, sbase, tmem, b, b_out, h, t, qt, fl, cnt, t_off, n_tiles, bad_set, ctl);
     }
 
     tc_fence_before();
@@ -741,9 +769,14 @@ bool stride_ok(const int64_t *s, int d)
     return s[2] >= d;
 }
 
+// Forward launch.  n_split == 1: O and LSE go to the caller's buffers.  n_split > 1:
+// every unit's key tiles are split into n_split ranges, CTA (unit, split) writes its
+// partial O / LSE into the workspace slices [split][B][H][Tq*P][d] (bf16, contiguous) and
+// [split][B][H][Tq*P] (fp32), and a k-way LSE merge writes the caller's O and LSE.
 template <int D>
 sfa_status launch(const sfa_attn_desc *d, const void *q, const void *k, const void *v, const int32_t *frames,
-                  const int32_t *counts, void *o, float *lse, int32_t *dev_status, cudaStream_t stream)
+                  const int32_t *counts, void *o, float *lse, int32_t *dev_status, cudaStream_t stream,
+                  int n_split = 1, void *ws_o = nullptr, float *ws_lse = nullptr)
 {
     using C = Cfg<D>;
     CUtensorMap tq, tk, tv, to;
@@ -753,9 +786,16 @@ sfa_status launch(const sfa_attn_desc *d, const void *q, const void *k, const vo
         const uint64_t st[4] = {(uint64_t)d->q_stride[2] * 2, P * d->q_stride[2] * 2, (uint64_t)d->q_stride[1] * 2,
                                 (uint64_t)d->q_stride[0] * 2};
         if (!encode(&tq, q, 5, dims, st)) return SFA_ERR_UNSUPPORTED;
-        const uint64_t so[4] = {(uint64_t)d->o_stride[2] * 2, P * d->o_stride[2] * 2, (uint64_t)d->o_stride[1] * 2,
-                                (uint64_t)d->o_stride[0] * 2};
-        if (!encode(&to, o, 5, dims, so)) return SFA_ERR_UNSUPPORTED;
+        if (n_split == 1) {
+            const uint64_t so[4] = {(uint64_t)d->o_stride[2] * 2, P * d->o_stride[2] * 2,
+                                    (uint64_t)d->o_stride[1] * 2, (uint64_t)d->o_stride[0] * 2};
+            if (!encode(&to, o, 5, dims, so)) return SFA_ERR_UNSUPPORTED;
+        } else {
+            const uint64_t Lq = Tq * P;
+            const uint64_t dims_w[5] = {(uint64_t)D, P, Tq, (uint64_t)d->H, (uint64_t)d->B * n_split};
+            const uint64_t sw[4] = {(uint64_t)D * 2, P * D * 2, Lq * D * 2, (uint64_t)d->H * Lq * D * 2};
+            if (!encode(&to, ws_o, 5, dims_w, sw)) return SFA_ERR_UNSUPPORTED;
+        }
     }
     {
         const uint64_t dims[4] = {(uint64_t)D, Lkv, (uint64_t)d->H, (uint64_t)d->B};
@@ -777,7 +817,7 @@ sfa_status launch(const sfa_attn_desc *d, const void *q, const void *k, const vo
     a.scale_log2 = d->scale * 1.4426950408889634f;
     a.frames = frames;
     a.counts = counts;
-    a.lse = lse;
+    a.lse = n_split == 1 ? lse : ws_lse;
     a.status = dev_status;
     a.timeout_ns = (uint64_t)(d->timeout_us ? d->timeout_us : DEFAULT_TIMEOUT_US) * 1000;
     a.debug_flags = d->debug_flags;
@@ -786,8 +826,50 @@ sfa_status launch(const sfa_attn_desc *d, const void *q, const void *k, const vo
     if (cudaFuncSetAttribute(sfa_forward_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
         cudaSuccess)
         return SFA_ERR_CUDA;
-    sfa_forward_kernel<D><<<(unsigned)grid, NUM_THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, to, a);
-    return launch_status();
+    sfa_forward_kernel<D><<<dim3((unsigned)grid, (unsigned)n_split), NUM_THREADS, C::SMEM_BYTES, stream>>>(
+        tq, tk, tv, to, a);
+    sfa_status st = launch_status();
+    if (st != SFA_OK || n_split == 1) return st;
+    const int64_t Lq = (int64_t)d->Tq * d->P;
+    return launch_lse_combine((int64_t)d->B * d->H * Lq, n_split, D, d->H, Lq, ws_o, ws_lse, o, d->o_stride, lse,
+                              stream);
+}
+
+size_t split_ws_o_bytes(const sfa_attn_desc *d, int n_split)
+{
+    const size_t rows = (size_t)d->B * d->H * d->Tq * d->P;
+    return ((size_t)n_split * rows * d->d * 2 + 255) / 256 * 256;
+}
+
+size_t split_ws_bytes(const sfa_attn_desc *d, int n_split)
+{
+    const size_t rows = (size_t)d->B * d->H * d->Tq * d->P;
+    return split_ws_o_bytes(d, n_split) + ((size_t)n_split * rows * 4 + 255) / 256 * 256;
+}
+
+sfa_status check_desc(const sfa_attn_desc *d)
+{
+    if (!d) return SFA_ERR_INVALID_ARG;
+    if (d->B < 0 || d->H < 1 || d->Tq < 1 || d->T_kv < 1 || d->P < 1 || d->Amax < 1) return SFA_ERR_INVALID_ARG;
+    if (d->d != 64 && d->d != 128) return SFA_ERR_UNSUPPORTED;
+    if (!(d->scale > 0.f) || !std::isfinite(d->scale)) return SFA_ERR_INVALID_ARG;
+    if ((int64_t)d->Tq * d->P >= ((int64_t)1 << 31) || (int64_t)d->T_kv * d->P >= ((int64_t)1 << 31))
+        return SFA_ERR_INVALID_ARG;
+    const int64_t grid = (int64_t)d->B * d->H * d->Tq * ((d->P + BM - 1) / BM);
+    if (grid >= ((int64_t)1 << 31)) return SFA_ERR_INVALID_ARG;
+    return SFA_OK;
+}
+
+sfa_status check_buffers(const sfa_attn_desc *d, const void *q, const void *k, const void *v, const int32_t *frames,
+                         const int32_t *counts, const void *o, const float *lse)
+{
+    if (!q || !k || !v || !o || !lse || !frames || !counts) return SFA_ERR_INVALID_ARG;
+    for (const void *p : {q, k, v, o})
+        if (reinterpret_cast<uintptr_t>(p) % 16) return SFA_ERR_INVALID_ARG;
+    if (!stride_ok(d->q_stride, d->d) || !stride_ok(d->k_stride, d->d) || !stride_ok(d->v_stride, d->d) ||
+        !stride_ok(d->o_stride, d->d))
+        return SFA_ERR_INVALID_ARG;
+    return SFA_OK;
 }
 
 }  // namespace
@@ -799,22 +881,43 @@ extern "C" sfa_status sfa_forward(const sfa_attn_desc *d, const void *q, const v
                                   const int32_t *frames, const int32_t *counts, void *o, float *lse,
                                   int32_t *dev_status, sfa_stream_t stream)
 {
-    if (!d) return SFA_ERR_INVALID_ARG;
-    if (d->B < 0 || d->H < 1 || d->Tq < 1 || d->T_kv < 1 || d->P < 1 || d->Amax < 1) return SFA_ERR_INVALID_ARG;
-    if (d->d != 64 && d->d != 128) return SFA_ERR_UNSUPPORTED;
-    if (!(d->scale > 0.f) || !std::isfinite(d->scale)) return SFA_ERR_INVALID_ARG;
-    if ((int64_t)d->Tq * d->P >= ((int64_t)1 << 31) || (int64_t)d->T_kv * d->P >= ((int64_t)1 << 31))
-        return SFA_ERR_INVALID_ARG;
-    const int64_t grid = (int64_t)d->B * d->H * d->Tq * ((d->P + BM - 1) / BM);
-    if (grid >= ((int64_t)1 << 31)) return SFA_ERR_INVALID_ARG;
+    sfa_status st = check_desc(d);
+    if (st != SFA_OK) return st;
     if (d->B == 0) return SFA_OK;
-    if (!q || !k || !v || !o || !lse || !frames || !counts) return SFA_ERR_INVALID_ARG;
-    for (const void *p : {q, k, v, (const void *)o})
-        if (reinterpret_cast<uintptr_t>(p) % 16) return SFA_ERR_INVALID_ARG;
-    if (!stride_ok(d->q_stride, d->d) || !stride_ok(d->k_stride, d->d) || !stride_ok(d->v_stride, d->d) ||
-        !stride_ok(d->o_stride, d->d))
-        return SFA_ERR_INVALID_ARG;
+    st = check_buffers(d, q, k, v, frames, counts, o, lse);
+    if (st != SFA_OK) return st;
     cudaStream_t s = as_cuda(stream);
     return d->d == 128 ? launch<128>(d, q, k, v, frames, counts, o, lse, dev_status, s)
                        : launch<64>(d, q, k, v, frames, counts, o, lse, dev_status, s);
+}
+
+extern "C" sfa_status sfa_forward_split_workspace(const sfa_attn_desc *d, int32_t n_split, size_t *bytes)
+{
+    sfa_status st = check_desc(d);
+    if (st != SFA_OK) return st;
+    if (!bytes || n_split < 1 || n_split > d->d / 8) return SFA_ERR_INVALID_ARG;
+    *bytes = n_split == 1 ? 0 : split_ws_bytes(d, n_split);
+    return SFA_OK;
+}
+
+extern "C" sfa_status sfa_forward_split(const sfa_attn_desc *d, const void *q, const void *k, const void *v,
+                                        const int32_t *frames, const int32_t *counts, void *o, float *lse,
+                                        int32_t n_split, void *workspace, size_t workspace_bytes,
+                                        int32_t *dev_status, sfa_stream_t stream)
+{
+    sfa_status st = check_desc(d);
+    if (st != SFA_OK) return st;
+    if (n_split < 1 || n_split > d->d / 8) return SFA_ERR_INVALID_ARG;
+    if (d->B == 0) return SFA_OK;
+    st = check_buffers(d, q, k, v, frames, counts, o, lse);
+    if (st != SFA_OK) return st;
+    cudaStream_t s = as_cuda(stream);
+    if (n_split == 1)
+        return d->d == 128 ? launch<128>(d, q, k, v, frames, counts, o, lse, dev_status, s)
+                           : launch<64>(d, q, k, v, frames, counts, o, lse, dev_status, s);
+    if (!workspace || reinterpret_cast<uintptr_t>(workspace) % 256 || workspace_bytes < split_ws_bytes(d, n_split))
+        return SFA_ERR_INVALID_ARG;
+    float *ws_lse = reinterpret_cast<float *>(static_cast<char *>(workspace) + split_ws_o_bytes(d, n_split));
+    return d->d == 128 ? launch<128>(d, q, k, v, frames, counts, o, lse, dev_status, s, n_split, workspace, ws_lse)
+                       : launch<64>(d, q, k, v, frames, counts, o, lse, dev_status, s, n_split, workspace, ws_lse);
 }

@@ -20,4 +20,8 @@ inline sfa_status launch_status()
 
 inline cudaStream_t as_cuda(sfa_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
 
+// k-way LSE merge of split-KV partials (sfa_merge.cu)
+sfa_status launch_lse_combine(int64_t rows, int S, int d, int H, int64_t Lq, const void *o_part,
+                              const float *lse_part, void *o, const int64_t *o_stride, float *lse, cudaStream_t s);
+
 }  // namespace sfa

@@ -72,7 +72,77 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(int64_t rows, const uint
     }
 }
 
+// k-way merge of split-KV partial results (the same LSE rule applied to S branches):
+// o_part bf16 [S][rows][D] and lse_part fp32 [S][rows] (rows = B*H*Lq in (b, h, i)
+// order) -> O at o + b*os0 + h*os1 + i*os2 and LSE [rows].  D/8 threads per row, the
+// lane s of a row's group holds branch s's weight (S <= D/8).
+template <int D>
+__global__ void __launch_bounds__(256) lse_combine_kernel(int64_t rows, int S, int H, int64_t Lq,
+                                                          const uint4 *__restrict__ o_part,
+                                                          const float *__restrict__ lse_part, uint16_t *o,
+                                                          int64_t os0, int64_t os1, int64_t os2, float *lse)
+{
+    constexpr int G = D / 8;
+    const int64_t gtid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int sub = threadIdx.x % G;
+    const unsigned group = ((1u << G) - 1u) << ((threadIdx.x % 32) & ~(G - 1));
+    const int64_t row_stride = (int64_t)gridDim.x * blockDim.x / G;
+    for (int64_t r = gtid / G; r < rows; r += row_stride) {
+        const float ls = sub < S ? lse_part[(int64_t)sub * rows + r] : -INFINITY;
+        float m = ls;
+#pragma unroll
+        for (int off = G / 2; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(group, m, off, G));
+        const float w = (ls == -INFINITY) ? 0.f : expf(ls - m);
+        float tot = w;
+#pragma unroll
+        for (int off = G / 2; off > 0; off >>= 1) tot += __shfl_xor_sync(group, tot, off, G);
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int sidx = 0; sidx < S; ++sidx) {
+            const float ws = __shfl_sync(group, w, sidx, G);
+            if (ws != 0.f) {
+                const uint4 v = o_part[((int64_t)sidx * rows + r) * G + sub];
+                const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    acc[2 * i] += ws * bf16_lo(vv[i]);
+                    acc[2 * i + 1] += ws * bf16_hi(vv[i]);
+                }
+            }
+        }
+        const bool empty = (m == -INFINITY);
+        const float inv = empty ? 0.f : 1.f / tot;
+        const int64_t b = r / ((int64_t)H * Lq), h = (r / Lq) % H, i = r % Lq;
+        uint4 out;
+        out.x = to_bf16x2(acc[0] * inv, acc[1] * inv);
+        out.y = to_bf16x2(acc[2] * inv, acc[3] * inv);
+        out.z = to_bf16x2(acc[4] * inv, acc[5] * inv);
+        out.w = to_bf16x2(acc[6] * inv, acc[7] * inv);
+        *reinterpret_cast<uint4 *>(o + b * os0 + h * os1 + i * os2 + sub * 8) = out;
+        if (sub == 0) lse[r] = empty ? -INFINITY : m + logf(tot);
+    }
+}
+
 }  // namespace
+
+sfa_status launch_lse_combine(int64_t rows, int S, int d, int H, int64_t Lq, const void *o_part,
+                              const float *lse_part, void *o, const int64_t *o_stride, float *lse, cudaStream_t s)
+{
+    if (rows == 0) return SFA_OK;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int threads = 256;
+    const int64_t need = (rows * (d / 8) + threads - 1) / threads;
+    const int64_t cap = (int64_t)sms * 8;
+    const int blocks = (int)(need < cap ? need : cap);
+    if (d == 128)
+        lse_combine_kernel<128><<<blocks, threads, 0, s>>>(rows, S, H, Lq, (const uint4 *)o_part, lse_part,
+                                                           (uint16_t *)o, o_stride[0], o_stride[1], o_stride[2], lse);
+    else
+        lse_combine_kernel<64><<<blocks, threads, 0, s>>>(rows, S, H, Lq, (const uint4 *)o_part, lse_part,
+                                                          (uint16_t *)o, o_stride[0], o_stride[1], o_stride[2], lse);
+    return launch_status();
+}
+
 }  // namespace sfa
 
 using namespace sfa;

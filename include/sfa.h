@@ -26,6 +26,7 @@
 #ifndef SFA_H_
 #define SFA_H_
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -173,6 +174,30 @@ typedef struct {
 sfa_status sfa_forward(const sfa_attn_desc *desc, const void *q, const void *k, const void *v,
                        const int32_t *frames, const int32_t *counts, void *o, float *lse,
                        int32_t *dev_status, sfa_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
+ * Split-KV forward (same result as sfa_forward, for short or uneven grids)
+ * ------------------------------------------------------------------------------------
+ * The key tiles of every (batch, head, query frame, 128-row query tile) are cut into
+ * n_split contiguous ranges that run as separate CTAs; each writes a partial O and LSE
+ * into the workspace, and the partials are merged by their LSE ("ISPA", §2.1: the LSE
+ * state makes partial attentions over disjoint key sets mergeable; the merge is
+ * sfa_lse_merge's rule over n_split branches).  Use it when B*H*Tq*ceil(P/128) is small
+ * next to the number of SMs or the sets differ a lot in size between heads.
+ *
+ * sfa_forward_split_workspace: bytes of device workspace for this descriptor and
+ *   n_split (0 when n_split == 1).  1 <= n_split <= d/8, else SFA_ERR_INVALID_ARG.
+ * sfa_forward_split: arguments as sfa_forward, plus n_split and a caller-owned device
+ *   workspace of at least that many bytes, 256-byte aligned (unused when n_split == 1;
+ *   its contents are scratch and are overwritten).  Partial O is rounded to bf16 before
+ *   the merge, in fp32, rounds it once more.
+ */
+sfa_status sfa_forward_split_workspace(const sfa_attn_desc *desc, int32_t n_split, size_t *bytes);
+
+sfa_status sfa_forward_split(const sfa_attn_desc *desc, const void *q, const void *k, const void *v,
+                             const int32_t *frames, const int32_t *counts, void *o, float *lse,
+                             int32_t n_split, void *workspace, size_t workspace_bytes, int32_t *dev_status,
+                             sfa_stream_t stream);
 
 /* ------------------------------------------------------------------------------------
  * LSE merge

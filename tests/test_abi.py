@@ -134,3 +134,22 @@ def test_no_oracle_in_product_path():
             if fn.endswith((".py", ".cu", ".cuh", ".h")):
                 text = open(os.path.join(dirpath, fn)).read()
                 assert "oracle" not in text.lower(), f"{fn} mentions the oracle"
+
+
+def test_split_workspace_and_arguments(sfa):
+    lib = sfa.load()
+    d = _desc(sfa)  # B=1, H=2, Tq=4, P=64, d=64: 512 query rows
+    out = ctypes.c_size_t(0)
+    assert lib.sfa_forward_split_workspace(ctypes.byref(d), 1, ctypes.byref(out)) == 0 and out.value == 0
+    assert lib.sfa_forward_split_workspace(ctypes.byref(d), 2, ctypes.byref(out)) == 0
+    assert out.value == 2 * 512 * 64 * 2 + 2 * 512 * 4
+    assert lib.sfa_forward_split_workspace(ctypes.byref(d), 9, ctypes.byref(out)) == 1   # > d/8
+    assert lib.sfa_forward_split_workspace(ctypes.byref(d), 0, ctypes.byref(out)) == 1
+    good = 1 << 20
+    # workspace missing, too small or misaligned: refused before any launch
+    assert lib.sfa_forward_split(ctypes.byref(d), good, good, good, good, good, good, good, 2, None, 0,
+                                 None, None) == 1
+    assert lib.sfa_forward_split(ctypes.byref(d), good, good, good, good, good, good, good, 2, good, 1024,
+                                 None, None) == 1
+    assert lib.sfa_forward_split(ctypes.byref(d), good, good, good, good, good, good, good, 2, good + 128,
+                                 out.value, None, None) == 1
