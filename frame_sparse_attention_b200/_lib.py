@@ -51,7 +51,7 @@ class AttnDesc(ctypes.Structure):
 
 _lib = None
 EXPORTS = ("sfa_error_string", "sfa_version", "sfa_set_max_count", "sfa_build_sets", "sfa_forward",
-           "sfa_forward_split_workspace", "sfa_forward_split", "sfa_lse_merge")
+           "sfa_forward_split_workspace", "sfa_forward_split", "sfa_forward_split_noalloc", "sfa_lse_merge")
 
 
 def load():
@@ -81,6 +81,8 @@ def load():
     lib.sfa_forward_split.restype = st
     lib.sfa_forward_split.argtypes = [ctypes.POINTER(AttnDesc), vp, vp, vp, vp, vp, vp, vp, i32, vp,
                                       ctypes.c_size_t, vp, vp]
+    lib.sfa_forward_split_noalloc.restype = st
+    lib.sfa_forward_split_noalloc.argtypes = [ctypes.POINTER(AttnDesc), vp, vp, vp, vp, vp, vp, vp, i32, vp, vp]
     lib.sfa_lse_merge.restype = st
     lib.sfa_lse_merge.argtypes = [i64, i32, vp, vp, vp, vp, vp, vp, vp]
     _lib = lib

@@ -921,3 +921,68 @@ extern "C" sfa_status sfa_forward_split(const sfa_attn_desc *d, const void *q, c
     return d->d == 128 ? launch<128>(d, q, k, v, frames, counts, o, lse, dev_status, s, n_split, workspace, ws_lse)
                        : launch<64>(d, q, k, v, frames, counts, o, lse, dev_status, s, n_split, workspace, ws_lse);
 }
+
+// ------------------------------------------------------------------------------------
+// Split-KV forward that allocates nothing.
+//
+// Some callers cannot hand this library a workspace: a process whose GPU memory is owned
+// by an allocator it may not call into (a custom caching pool, a framework that forbids
+// allocation while it is running), or code paths that must never call cudaMalloc or
+// cudaFree because those synchronise the device.  For them the split-KV scratch lives in
+// a fixed array of device memory inside this library, reserved once per GPU when the
+// library's kernels are loaded there and kept until the process exits.
+// ------------------------------------------------------------------------------------
+namespace sfa {
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[SFA_NOALLOC_SCRATCH_BYTES];
+
+constexpr int NOALLOC_MAX_DEVICES = 256;
+std::mutex g_noalloc_mutex;
+void *g_noalloc_ptr[NOALLOC_MAX_DEVICES] = {};
+
+// Device address of the scratch array on the current device.  In host code the array's
+// name only stands for it, so the address is looked up once per device, with that device
+// current, and cached.
+sfa_status noalloc_scratch(void **out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SFA_ERR_CUDA;
+    if (dev < 0 || dev >= NOALLOC_MAX_DEVICES) return SFA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return SFA_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return SFA_OK;
+}
+
+}  // namespace
+}  // namespace sfa
+
+extern "C" sfa_status sfa_forward_split_noalloc(const sfa_attn_desc *d, const void *q, const void *k,
+                                                const void *v, const int32_t *frames, const int32_t *counts,
+                                                void *o, float *lse, int32_t n_split, int32_t *dev_status,
+                                                sfa_stream_t stream)
+{
+    sfa_status st = check_desc(d);
+    if (st != SFA_OK) return st;
+    if (n_split < 1 || n_split > d->d / 8) return SFA_ERR_INVALID_ARG;
+    if (n_split > 1 && split_ws_bytes(d, n_split) > (size_t)SFA_NOALLOC_SCRATCH_BYTES)
+        return SFA_ERR_INVALID_ARG;  // needs more scratch than the fixed array holds
+    if (d->B == 0) return SFA_OK;
+    st = check_buffers(d, q, k, v, frames, counts, o, lse);
+    if (st != SFA_OK) return st;
+    cudaStream_t s = as_cuda(stream);
+    if (n_split == 1)
+        return d->d == 128 ? launch<128>(d, q, k, v, frames, counts, o, lse, dev_status, s)
+                           : launch<64>(d, q, k, v, frames, counts, o, lse, dev_status, s);
+    void *scratch = nullptr;
+    st = noalloc_scratch(&scratch);
+    if (st != SFA_OK) return st;
+    float *ws_lse = reinterpret_cast<float *>(static_cast<char *>(scratch) + split_ws_o_bytes(d, n_split));
+    return d->d == 128 ? launch<128>(d, q, k, v, frames, counts, o, lse, dev_status, s, n_split, scratch, ws_lse)
+                       : launch<64>(d, q, k, v, frames, counts, o, lse, dev_status, s, n_split, scratch, ws_lse);
+}

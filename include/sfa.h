@@ -199,6 +199,32 @@ sfa_status sfa_forward_split(const sfa_attn_desc *desc, const void *q, const voi
                              int32_t n_split, void *workspace, size_t workspace_bytes, int32_t *dev_status,
                              sfa_stream_t stream);
 
+/*
+ * sfa_forward_split_noalloc: sfa_forward_split for callers that cannot allocate device
+ * memory for the library (their memory belongs to an allocator they may not call into,
+ * or they must not call cudaMalloc / cudaFree, which synchronise the device).  The pages
+ * have no counterpart: this is an interface convenience, not part of the method.
+ *   - The workspace is a fixed array of SFA_NOALLOC_SCRATCH_BYTES inside the library,
+ *     reserved on every GPU where the library's kernels are loaded and held until the
+ *     process exits.  The call allocates nothing (no cudaMalloc, no cudaFree, no
+ *     allocating library routine); the caller still passes inputs and outputs.
+ *   - The first call on a device looks up the array's device address with that device
+ *     current (cudaGetSymbolAddress) and caches it; make that first call before any
+ *     stream capture on the device.
+ *   - Requests needing more than SFA_NOALLOC_SCRATCH_BYTES of workspace (see
+ *     sfa_forward_split_workspace) return SFA_ERR_INVALID_ARG without launching.
+ *     n_split == 1 needs no workspace.
+ *   - Every call shares the one array, which keeps the previous call's contents (nothing
+ *     in it has to start at zero: each call writes every partial it reads).  Calls
+ *     that can overlap on the GPU (different streams, or different host threads on the
+ *     same device) race on it: serialise them.
+ */
+#define SFA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+sfa_status sfa_forward_split_noalloc(const sfa_attn_desc *desc, const void *q, const void *k, const void *v,
+                                     const int32_t *frames, const int32_t *counts, void *o, float *lse,
+                                     int32_t n_split, int32_t *dev_status, sfa_stream_t stream);
+
 /* ------------------------------------------------------------------------------------
  * LSE merge
  * ------------------------------------------------------------------------------------
