@@ -57,11 +57,11 @@ def measured_peaks():
     return p
 
 
-# DRAM bytes (read + write) of one forward launch on this workload: one ncu capture of the
-# same kernel on the 4-head version of the workload (196.77 MB read + 52.34 MB written),
-# scaled by 3 to 12 heads (the traffic is per (head, frame, query tile) unit).  Must be
-# re-measured whenever the forward kernel changes.
-NCU_TRAFFIC_BYTES = 3 * (196_768_512 + 52_340_736)
+# DRAM bytes (read + write) of one forward launch on this workload, from one ncu capture
+# of the same kernel on the 4-head version of the workload scaled by 3 to 12 heads (the
+# traffic is per (head, frame, query tile) unit); None until it is re-measured after a
+# change to the forward kernel.
+NCU_TRAFFIC_BYTES = None
 
 
 def max_over_ranks(x: float, device) -> float:

@@ -51,7 +51,8 @@ class AttnDesc(ctypes.Structure):
 
 _lib = None
 EXPORTS = ("sfa_error_string", "sfa_version", "sfa_set_max_count", "sfa_build_sets", "sfa_forward",
-           "sfa_forward_split_workspace", "sfa_forward_split", "sfa_forward_split_noalloc", "sfa_lse_merge")
+           "sfa_forward_split_workspace", "sfa_forward_split", "sfa_forward_split_noalloc", "sfa_forward_paged",
+           "sfa_lse_merge")
 
 
 def load():
@@ -83,6 +84,8 @@ def load():
                                       ctypes.c_size_t, vp, vp]
     lib.sfa_forward_split_noalloc.restype = st
     lib.sfa_forward_split_noalloc.argtypes = [ctypes.POINTER(AttnDesc), vp, vp, vp, vp, vp, vp, vp, i32, vp, vp]
+    lib.sfa_forward_paged.restype = st
+    lib.sfa_forward_paged.argtypes = [ctypes.POINTER(AttnDesc), vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp]
     lib.sfa_lse_merge.restype = st
     lib.sfa_lse_merge.argtypes = [i64, i32, vp, vp, vp, vp, vp, vp, vp]
     _lib = lib
@@ -192,6 +195,28 @@ def forward(q, k, v, frames, counts, P: int, scale: float | None = None, out=Non
     _check(load().sfa_forward(ctypes.byref(desc), q.data_ptr(), k.data_ptr(), v.data_ptr(),
                               frames.data_ptr(), counts.data_ptr(), out.data_ptr(), lse.data_ptr(),
                               _ptr(dev_status), _stream(stream)), "sfa_forward")
+    return out, lse
+
+
+def forward_paged(q, k_cache, v_cache, slots, frames, counts, P: int, T_kv: int, scale: float | None = None,
+                  out=None, lse=None, dev_status=None, stream=None, timeout_us: int = 0):
+    """Frame-sparse attention with K/V read through a per-head slot table [H, T_kv]
+    (logical frame -> physical frame slot of k_cache / v_cache [B, H, n_slots*P, d])."""
+    B, H, Lq, d = q.shape
+    n_slots = k_cache.shape[2] // P
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, Lq), dtype=torch.float32, device=q.device)
+    assert slots.dtype == torch.int32 and slots.is_contiguous() and tuple(slots.shape) == (H, T_kv)
+    assert frames.dtype == torch.int32 and counts.dtype == torch.int32
+    assert frames.is_contiguous() and counts.is_contiguous() and lse.is_contiguous()
+    desc = attn_desc(q, k_cache, v_cache, out, P, frames.shape[2], scale, timeout_us)
+    desc.T_kv = T_kv
+    _check(load().sfa_forward_paged(ctypes.byref(desc), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                                    slots.data_ptr(), n_slots, frames.data_ptr(), counts.data_ptr(),
+                                    out.data_ptr(), lse.data_ptr(), _ptr(dev_status), _stream(stream)),
+           "sfa_forward_paged")
     return out, lse
 
 

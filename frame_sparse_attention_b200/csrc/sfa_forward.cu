@@ -95,6 +95,8 @@ struct FwdArgs {
     float scale_log2;  // softmax scale * log2(e)
     const int32_t *frames;
     const int32_t *counts;
+    const int32_t *slots;  // [H][T_kv] physical frame slot of each logical frame, or null
+    int32_t n_slots;       // frames held by the K/V buffers (T_kv without a slot table)
     float *lse;
     int32_t *status;
     uint64_t timeout_ns;
@@ -151,23 +153,33 @@ __device__ __noinline__ void wait_drain(uint32_t bar, uint32_t parity)
 }
 
 // ----------------------------------------------------------------- attended key tiles
+// Physical frame slot of a logical key/value frame: a per-head slot table (paged caches)
+// or the identity.
+__device__ __forceinline__ int slot_of(const int32_t *srow, int f) { return srow ? __ldg(srow + f) : f; }
+
 // Number of K/V tiles for a frame list, or -1 if the list is not strictly increasing
-// inside [0, T_kv).
-__device__ int count_tiles(const int32_t *fl, int cnt, int T_kv, int P)
+// inside [0, T_kv) or a slot lies outside [0, n_slots).  A run is a stretch of list
+// entries whose slots are consecutive, i.e. one contiguous token interval.
+__device__ int count_tiles(const int32_t *fl, int cnt, int T_kv, int P, const int32_t *srow, int n_slots)
 {
     int tiles = 0, a = 0, prev = -1;
     while (a < cnt) {
         const int f0 = __ldg(fl + a);
         if (f0 <= prev || f0 >= T_kv) return -1;
-        int f1 = f0;
+        const int s0 = slot_of(srow, f0);
+        if (s0 < 0 || s0 >= n_slots) return -1;
+        int s1 = s0;
+        prev = f0;
         ++a;
-        while (a < cnt && __ldg(fl + a) == f1 + 1) {
-            ++f1;
+        while (a < cnt) {
+            const int f = __ldg(fl + a);
+            if (f <= prev || f >= T_kv) return -1;
+            if (slot_of(srow, f) != s1 + 1 || s1 + 1 >= n_slots) break;
+            ++s1;
+            prev = f;
             ++a;
         }
-        if (f1 >= T_kv) return -1;
-        prev = f1;
-        tiles += ((f1 - f0 + 1) * P + BN - 1) / BN;
+        tiles += ((s1 - s0 + 1) * P + BN - 1) / BN;
     }
     return tiles;
 }
@@ -175,10 +187,12 @@ __device__ int count_tiles(const int32_t *fl, int cnt, int T_kv, int P)
 // Walks the attended tokens as runs of consecutive frames, 128 keys at a time.
 struct KvIter {
     const int32_t *fl;
+    const int32_t *srow;
     int n, a, P, pos, end;
-    __device__ void init(const int32_t *f, int cnt, int P_)
+    __device__ void init(const int32_t *f, int cnt, int P_, const int32_t *slot_row)
     {
         fl = f;
+        srow = slot_row;
         n = cnt;
         a = 0;
         P = P_;
@@ -187,15 +201,15 @@ struct KvIter {
     }
     __device__ void open_run()
     {
-        const int f0 = __ldg(fl + a);
-        int f1 = f0;
+        const int s0 = slot_of(srow, __ldg(fl + a));
+        int s1 = s0;
         ++a;
-        while (a < n && __ldg(fl + a) == f1 + 1) {
-            ++f1;
+        while (a < n && slot_of(srow, __ldg(fl + a)) == s1 + 1) {
+            ++s1;
             ++a;
         }
-        pos = f0 * P;
-        end = (f1 + 1) * P;
+        pos = s0 * P;
+        end = (s1 + 1) * P;
     }
     __device__ void next(int &start, int &nvalid)
     {
@@ -247,7 +261,7 @@ __device__ void loader_role(const CUtensorMap *tm_q, const CUtensorMap *tm_kv, c
     // K/V of one (h, t) are re-read by every query tile of the frame: keep them in L2
     const uint64_t policy = l2_policy_evict_last();
     KvIter it;
-    it.init(fl, cnt, a.P);
+    it.init(fl, cnt, a.P, a.slots ? a.slots + (int64_t)h * a.T_kv : nullptr);
     it.skip(t_off);
     int j = 0;
     for (; j < n_tiles; ++j) {
@@ -325,8 +339,8 @@ __device__ __forceinline__ void commit_one(uint32_t bar)
 }
 
 template <int D>
-__device__ void mma_role(const FwdArgs &a, uint32_t sbase, uint32_t tmem, const int32_t *fl, int cnt, int t_off,
-                         int n_tiles, const Ctl &ctl)
+__device__ void mma_role(const FwdArgs &a, uint32_t sbase, uint32_t tmem, int h, const int32_t *fl, int cnt,
+                         int t_off, int n_tiles, const Ctl &ctl)
 {
     using C = Cfg<D>;
     const Bars<D> bar{sbase + C::SMEM_BAR};
@@ -337,7 +351,7 @@ __device__ void mma_role(const FwdArgs &a, uint32_t sbase, uint32_t tmem, const 
     const uint64_t dp = sdesc_sw128(sbase + C::SMEM_P, 16, 1024);
     bool issued = false;
     KvIter it;
-    it.init(fl, cnt, a.P);
+    it.init(fl, cnt, a.P, a.slots ? a.slots + (int64_t)h * a.T_kv : nullptr);
     it.skip(t_off);
     // valid keys of tiles j, j+1, j+2 (S runs two tiles ahead of P V)
     int st, nv0 = 0, nv1 = 0, nv2 = 0;
@@ -368,6 +382,20 @@ __device__ void mma_role(const FwdArgs &a, uint32_t sbase, uint32_t tmem, const 
         }
         const int sv = j % C::NSV;
         if (!__all_sync(0xffffffffu, wait_bar(bar.v_full(sv), (j / C::NSV) & 1, ctl))) break;
+        if (nv0 & 15) {
+            // P V reads V up to the next multiple of 16 keys, where P is 0; those few rows
+            // hold whatever follows the run in memory (another frame, an unused cache
+            // slot), so they are zeroed first: 0 * (non-finite) would poison O
+            const int r0 = nv0, r1 = (nv0 + 15) & ~15;
+            const uint32_t vslot = sbase + C::SMEM_V + sv * C::TILE_BYTES;
+            const uint32_t zero[4] = {0u, 0u, 0u, 0u};
+            for (int idx = (int)(threadIdx.x & 31); idx < (r1 - r0) * C::KBOX * 8; idx += 32) {
+                const int r = r0 + idx / (C::KBOX * 8), kb = (idx / 8) % C::KBOX, ch = idx % 8;
+                st_shared_v4(vslot + kb * C::BOX_BYTES + r * 128 + ch * 16, zero);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+        }
         tc_fence_after();
         issue_pv<D>(tmem + TM_O, desc_add(dp, (j & 1) * C::P_BYTES), desc_add(dv, sv * C::TILE_BYTES), mma_n(nv0),
                     j > 0);
@@ -558,7 +586,7 @@ __device__ void softmax_role(const CUtensorMap *tm_o, const FwdArgs &a, uint8_t 
     float l = 0.f;             // running row sum of exp2(s*sl2 - m_used)
     bool alive = true;
     KvIter it;
-    it.init(fl, cnt, a.P);
+    it.init(fl, cnt, a.P, a.slots ? a.slots + (int64_t)h * a.T_kv : nullptr);
     it.skip(t_off);
     for (int j = 0; j < n_tiles; ++j) {
         int st, nv;
@@ -666,7 +694,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int b = x / a.H;
     const int32_t *fl = a.frames + ((int64_t)h * a.Tq + t) * a.Amax;
     const int cnt = __ldg(a.counts + h * a.Tq + t);
-    int n_all = (cnt >= 0 && cnt <= a.Amax) ? count_tiles(fl, cnt, a.T_kv, a.P) : -1;
+    int n_all = (cnt >= 0 && cnt <= a.Amax)
+                    ? count_tiles(fl, cnt, a.T_kv, a.P, a.slots ? a.slots + (int64_t)h * a.T_kv : nullptr, a.n_slots)
+                    : -1;
     const bool bad_set = n_all < 0;
     if (bad_set) n_all = 0;
     // split-KV: CTA (unit, split) takes the unit's key tiles [t_off, t_off + n_tiles) and
@@ -711,7 +741,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     } else if (warp == V_LOAD_WARP) {
         loader_role<D, false>(&tm_q, &tm_v, a, sbase, b, h, t, qt, fl, cnt, t_off, n_tiles, ctl);
     } else if (warp == MMA_WARP) {
-        mma_role<D>(a, sbase, tmem, fl, cnt, t_off, n_tiles, ctl);
+        mma_role<D>(a, sbase, tmem, h, fl, cnt, t_off, n_tiles, ctl);
     } else {
         if (!skipped)
             softmax_role<D>(&tm_o, a, smem, sbase, tmem, b, b_out, h, t, qt, fl, cnt, t_off, n_tiles, bad_set, ctl);
@@ -776,11 +806,13 @@ bool stride_ok(const int64_t *s, int d)
 template <int D>
 sfa_status launch(const sfa_attn_desc *d, const void *q, const void *k, const void *v, const int32_t *frames,
                   const int32_t *counts, void *o, float *lse, int32_t *dev_status, cudaStream_t stream,
-                  int n_split = 1, void *ws_o = nullptr, float *ws_lse = nullptr)
+                  int n_split = 1, void *ws_o = nullptr, float *ws_lse = nullptr, const int32_t *slots = nullptr,
+                  int n_slots = 0)
 {
     using C = Cfg<D>;
     CUtensorMap tq, tk, tv, to;
-    const uint64_t P = d->P, Tq = d->Tq, Lkv = (uint64_t)d->T_kv * d->P;
+    const int kv_frames = slots ? n_slots : d->T_kv;  // frames held by the K/V buffers
+    const uint64_t P = d->P, Tq = d->Tq, Lkv = (uint64_t)kv_frames * d->P;
     {
         const uint64_t dims[5] = {(uint64_t)D, P, Tq, (uint64_t)d->H, (uint64_t)d->B};
         const uint64_t st[4] = {(uint64_t)d->q_stride[2] * 2, P * d->q_stride[2] * 2, (uint64_t)d->q_stride[1] * 2,
@@ -817,6 +849,8 @@ sfa_status launch(const sfa_attn_desc *d, const void *q, const void *k, const vo
     a.scale_log2 = d->scale * 1.4426950408889634f;
     a.frames = frames;
     a.counts = counts;
+    a.slots = slots;
+    a.n_slots = kv_frames;
     a.lse = n_split == 1 ? lse : ws_lse;
     a.status = dev_status;
     a.timeout_ns = (uint64_t)(d->timeout_us ? d->timeout_us : DEFAULT_TIMEOUT_US) * 1000;
@@ -985,4 +1019,28 @@ extern "C" sfa_status sfa_forward_split_noalloc(const sfa_attn_desc *d, const vo
     float *ws_lse = reinterpret_cast<float *>(static_cast<char *>(scratch) + split_ws_o_bytes(d, n_split));
     return d->d == 128 ? launch<128>(d, q, k, v, frames, counts, o, lse, dev_status, s, n_split, scratch, ws_lse)
                        : launch<64>(d, q, k, v, frames, counts, o, lse, dev_status, s, n_split, scratch, ws_lse);
+}
+
+// ------------------------------------------------------------------------------------
+// Paged key/value caches: a per-head table maps each logical key/value frame to the
+// physical frame slot that holds it, so per-head caches of different contents need no
+// compaction.
+// ------------------------------------------------------------------------------------
+extern "C" sfa_status sfa_forward_paged(const sfa_attn_desc *d, const void *q, const void *k_cache,
+                                        const void *v_cache, const int32_t *slots, int32_t n_slots,
+                                        const int32_t *frames, const int32_t *counts, void *o, float *lse,
+                                        int32_t *dev_status, sfa_stream_t stream)
+{
+    sfa_status st = check_desc(d);
+    if (st != SFA_OK) return st;
+    if (n_slots < 1 || (int64_t)n_slots * d->P >= ((int64_t)1 << 31)) return SFA_ERR_INVALID_ARG;
+    if (d->B == 0) return SFA_OK;
+    if (!slots) return SFA_ERR_INVALID_ARG;
+    st = check_buffers(d, q, k_cache, v_cache, frames, counts, o, lse);
+    if (st != SFA_OK) return st;
+    cudaStream_t s = as_cuda(stream);
+    return d->d == 128 ? launch<128>(d, q, k_cache, v_cache, frames, counts, o, lse, dev_status, s, 1, nullptr,
+                                     nullptr, slots, n_slots)
+                       : launch<64>(d, q, k_cache, v_cache, frames, counts, o, lse, dev_status, s, 1, nullptr,
+                                    nullptr, slots, n_slots);
 }

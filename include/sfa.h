@@ -176,6 +176,26 @@ sfa_status sfa_forward(const sfa_attn_desc *desc, const void *q, const void *k, 
                        int32_t *dev_status, sfa_stream_t stream);
 
 /* ------------------------------------------------------------------------------------
+ * Paged key/value caches
+ * ------------------------------------------------------------------------------------
+ * ("Head Forcing", §2: every head keeps its own cache — local, anchor or memory — of
+ *  different frames.)  sfa_forward with the keys and values read through a per-head slot
+ * table: logical key/value frame f of head h lives in physical frame slot
+ * slots[h * T_kv + f] of k_cache / v_cache, so caches are updated by rewriting slots and
+ * the table, never by compacting tensors.
+ *   k_cache, v_cache  bf16 [B][H][n_slots * P][d] with desc->k_stride / v_stride.
+ *   slots             device int32 [H][T_kv] (shared by the batch); only entries of
+ *                     frames that appear in a list are read, each must lie in
+ *                     [0, n_slots) (else SFA_ERR_BAD_SET through dev_status).
+ *   desc->T_kv        logical frames (the range of the frame lists), n_slots >= 1.
+ * List entries whose slots are consecutive are read as one contiguous run.  Every slot
+ * may hold arbitrary data: rows past a run's end are never used.
+ */
+sfa_status sfa_forward_paged(const sfa_attn_desc *desc, const void *q, const void *k_cache, const void *v_cache,
+                             const int32_t *slots, int32_t n_slots, const int32_t *frames, const int32_t *counts,
+                             void *o, float *lse, int32_t *dev_status, sfa_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
  * Split-KV forward (same result as sfa_forward, for short or uneven grids)
  * ------------------------------------------------------------------------------------
  * The key tiles of every (batch, head, query frame, 128-row query tile) are cut into

@@ -59,4 +59,4 @@ def test_single_process_helpers():
     import bench
     assert bench.max_over_ranks(3.5, "cpu") == 3.5
     assert bench.job_rate_tflops(1e12, 1, 1.0) == pytest.approx(1000.0)
-    assert bench.NCU_TRAFFIC_BYTES > 0
+    assert bench.NCU_TRAFFIC_BYTES is None or bench.NCU_TRAFFIC_BYTES > 0
