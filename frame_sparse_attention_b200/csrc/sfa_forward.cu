@@ -6,22 +6,26 @@
 // of O(T P d).  Per row it also emits the log-sum-exp of its scaled scores, the state
 // that "ISPA" (§2.1, Atención Descomponible) uses to merge partial attentions.
 //
-// How, on one SM per work unit (b, h, t, 128-row query tile):
+// How, on one SM per work unit (b, h, t, pair of 128-row query tiles A and B):
 //   * the frame list of (h, t) is walked as runs of consecutive frames; each run is one
 //     contiguous token interval, cut into 128-key tiles, so unattended frames are never
 //     loaded and only the last tile of a run is partial;
-//   * warp 4 (one thread) streams Q once and K/V tiles through a 3-stage (d = 128) or
-//     4-stage (d = 64) shared-memory ring with TMA, 128-byte swizzled;
-//   * warp 5 (one thread) issues tcgen05.mma: S = Q K^T into one of two TMEM S buffers
-//     (two tiles ahead of the softmax), then O += P V with P read from shared memory
-//     (both operands in shared memory: the tensor-memory-A form of this MMA runs at
-//     ~0.6x the rate on sm_100); a partial last tile uses an MMA N (for S) and K (for
-//     P V) rounded up to 16 only;
-//   * warps 0-3 (one thread per query row = TMEM lane) run the online softmax in fp32
-//     (exp2 with the scale folded into one FMA; O is rescaled only when a row's running
-//     max grows by more than 2^8, otherwise the stale max is kept), write P as bf16 into
-//     a 128-byte-swizzled shared-memory tile, and finally normalise O, stage it in shared
-//     memory and TMA-store it, clipped to the frame, plus the fp32 LSE.
+//   * warp 8 loads Q of both tiles once and streams K tiles through a 2-slot ring, warp
+//     10 streams V tiles (1 slot at d = 128, 2 at d = 64), all with TMA, 128-byte
+//     swizzled; a K slot frees once S of both tiles has read it, a V slot once P V of
+//     both has;
+//   * warp 9 (one elected lane) issues tcgen05.mma for both tiles in the order
+//     S_A(0) S_B(0) | P V_A(j) S_A(j+1) P V_B(j) S_B(j+1) ..., S into TMEM (one buffer per
+//     tile), O += P V with P read from shared memory (both operands in shared memory: the
+//     tensor-memory-A form of this MMA runs at ~0.6x the rate on sm_100); a partial last
+//     tile uses an MMA N (for S) and K (for P V) rounded up to 16 only.  While the
+//     softmax of one tile runs, the tensor cores work on the other;
+//   * warps 0-3 (tile A) and 4-7 (tile B), one thread per query row = TMEM lane, run the
+//     online softmax in fp32 (exp2 with the scale folded into one FMA; O is rescaled only
+//     when a row's running max grows by more than 2^8, otherwise the stale max is kept),
+//     write P as bf16 into a 128-byte-swizzled shared-memory tile, and finally normalise
+//     O, stage it in shared memory and TMA-store it, clipped to the frame, plus the fp32
+//     LSE.
 // Every mbarrier wait is bounded; a wait that runs out records SFA_ERR_TIMEOUT, the CTA
 // drains its in-flight copies and MMAs, frees its TMEM and returns.
 #include <cuda.h>
@@ -41,36 +45,39 @@ namespace {
 
 constexpr int BM = 128;                 // query rows per tile = MMA M = TMEM lanes
 constexpr int BN = 128;                 // keys per K/V tile (largest MMA N used)
-constexpr int NUM_THREADS = 224;        // warps 0-3 softmax, 4 Q+K loader, 5 MMA issuer, 6 V loader
-constexpr int K_LOAD_WARP = 4;
-constexpr int MMA_WARP = 5;
-constexpr int V_LOAD_WARP = 6;
+// warps 0-3 softmax of query tile A, 4-7 softmax of query tile B, 8 Q+K loader,
+// 9 MMA issuer, 10 V loader
+constexpr int NUM_THREADS = 352;
+constexpr int K_LOAD_WARP = 8;
+constexpr int MMA_WARP = 9;
+constexpr int V_LOAD_WARP = 10;
 constexpr float RESCALE_LOG2 = 8.0f;    // keep a stale row max while the new one is < 2^8 above
 constexpr uint32_t DEFAULT_TIMEOUT_US = 2000000;  // 2 s; a healthy wait lasts microseconds
 constexpr uint32_t DRAIN_TIMEOUT_US = 2000000;
 constexpr uint32_t MAX_SPINS = 1u << 30;           // backstop should the timer not advance
 
-// tensor-memory columns (512 allocated: 2 x S fp32, O fp32)
-constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_O = 256, TM_COLS = 512;
+// tensor-memory columns (512 allocated): S of tile A / B, O of tile A / B (fp32)
+constexpr uint32_t TM_COLS = 512;
+__host__ __device__ constexpr uint32_t tcol_s(int x) { return (uint32_t)x * 128; }
+__host__ __device__ constexpr uint32_t tcol_o(int x) { return 256 + (uint32_t)x * 128; }
 
 template <int D>
 struct Cfg {
     static constexpr int KBOX = D / 64;                 // 128-byte swizzle boxes per row
     static constexpr int BOX_BYTES = 128 * 128;         // 128 rows x 64 bf16
     static constexpr int TILE_BYTES = BM * D * 2;       // one Q / K / V / O tile
-    // separate two-slot K and V rings: a K slot frees once S of its tile is computed (the
-    // loader waits on that S's own barrier), a V slot once P V is (it waits on the P
-    // buffer's release), so no extra tensor-core commits are needed for the rings
+    // K and V rings: a K slot frees once S of both query tiles is computed from it, a V
+    // slot once P V of both is (d = 128 leaves room for one V slot only)
     static constexpr int NSK = 2;
-    static constexpr int NSV = 2;
+    static constexpr int NSV = D == 128 ? 1 : 2;
     static constexpr int P_BYTES = BM * BN * 2;          // one bf16 probability tile
-    static constexpr int SMEM_Q = 0;
-    static constexpr int SMEM_P = TILE_BYTES;             // two P tiles (double buffer)
+    static constexpr int SMEM_Q = 0;                      // Q tiles A and B
+    static constexpr int SMEM_P = 2 * TILE_BYTES;         // P tiles A and B
     static constexpr int SMEM_K = SMEM_P + 2 * P_BYTES;
     static constexpr int SMEM_V = SMEM_K + NSK * TILE_BYTES;
     static constexpr int SMEM_BAR = SMEM_V + NSV * TILE_BYTES;
     static constexpr int SMEM_BYTES = SMEM_BAR + 256 + 1024;  // + barriers, + alignment slack
-    static_assert(NSK + NSV + 9 <= 28, "mbarriers must fit in 224 bytes");
+    static_assert(2 * NSK + 2 * NSV + 7 <= 20, "mbarriers must fit in 160 bytes");
     static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 };
 
@@ -79,14 +86,15 @@ template <int D>
 struct Bars {
     uint32_t base;
     __device__ uint32_t k_full(int s) const { return base + 8 * s; }
-    __device__ uint32_t v_full(int s) const { return base + 8 * (Cfg<D>::NSK + s); }
-    __device__ uint32_t q_full() const { return base + 8 * (Cfg<D>::NSK + Cfg<D>::NSV); }
-    __device__ uint32_t s_full(int b) const { return q_full() + 8 + 8 * b; }   // S of a tile in TMEM
-    __device__ uint32_t p_full(int b) const { return q_full() + 24 + 8 * b; }  // P of a tile in TMEM
-    __device__ uint32_t p_free(int b) const { return q_full() + 40 + 8 * b; }  // P V done with a P buffer
-    __device__ uint32_t drain() const { return q_full() + 56; }
-    __device__ uint32_t o_final() const { return q_full() + 64; }              // after the last P V
-    static constexpr int COUNT = Cfg<D>::NSK + Cfg<D>::NSV + 9;
+    __device__ uint32_t k_free(int s) const { return base + 8 * (Cfg<D>::NSK + s); }
+    __device__ uint32_t v_full(int s) const { return base + 8 * (2 * Cfg<D>::NSK + s); }
+    __device__ uint32_t v_free(int s) const { return base + 8 * (2 * Cfg<D>::NSK + Cfg<D>::NSV + s); }
+    __device__ uint32_t q_full() const { return base + 8 * (2 * Cfg<D>::NSK + 2 * Cfg<D>::NSV); }
+    __device__ uint32_t s_full(int x) const { return q_full() + 8 + 8 * x; }   // S of query tile x in TMEM
+    __device__ uint32_t p_full(int x) const { return q_full() + 24 + 8 * x; }  // P of query tile x in smem
+    __device__ uint32_t o_final() const { return q_full() + 40; }              // after the last P V
+    __device__ uint32_t drain() const { return q_full() + 48; }
+    static constexpr int COUNT = 2 * Cfg<D>::NSK + 2 * Cfg<D>::NSV + 7;
 };
 
 struct FwdArgs {
@@ -238,13 +246,14 @@ struct KvIter {
 __device__ __forceinline__ uint32_t mma_n(int nvalid) { return (uint32_t)((nvalid + 15) & ~15); }
 
 // ----------------------------------------------------------------- roles
-// Streams the K tiles (IS_K, plus the Q tile first) or the V tiles of the attended
+// Streams the K tiles (IS_K, plus the query tiles first) or the V tiles of the attended
 // frames into their ring.  The whole warp runs the loop (its state stays warp-uniform);
-// one elected lane issues each copy.
+// one elected lane issues each copy.  A slot is reused once the MMA warp has released
+// it (k_free / v_free: committed after the last MMA that reads the slot).
 template <int D, bool IS_K>
 __device__ void loader_role(const CUtensorMap *tm_q, const CUtensorMap *tm_kv, const FwdArgs &a, uint32_t sbase,
-                            int b, int h, int t, int qt, const int32_t *fl, int cnt, int t_off, int n_tiles,
-                            const Ctl &ctl)
+                            int b, int h, int t, int qt_a, bool has_b, const int32_t *fl, int cnt, int t_off,
+                            int n_tiles, const Ctl &ctl)
 {
     using C = Cfg<D>;
     constexpr int NSR = IS_K ? C::NSK : C::NSV;
@@ -252,10 +261,12 @@ __device__ void loader_role(const CUtensorMap *tm_q, const CUtensorMap *tm_kv, c
     const uint32_t ring = sbase + (IS_K ? C::SMEM_K : C::SMEM_V);
     if (n_tiles <= 0) return;
     if (IS_K && elect_one()) {
-        mbar_arrive_expect_tx(bar.q_full(), C::TILE_BYTES);
+        mbar_arrive_expect_tx(bar.q_full(), C::TILE_BYTES * (has_b ? 2 : 1));
+        for (int x = 0; x < (has_b ? 2 : 1); ++x)
 #pragma unroll
-        for (int kb = 0; kb < C::KBOX; ++kb)
-            tma_load_5d(sbase + C::SMEM_Q + kb * C::BOX_BYTES, tm_q, bar.q_full(), kb * 64, qt * BM, t, h, b);
+            for (int kb = 0; kb < C::KBOX; ++kb)
+                tma_load_5d(sbase + C::SMEM_Q + x * C::TILE_BYTES + kb * C::BOX_BYTES, tm_q, bar.q_full(), kb * 64,
+                            (qt_a + x) * BM, t, h, b);
     }
     __syncwarp();
     // K/V of one (h, t) are re-read by every query tile of the frame: keep them in L2
@@ -267,14 +278,9 @@ __device__ void loader_role(const CUtensorMap *tm_q, const CUtensorMap *tm_kv, c
     for (; j < n_tiles; ++j) {
         const int s = j % NSR;
         const uint32_t full = IS_K ? bar.k_full(s) : bar.v_full(s);
-        // slot s last held tile j-2: wait for its S (K ring) or P V (V ring).  Both
-        // barriers belong to buffer (j-2) & 1 and have exactly one pending phase here,
-        // because tile j's S or P V cannot run before this very load.
-        static_assert(NSR == 2, "the release waits below assume two-slot rings");
-        if (j >= 2) {
-            const int jj = j - 2;
-            const uint32_t rel = IS_K ? bar.s_full(jj & 1) : bar.p_free(jj & 1);
-            if (!__all_sync(0xffffffffu, wait_bar(rel, (jj >> 1) & 1, ctl))) break;
+        if (j >= NSR) {  // one release per use of the slot: exactly one pending phase here
+            const uint32_t rel = IS_K ? bar.k_free(s) : bar.v_free(s);
+            if (!__all_sync(0xffffffffu, wait_bar(rel, ((j - NSR) / NSR) & 1, ctl))) break;
         }
         int start, nv;
         it.next(start, nv);
@@ -338,9 +344,15 @@ __device__ __forceinline__ void commit_one(uint32_t bar)
     __syncwarp();
 }
 
+// One warp issues all tensor-core work, in the order
+//   S_A(0) S_B(0) | P V_A(j) S_A(j+1) P V_B(j) S_B(j+1) | ...
+// While one softmax warpgroup works on its tile, the tensor cores run the other tile's
+// P V and next S.  Because one thread issues everything and a commit tracks every MMA it
+// issued before, the completion of S_x(j+1) implies P V_x(j) is done: the softmax can
+// then overwrite P_x and rescale O_x without further waits.
 template <int D>
-__device__ void mma_role(const FwdArgs &a, uint32_t sbase, uint32_t tmem, int h, const int32_t *fl, int cnt,
-                         int t_off, int n_tiles, const Ctl &ctl)
+__device__ void mma_role(const FwdArgs &a, uint32_t sbase, uint32_t tmem, int h, bool has_b, const int32_t *fl,
+                         int cnt, int t_off, int n_tiles, const Ctl &ctl)
 {
     using C = Cfg<D>;
     const Bars<D> bar{sbase + C::SMEM_BAR};
@@ -349,62 +361,64 @@ __device__ void mma_role(const FwdArgs &a, uint32_t sbase, uint32_t tmem, int h,
     const uint64_t dk = sdesc_sw128(sbase + C::SMEM_K, 16, 1024);
     const uint64_t dv = sdesc_sw128(sbase + C::SMEM_V, C::BOX_BYTES, 1024);
     const uint64_t dp = sdesc_sw128(sbase + C::SMEM_P, 16, 1024);
+    const int nx = has_b ? 2 : 1;
     bool issued = false;
     KvIter it;
     it.init(fl, cnt, a.P, a.slots ? a.slots + (int64_t)h * a.T_kv : nullptr);
     it.skip(t_off);
-    // valid keys of tiles j, j+1, j+2 (S runs two tiles ahead of P V)
-    int st, nv0 = 0, nv1 = 0, nv2 = 0;
-    it.next(st, nv0);
-    if (n_tiles > 1) it.next(st, nv1);
+    int st, nv_cur = 0, nv_next = 0;
+    it.next(st, nv_cur);
     if (!__all_sync(0xffffffffu, wait_bar(bar.q_full(), 0, ctl))) goto done;
-    // S of the first two tiles into the two S buffers
-    for (int j = 0; j < 2 && j < n_tiles; ++j) {
-        if (!__all_sync(0xffffffffu, wait_bar(bar.k_full(j), 0, ctl))) goto done;
-        tc_fence_after();
-        issue_s<D>(tmem + (j ? TM_S1 : TM_S0), dq, desc_add(dk, j * C::TILE_BYTES),
-                   idesc_bf16_f32(BM, mma_n(j ? nv1 : nv0), false));
-        commit_one(bar.s_full(j));
-        issued = true;
+    if (!__all_sync(0xffffffffu, wait_bar(bar.k_full(0), 0, ctl))) goto done;
+    tc_fence_after();
+    for (int x = 0; x < nx; ++x) {
+        issue_s<D>(tmem + tcol_s(x), desc_add(dq, x * C::TILE_BYTES), dk, idesc_bf16_f32(BM, mma_n(nv_cur), false));
+        commit_one(bar.s_full(x));
     }
+    commit_one(bar.k_free(0));
+    issued = true;
     for (int j = 0; j < n_tiles; ++j) {
-        // P of tile j published: its S buffer is free again, so S of tile j+2 goes to the
-        // tensor cores first (the softmax waits for it), P V of tile j after it
-        if (!__all_sync(0xffffffffu, wait_bar(bar.p_full(j & 1), (j >> 1) & 1, ctl))) break;
-        if (j + 2 < n_tiles) {
-            it.next(st, nv2);
-            const int sk = (j + 2) % C::NSK;
-            if (!__all_sync(0xffffffffu, wait_bar(bar.k_full(sk), ((j + 2) / C::NSK) & 1, ctl))) break;
-            tc_fence_after();
-            issue_s<D>(tmem + ((j & 1) ? TM_S1 : TM_S0), dq, desc_add(dk, sk * C::TILE_BYTES),
-                       idesc_bf16_f32(BM, mma_n(nv2), false));
-            commit_one(bar.s_full(j & 1));  // S ready; also frees its K slot
-        }
-        const int sv = j % C::NSV;
-        if (!__all_sync(0xffffffffu, wait_bar(bar.v_full(sv), (j / C::NSV) & 1, ctl))) break;
-        if (nv0 & 15) {
-            // P V reads V up to the next multiple of 16 keys, where P is 0; those few rows
-            // hold whatever follows the run in memory (another frame, an unused cache
-            // slot), so they are zeroed first: 0 * (non-finite) would poison O
-            const int r0 = nv0, r1 = (nv0 + 15) & ~15;
-            const uint32_t vslot = sbase + C::SMEM_V + sv * C::TILE_BYTES;
-            const uint32_t zero[4] = {0u, 0u, 0u, 0u};
-            for (int idx = (int)(threadIdx.x & 31); idx < (r1 - r0) * C::KBOX * 8; idx += 32) {
-                const int r = r0 + idx / (C::KBOX * 8), kb = (idx / 8) % C::KBOX, ch = idx % 8;
-                st_shared_v4(vslot + kb * C::BOX_BYTES + r * 128 + ch * 16, zero);
+        if (j + 1 < n_tiles) it.next(st, nv_next);
+        const int sv = j % C::NSV, sk = (j + 1) % C::NSK;
+        for (int x = 0; x < nx; ++x) {
+            if (!__all_sync(0xffffffffu, wait_bar(bar.p_full(x), j & 1, ctl))) goto done;
+            if (x == 0) {
+                if (!__all_sync(0xffffffffu, wait_bar(bar.v_full(sv), (j / C::NSV) & 1, ctl))) goto done;
+                if (nv_cur & 15) {
+                    // P V reads V up to the next multiple of 16 keys, where P is 0; those
+                    // few rows hold whatever follows the run in memory (another frame, an
+                    // unused cache slot), so they are zeroed first: 0 * (non-finite)
+                    // would poison O
+                    const int r0 = nv_cur, r1 = (nv_cur + 15) & ~15;
+                    const uint32_t vslot = sbase + C::SMEM_V + sv * C::TILE_BYTES;
+                    const uint32_t zero[4] = {0u, 0u, 0u, 0u};
+                    for (int idx = (int)(threadIdx.x & 31); idx < (r1 - r0) * C::KBOX * 8; idx += 32) {
+                        const int r = r0 + idx / (C::KBOX * 8), kb = (idx / 8) % C::KBOX, ch = idx % 8;
+                        st_shared_v4(vslot + kb * C::BOX_BYTES + r * 128 + ch * 16, zero);
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                }
             }
-            fence_proxy_async_smem();
-            __syncwarp();
+            tc_fence_after();
+            issue_pv<D>(tmem + tcol_o(x), desc_add(dp, x * C::P_BYTES), desc_add(dv, sv * C::TILE_BYTES),
+                        mma_n(nv_cur), j > 0);
+            if (x == nx - 1) {
+                commit_one(bar.v_free(sv));  // both tiles' P V have read this V slot
+                // single-phase signal for the epilogues: O of both tiles is complete
+                if (j == n_tiles - 1) commit_one(bar.o_final());
+            }
+            if (j + 1 < n_tiles) {
+                if (x == 0 && !__all_sync(0xffffffffu, wait_bar(bar.k_full(sk), ((j + 1) / C::NSK) & 1, ctl)))
+                    goto done;
+                tc_fence_after();
+                issue_s<D>(tmem + tcol_s(x), desc_add(dq, x * C::TILE_BYTES), desc_add(dk, sk * C::TILE_BYTES),
+                           idesc_bf16_f32(BM, mma_n(nv_next), false));
+                commit_one(bar.s_full(x));
+                if (x == nx - 1) commit_one(bar.k_free(sk));  // both tiles' S have read this K slot
+            }
         }
-        tc_fence_after();
-        issue_pv<D>(tmem + TM_O, desc_add(dp, (j & 1) * C::P_BYTES), desc_add(dv, sv * C::TILE_BYTES), mma_n(nv0),
-                    j > 0);
-        commit_one(bar.p_free(j & 1));  // P buffer and V slot free, O holds tiles 0..j
-        // single-phase signal for the epilogue: with parity waits alone, the P V of the
-        // last two tiles can both be pending and would be indistinguishable
-        if (j == n_tiles - 1) commit_one(bar.o_final());
-        nv0 = nv1;
-        nv1 = nv2;
+        nv_cur = nv_next;
     }
 done:
     // (warp-uniform decision: the drain commit below is issued by an elected lane)
@@ -480,24 +494,17 @@ __device__ __forceinline__ float sum8(const float (&acc)[8])
 }
 
 // One K/V tile of the online softmax for this thread's query row (thread = TMEM lane):
-// S (fp32, TMEM) -> P = exp2(S * scale * log2e - m) as bf16 into TMEM, running max m and
-// sum l.  A row keeps a stale max m until a tile's max exceeds it by 2^RESCALE_LOG2, so
+// S (fp32, TMEM) -> P = exp2(S * scale * log2e - m) as bf16 into shared memory, running
+// max m and sum l.  A row keeps a stale max m until a tile's max exceeds it by 2^RESCALE_LOG2, so
 // the common case streams S through registers 32 columns at a time against the current
 // max.  The first tile, and a tile on which any lane of the warp finds a larger max,
-// take the exact two-pass path: row max first, then P (S is re-read from TMEM; P has
-// its own columns), and O is rescaled in place.  FULL: all 128 keys valid.
-// Returns false if a wait was abandoned.
+// take the exact two-pass path: row max first, then P (S is re-read from TMEM; P lives
+// in shared memory), and O is rescaled in place.  FULL: all 128 keys valid.
 template <int D, bool FULL>
-__device__ __forceinline__ bool softmax_tile(uint32_t t_s, uint32_t p_row, int row, uint32_t t_o, int nv, float sl2,
-                                          float &m_used, float &l, int j, uint32_t p_free0, const Ctl &ctl)
+__device__ __forceinline__ void softmax_tile(uint32_t t_s, uint32_t p_row, int row, uint32_t t_o, int nv, float sl2,
+                                             float &m_used, float &l, int j)
 {
     const int nch = FULL ? 4 : (nv + 31) >> 5;
-    // P of tile j goes to the buffer that P V of tile j-2 read: wait until it is done (S of
-    // tile j was committed after P V of tile j-3, so that is the only pending use)
-    if (j >= 2) {
-        const bool done = wait_bar(p_free0 + 8 * (j & 1), ((j >> 1) - 1) & 1, ctl);
-        if (!__all_sync(0xffffffffu, done)) return false;
-    }
     if (j > 0) {  // streaming pass against the current max
         float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         bool grow = false;
@@ -519,7 +526,7 @@ __device__ __forceinline__ bool softmax_tile(uint32_t t_s, uint32_t p_row, int r
         }
         if (!__any_sync(0xffffffffu, grow)) {
             l += sum8(acc);
-            return true;
+            return;
         }
     }
     // exact pass: row max over the tile, then P against the new max
@@ -546,12 +553,9 @@ __device__ __forceinline__ bool softmax_tile(uint32_t t_s, uint32_t p_row, int r
         }
     }
     // O must be rescaled before P V of this tile accumulates into it; the warp does it
-    // together (tcgen05.ld/st are warp-wide) once P V of tile j-1 (and so every earlier
-    // one) is done.  Tile j-1's P buffer has no other pending use, so the parity is exact.
+    // together (tcgen05.ld/st are warp-wide).  P V of the previous tile is already done:
+    // S of this tile was issued after it, and its completion was waited for.
     if (j > 0 && __any_sync(0xffffffffu, resc)) {
-        const bool done = wait_bar(p_free0 + 8 * ((j - 1) & 1), ((j - 1) >> 1) & 1, ctl);
-        if (!__all_sync(0xffffffffu, done)) return false;
-        tc_fence_after();
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
@@ -564,22 +568,24 @@ __device__ __forceinline__ bool softmax_tile(uint32_t t_s, uint32_t p_row, int r
     }
     l = l * alpha + sum8(acc);
     m_used = m_new;
-    return true;
 }
 
+// Softmax and epilogue of query tile x (0: warps 0-3, 1: warps 4-7), one thread per
+// query row.
 template <int D>
 __device__ void softmax_role(const CUtensorMap *tm_o, const FwdArgs &a, uint8_t *smem, uint32_t sbase,
-                             uint32_t tmem, int b, int b_out, int h, int t, int qt, const int32_t *fl, int cnt,
-                             int t_off, int n_tiles, bool bad_set, const Ctl &ctl)
+                             uint32_t tmem, int x, int b, int b_out, int h, int t, int qt, const int32_t *fl,
+                             int cnt, int t_off, int n_tiles, bool bad_set, const Ctl &ctl)
 {
     using C = Cfg<D>;
     const Bars<D> bar{sbase + C::SMEM_BAR};
-    const uint32_t s_full0 = bar.s_full(0), p_full0 = bar.p_full(0), p_free0 = bar.p_free(0);
-    const uint32_t o_final = bar.o_final();
-    volatile int32_t *epi_ok = reinterpret_cast<volatile int32_t *>(smem + C::SMEM_BAR + 224);
-    const int row = threadIdx.x;  // query row inside the tile == TMEM lane
-    const int warp = row >> 5;
+    // 8 flags after the mbarriers (at most 15 x 8 bytes) and before the words at +240
+    volatile int32_t *epi_ok = reinterpret_cast<volatile int32_t *>(smem + C::SMEM_BAR + 160) + 4 * x;
+    const int row = threadIdx.x & 127;  // query row inside the tile == TMEM lane
+    const int warp = (threadIdx.x >> 5) & 3;
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t t_s = lane_base + tcol_s(x), t_o = lane_base + tcol_o(x);
+    const uint32_t p_row = sbase + C::SMEM_P + x * C::P_BYTES + row * 128;
     const float sl2 = a.scale_log2;
 
     float m_used = -INFINITY;  // running row max (log2 units, scale folded in)
@@ -591,45 +597,40 @@ __device__ void softmax_role(const CUtensorMap *tm_o, const FwdArgs &a, uint8_t 
     for (int j = 0; j < n_tiles; ++j) {
         int st, nv;
         it.next(st, nv);
-        const bool got = wait_bar(s_full0 + 8 * (j & 1), (j >> 1) & 1, ctl);
+        // S of tile j has one pending phase: S of tile j+1 waits for P of tile j
+        const bool got = wait_bar(bar.s_full(x), j & 1, ctl);
         if (!__all_sync(0xffffffffu, got)) {
             alive = false;
             break;
         }
         tc_fence_after();
-        const uint32_t t_s = lane_base + ((j & 1) ? TM_S1 : TM_S0);
-        const uint32_t p_row = sbase + C::SMEM_P + (j & 1) * C::P_BYTES + row * 128;
-        const bool ok = nv >= BN
-                            ? softmax_tile<D, true>(t_s, p_row, row, lane_base + TM_O, nv, sl2, m_used, l, j, p_free0, ctl)
-                            : softmax_tile<D, false>(t_s, p_row, row, lane_base + TM_O, nv, sl2, m_used, l, j, p_free0, ctl);
-        if (!ok) {
-            alive = false;
-            break;
-        }
+        if (nv >= BN) softmax_tile<D, true>(t_s, p_row, row, t_o, nv, sl2, m_used, l, j);
+        else softmax_tile<D, false>(t_s, p_row, row, t_o, nv, sl2, m_used, l, j);
         tmem_wait_st();            // O rescale stores, if any
         fence_proxy_async_smem();  // P written with st.shared is read by the tensor cores
         tc_fence_before();
-        if (!((a.debug_flags & SFA_DEBUG_STALL_SOFTMAX) && j == 0)) mbar_arrive(p_full0 + 8 * (j & 1));
+        if (!((a.debug_flags & SFA_DEBUG_STALL_SOFTMAX) && j == 0)) mbar_arrive(bar.p_full(x));
     }
 
-    // ---- epilogue: O / l -> bf16 -> swizzled smem (the Q tile's space) -> TMA store
+    // ---- epilogue: O / l -> bf16 -> swizzled smem (this tile's Q space) -> TMA store
     bool have = alive;
     if (have && n_tiles > 0) {
-        const bool done = wait_bar(o_final, 0, ctl);
+        const bool done = wait_bar(bar.o_final(), 0, ctl);
         have = __all_sync(0xffffffffu, done);
     }
-    if ((row & 31) == 0) epi_ok[warp] = have ? 1 : 0;
-    named_bar_sync(1, BM);
+    if ((threadIdx.x & 31) == 0) epi_ok[warp] = have ? 1 : 0;
+    named_bar_sync(1 + x, BM);
     const bool write = epi_ok[0] && epi_ok[1] && epi_ok[2] && epi_ok[3];
+    const uint32_t s_o_addr = sbase + C::SMEM_Q + x * C::TILE_BYTES;
     if (write) {
         const float inv_l = n_tiles > 0 ? 1.f / l : 0.f;
-        uint8_t *s_o = smem + C::SMEM_Q;
+        uint8_t *s_o = smem + C::SMEM_Q + x * C::TILE_BYTES;
         if (n_tiles > 0) tc_fence_after();
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
             if (n_tiles > 0) {
-                tmem_ld32(lane_base + TM_O + c * 32, o);
+                tmem_ld32(t_o + c * 32, o);
                 tmem_wait_ld_regs(o);
             } else {
 #pragma unroll
@@ -649,11 +650,11 @@ __device__ void softmax_role(const CUtensorMap *tm_o, const FwdArgs &a, uint8_t 
         }
         fence_proxy_async_smem();
     }
-    named_bar_sync(1, BM);
+    named_bar_sync(1 + x, BM);
     if (write && row == 0) {
 #pragma unroll
         for (int kb = 0; kb < C::KBOX; ++kb)
-            tma_store_5d(tm_o, sbase + C::SMEM_Q + kb * C::BOX_BYTES, kb * 64, qt * BM, t, h, b_out);
+            tma_store_5d(tm_o, s_o_addr + kb * C::BOX_BYTES, kb * 64, qt * BM, t, h, b_out);
         tma_store_commit();
         tma_store_wait_read_all();
     }
@@ -683,11 +684,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // work unit: (b, h, t, query tile), query tile fastest so that the tiles sharing
-    // one frame's K/V run side by side
+    // work unit: (b, h, t, pair of query tiles), pair fastest so that the tiles sharing
+    // one frame's K/V run side by side; the last pair of a frame may hold one tile only
+    const int n_pairs = (a.n_qtiles + 1) / 2;
     int x = blockIdx.x;
-    const int qt = x % a.n_qtiles;
-    x /= a.n_qtiles;
+    const int qt_a = 2 * (x % n_pairs);
+    const bool has_b = qt_a + 1 < a.n_qtiles;
+    x /= n_pairs;
     const int t = x % a.Tq;
     x /= a.Tq;
     const int h = x % a.H;
@@ -710,7 +713,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (threadIdx.x == 0) {
         const Bars<D> bar{bars};
         for (int i = 0; i < Bars<D>::COUNT; ++i) mbar_init(bars + 8 * i, 1);
-        mbar_init(bar.p_full(0), BM);    // P full: every softmax thread arrives
+        mbar_init(bar.p_full(0), BM);    // P full: every softmax thread of the tile arrives
         mbar_init(bar.p_full(1), BM);
         *abort_flag = 0;
         // once a CTA has timed out, the ones that start later skip their work
@@ -737,14 +740,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (skipped) n_tiles = 0;
 
     if (warp == K_LOAD_WARP) {
-        loader_role<D, true>(&tm_q, &tm_k, a, sbase, b, h, t, qt, fl, cnt, t_off, n_tiles, ctl);
+        loader_role<D, true>(&tm_q, &tm_k, a, sbase, b, h, t, qt_a, has_b, fl, cnt, t_off, n_tiles, ctl);
     } else if (warp == V_LOAD_WARP) {
-        loader_role<D, false>(&tm_q, &tm_v, a, sbase, b, h, t, qt, fl, cnt, t_off, n_tiles, ctl);
+        loader_role<D, false>(&tm_q, &tm_v, a, sbase, b, h, t, qt_a, has_b, fl, cnt, t_off, n_tiles, ctl);
     } else if (warp == MMA_WARP) {
-        mma_role<D>(a, sbase, tmem, h, fl, cnt, t_off, n_tiles, ctl);
-    } else {
-        if (!skipped)
-            softmax_role<D>(&tm_o, a, smem, sbase, tmem, b, b_out, h, t, qt, fl, cnt, t_off, n_tiles, bad_set, ctl);
+        mma_role<D>(a, sbase, tmem, h, has_b, fl, cnt, t_off, n_tiles, ctl);
+    } else if (warp < 8) {
+        const int xt = warp >> 2;  // query tile of this softmax warpgroup
+        if (!skipped && (xt == 0 || has_b))
+            softmax_role<D>(&tm_o, a, smem, sbase, tmem, xt, b, b_out, h, t, qt_a + xt, fl, cnt, t_off, n_tiles,
+                            bad_set, ctl);
     }
 
     tc_fence_before();
@@ -856,7 +861,7 @@ sfa_status launch(const sfa_attn_desc *d, const void *q, const void *k, const vo
     a.timeout_ns = (uint64_t)(d->timeout_us ? d->timeout_us : DEFAULT_TIMEOUT_US) * 1000;
     a.debug_flags = d->debug_flags;
 
-    const int64_t grid = (int64_t)d->B * d->H * d->Tq * a.n_qtiles;
+    const int64_t grid = (int64_t)d->B * d->H * d->Tq * ((a.n_qtiles + 1) / 2);
     if (cudaFuncSetAttribute(sfa_forward_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
         cudaSuccess)
         return SFA_ERR_CUDA;
