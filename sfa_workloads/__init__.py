@@ -10,6 +10,8 @@ Shapes follow the video-DiT workloads the method is described on:
     Wan-2.1-1.3B-like: 30x52 patch grid -> P = 1560, H = 12, d = 128, C = 21.
   * "Head Forcing", §2 (per-head KV caches): local / anchor / memory heads.
   * "ISPA", §2.1 Dual-Stream Warmup: local (current + sink) and history branches.
+  * "Resumen Técnico: LIGHT FORCING", §2.2 (HSA): an autoregressive chunk that
+    selects history frames, then blocks, by mean-pooled keys.
 
 The real activations of those models are not available; Q, K and V are drawn
 i.i.d. N(0, 1) in fp32 and rounded to bf16, which has the right shapes, dtype
@@ -50,6 +52,9 @@ class Workload:
     n_prev: int = 0
     chunk_len: int = 1
     heads: tuple = field(default_factory=tuple)   # one SetSpec per head
+    # hierarchical selection (HSA): history frames kept per query block, then key blocks
+    k_frames: int = 0
+    k_blocks: int = 0
 
     @property
     def Lq(self) -> int:
@@ -109,6 +114,11 @@ WORKLOADS = {
                               d=128, heads=(SetSpec("explicit", extra=tuple(range(1, 13))),) * 12),
     "lsemerge_full": Workload("lsemerge_full", B=1, H=12, Tq=1, Tkv=14, q_off=13, P=1560,
                               d=128, heads=(SetSpec("dense"),) * 12),
+    # HSA: the streaming chunk of "stream"; sink + local window always, plus the 24 best
+    # 128-token blocks of the 4 best history frames (of 17) per 256-row query block
+    "hsa": Workload("hsa", B=1, H=12, Tq=3, Tkv=24, q_off=21, P=1560, d=128,
+                    n_sink=1, n_prev=3, chunk_len=3, k_frames=4, k_blocks=24,
+                    heads=(SetSpec("hsa"),) * 12),
 }
 
 
@@ -126,7 +136,38 @@ def qkv(B: int, H: int, Lq: int, Lkv: int, d: int, seed: int = 0):
 
 
 def workload_qkv(w: Workload, seed: int = 0):
+    if w.k_frames:
+        return qkv_structured(w.B, w.H, w.Tq, w.Tkv, w.P, w.d, seed)
     return qkv(w.B, w.H, w.Lq, w.Lkv, w.d, seed)
+
+
+def qkv_structured(B: int, H: int, Tq: int, Tkv: int, P: int, d: int, seed: int = 0, sigma: float = 0.5,
+                   key_block: int = 128, query_block: int = 256):
+    """Q, K, V as in ``qkv`` plus per-frame and per-block offsets, so that pooled keys differ.
+
+    Real video features are correlated within a frame and within a spatial block; an
+    i.i.d. draw pools to almost nothing and makes any selection among frames arbitrary.
+    After the Q, K, V draws of ``qkv`` the same generator draws, in this order,
+    N(0, sigma^2) offset vectors per (b, h, KV frame), per (b, h, KV frame, key block of
+    ``key_block`` tokens) and per (b, h, query frame, query block of ``query_block``
+    rows); each K token gets its frame's and its block's offsets added, each Q row its
+    block's, in fp32 before the rounding to bf16.  V is unchanged.
+    """
+    g = torch.Generator("cpu").manual_seed(seed)
+    q = torch.randn(B, H, Tq * P, d, generator=g, dtype=torch.float32)
+    k = torch.randn(B, H, Tkv * P, d, generator=g, dtype=torch.float32)
+    v = torch.randn(B, H, Tkv * P, d, generator=g, dtype=torch.float32)
+    nkb = (P + key_block - 1) // key_block
+    nqb = (P + query_block - 1) // query_block
+    frame_off = sigma * torch.randn(B, H, Tkv, d, generator=g, dtype=torch.float32)
+    block_off = sigma * torch.randn(B, H, Tkv, nkb, d, generator=g, dtype=torch.float32)
+    query_off = sigma * torch.randn(B, H, Tq, nqb, d, generator=g, dtype=torch.float32)
+    kb_of_token = torch.arange(P) // key_block
+    qb_of_row = torch.arange(P) // query_block
+    k = k.view(B, H, Tkv, P, d) + frame_off[:, :, :, None, :] + block_off[:, :, :, kb_of_token, :]
+    q = q.view(B, H, Tq, P, d) + query_off[:, :, :, qb_of_row, :]
+    return (q.reshape(B, H, Tq * P, d).to(torch.bfloat16), k.reshape(B, H, Tkv * P, d).to(torch.bfloat16),
+            v.to(torch.bfloat16))
 
 
 def sample_rows(w: Workload, n_per_head: int, seed: int = 0, frames=()):
