@@ -9,16 +9,20 @@ Python face of libsfa.so (C ABI in include/sfa.h):
                     partials merged by LSE (short or uneven grids)
 * ``forward_paged`` - the same with K/V read through a per-head frame -> slot table
 * ``lse_merge``   - merge of two partial attentions (local + history branch) by LSE
+* ``hsa_select``  - hierarchical selection (Light Forcing HSA): pooled keys, top history
+                    frames, then top 128-token key blocks, per 256-row query block
+* ``forward_blocks`` - attention of every query block over its key-block list
 
 Tensors are PyTorch CUDA tensors; calls run on the current CUDA stream.
 """
 from ._lib import (SET_KINDS, SFA_DEBUG_STALL_SOFTMAX, SFA_ERR_BAD_SET, SFA_ERR_CUDA,
                    SFA_ERR_INVALID_ARG, SFA_ERR_TIMEOUT, SFA_ERR_UNSUPPORTED, SFA_OK, AttnDesc,
-                   SetParams, SfaError, attn_desc, build_sets, error_string, forward, forward_paged,
-                   forward_split, load, lse_merge, set_max_count, set_params, split_workspace_bytes, version)
+                   SetParams, SfaError, attn_desc, build_sets, error_string, forward, forward_blocks,
+                   forward_paged, forward_split, hsa_max_count, hsa_select, load, lse_merge, set_max_count,
+                   set_params, split_workspace_bytes, version)
 
 __all__ = ["SET_KINDS", "SFA_DEBUG_STALL_SOFTMAX", "SFA_ERR_BAD_SET", "SFA_ERR_CUDA",
            "SFA_ERR_INVALID_ARG", "SFA_ERR_TIMEOUT", "SFA_ERR_UNSUPPORTED", "SFA_OK", "AttnDesc",
-           "SetParams", "SfaError", "attn_desc", "build_sets", "error_string", "forward", "forward_paged",
-           "forward_split",
+           "SetParams", "SfaError", "attn_desc", "build_sets", "error_string", "forward", "forward_blocks",
+           "forward_paged", "forward_split", "hsa_max_count", "hsa_select",
            "load", "lse_merge", "set_max_count", "set_params", "split_workspace_bytes", "version"]

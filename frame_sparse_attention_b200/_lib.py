@@ -52,7 +52,7 @@ class AttnDesc(ctypes.Structure):
 _lib = None
 EXPORTS = ("sfa_error_string", "sfa_version", "sfa_set_max_count", "sfa_build_sets", "sfa_forward",
            "sfa_forward_split_workspace", "sfa_forward_split", "sfa_forward_split_noalloc", "sfa_forward_paged",
-           "sfa_lse_merge")
+           "sfa_lse_merge", "sfa_hsa_max_count", "sfa_hsa_workspace", "sfa_hsa_select", "sfa_forward_blocks")
 
 
 def load():
@@ -88,6 +88,15 @@ def load():
     lib.sfa_forward_paged.argtypes = [ctypes.POINTER(AttnDesc), vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp]
     lib.sfa_lse_merge.restype = st
     lib.sfa_lse_merge.argtypes = [i64, i32, vp, vp, vp, vp, vp, vp, vp]
+    lib.sfa_hsa_max_count.restype = st
+    lib.sfa_hsa_max_count.argtypes = [ctypes.POINTER(SetParams), i32, i32, i32, ctypes.POINTER(i32)]
+    lib.sfa_hsa_workspace.restype = st
+    lib.sfa_hsa_workspace.argtypes = [ctypes.POINTER(AttnDesc), ctypes.POINTER(ctypes.c_size_t)]
+    lib.sfa_hsa_select.restype = st
+    lib.sfa_hsa_select.argtypes = [ctypes.POINTER(AttnDesc), ctypes.POINTER(SetParams), i32, i32, vp, vp, vp,
+                                   ctypes.c_size_t, vp, vp, vp]
+    lib.sfa_forward_blocks.restype = st
+    lib.sfa_forward_blocks.argtypes = [ctypes.POINTER(AttnDesc), vp, vp, vp, vp, vp, vp, vp, vp, vp]
     _lib = lib
     return lib
 
@@ -265,4 +274,58 @@ def lse_merge(o1, lse1, o2, lse2, out=None, lse=None, stream=None):
         lse = torch.empty_like(lse1)
     _check(load().sfa_lse_merge(rows, d, o1.data_ptr(), lse1.data_ptr(), o2.data_ptr(), lse2.data_ptr(),
                                 out.data_ptr(), lse.data_ptr(), _stream(stream)), "sfa_lse_merge")
+    return out, lse
+
+
+KEY_BLOCK = 128    # tokens per key block of the hierarchical selection
+QUERY_BLOCK = 256  # query rows per query block
+
+
+def hsa_max_count(params: SetParams, P: int, k_frames: int, k_blocks: int) -> int:
+    """Length bound of a key-block list: the smallest Amax that hsa_select accepts."""
+    out = ctypes.c_int32(0)
+    _check(load().sfa_hsa_max_count(ctypes.byref(params), P, k_frames, k_blocks, ctypes.byref(out)),
+           "sfa_hsa_max_count")
+    return out.value
+
+
+def hsa_select(q, k, params: SetParams, k_frames: int, k_blocks: int, Amax: int | None = None, workspace=None,
+               stream=None):
+    """Hierarchical selection (pooled keys, top frames, then top blocks): (blocks int32
+    [B, H, Tq, nqb, Amax] sorted key-block ids with -1 padding, counts int32 [B, H, Tq, nqb])."""
+    B, H, Lq, d = q.shape
+    P = Lq // params.Tq
+    if Amax is None:
+        Amax = hsa_max_count(params, P, k_frames, k_blocks)
+    nqb = (P + QUERY_BLOCK - 1) // QUERY_BLOCK
+    desc = attn_desc(q, k, k, q, P, Amax)
+    nbytes = ctypes.c_size_t(0)
+    _check(load().sfa_hsa_workspace(ctypes.byref(desc), ctypes.byref(nbytes)), "sfa_hsa_workspace")
+    if workspace is None:
+        workspace = torch.empty(max(nbytes.value, 1), dtype=torch.uint8, device=q.device)
+    blocks = torch.empty((B, H, params.Tq, nqb, Amax), dtype=torch.int32, device=q.device)
+    counts = torch.empty((B, H, params.Tq, nqb), dtype=torch.int32, device=q.device)
+    _check(load().sfa_hsa_select(ctypes.byref(desc), ctypes.byref(params), k_frames, k_blocks, q.data_ptr(),
+                                 k.data_ptr(), workspace.data_ptr(), workspace.numel(), blocks.data_ptr(),
+                                 counts.data_ptr(), _stream(stream)), "sfa_hsa_select")
+    return blocks, counts
+
+
+def forward_blocks(q, k, v, blocks, counts, P: int, scale: float | None = None, out=None, lse=None,
+                   dev_status=None, stream=None, timeout_us: int = 0):
+    """Attention of every query block over its key-block list: (O bf16 like q, LSE fp32)."""
+    B, H, Lq, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, Lq), dtype=torch.float32, device=q.device)
+    assert lse.is_contiguous() and lse.dtype == torch.float32
+    assert blocks.dtype == torch.int32 and counts.dtype == torch.int32
+    assert blocks.is_contiguous() and counts.is_contiguous()
+    desc = attn_desc(q, k, v, out, P, blocks.shape[-1], scale, timeout_us)
+    nqb = (P + QUERY_BLOCK - 1) // QUERY_BLOCK
+    assert tuple(blocks.shape[:4]) == (B, H, desc.Tq, nqb) and tuple(counts.shape) == (B, H, desc.Tq, nqb)
+    _check(load().sfa_forward_blocks(ctypes.byref(desc), q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                     blocks.data_ptr(), counts.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                     _ptr(dev_status), _stream(stream)), "sfa_forward_blocks")
     return out, lse

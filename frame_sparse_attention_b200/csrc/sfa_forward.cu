@@ -45,6 +45,7 @@ namespace {
 
 constexpr int BM = 128;                 // query rows per tile = MMA M = TMEM lanes
 constexpr int BN = 128;                 // keys per K/V tile (largest MMA N used)
+constexpr int KEY_BLOCK = 128;          // tokens per key block of a key-block list
 // warps 0-3 softmax of query tile A, 4-7 softmax of query tile B, 8 Q+K loader,
 // 9 MMA issuer, 10 V loader
 constexpr int NUM_THREADS = 352;
@@ -105,6 +106,8 @@ struct FwdArgs {
     const int32_t *counts;
     const int32_t *slots;  // [H][T_kv] physical frame slot of each logical frame, or null
     int32_t n_slots;       // frames held by the K/V buffers (T_kv without a slot table)
+    int32_t nblk;          // > 0: the lists hold key blocks of KEY_BLOCK tokens (nblk per frame),
+                           // one list per (b, h, t, query block of 2 tiles); 0: frame lists per (h, t)
     float *lse;
     int32_t *status;
     uint64_t timeout_ns;
@@ -165,59 +168,88 @@ __device__ __noinline__ void wait_drain(uint32_t bar, uint32_t parity)
 // or the identity.
 __device__ __forceinline__ int slot_of(const int32_t *srow, int f) { return srow ? __ldg(srow + f) : f; }
 
-// Number of K/V tiles for a frame list, or -1 if the list is not strictly increasing
-// inside [0, T_kv) or a slot lies outside [0, n_slots).  A run is a stretch of list
-// entries whose slots are consecutive, i.e. one contiguous token interval.
-__device__ int count_tiles(const int32_t *fl, int cnt, int T_kv, int P, const int32_t *srow, int n_slots)
+// Token interval [lo, hi) of list entry x: frame x (through the slot table) or, with
+// key-block lists (nblk > 0), block x % nblk of frame x / nblk.
+__device__ __forceinline__ void entry_range(int x, int P, int nblk, const int32_t *srow, int &lo, int &hi)
+{
+    if (nblk) {
+        const int f = x / nblk, b = x - f * nblk;
+        lo = f * P + b * KEY_BLOCK;
+        hi = f * P + min(b * KEY_BLOCK + KEY_BLOCK, P);
+    } else {
+        lo = slot_of(srow, x) * P;
+        hi = lo + P;
+    }
+}
+
+// Number of K/V tiles for a list, or -1 if the list is not strictly increasing inside
+// [0, n_entries) or a frame's slot lies outside [0, n_slots).  A run is a stretch of
+// entries whose token intervals follow one another, i.e. one contiguous token interval.
+__device__ int count_tiles(const int32_t *fl, int cnt, int n_entries, int P, int nblk, const int32_t *srow,
+                           int n_slots)
 {
     int tiles = 0, a = 0, prev = -1;
     while (a < cnt) {
-        const int f0 = __ldg(fl + a);
-        if (f0 <= prev || f0 >= T_kv) return -1;
-        const int s0 = slot_of(srow, f0);
-        if (s0 < 0 || s0 >= n_slots) return -1;
-        int s1 = s0;
-        prev = f0;
+        const int x0 = __ldg(fl + a);
+        if (x0 <= prev || x0 >= n_entries) return -1;
+        if (!nblk) {
+            const int s0 = slot_of(srow, x0);
+            if (s0 < 0 || s0 >= n_slots) return -1;
+        }
+        int lo, hi;
+        entry_range(x0, P, nblk, srow, lo, hi);
+        const int run_lo = lo;
+        prev = x0;
         ++a;
         while (a < cnt) {
-            const int f = __ldg(fl + a);
-            if (f <= prev || f >= T_kv) return -1;
-            if (slot_of(srow, f) != s1 + 1 || s1 + 1 >= n_slots) break;
-            ++s1;
-            prev = f;
+            const int x = __ldg(fl + a);
+            if (x <= prev || x >= n_entries) return -1;
+            if (!nblk) {
+                const int s = slot_of(srow, x);
+                if (s < 0 || s >= n_slots) return -1;
+            }
+            int lo2, hi2;
+            entry_range(x, P, nblk, srow, lo2, hi2);
+            if (lo2 != hi) break;
+            hi = hi2;
+            prev = x;
             ++a;
         }
-        tiles += ((s1 - s0 + 1) * P + BN - 1) / BN;
+        tiles += (hi - run_lo + BN - 1) / BN;
     }
     return tiles;
 }
 
-// Walks the attended tokens as runs of consecutive frames, 128 keys at a time.
+// Walks the attended tokens as runs of contiguous list entries, 128 keys at a time.
 struct KvIter {
     const int32_t *fl;
     const int32_t *srow;
-    int n, a, P, pos, end;
-    __device__ void init(const int32_t *f, int cnt, int P_, const int32_t *slot_row)
+    int n, a, P, nblk, pos, end;
+    __device__ void init(const int32_t *f, int cnt, int P_, const int32_t *slot_row, int nblk_ = 0)
     {
         fl = f;
         srow = slot_row;
         n = cnt;
         a = 0;
         P = P_;
+        nblk = nblk_;
         pos = 0;
         end = 0;
     }
     __device__ void open_run()
     {
-        const int s0 = slot_of(srow, __ldg(fl + a));
-        int s1 = s0;
+        int lo, hi;
+        entry_range(__ldg(fl + a), P, nblk, srow, lo, hi);
         ++a;
-        while (a < n && slot_of(srow, __ldg(fl + a)) == s1 + 1) {
-            ++s1;
+        while (a < n) {
+            int lo2, hi2;
+            entry_range(__ldg(fl + a), P, nblk, srow, lo2, hi2);
+            if (lo2 != hi) break;
+            hi = hi2;
             ++a;
         }
-        pos = s0 * P;
-        end = (s1 + 1) * P;
+        pos = lo;
+        end = hi;
     }
     __device__ void next(int &start, int &nvalid)
     {
@@ -272,7 +304,7 @@ __device__ void loader_role(const CUtensorMap *tm_q, const CUtensorMap *tm_kv, c
     // K/V of one (h, t) are re-read by every query tile of the frame: keep them in L2
     const uint64_t policy = l2_policy_evict_last();
     KvIter it;
-    it.init(fl, cnt, a.P, a.slots ? a.slots + (int64_t)h * a.T_kv : nullptr);
+    it.init(fl, cnt, a.P, a.slots ? a.slots + (int64_t)h * a.T_kv : nullptr, a.nblk);
     it.skip(t_off);
     int j = 0;
     for (; j < n_tiles; ++j) {
@@ -364,7 +396,7 @@ __device__ void mma_role(const FwdArgs &a, uint32_t sbase, uint32_t tmem, int h,
     const int nx = has_b ? 2 : 1;
     bool issued = false;
     KvIter it;
-    it.init(fl, cnt, a.P, a.slots ? a.slots + (int64_t)h * a.T_kv : nullptr);
+    it.init(fl, cnt, a.P, a.slots ? a.slots + (int64_t)h * a.T_kv : nullptr, a.nblk);
     it.skip(t_off);
     int st, nv_cur = 0, nv_next = 0;
     it.next(st, nv_cur);
@@ -592,7 +624,7 @@ __device__ void softmax_role(const CUtensorMap *tm_o, const FwdArgs &a, uint8_t 
     float l = 0.f;             // running row sum of exp2(s*sl2 - m_used)
     bool alive = true;
     KvIter it;
-    it.init(fl, cnt, a.P, a.slots ? a.slots + (int64_t)h * a.T_kv : nullptr);
+    it.init(fl, cnt, a.P, a.slots ? a.slots + (int64_t)h * a.T_kv : nullptr, a.nblk);
     it.skip(t_off);
     for (int j = 0; j < n_tiles; ++j) {
         int st, nv;
@@ -695,10 +727,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     x /= a.Tq;
     const int h = x % a.H;
     const int b = x / a.H;
-    const int32_t *fl = a.frames + ((int64_t)h * a.Tq + t) * a.Amax;
-    const int cnt = __ldg(a.counts + h * a.Tq + t);
+    // the unit's list: frames of (h, t), or key blocks of (b, h, t, query block = pair)
+    const int64_t list = a.nblk ? ((((int64_t)b * a.H + h) * a.Tq + t) * n_pairs + qt_a / 2) : (int64_t)h * a.Tq + t;
+    const int32_t *fl = a.frames + list * a.Amax;
+    const int cnt = __ldg(a.counts + list);
     int n_all = (cnt >= 0 && cnt <= a.Amax)
-                    ? count_tiles(fl, cnt, a.T_kv, a.P, a.slots ? a.slots + (int64_t)h * a.T_kv : nullptr, a.n_slots)
+                    ? count_tiles(fl, cnt, a.nblk ? a.T_kv * a.nblk : a.T_kv, a.P, a.nblk,
+                                  a.slots ? a.slots + (int64_t)h * a.T_kv : nullptr, a.n_slots)
                     : -1;
     const bool bad_set = n_all < 0;
     if (bad_set) n_all = 0;
@@ -812,7 +847,7 @@ template <int D>
 sfa_status launch(const sfa_attn_desc *d, const void *q, const void *k, const void *v, const int32_t *frames,
                   const int32_t *counts, void *o, float *lse, int32_t *dev_status, cudaStream_t stream,
                   int n_split = 1, void *ws_o = nullptr, float *ws_lse = nullptr, const int32_t *slots = nullptr,
-                  int n_slots = 0)
+                  int n_slots = 0, int nblk = 0)
 {
     using C = Cfg<D>;
     CUtensorMap tq, tk, tv, to;
@@ -856,6 +891,7 @@ sfa_status launch(const sfa_attn_desc *d, const void *q, const void *k, const vo
     a.counts = counts;
     a.slots = slots;
     a.n_slots = kv_frames;
+    a.nblk = nblk;
     a.lse = n_split == 1 ? lse : ws_lse;
     a.status = dev_status;
     a.timeout_ns = (uint64_t)(d->timeout_us ? d->timeout_us : DEFAULT_TIMEOUT_US) * 1000;
@@ -1024,6 +1060,28 @@ extern "C" sfa_status sfa_forward_split_noalloc(const sfa_attn_desc *d, const vo
     float *ws_lse = reinterpret_cast<float *>(static_cast<char *>(scratch) + split_ws_o_bytes(d, n_split));
     return d->d == 128 ? launch<128>(d, q, k, v, frames, counts, o, lse, dev_status, s, n_split, scratch, ws_lse)
                        : launch<64>(d, q, k, v, frames, counts, o, lse, dev_status, s, n_split, scratch, ws_lse);
+}
+
+// ------------------------------------------------------------------------------------
+// Key-block lists (hierarchical selection): each (b, h, t, query block of 256 rows) has
+// its own sorted list of 128-token key blocks.
+// ------------------------------------------------------------------------------------
+extern "C" sfa_status sfa_forward_blocks(const sfa_attn_desc *d, const void *q, const void *k, const void *v,
+                                         const int32_t *blocks, const int32_t *counts, void *o, float *lse,
+                                         int32_t *dev_status, sfa_stream_t stream)
+{
+    sfa_status st = check_desc(d);
+    if (st != SFA_OK) return st;
+    if ((int64_t)d->T_kv * ((d->P + KEY_BLOCK - 1) / KEY_BLOCK) >= ((int64_t)1 << 31)) return SFA_ERR_INVALID_ARG;
+    if (d->B == 0) return SFA_OK;
+    st = check_buffers(d, q, k, v, blocks, counts, o, lse);
+    if (st != SFA_OK) return st;
+    cudaStream_t s = as_cuda(stream);
+    const int nblk = (d->P + KEY_BLOCK - 1) / KEY_BLOCK;
+    return d->d == 128 ? launch<128>(d, q, k, v, blocks, counts, o, lse, dev_status, s, 1, nullptr, nullptr, nullptr, 0,
+                                     nblk)
+                       : launch<64>(d, q, k, v, blocks, counts, o, lse, dev_status, s, 1, nullptr, nullptr, nullptr, 0,
+                                    nblk);
 }
 
 // ------------------------------------------------------------------------------------

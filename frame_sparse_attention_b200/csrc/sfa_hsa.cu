@@ -1,0 +1,398 @@
+// Hierarchical sparse attention (HSA): the two-level selection of key blocks.
+//
+// "Resumen Técnico: LIGHT FORCING", §2.2 Atención Dispersa Jerárquica: query and key
+// tokens are mean-pooled per block and per frame (token compression); each query block
+// retrieves a few history frames with the frame-level pooled keys (frame selection), then
+// the critical blocks inside those frames with the block-level pooled keys (block
+// selection); attention then runs over the selected frame-block pairs only
+// (sfa_forward_blocks, in sfa_forward.cu).
+//
+// Two kernels:
+//   * hsa_pool_kernel: one CTA per (frame, h, b) of keys or queries; 16-byte loads,
+//     fp32 sums per column, one mean per segment (128-token key block or 256-row query
+//     block) and, for keys, one per frame.  HBM-bound: every K and Q element is read once.
+//   * hsa_select_kernel: one CTA per (b, h, t, query block): scores of the history
+//     frames, top k_frames, scores of their blocks, top k_blocks, then the sorted union
+//     with the always-attended blocks, compacted with a block-wide prefix count.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+
+#include "sfa.h"
+#include "sfa_internal.h"
+
+namespace sfa {
+namespace {
+
+constexpr int KEY_BLOCK = 128;    // tokens per key block
+constexpr int QUERY_BLOCK = 256;  // query rows per query block
+constexpr int POOL_THREADS = 256;
+constexpr int SELECT_THREADS = 256;
+constexpr int MAX_ENTRIES = 65536;  // T_kv * nblk bound (the block flags live in shared memory)
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Means of the segments of `seg` rows of one frame of x (P rows of D bf16, row stride
+// `row_stride` elements), written to seg_out[nseg][D]; with frame_out, also the mean of
+// the whole frame.  Thread layout: D/8 threads per row (8 columns, one 16-byte load
+// each), POOL_THREADS / (D/8) rows at a time; a shared-memory pass adds the row groups.
+template <int D>
+__global__ void __launch_bounds__(POOL_THREADS) hsa_pool_kernel(const uint16_t *x, int64_t s_b, int64_t s_h,
+                                                                  int64_t s_row, int P, int seg, int n_frames,
+                                                                  float *seg_out, float *frame_out)
+{
+    constexpr int TPR = D / 8;                 // threads per row
+    constexpr int RG = POOL_THREADS / TPR;     // rows in flight
+    __shared__ float part[RG][D];
+    __shared__ float frame_acc[D];
+    const int f = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int H = gridDim.y;
+    const int cg = threadIdx.x % TPR, rg = threadIdx.x / TPR;
+    const uint16_t *base = x + b * s_b + h * s_h + (int64_t)f * P * s_row + cg * 8;
+    const int nseg = (P + seg - 1) / seg;
+    float *out = seg_out + (((int64_t)b * H + h) * n_frames + f) * nseg * D;
+    if (threadIdx.x < D) frame_acc[threadIdx.x] = 0.f;
+    for (int sg = 0; sg < nseg; ++sg) {
+        const int r0 = sg * seg, r1 = min(r0 + seg, P);
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int r = r0 + rg; r < r1; r += RG) {
+            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(base + (int64_t)r * s_row));
+            acc[0] += bf16_lo(v.x);
+            acc[1] += bf16_hi(v.x);
+            acc[2] += bf16_lo(v.y);
+            acc[3] += bf16_hi(v.y);
+            acc[4] += bf16_lo(v.z);
+            acc[5] += bf16_hi(v.z);
+            acc[6] += bf16_lo(v.w);
+            acc[7] += bf16_hi(v.w);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) part[rg][cg * 8 + i] = acc[i];
+        __syncthreads();
+        if (threadIdx.x < D) {
+            float s = 0.f;
+            for (int g = 0; g < RG; ++g) s += part[g][threadIdx.x];
+            out[(int64_t)sg * D + threadIdx.x] = s / (float)(r1 - r0);
+            frame_acc[threadIdx.x] += s;
+        }
+        __syncthreads();
+    }
+    if (frame_out && threadIdx.x < D)
+        frame_out[(((int64_t)b * H + h) * n_frames + f) * D + threadIdx.x] = frame_acc[threadIdx.x] / (float)P;
+}
+
+struct SelectArgs {
+    int B, H, Tq, T_kv, P, nblk, nqb, Amax;
+    int q_off, n_sink, n_prev, chunk_len, k_frames, k_blocks;
+    const float *kf;  // [B][H][T_kv][D]
+    const float *kb;  // [B][H][T_kv][nblk][D]
+    const float *qb;  // [B][H][Tq][nqb][D]
+    int32_t *blocks;  // [B][H][Tq][nqb][Amax]
+    int32_t *counts;  // [B][H][Tq][nqb]
+};
+
+// a > b in the selection order: larger score, then smaller id
+__device__ __forceinline__ bool ranks_before(float sa, int ia, float sb, int ib)
+{
+    return sa > sb || (sa == sb && ia < ib);
+}
+
+// One warp: the index (into ids/scores[0, n)) of the best entry not yet taken, or -1.
+__device__ int warp_best(const float *scores, const int *ids, const uint8_t *taken, int n)
+{
+    const int lane = threadIdx.x & 31;
+    float bs = -INFINITY;
+    int bi = -1, bid = 0x7fffffff;
+    for (int i = lane; i < n; i += 32) {
+        if (taken[i]) continue;
+        if (bi < 0 || ranks_before(scores[i], ids[i], bs, bid)) {
+            bs = scores[i];
+            bi = i;
+            bid = ids[i];
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        const float os = __shfl_xor_sync(0xffffffffu, bs, off);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+        const int oid = __shfl_xor_sync(0xffffffffu, bid, off);
+        if (oi >= 0 && (bi < 0 || ranks_before(os, oid, bs, bid))) {
+            bs = os;
+            bi = oi;
+            bid = oid;
+        }
+    }
+    return bi;
+}
+
+// dot(q, key) of D floats by one warp
+template <int D>
+__device__ __forceinline__ float warp_dot(const float *q, const float *key)
+{
+    const int lane = threadIdx.x & 31;
+    float s = 0.f;
+#pragma unroll
+    for (int i = lane; i < D; i += 32) s = fmaf(q[i], __ldg(key + i), s);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    return s;
+}
+
+// Dynamic shared memory: frame scores/ids/taken [T_kv], block scores/ids/taken
+// [k_frames' * nblk], entry flags [T_kv * nblk], warp totals.
+template <int D>
+__global__ void __launch_bounds__(SELECT_THREADS) hsa_select_kernel(const __grid_constant__ SelectArgs a)
+{
+    extern __shared__ __align__(16) uint8_t sm[];
+    __shared__ float qv[D];
+    __shared__ int n_hist_s, n_sel_s;
+    __shared__ int warp_tot[SELECT_THREADS / 32];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = SELECT_THREADS / 32;
+    int u = blockIdx.x;
+    const int qi = u % a.nqb;
+    u /= a.nqb;
+    const int t = u % a.Tq;
+    u /= a.Tq;
+    const int h = u % a.H;
+    const int b = u / a.H;
+    const int n_sel_max = min(a.k_frames, a.T_kv);
+    const int n_bc_max = n_sel_max * a.nblk;
+    const int n_entries = a.T_kv * a.nblk;
+    float *f_score = reinterpret_cast<float *>(sm);
+    int *f_id = reinterpret_cast<int *>(f_score + a.T_kv);
+    float *b_score = reinterpret_cast<float *>(f_id + a.T_kv);
+    int *b_id = reinterpret_cast<int *>(b_score + n_bc_max);
+    int *sel = b_id + n_bc_max;                                         // [n_sel_max]
+    uint8_t *f_taken = reinterpret_cast<uint8_t *>(sel + n_sel_max);   // [T_kv]
+    uint8_t *b_taken = f_taken + a.T_kv;                                // [n_bc_max]
+    uint8_t *flag = b_taken + n_bc_max;                                 // [n_entries]
+
+    const int c = t + a.q_off;
+    const int c0 = c - c % a.chunk_len;
+    const int w_lo = c0 - a.n_prev, w_hi = c0 + a.chunk_len;  // local window [w_lo, w_hi)
+    const int64_t bh = (int64_t)b * a.H + h;
+    for (int i = threadIdx.x; i < D; i += SELECT_THREADS)
+        qv[i] = a.qb[(((bh * a.Tq + t) * a.nqb) + qi) * D + i];
+    for (int i = threadIdx.x; i < n_entries; i += SELECT_THREADS) flag[i] = 0;
+    if (threadIdx.x == 0) {
+        // history candidates in ascending order
+        int n = 0;
+        for (int f = 0; f < min(c0, a.T_kv); ++f)
+            if (!(f < a.n_sink || (f >= w_lo && f < w_hi))) f_id[n++] = f;
+        n_hist_s = n;
+    }
+    __syncthreads();
+    const int n_hist = n_hist_s;
+    // frame scores
+    for (int i = warp; i < n_hist; i += nwarps) {
+        const float s = warp_dot<D>(qv, a.kf + (bh * a.T_kv + f_id[i]) * D);
+        if (lane == 0) {
+            f_score[i] = s;
+            f_taken[i] = 0;
+        }
+    }
+    __syncthreads();
+    // top k_frames (warp 0)
+    if (warp == 0) {
+        const int n_sel = min(a.k_frames, n_hist);
+        for (int k = 0; k < n_sel; ++k) {
+            const int bi = warp_best(f_score, f_id, f_taken, n_hist);
+            if (lane == 0) {
+                f_taken[bi] = 1;
+                sel[k] = f_id[bi];
+            }
+            __syncwarp();
+        }
+        if (lane == 0) n_sel_s = n_sel;
+    }
+    __syncthreads();
+    const int n_sel = n_sel_s;
+    const int n_bc = n_sel * a.nblk;
+    // block scores of the selected frames
+    for (int i = warp; i < n_bc; i += nwarps) {
+        const int f = sel[i / a.nblk], bb = i % a.nblk;
+        const float s = warp_dot<D>(qv, a.kb + ((bh * a.T_kv + f) * a.nblk + bb) * D);
+        if (lane == 0) {
+            b_score[i] = s;
+            b_id[i] = f * a.nblk + bb;
+            b_taken[i] = 0;
+        }
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const int n_pick = min(a.k_blocks, n_bc);
+        for (int k = 0; k < n_pick; ++k) {
+            const int bi = warp_best(b_score, b_id, b_taken, n_bc);
+            if (lane == 0) {
+                b_taken[bi] = 1;
+                flag[b_id[bi]] = 1;
+            }
+            __syncwarp();
+        }
+    }
+    // always-attended frames: every block
+    for (int i = threadIdx.x; i < n_entries; i += SELECT_THREADS) {
+        const int f = i / a.nblk;
+        if (f < a.n_sink || (f >= w_lo && f < w_hi)) flag[i] = 1;
+    }
+    __syncthreads();
+    // compaction in id order: block-wide prefix count, SELECT_THREADS ids per round
+    int32_t *out = a.blocks + (((bh * a.Tq + t) * a.nqb) + qi) * a.Amax;
+    int base = 0;
+    for (int r0 = 0; r0 < n_entries; r0 += SELECT_THREADS) {
+        const int i = r0 + threadIdx.x;
+        const bool on = i < n_entries && flag[i];
+        const unsigned m = __ballot_sync(0xffffffffu, on);
+        if (lane == 0) warp_tot[warp] = __popc(m);
+        __syncthreads();
+        int before = base;
+        for (int w = 0; w < warp; ++w) before += warp_tot[w];
+        before += __popc(m & ((1u << lane) - 1u));
+        if (on && before < a.Amax) out[before] = i;
+        int total = 0;
+        for (int w = 0; w < nwarps; ++w) total += warp_tot[w];
+        base += total;
+        __syncthreads();
+    }
+    for (int i = base + threadIdx.x; i < a.Amax; i += SELECT_THREADS) out[i] = -1;
+    if (threadIdx.x == 0) a.counts[((bh * a.Tq + t) * a.nqb) + qi] = min(base, a.Amax);
+}
+
+bool params_ok(const sfa_set_params *p, int P, int k_frames, int k_blocks)
+{
+    if (!p || P < 1 || k_frames < 0 || k_blocks < 0) return false;
+    if (p->T_kv < 1 || p->Tq < 1 || p->q_off < 0 || (int64_t)p->q_off + p->Tq > p->T_kv) return false;
+    if (p->n_sink < 0 || p->n_prev < 0 || p->chunk_len < 1) return false;
+    const int64_t nblk = (P + KEY_BLOCK - 1) / KEY_BLOCK;
+    return (int64_t)p->T_kv * nblk <= MAX_ENTRIES;
+}
+
+int64_t max_count(const sfa_set_params *p, int P, int k_frames, int k_blocks)
+{
+    const int64_t nblk = (P + KEY_BLOCK - 1) / KEY_BLOCK;
+    const int64_t always = std::min<int64_t>((int64_t)p->n_sink + p->n_prev + p->chunk_len, p->T_kv) * nblk;
+    return always + std::min<int64_t>(k_blocks, (int64_t)k_frames * nblk);
+}
+
+struct WsLayout {
+    size_t kf, kb, qb, total;
+};
+
+WsLayout ws_layout(const sfa_attn_desc *d)
+{
+    auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+    const size_t nblk = (d->P + KEY_BLOCK - 1) / KEY_BLOCK, nqb = (d->P + QUERY_BLOCK - 1) / QUERY_BLOCK;
+    const size_t bh = (size_t)d->B * d->H;
+    WsLayout w;
+    w.kf = 0;
+    w.kb = up(bh * d->T_kv * d->d * 4);
+    w.qb = w.kb + up(bh * d->T_kv * nblk * d->d * 4);
+    w.total = w.qb + up(bh * d->Tq * nqb * d->d * 4);
+    return w;
+}
+
+bool desc_ok(const sfa_attn_desc *d)
+{
+    if (!d || d->B < 0 || d->H < 1 || d->Tq < 1 || d->T_kv < 1 || d->P < 1 || d->Amax < 1) return false;
+    if ((int64_t)d->Tq * d->P >= ((int64_t)1 << 31) || (int64_t)d->T_kv * d->P >= ((int64_t)1 << 31)) return false;
+    if (d->H > 65535 || d->B > 65535) return false;  // grid y / z of the pooling launch
+    return true;
+}
+
+bool stride_ok(const int64_t *s, int d)
+{
+    return s[2] >= d && s[0] >= 0 && s[1] >= 0 && s[0] % 8 == 0 && s[1] % 8 == 0 && s[2] % 8 == 0;
+}
+
+template <int D>
+sfa_status run_select(const sfa_attn_desc *d, const sfa_set_params *p, int k_frames, int k_blocks, const void *q,
+                      const void *k, uint8_t *ws, int32_t *blocks, int32_t *counts, cudaStream_t s)
+{
+    const WsLayout w = ws_layout(d);
+    float *kf = reinterpret_cast<float *>(ws + w.kf), *kb = reinterpret_cast<float *>(ws + w.kb);
+    float *qb = reinterpret_cast<float *>(ws + w.qb);
+    hsa_pool_kernel<D><<<dim3(d->T_kv, d->H, d->B), POOL_THREADS, 0, s>>>(
+        static_cast<const uint16_t *>(k), d->k_stride[0], d->k_stride[1], d->k_stride[2], d->P, KEY_BLOCK, d->T_kv, kb,
+        kf);
+    hsa_pool_kernel<D><<<dim3(d->Tq, d->H, d->B), POOL_THREADS, 0, s>>>(
+        static_cast<const uint16_t *>(q), d->q_stride[0], d->q_stride[1], d->q_stride[2], d->P, QUERY_BLOCK, d->Tq,
+        qb, nullptr);
+    SelectArgs a;
+    a.B = d->B;
+    a.H = d->H;
+    a.Tq = d->Tq;
+    a.T_kv = d->T_kv;
+    a.P = d->P;
+    a.nblk = (d->P + KEY_BLOCK - 1) / KEY_BLOCK;
+    a.nqb = (d->P + QUERY_BLOCK - 1) / QUERY_BLOCK;
+    a.Amax = d->Amax;
+    a.q_off = p->q_off;
+    a.n_sink = p->n_sink;
+    a.n_prev = p->n_prev;
+    a.chunk_len = p->chunk_len;
+    a.k_frames = k_frames;
+    a.k_blocks = k_blocks;
+    a.kf = kf;
+    a.kb = kb;
+    a.qb = qb;
+    a.blocks = blocks;
+    a.counts = counts;
+    const int n_sel_max = std::min(k_frames, d->T_kv);
+    const size_t n_bc_max = (size_t)n_sel_max * a.nblk;
+    const size_t smem = (size_t)d->T_kv * 8 + n_bc_max * 8 + (size_t)n_sel_max * 4 + d->T_kv + n_bc_max +
+                        (size_t)d->T_kv * a.nblk;
+    if (smem > 200 * 1024) return SFA_ERR_UNSUPPORTED;
+    if (cudaFuncSetAttribute(hsa_select_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+        return SFA_ERR_CUDA;
+    const int64_t grid = (int64_t)d->B * d->H * d->Tq * a.nqb;
+    hsa_select_kernel<D><<<(unsigned)grid, SELECT_THREADS, smem, s>>>(a);
+    return launch_status();
+}
+
+}  // namespace
+}  // namespace sfa
+
+using namespace sfa;
+
+extern "C" sfa_status sfa_hsa_max_count(const sfa_set_params *p, int32_t P, int32_t k_frames, int32_t k_blocks,
+                                        int32_t *amax_out)
+{
+    if (!amax_out || !params_ok(p, P, k_frames, k_blocks)) return SFA_ERR_INVALID_ARG;
+    const int64_t m = max_count(p, P, k_frames, k_blocks);
+    if (m > INT32_MAX) return SFA_ERR_INVALID_ARG;
+    *amax_out = (int32_t)std::max<int64_t>(m, 1);
+    return SFA_OK;
+}
+
+extern "C" sfa_status sfa_hsa_workspace(const sfa_attn_desc *d, size_t *bytes)
+{
+    if (!bytes || !desc_ok(d)) return SFA_ERR_INVALID_ARG;
+    if (d->d != 64 && d->d != 128) return SFA_ERR_UNSUPPORTED;
+    *bytes = ws_layout(d).total;
+    return SFA_OK;
+}
+
+extern "C" sfa_status sfa_hsa_select(const sfa_attn_desc *d, const sfa_set_params *p, int32_t k_frames,
+                                     int32_t k_blocks, const void *q, const void *k, void *workspace,
+                                     size_t workspace_bytes, int32_t *blocks, int32_t *counts, sfa_stream_t stream)
+{
+    if (!desc_ok(d) || !params_ok(p, d ? d->P : 0, k_frames, k_blocks)) return SFA_ERR_INVALID_ARG;
+    if (d->d != 64 && d->d != 128) return SFA_ERR_UNSUPPORTED;
+    if (p->T_kv != d->T_kv || p->Tq != d->Tq) return SFA_ERR_INVALID_ARG;
+    if (max_count(p, d->P, k_frames, k_blocks) > d->Amax) return SFA_ERR_INVALID_ARG;
+    if (d->B == 0) return SFA_OK;
+    if (!q || !k || !workspace || !blocks || !counts) return SFA_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(q) % 16 || reinterpret_cast<uintptr_t>(k) % 16 ||
+        reinterpret_cast<uintptr_t>(workspace) % 256)
+        return SFA_ERR_INVALID_ARG;
+    if (!stride_ok(d->q_stride, d->d) || !stride_ok(d->k_stride, d->d)) return SFA_ERR_INVALID_ARG;
+    if (workspace_bytes < ws_layout(d).total) return SFA_ERR_INVALID_ARG;
+    cudaStream_t s = as_cuda(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    return d->d == 128 ? run_select<128>(d, p, k_frames, k_blocks, q, k, ws, blocks, counts, s)
+                       : run_select<64>(d, p, k_frames, k_blocks, q, k, ws, blocks, counts, s);
+}

@@ -9,6 +9,9 @@
  *                   only, writing O (bf16) and the per-row log-sum-exp (fp32)
  *   sfa_lse_merge   merge of two partial attentions (e.g. local + history branch)
  *
+ * plus variants of the forward (paged caches, split-KV) and the hierarchical block
+ * selection of Light Forcing (sfa_hsa_select + sfa_forward_blocks).
+ *
  * Conventions
  *   - A video has T latent frames of P tokens each; token i belongs to frame i / P.
  *     Query frame t (0 <= t < Tq) sits at frame t + q_off of the key/value timeline
@@ -244,6 +247,66 @@ sfa_status sfa_forward_split(const sfa_attn_desc *desc, const void *q, const voi
 sfa_status sfa_forward_split_noalloc(const sfa_attn_desc *desc, const void *q, const void *k, const void *v,
                                      const int32_t *frames, const int32_t *counts, void *o, float *lse,
                                      int32_t n_split, int32_t *dev_status, sfa_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
+ * Hierarchical sparse attention (HSA): selection of key blocks, and attention over them
+ * ------------------------------------------------------------------------------------
+ * ("Resumen Técnico: LIGHT FORCING", §2.2 Atención Dispersa Jerárquica: query and key
+ *  tokens are mean-pooled per block and per frame; each query block picks a few history
+ *  frames with the frame-level pooled keys, then the critical blocks inside them with the
+ *  block-level pooled keys; attention runs over the picked frame-block pairs only.)
+ *
+ * Blocks.  A key block is 128 consecutive tokens of one frame: block b of frame f holds
+ * tokens [f*P + 128 b, f*P + min(128 (b+1), P)) and has id f * nblk + b, with
+ * nblk = ceil(P / 128).  A query block is 256 consecutive query rows of one frame (the
+ * last one of a frame holds the rest): nqb = ceil(P / 256) per frame.
+ *
+ * Selection, per (b, h, query frame t, query block), with c = t + q_off and the chunk
+ * [c0, c0 + chunk_len), c0 = c - c mod chunk_len:
+ *   always  = every block of the frames {0 .. n_sink-1} ∪ [c0 - n_prev, c0 + chunk_len)
+ *             (the sink and the local window; clipped to [0, T_kv));
+ *   history = the other frames before c0;
+ *   score   = (mean of the block's query rows) . (mean of the frame's or block's keys),
+ *             in fp32;
+ *   frames  = the k_frames history frames of highest score; then
+ *   picked  = the k_blocks blocks of highest score among all blocks of those frames
+ *             (equal scores: the smaller id first; k larger than the candidates keeps
+ *             them all);
+ *   list    = always ∪ picked, sorted ascending.
+ *
+ * sfa_hsa_max_count: the list length bound for these parameters,
+ *   (n_sink + n_prev + chunk_len) * nblk + min(k_blocks, k_frames * nblk): the smallest
+ *   Amax that sfa_hsa_select accepts.
+ * sfa_hsa_workspace: bytes of device workspace sfa_hsa_select needs (the pooled keys
+ *   and queries, fp32).
+ * sfa_hsa_select: writes the lists.
+ *   desc      B, H, Tq, T_kv, P, d, q_stride, k_stride as for sfa_forward; desc->Amax =
+ *             list capacity (>= sfa_hsa_max_count); scale, v/o strides unused.
+ *   p         q_off, n_sink, n_prev, chunk_len used (p->T_kv, p->Tq must equal the
+ *             descriptor's); the LVSA fields are ignored.
+ *   q, k      bf16, laid out as for sfa_forward.
+ *   workspace caller-owned device memory, >= sfa_hsa_workspace bytes, 256-byte aligned;
+ *             scratch, overwritten.
+ *   blocks    device int32 [B][H][Tq][nqb][Amax], written: the sorted list, -1 padding.
+ *   counts    device int32 [B][H][Tq][nqb], written: list lengths.
+ *   k_frames >= 0, k_blocks >= 0; T_kv * nblk <= 65536.
+ * sfa_forward_blocks: sfa_forward over key-block lists: query rows of query block i of
+ *   frame t attend to the tokens of the blocks in blocks[b][h][t][i] (layout and Amax as
+ *   sfa_hsa_select writes them; each list strictly increasing inside [0, T_kv * nblk),
+ *   else SFA_ERR_BAD_SET through dev_status).  Other arguments as sfa_forward.
+ */
+sfa_status sfa_hsa_max_count(const sfa_set_params *p, int32_t P, int32_t k_frames, int32_t k_blocks,
+                             int32_t *amax_out);
+
+sfa_status sfa_hsa_workspace(const sfa_attn_desc *desc, size_t *bytes);
+
+sfa_status sfa_hsa_select(const sfa_attn_desc *desc, const sfa_set_params *p, int32_t k_frames,
+                          int32_t k_blocks, const void *q, const void *k, void *workspace,
+                          size_t workspace_bytes, int32_t *blocks, int32_t *counts, sfa_stream_t stream);
+
+sfa_status sfa_forward_blocks(const sfa_attn_desc *desc, const void *q, const void *k, const void *v,
+                              const int32_t *blocks, const int32_t *counts, void *o, float *lse,
+                              int32_t *dev_status, sfa_stream_t stream);
 
 /* ------------------------------------------------------------------------------------
  * LSE merge

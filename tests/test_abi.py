@@ -153,3 +153,37 @@ def test_split_workspace_and_arguments(sfa):
                                  None, None) == 1
     assert lib.sfa_forward_split(ctypes.byref(d), good, good, good, good, good, good, good, 2, good + 128,
                                  out.value, None, None) == 1
+
+
+def test_hsa_host_checks(sfa):
+    lib = sfa.load()
+    P = sfa.set_params
+    # (n_sink + n_prev + chunk_len) * nblk + min(k_blocks, k_frames * nblk); P = 1560 -> 13 blocks
+    p = P(T_kv=24, Tq=3, q_off=21, n_sink=1, n_prev=3, chunk_len=3)
+    assert sfa.hsa_max_count(p, 1560, 4, 24) == 7 * 13 + 24
+    assert sfa.hsa_max_count(p, 1560, 1, 24) == 7 * 13 + 13
+    assert sfa.hsa_max_count(p, 200, 0, 5) == 7 * 2
+    with pytest.raises(sfa.SfaError):
+        sfa.hsa_max_count(p, 1560, -1, 3)
+    d = _desc(sfa, Tq=3, T_kv=24, P=1560, Amax=7 * 13 + 24 - 1)
+    good = 1 << 20
+    ws = ctypes.c_size_t(0)
+    assert lib.sfa_hsa_workspace(ctypes.byref(d), ctypes.byref(ws)) == 0 and ws.value > 0
+    # Amax below the bound, Tq mismatch, misaligned workspace: refused before any launch
+    assert lib.sfa_hsa_select(ctypes.byref(d), ctypes.byref(p), 4, 24, good, good, good, ws.value, good, good,
+                              None) == sfa.SFA_ERR_INVALID_ARG
+    d.Amax = 7 * 13 + 24
+    p2 = P(T_kv=24, Tq=2, q_off=21, n_sink=1, n_prev=3, chunk_len=3)
+    assert lib.sfa_hsa_select(ctypes.byref(d), ctypes.byref(p2), 4, 24, good, good, good, ws.value, good, good,
+                              None) == sfa.SFA_ERR_INVALID_ARG
+    assert lib.sfa_hsa_select(ctypes.byref(d), ctypes.byref(p), 4, 24, good, good, good + 16, ws.value, good,
+                              good, None) == sfa.SFA_ERR_INVALID_ARG
+    assert lib.sfa_hsa_select(ctypes.byref(d), ctypes.byref(p), 4, 24, good, good, good, ws.value - 1, good,
+                              good, None) == sfa.SFA_ERR_INVALID_ARG
+    d.B = 0  # nothing to do
+    assert lib.sfa_hsa_select(ctypes.byref(d), ctypes.byref(p), 4, 24, good, good, good, ws.value, good, good,
+                              None) == 0
+    d = _desc(sfa, d=96)
+    assert lib.sfa_forward_blocks(ctypes.byref(d), good, good, good, good, good, good, good, None, None) == 2
+    d = _desc(sfa)
+    assert lib.sfa_forward_blocks(ctypes.byref(d), good, good, good, None, good, good, good, None, None) == 1

@@ -1,0 +1,167 @@
+"""Hierarchical sparse attention on the GPU against the oracle ("Resumen Técnico: LIGHT
+FORCING", §2.2): the block lists of sfa_hsa_select against oracle.hsa's selection, and
+sfa_forward_blocks against oracle.hsa.attention_blocks on the oracle's own lists.
+
+Selection is an integer result decided by floating-point scores: the GPU ranks fp32
+means and dot products, the oracle fp64 ones.  Lists must be identical wherever the
+oracle's scores separate the kept from the dropped candidates by more than SCORE_EPS (a
+bound far above the fp32 error of a mean over <= 1560 values and a d-term dot product);
+where they do not, the GPU list must still be a valid selection under the fp64 scores
+within SCORE_EPS.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import hsa
+from sfa_workloads import WORKLOADS, Workload, SetSpec, qkv, sample_rows, workload_qkv
+
+from gpu_helpers import compare, sfa
+
+pytestmark = pytest.mark.gpu
+
+SCORE_EPS = 1e-4
+
+
+def _params(w):
+    return sfa().set_params(T_kv=w.Tkv, Tq=w.Tq, q_off=w.q_off, n_sink=w.n_sink, n_prev=w.n_prev,
+                            chunk_len=w.chunk_len)
+
+
+def _kw(w):
+    return dict(P=w.P, T_kv=w.Tkv, q_off=w.q_off, chunk_len=w.chunk_len, n_prev=w.n_prev, n_sink=w.n_sink,
+                k_frames=w.k_frames, k_blocks=w.k_blocks)
+
+
+def _check_selection(w, q, k, lists_gpu, counts_gpu):
+    """Exact where the fp64 scores decide clearly; a valid selection elsewhere."""
+    kw = _kw(w)
+    Amax = lists_gpu.shape[-1]
+    o_lists, o_counts = hsa.build_block_lists(q.float().numpy(), k.float().numpy(), Bmax=Amax, **kw)
+    kf, kb = hsa.pool_keys(k.float().numpy(), w.P)
+    qb = hsa.pool_queries(q.float().numpy(), w.P)
+    nb = hsa.n_key_blocks(w.P)
+    fw = {x: kw[x] for x in ("T_kv", "q_off", "chunk_len", "n_prev", "n_sink")}
+    n_close = 0
+    B, H, Tq, nq = o_counts.shape
+    for b in range(B):
+        for h in range(H):
+            for t in range(Tq):
+                always = hsa.always_frames(t, **fw)
+                hist = hsa.history_frames(t, **fw)
+                for i in range(nq):
+                    got = lists_gpu[b, h, t, i, :counts_gpu[b, h, t, i]].tolist()
+                    assert all(x == -1 for x in lists_gpu[b, h, t, i, counts_gpu[b, h, t, i]:])
+                    want = o_lists[b, h, t, i, :o_counts[b, h, t, i]].tolist()
+                    if got == want:
+                        continue
+                    n_close += 1
+                    # not identical: both selections must be equally good within SCORE_EPS
+                    fs = {f: float(np.dot(qb[b, h, t, i], kf[b, h, f])) for f in hist}
+                    n_sel = min(w.k_frames, len(hist))
+                    kth = sorted(fs.values(), reverse=True)[n_sel - 1] if n_sel else math.inf
+                    assert got == sorted(set(got))
+                    assert all(f * nb + x in got for f in always for x in range(nb))
+                    picked = [g for g in got if g // nb not in always]
+                    assert len(picked) == min(w.k_blocks, n_sel * nb)
+                    assert all(fs[g // nb] >= kth - SCORE_EPS for g in picked)
+    return n_close
+
+
+SMALL = [
+    Workload("hsa_p200", B=2, H=2, Tq=2, Tkv=9, q_off=7, P=200, d=128, n_sink=1, n_prev=2, chunk_len=2,
+             k_frames=2, k_blocks=3, heads=(SetSpec("hsa"),) * 2),
+    Workload("hsa_p300_d64", B=1, H=3, Tq=3, Tkv=12, q_off=9, P=300, d=64, n_sink=2, n_prev=1, chunk_len=3,
+             k_frames=3, k_blocks=5, heads=(SetSpec("hsa"),) * 3),
+    Workload("hsa_p1", B=1, H=2, Tq=2, Tkv=10, q_off=8, P=1, d=128, n_sink=0, n_prev=1, chunk_len=1,
+             k_frames=4, k_blocks=2, heads=(SetSpec("hsa"),) * 2),
+    Workload("hsa_nohist", B=1, H=1, Tq=2, Tkv=4, q_off=2, P=136, d=128, n_sink=1, n_prev=1, chunk_len=2,
+             k_frames=3, k_blocks=4, heads=(SetSpec("hsa"),)),
+    Workload("hsa_k0", B=1, H=2, Tq=1, Tkv=8, q_off=7, P=260, d=128, n_sink=1, n_prev=1, chunk_len=1,
+             k_frames=0, k_blocks=6, heads=(SetSpec("hsa"),) * 2),
+]
+
+
+@pytest.mark.parametrize("w", SMALL, ids=[w.name for w in SMALL])
+def test_selection_matches_oracle(w):
+    q, k, v = workload_qkv(w, seed=2)
+    blocks, counts = sfa().hsa_select(q.cuda(), k.cuda(), _params(w), w.k_frames, w.k_blocks)
+    torch.cuda.synchronize()
+    n_close = _check_selection(w, q, k, blocks.cpu().numpy(), counts.cpu().numpy())
+    assert n_close == 0, f"{n_close} lists decided by near-ties"
+
+
+@pytest.mark.parametrize("w", SMALL, ids=[w.name for w in SMALL])
+def test_forward_blocks_matches_oracle_full_rows(w):
+    q, k, v = workload_qkv(w, seed=3)
+    Amax = sfa().hsa_max_count(_params(w), w.P, w.k_frames, w.k_blocks)
+    lists, counts = hsa.build_block_lists(q.float().numpy(), k.float().numpy(), Bmax=Amax, **_kw(w))
+    scale = 1 / math.sqrt(w.d)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o, lse = sfa().forward_blocks(q.cuda(), k.cuda(), v.cuda(), torch.from_numpy(lists).cuda(),
+                                  torch.from_numpy(counts).cuda(), w.P, dev_status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    o_ref, l_ref = hsa.attention_blocks(q.float().numpy(), k.float().numpy(), v.float().numpy(), lists, counts,
+                                        w.P, scale)
+    compare(o.float().cpu().reshape(-1, w.d).numpy(), lse.cpu().reshape(-1).numpy(), o_ref.reshape(-1, w.d),
+            l_ref.reshape(-1))
+
+
+def test_whole_frame_block_lists_equal_frame_lists():
+    # lists naming every block of some frames attend to exactly those frames' tokens
+    w = Workload("frames", B=1, H=2, Tq=2, Tkv=6, q_off=0, P=200, d=128, heads=(SetSpec("explicit"),) * 2)
+    q, k, v = (x.cuda() for x in qkv(w.B, w.H, w.Lq, w.Lkv, w.d, seed=6))
+    frame_sets = [[0, 2, 3], [1, 5]]
+    nb = hsa.n_key_blocks(w.P)
+    nq = hsa.n_query_blocks(w.P)
+    frames = torch.full((w.H, w.Tq, 3), -1, dtype=torch.int32)
+    fcounts = torch.zeros((w.H, w.Tq), dtype=torch.int32)
+    blocks = torch.full((w.B, w.H, w.Tq, nq, 3 * nb), -1, dtype=torch.int32)
+    bcounts = torch.zeros((w.B, w.H, w.Tq, nq), dtype=torch.int32)
+    for h in range(w.H):
+        for t in range(w.Tq):
+            fs = frame_sets[(h + t) % 2]
+            frames[h, t, :len(fs)] = torch.tensor(fs)
+            fcounts[h, t] = len(fs)
+            ids = [f * nb + x for f in fs for x in range(nb)]
+            blocks[:, h, t, :, :len(ids)] = torch.tensor(ids, dtype=torch.int32)
+            bcounts[:, h, t, :] = len(ids)
+    o1, l1 = sfa().forward(q, k, v, frames.cuda(), fcounts.cuda(), w.P)
+    o2, l2 = sfa().forward_blocks(q, k, v, blocks.cuda(), bcounts.cuda(), w.P)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_bad_block_list_reported():
+    w = SMALL[0]
+    q, k, v = (x.cuda() for x in workload_qkv(w, seed=1))
+    Amax = sfa().hsa_max_count(_params(w), w.P, w.k_frames, w.k_blocks)
+    blocks, counts = sfa().hsa_select(q, k, _params(w), w.k_frames, w.k_blocks, Amax=Amax)
+    bad = blocks.clone()
+    bad[0, 1, 1, 0, 0] = w.Tkv * hsa.n_key_blocks(w.P)  # one past the last block
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sfa().forward_blocks(q, k, v, bad, counts, w.P, dev_status=status)
+    torch.cuda.synchronize()
+    assert status.item() == sfa().SFA_ERR_BAD_SET
+
+
+def test_hsa_workload_selection_and_sampled_attention():
+    w = WORKLOADS["hsa"]
+    q, k, v = workload_qkv(w, seed=0)
+    blocks, counts = sfa().hsa_select(q.cuda(), k.cuda(), _params(w), w.k_frames, w.k_blocks)
+    torch.cuda.synchronize()
+    n_close = _check_selection(w, q, k, blocks.cpu().numpy(), counts.cpu().numpy())
+    assert n_close <= 2, f"{n_close} lists decided by near-ties"
+    # attention on the oracle's lists, sampled rows (all rows of query frame 0, 256 per head)
+    Amax = blocks.shape[-1]
+    lists, cnts = hsa.build_block_lists(q.float().numpy(), k.float().numpy(), Bmax=Amax, **_kw(w))
+    o, lse = sfa().forward_blocks(q.cuda(), k.cuda(), v.cuda(), torch.from_numpy(lists).cuda(),
+                                  torch.from_numpy(cnts).cuda(), w.P)
+    torch.cuda.synchronize()
+    rows = sample_rows(w, 256, seed=1, frames=(0,))
+    o_ref, l_ref = hsa.attention_blocks(q.float().numpy(), k.float().numpy(), v.float().numpy(), lists, cnts,
+                                        w.P, 1 / math.sqrt(w.d), rows=rows)
+    compare(o.float().cpu().reshape(-1, w.d).numpy()[rows], lse.cpu().reshape(-1).numpy()[rows], o_ref, l_ref)

@@ -199,3 +199,24 @@ def test_planted_mistakes_are_caught():
     g = _golden()
     wrong = hsa.top_k([1, 2, 3, 4], [-x for x in g["frame_scores"][1:5]], 2)
     assert wrong != [2, 4]
+
+
+def test_structured_inputs_give_clear_selections():
+    # the synthetic offsets make the pooled keys distinct: on the small cases the
+    # oracle's k-th and (k+1)-th frame scores are far apart for nearly every query block
+    from sfa_workloads import Workload, SetSpec, qkv_structured
+    w = Workload("hsa_p300_d64", B=1, H=3, Tq=3, Tkv=12, q_off=9, P=300, d=64, n_sink=2, n_prev=1, chunk_len=3,
+                 k_frames=3, k_blocks=5, heads=(SetSpec("hsa"),) * 3)
+    q, k, _ = qkv_structured(w.B, w.H, w.Tq, w.Tkv, w.P, w.d, seed=2)
+    kf, _ = hsa.pool_keys(k.float().numpy(), w.P)
+    qb = hsa.pool_queries(q.float().numpy(), w.P)
+    fw = dict(T_kv=w.Tkv, q_off=w.q_off, chunk_len=w.chunk_len, n_prev=w.n_prev, n_sink=w.n_sink)
+    gaps = []
+    for h in range(w.H):
+        for t in range(w.Tq):
+            hist = hsa.history_frames(t, **fw)
+            for i in range(qb.shape[3]):
+                s = sorted((float(np.dot(qb[0, h, t, i], kf[0, h, f])) for f in hist), reverse=True)
+                if len(s) > w.k_frames:
+                    gaps.append(s[w.k_frames - 1] - s[w.k_frames])
+    assert min(gaps) > 1e-3
