@@ -59,9 +59,9 @@ def measured_peaks():
 
 # DRAM bytes (read + write) of one forward launch on this workload, from one ncu capture
 # of the same kernel on the 4-head version of the workload scaled by 3 to 12 heads (the
-# traffic is per (head, frame, query tile) unit); None until it is re-measured after a
-# change to the forward kernel.
-NCU_TRAFFIC_BYTES = None
+# traffic is per (head, frame, query tile) unit): 3 x (197.487872 + 53.305344) MB.  Set
+# back to None whenever the forward kernel changes, until it is re-measured.
+NCU_TRAFFIC_BYTES = 752_379_648
 
 
 def max_over_ranks(x: float, device) -> float:
@@ -239,6 +239,7 @@ def run_ours(args, rank, world, local_rank):
     d2h = o_p.numel() * o_p.element_size() + lse_p.numel() * lse_p.element_size()
 
     merge = bench_merge(sfa, dev, stream, flush) if rank == 0 else None
+    hsa_rec = bench_hsa(sfa, dev, stream, flush) if rank == 0 else None
 
     if rank != 0:
         return None
@@ -279,6 +280,7 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": 2 * args.steps,
         "clocks": clk,
         "merge": merge,
+        "hsa": hsa_rec,
     }
     if world == 1 and not args.no_cpu_baseline:
         rec["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
@@ -315,6 +317,64 @@ def bench_merge(sfa, dev, stream, flush, reps=20):
     return {"kernel": "lse_merge_kernel<128>", "rows": rows, "bytes": nbytes, "us": round(ms * 1e3, 2),
             "achieved_gbs": round(gbs, 1), "peak_gbs": float(peaks["hbm_gbs"]), "bound": "hbm",
             "frac": round(gbs / float(peaks["hbm_gbs"]), 4)}
+
+
+def block_list_flops(blocks: np.ndarray, counts: np.ndarray, P: int, d: int) -> float:
+    """4*d * sum over query blocks of (query rows) x (tokens of the listed key blocks)."""
+    nb = (P + 127) // 128
+    size = np.array([min(b * 128 + 128, P) - b * 128 for b in range(nb)], dtype=np.int64)
+    rows = np.array([min(256, P - 256 * i) for i in range((P + 255) // 256)], dtype=np.int64)
+    keys = np.zeros(counts.shape, dtype=np.int64)
+    for idx in np.ndindex(counts.shape):
+        ids = blocks[idx][:counts[idx]]
+        keys[idx] = int(size[ids % nb].sum())
+    return 4.0 * d * float((keys * rows).sum())
+
+
+def bench_hsa(sfa, dev, stream, flush, reps=20):
+    """Light Forcing HSA on the hsa workload: selection, then attention over the lists."""
+    w = WORKLOADS["hsa"]
+    q_h, k_h, v_h = workload_qkv(w, seed=0)
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    params = sfa.set_params(T_kv=w.Tkv, Tq=w.Tq, q_off=w.q_off, n_sink=w.n_sink, n_prev=w.n_prev,
+                            chunk_len=w.chunk_len)
+    blocks, counts = sfa.hsa_select(q, k, params, w.k_frames, w.k_blocks, stream=stream)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.Lq), dtype=torch.float32, device=dev)
+    desc = sfa.attn_desc(q, k, k, q, w.P, blocks.shape[-1])
+    import ctypes
+    nbytes = ctypes.c_size_t(0)
+    sfa.load().sfa_hsa_workspace(ctypes.byref(desc), ctypes.byref(nbytes))
+    wsp = torch.empty(max(nbytes.value, 1), dtype=torch.uint8, device=dev)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            ts.append(a.elapsed_time(b))
+        return float(np.median(ts))
+
+    sel_ms = timed(lambda: sfa.hsa_select(q, k, params, w.k_frames, w.k_blocks, workspace=wsp, stream=stream))
+    fwd_ms = timed(lambda: sfa.forward_blocks(q, k, v, blocks, counts, w.P, out=o, lse=lse, stream=stream))
+    flops = block_list_flops(blocks.cpu().numpy(), counts.cpu().numpy(), w.P, w.d)
+    peak = float(measured_peaks()["bf16_tflops"])
+    tf = flops / (fwd_ms * 1e-3) / 1e12
+    pool_bytes = (k.numel() + q.numel()) * 2
+    return {"workload": "hsa: 3 query frames after 21 history frames, P=1560, H=12, d=128; sink 1 + "
+                        "local 6 frames always, 24 blocks of the 4 best history frames per 256-row query block",
+            "select_ms": round(sel_ms, 4), "select_pool_bytes": pool_bytes,
+            "forward_blocks_ms": round(fwd_ms, 4), "attended_tflop": round(flops / 1e12, 4),
+            "forward_tflops": round(tf, 1), "forward_frac": round(tf / peak, 4),
+            "step_tflops": round(flops / ((sel_ms + fwd_ms) * 1e-3) / 1e12, 1),
+            "mean_blocks_per_list": round(float(counts.float().mean().item()), 2)}
 
 
 # ----------------------------------------------------------------------------- oracle timing
@@ -477,7 +537,7 @@ def main():
                     help="run the workload with this many heads instead of 12 (smaller profiling case)")
     ap.add_argument("--skip-extras", action="store_true",
                     help="time the device step only: no end-to-end, merge or CPU-baseline legs")
-    ap.add_argument("--workload", choices=["lvsa41", "long121", "stream", "lsemerge"], default="lvsa41",
+    ap.add_argument("--workload", choices=["lvsa41", "long121", "stream", "lsemerge", "hsa"], default="lvsa41",
                     help="other workloads are timed on the device only (one JSON line, not the bench line)")
     ap.add_argument("--split", type=int, default=1,
                     help="split-KV ranges per unit for --workload other than lvsa41 (sfa_forward_split)")
@@ -491,7 +551,15 @@ def main():
 
     if args.workload != "lvsa41":
         if rank == 0:
-            print(json.dumps(run_other_workload(args)), flush=True)
+            if args.workload == "hsa":
+                import frame_sparse_attention_b200 as sfa
+                sfa.load()
+                dev = torch.device("cuda", 0)
+                flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+                rec = bench_hsa(sfa, dev, torch.cuda.current_stream(dev), flush, reps=args.steps)
+            else:
+                rec = run_other_workload(args)
+            print(json.dumps(rec), flush=True)
         return
 
     if args.impl == "reference":

@@ -8,9 +8,10 @@
 // (sfa_forward_blocks, in sfa_forward.cu).
 //
 // Two kernels:
-//   * hsa_pool_kernel: one CTA per (frame, h, b) of keys or queries; 16-byte loads,
-//     fp32 sums per column, one mean per segment (128-token key block or 256-row query
-//     block) and, for keys, one per frame.  HBM-bound: every K and Q element is read once.
+//   * hsa_pool_kernel: one CTA per segment (128-token key block or 256-row query block)
+//     of keys or queries; 16-byte loads, fp32 sums per column, one mean per segment.
+//     HBM-bound: every K and Q element is read once.  hsa_frame_mean_kernel then forms
+//     each frame's mean as the token-weighted average of its block means.
 //   * hsa_select_kernel: one CTA per (b, h, t, query block): scores of the history
 //     frames, top k_frames, scores of their blocks, top k_blocks, then the sorted union
 //     with the always-attended blocks, compacted with a block-wide prefix count.
@@ -35,53 +36,58 @@ constexpr int MAX_ENTRIES = 65536;  // T_kv * nblk bound (the block flags live i
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
-// Means of the segments of `seg` rows of one frame of x (P rows of D bf16, row stride
-// `row_stride` elements), written to seg_out[nseg][D]; with frame_out, also the mean of
-// the whole frame.  Thread layout: D/8 threads per row (8 columns, one 16-byte load
-// each), POOL_THREADS / (D/8) rows at a time; a shared-memory pass adds the row groups.
+// Mean of one segment of `seg` rows of one frame of x (P rows of D bf16, row stride
+// s_row elements), written to out[((b*H + h)*n_frames + f)*nseg + sg][D]; the last
+// segment of a frame holds the remaining rows.  One CTA per (segment, frame, b*H + h):
+// D/8 threads per row (8 columns, one 16-byte load each), POOL_THREADS / (D/8) rows at a
+// time, then a shared-memory pass adds the row groups.
 template <int D>
 __global__ void __launch_bounds__(POOL_THREADS) hsa_pool_kernel(const uint16_t *x, int64_t s_b, int64_t s_h,
-                                                                  int64_t s_row, int P, int seg, int n_frames,
-                                                                  float *seg_out, float *frame_out)
+                                                                  int64_t s_row, int H, int P, int seg,
+                                                                  int n_frames, float *out)
 {
     constexpr int TPR = D / 8;                 // threads per row
     constexpr int RG = POOL_THREADS / TPR;     // rows in flight
     __shared__ float part[RG][D];
-    __shared__ float frame_acc[D];
-    const int f = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int H = gridDim.y;
+    const int sg = blockIdx.x, f = blockIdx.y, bh = blockIdx.z;
+    const int nseg = gridDim.x;
     const int cg = threadIdx.x % TPR, rg = threadIdx.x / TPR;
-    const uint16_t *base = x + b * s_b + h * s_h + (int64_t)f * P * s_row + cg * 8;
-    const int nseg = (P + seg - 1) / seg;
-    float *out = seg_out + (((int64_t)b * H + h) * n_frames + f) * nseg * D;
-    if (threadIdx.x < D) frame_acc[threadIdx.x] = 0.f;
-    for (int sg = 0; sg < nseg; ++sg) {
-        const int r0 = sg * seg, r1 = min(r0 + seg, P);
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int r = r0 + rg; r < r1; r += RG) {
-            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(base + (int64_t)r * s_row));
-            acc[0] += bf16_lo(v.x);
-            acc[1] += bf16_hi(v.x);
-            acc[2] += bf16_lo(v.y);
-            acc[3] += bf16_hi(v.y);
-            acc[4] += bf16_lo(v.z);
-            acc[5] += bf16_hi(v.z);
-            acc[6] += bf16_lo(v.w);
-            acc[7] += bf16_hi(v.w);
-        }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) part[rg][cg * 8 + i] = acc[i];
-        __syncthreads();
-        if (threadIdx.x < D) {
-            float s = 0.f;
-            for (int g = 0; g < RG; ++g) s += part[g][threadIdx.x];
-            out[(int64_t)sg * D + threadIdx.x] = s / (float)(r1 - r0);
-            frame_acc[threadIdx.x] += s;
-        }
-        __syncthreads();
+    const int r0 = sg * seg, r1 = min(r0 + seg, P);
+    const uint16_t *base = x + (int64_t)(bh / H) * s_b + (int64_t)(bh % H) * s_h + (int64_t)f * P * s_row + cg * 8;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int r = r0 + rg; r < r1; r += RG) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(base + (int64_t)r * s_row));
+        acc[0] += bf16_lo(v.x);
+        acc[1] += bf16_hi(v.x);
+        acc[2] += bf16_lo(v.y);
+        acc[3] += bf16_hi(v.y);
+        acc[4] += bf16_lo(v.z);
+        acc[5] += bf16_hi(v.z);
+        acc[6] += bf16_lo(v.w);
+        acc[7] += bf16_hi(v.w);
     }
-    if (frame_out && threadIdx.x < D)
-        frame_out[(((int64_t)b * H + h) * n_frames + f) * D + threadIdx.x] = frame_acc[threadIdx.x] / (float)P;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) part[rg][cg * 8 + i] = acc[i];
+    __syncthreads();
+    if (threadIdx.x < D) {
+        float sum = 0.f;
+        for (int g = 0; g < RG; ++g) sum += part[g][threadIdx.x];
+        out[(((int64_t)bh * n_frames + f) * nseg + sg) * D + threadIdx.x] = sum / (float)(r1 - r0);
+    }
+}
+
+// Frame means from the block means: the token-weighted average of a frame's blocks.
+// One thread per (b*H + h, frame, column).
+template <int D>
+__global__ void hsa_frame_mean_kernel(const float *kb, int64_t n, int P, int nblk, float *kf)
+{
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n) return;
+    const int64_t fr = i / D, c = i % D;
+    const float *src = kb + fr * nblk * D + c;
+    float s = 0.f;
+    for (int b = 0; b < nblk; ++b) s += src[(int64_t)b * D] * (float)(min(b * KEY_BLOCK + KEY_BLOCK, P) - b * KEY_BLOCK);
+    kf[i] = s / (float)P;
 }
 
 struct SelectArgs {
@@ -298,7 +304,7 @@ bool desc_ok(const sfa_attn_desc *d)
 {
     if (!d || d->B < 0 || d->H < 1 || d->Tq < 1 || d->T_kv < 1 || d->P < 1 || d->Amax < 1) return false;
     if ((int64_t)d->Tq * d->P >= ((int64_t)1 << 31) || (int64_t)d->T_kv * d->P >= ((int64_t)1 << 31)) return false;
-    if (d->H > 65535 || d->B > 65535) return false;  // grid y / z of the pooling launch
+    if ((int64_t)d->B * d->H > 65535 || d->T_kv > 65535) return false;  // grid z / y of the pooling launch
     return true;
 }
 
@@ -314,12 +320,16 @@ sfa_status run_select(const sfa_attn_desc *d, const sfa_set_params *p, int k_fra
     const WsLayout w = ws_layout(d);
     float *kf = reinterpret_cast<float *>(ws + w.kf), *kb = reinterpret_cast<float *>(ws + w.kb);
     float *qb = reinterpret_cast<float *>(ws + w.qb);
-    hsa_pool_kernel<D><<<dim3(d->T_kv, d->H, d->B), POOL_THREADS, 0, s>>>(
-        static_cast<const uint16_t *>(k), d->k_stride[0], d->k_stride[1], d->k_stride[2], d->P, KEY_BLOCK, d->T_kv, kb,
-        kf);
-    hsa_pool_kernel<D><<<dim3(d->Tq, d->H, d->B), POOL_THREADS, 0, s>>>(
-        static_cast<const uint16_t *>(q), d->q_stride[0], d->q_stride[1], d->q_stride[2], d->P, QUERY_BLOCK, d->Tq,
-        qb, nullptr);
+    const int nblk = (d->P + KEY_BLOCK - 1) / KEY_BLOCK, nqb = (d->P + QUERY_BLOCK - 1) / QUERY_BLOCK;
+    const unsigned bh = (unsigned)d->B * d->H;
+    hsa_pool_kernel<D><<<dim3(nblk, d->T_kv, bh), POOL_THREADS, 0, s>>>(
+        static_cast<const uint16_t *>(k), d->k_stride[0], d->k_stride[1], d->k_stride[2], d->H, d->P, KEY_BLOCK,
+        d->T_kv, kb);
+    hsa_pool_kernel<D><<<dim3(nqb, d->Tq, bh), POOL_THREADS, 0, s>>>(
+        static_cast<const uint16_t *>(q), d->q_stride[0], d->q_stride[1], d->q_stride[2], d->H, d->P, QUERY_BLOCK,
+        d->Tq, qb);
+    const int64_t n_kf = (int64_t)bh * d->T_kv * D;
+    hsa_frame_mean_kernel<D><<<(unsigned)((n_kf + 255) / 256), 256, 0, s>>>(kb, n_kf, d->P, nblk, kf);
     SelectArgs a;
     a.B = d->B;
     a.H = d->H;
