@@ -493,7 +493,28 @@ def run_other_workload(args):
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    dual = getattr(args, "dual", False) and len(branches) == 2
+    if dual:  # both branches in one launch, local result + their merge (sfa_forward_dual)
+        Amax = max(b[4] for b in branches)
+        for i, b in enumerate(branches):
+            w_, p_, k_, e_ = b[0], b[1], b[2], b[3]
+            fr = torch.empty((w_.H, w_.Tq, Amax), dtype=torch.int32, device=dev)
+            branches[i] = (w_, p_, k_, e_, Amax, fr, torch.empty_like(b[6])) + b[7:]
+        import ctypes
+        nbytes = ctypes.c_size_t(0)
+        ddesc = sfa.attn_desc(q, k, v, merged[0], branches[0][0].P, Amax)
+        if sfa.load().sfa_forward_dual_workspace(ctypes.byref(ddesc), args.split, ctypes.byref(nbytes)) != 0:
+            raise SystemExit("--dual: bad --split for this head dimension")
+        dual_ws = torch.empty(max(1, nbytes.value), dtype=torch.uint8, device=dev)
+
     def step():
+        if dual:
+            (w0, p0, k0, e0, A0, f0, c0, o0, l0, _), (w1, p1, k1, e1, A1, f1, c1, o1, l1, _) = branches
+            sfa.build_sets(p0, k0, e0, A0, f0, c0, stream=stream)
+            sfa.build_sets(p1, k1, e1, A1, f1, c1, stream=stream)
+            sfa.forward_dual(q, k, v, f0, c0, f1, c1, w0.P, args.split, out_local=o0, lse_local=l0,
+                             out_full=merged[0], lse_full=merged[1], workspace=dual_ws, stream=stream)
+            return
         for (w, params, kinds, extra, Amax, fr, cn, o, lse, wsp) in branches:
             sfa.build_sets(params, kinds, extra, Amax, fr, cn, stream=stream)
             if args.split > 1:
@@ -520,7 +541,8 @@ def run_other_workload(args):
         torch.cuda.synchronize(dev)
         times.append(e0.elapsed_time(e1))
     ms = float(np.median(times))
-    return {"workload": args.workload, "branches": names, "split": args.split, "attended_tflop_per_step": round(flops / 1e12, 4),
+    return {"workload": args.workload, "branches": names, "split": args.split, "dual_launch": dual,
+            "attended_tflop_per_step": round(flops / 1e12, 4),
             "ms_per_step": round(ms, 4), "tflops": round(flops / (ms * 1e-3) / 1e12, 1),
             "steps": args.steps, "warmup": args.warmup, "note": "device time, median, L2 flushed between steps"}
 
@@ -539,6 +561,8 @@ def main():
                     help="time the device step only: no end-to-end, merge or CPU-baseline legs")
     ap.add_argument("--workload", choices=["lvsa41", "long121", "stream", "lsemerge", "hsa"], default="lvsa41",
                     help="other workloads are timed on the device only (one JSON line, not the bench line)")
+    ap.add_argument("--dual", action="store_true",
+                    help="--workload lsemerge: both branches in one launch (sfa_forward_dual)")
     ap.add_argument("--split", type=int, default=1,
                     help="split-KV ranges per unit for --workload other than lvsa41 (sfa_forward_split)")
     args = ap.parse_args()

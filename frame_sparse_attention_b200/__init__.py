@@ -8,6 +8,8 @@ Python face of libsfa.so (C ABI in include/sfa.h):
 * ``forward_split`` - the same with each unit's key tiles split over several CTAs and the
                     partials merged by LSE (short or uneven grids)
 * ``forward_paged`` - the same with K/V read through a per-head frame -> slot table
+* ``forward_dual`` - local and history branches in one launch: the local result and their
+                    LSE merge (the full attention)
 * ``lse_merge``   - merge of two partial attentions (local + history branch) by LSE
 * ``hsa_select``  - hierarchical selection (Light Forcing HSA): pooled keys, top history
                     frames, then top 128-token key blocks, per 256-row query block
@@ -17,12 +19,13 @@ Tensors are PyTorch CUDA tensors; calls run on the current CUDA stream.
 """
 from ._lib import (SET_KINDS, SFA_DEBUG_STALL_SOFTMAX, SFA_ERR_BAD_SET, SFA_ERR_CUDA,
                    SFA_ERR_INVALID_ARG, SFA_ERR_TIMEOUT, SFA_ERR_UNSUPPORTED, SFA_OK, AttnDesc,
-                   SetParams, SfaError, attn_desc, build_sets, error_string, forward, forward_blocks,
+                   SetParams, SfaError, attn_desc, build_sets, error_string, forward, forward_blocks, forward_dual,
                    forward_paged, forward_split, hsa_max_count, hsa_select, load, lse_merge, set_max_count,
                    set_params, split_workspace_bytes, version)
 
 __all__ = ["SET_KINDS", "SFA_DEBUG_STALL_SOFTMAX", "SFA_ERR_BAD_SET", "SFA_ERR_CUDA",
            "SFA_ERR_INVALID_ARG", "SFA_ERR_TIMEOUT", "SFA_ERR_UNSUPPORTED", "SFA_OK", "AttnDesc",
            "SetParams", "SfaError", "attn_desc", "build_sets", "error_string", "forward", "forward_blocks",
+           "forward_dual",
            "forward_paged", "forward_split", "hsa_max_count", "hsa_select",
            "load", "lse_merge", "set_max_count", "set_params", "split_workspace_bytes", "version"]

@@ -52,7 +52,8 @@ class AttnDesc(ctypes.Structure):
 _lib = None
 EXPORTS = ("sfa_error_string", "sfa_version", "sfa_set_max_count", "sfa_build_sets", "sfa_forward",
            "sfa_forward_split_workspace", "sfa_forward_split", "sfa_forward_split_noalloc", "sfa_forward_paged",
-           "sfa_lse_merge", "sfa_hsa_max_count", "sfa_hsa_workspace", "sfa_hsa_select", "sfa_forward_blocks")
+           "sfa_lse_merge", "sfa_hsa_max_count", "sfa_hsa_workspace", "sfa_hsa_select", "sfa_forward_blocks",
+           "sfa_forward_dual_workspace", "sfa_forward_dual")
 
 
 def load():
@@ -95,6 +96,11 @@ def load():
     lib.sfa_hsa_select.restype = st
     lib.sfa_hsa_select.argtypes = [ctypes.POINTER(AttnDesc), ctypes.POINTER(SetParams), i32, i32, vp, vp, vp,
                                    ctypes.c_size_t, vp, vp, vp]
+    lib.sfa_forward_dual_workspace.restype = st
+    lib.sfa_forward_dual_workspace.argtypes = [ctypes.POINTER(AttnDesc), i32, ctypes.POINTER(ctypes.c_size_t)]
+    lib.sfa_forward_dual.restype = st
+    lib.sfa_forward_dual.argtypes = [ctypes.POINTER(AttnDesc), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp,
+                                     ctypes.c_size_t, vp, vp]
     lib.sfa_forward_blocks.restype = st
     lib.sfa_forward_blocks.argtypes = [ctypes.POINTER(AttnDesc), vp, vp, vp, vp, vp, vp, vp, vp, vp]
     _lib = lib
@@ -329,3 +335,33 @@ def forward_blocks(q, k, v, blocks, counts, P: int, scale: float | None = None, 
                                      blocks.data_ptr(), counts.data_ptr(), out.data_ptr(), lse.data_ptr(),
                                      _ptr(dev_status), _stream(stream)), "sfa_forward_blocks")
     return out, lse
+
+
+def forward_dual(q, k, v, frames_local, counts_local, frames_hist, counts_hist, P: int, n_split: int = 1,
+                 scale: float | None = None, out_local=None, lse_local=None, out_full=None, lse_full=None,
+                 workspace=None, dev_status=None, stream=None, timeout_us: int = 0):
+    """Local and history branches in one launch: (O_local, LSE_local, O_full, LSE_full), the
+    full result being the LSE merge of both branches."""
+    B, H, Lq, d = q.shape
+    out_local = torch.empty_like(q) if out_local is None else out_local
+    out_full = torch.empty_like(q) if out_full is None else out_full
+    if lse_local is None:
+        lse_local = torch.empty((B, H, Lq), dtype=torch.float32, device=q.device)
+    if lse_full is None:
+        lse_full = torch.empty((B, H, Lq), dtype=torch.float32, device=q.device)
+    for f, c in ((frames_local, counts_local), (frames_hist, counts_hist)):
+        assert f.dtype == torch.int32 and c.dtype == torch.int32 and f.is_contiguous() and c.is_contiguous()
+    assert frames_local.shape == frames_hist.shape
+    assert tuple(out_local.stride()) == tuple(out_full.stride())
+    desc = attn_desc(q, k, v, out_full, P, frames_local.shape[2], scale, timeout_us)
+    nbytes = ctypes.c_size_t(0)
+    _check(load().sfa_forward_dual_workspace(ctypes.byref(desc), n_split, ctypes.byref(nbytes)),
+           "sfa_forward_dual_workspace")
+    if workspace is None:
+        workspace = torch.empty(max(nbytes.value, 1), dtype=torch.uint8, device=q.device)
+    _check(load().sfa_forward_dual(ctypes.byref(desc), q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                   frames_local.data_ptr(), counts_local.data_ptr(), frames_hist.data_ptr(),
+                                   counts_hist.data_ptr(), out_local.data_ptr(), lse_local.data_ptr(),
+                                   out_full.data_ptr(), lse_full.data_ptr(), n_split, workspace.data_ptr(),
+                                   workspace.numel(), _ptr(dev_status), _stream(stream)), "sfa_forward_dual")
+    return out_local, lse_local, out_full, lse_full

@@ -108,6 +108,9 @@ struct FwdArgs {
     int32_t n_slots;       // frames held by the K/V buffers (T_kv without a slot table)
     int32_t nblk;          // > 0: the lists hold key blocks of KEY_BLOCK tokens (nblk per frame),
                            // one list per (b, h, t, query block of 2 tiles); 0: frame lists per (h, t)
+    const int32_t *frames2;  // second list set (two-branch launch: grid y = 2 x splits), or null
+    const int32_t *counts2;
+    int32_t n_lists;         // 1, or 2 with frames2 / counts2
     float *lse;
     int32_t *status;
     uint64_t timeout_ns;
@@ -727,10 +730,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     x /= a.Tq;
     const int h = x % a.H;
     const int b = x / a.H;
+    // grid y = list set x split: CTA (unit, y) takes list set y / n_split and key-tile range
+    // y mod n_split of it, and with more than one y writes slice y of the partial outputs
+    const int n_split = gridDim.y / a.n_lists;
+    const int li = blockIdx.y / n_split, split = blockIdx.y - li * n_split;
     // the unit's list: frames of (h, t), or key blocks of (b, h, t, query block = pair)
     const int64_t list = a.nblk ? ((((int64_t)b * a.H + h) * a.Tq + t) * n_pairs + qt_a / 2) : (int64_t)h * a.Tq + t;
-    const int32_t *fl = a.frames + list * a.Amax;
-    const int cnt = __ldg(a.counts + list);
+    const int32_t *fl = (li ? a.frames2 : a.frames) + list * a.Amax;
+    const int cnt = __ldg((li ? a.counts2 : a.counts) + list);
     int n_all = (cnt >= 0 && cnt <= a.Amax)
                     ? count_tiles(fl, cnt, a.nblk ? a.T_kv * a.nblk : a.T_kv, a.P, a.nblk,
                                   a.slots ? a.slots + (int64_t)h * a.T_kv : nullptr, a.n_slots)
@@ -738,11 +745,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const bool bad_set = n_all < 0;
     if (bad_set) n_all = 0;
     // split-KV: CTA (unit, split) takes the unit's key tiles [t_off, t_off + n_tiles) and
-    // writes a partial result into slice `split` of the output (batch index b_out)
-    const int split = blockIdx.y, n_split = gridDim.y;
+    // writes a partial result into slice blockIdx.y of the output (batch index b_out)
     const int t_off = (int)(((int64_t)n_all * split) / n_split);
     int n_tiles = (int)(((int64_t)n_all * (split + 1)) / n_split) - t_off;
-    const int b_out = split * a.B + b;
+    const int b_out = blockIdx.y * a.B + b;
     volatile int32_t *skip = reinterpret_cast<volatile int32_t *>(smem + C::SMEM_BAR + 248);
 
     if (threadIdx.x == 0) {
@@ -847,9 +853,12 @@ template <int D>
 sfa_status launch(const sfa_attn_desc *d, const void *q, const void *k, const void *v, const int32_t *frames,
                   const int32_t *counts, void *o, float *lse, int32_t *dev_status, cudaStream_t stream,
                   int n_split = 1, void *ws_o = nullptr, float *ws_lse = nullptr, const int32_t *slots = nullptr,
-                  int n_slots = 0, int nblk = 0)
+                  int n_slots = 0, int nblk = 0, const int32_t *frames2 = nullptr, const int32_t *counts2 = nullptr,
+                  void *o_first = nullptr, float *lse_first = nullptr)
 {
     using C = Cfg<D>;
+    const int n_lists = frames2 ? 2 : 1;
+    const int slices = n_lists * n_split;  // partial outputs (1: straight to o / lse)
     CUtensorMap tq, tk, tv, to;
     const int kv_frames = slots ? n_slots : d->T_kv;  // frames held by the K/V buffers
     const uint64_t P = d->P, Tq = d->Tq, Lkv = (uint64_t)kv_frames * d->P;
@@ -858,13 +867,13 @@ sfa_status launch(const sfa_attn_desc *d, const void *q, const void *k, const vo
         const uint64_t st[4] = {(uint64_t)d->q_stride[2] * 2, P * d->q_stride[2] * 2, (uint64_t)d->q_stride[1] * 2,
                                 (uint64_t)d->q_stride[0] * 2};
         if (!encode(&tq, q, 5, dims, st)) return SFA_ERR_UNSUPPORTED;
-        if (n_split == 1) {
+        if (slices == 1) {
             const uint64_t so[4] = {(uint64_t)d->o_stride[2] * 2, P * d->o_stride[2] * 2,
                                     (uint64_t)d->o_stride[1] * 2, (uint64_t)d->o_stride[0] * 2};
             if (!encode(&to, o, 5, dims, so)) return SFA_ERR_UNSUPPORTED;
         } else {
             const uint64_t Lq = Tq * P;
-            const uint64_t dims_w[5] = {(uint64_t)D, P, Tq, (uint64_t)d->H, (uint64_t)d->B * n_split};
+            const uint64_t dims_w[5] = {(uint64_t)D, P, Tq, (uint64_t)d->H, (uint64_t)d->B * slices};
             const uint64_t sw[4] = {(uint64_t)D * 2, P * D * 2, Lq * D * 2, (uint64_t)d->H * Lq * D * 2};
             if (!encode(&to, ws_o, 5, dims_w, sw)) return SFA_ERR_UNSUPPORTED;
         }
@@ -892,7 +901,10 @@ sfa_status launch(const sfa_attn_desc *d, const void *q, const void *k, const vo
     a.slots = slots;
     a.n_slots = kv_frames;
     a.nblk = nblk;
-    a.lse = n_split == 1 ? lse : ws_lse;
+    a.lse = slices == 1 ? lse : ws_lse;
+    a.frames2 = frames2;
+    a.counts2 = counts2;
+    a.n_lists = n_lists;
     a.status = dev_status;
     a.timeout_ns = (uint64_t)(d->timeout_us ? d->timeout_us : DEFAULT_TIMEOUT_US) * 1000;
     a.debug_flags = d->debug_flags;
@@ -901,13 +913,13 @@ sfa_status launch(const sfa_attn_desc *d, const void *q, const void *k, const vo
     if (cudaFuncSetAttribute(sfa_forward_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
         cudaSuccess)
         return SFA_ERR_CUDA;
-    sfa_forward_kernel<D><<<dim3((unsigned)grid, (unsigned)n_split), NUM_THREADS, C::SMEM_BYTES, stream>>>(
+    sfa_forward_kernel<D><<<dim3((unsigned)grid, (unsigned)slices), NUM_THREADS, C::SMEM_BYTES, stream>>>(
         tq, tk, tv, to, a);
     sfa_status st = launch_status();
-    if (st != SFA_OK || n_split == 1) return st;
+    if (st != SFA_OK || slices == 1) return st;
     const int64_t Lq = (int64_t)d->Tq * d->P;
-    return launch_lse_combine((int64_t)d->B * d->H * Lq, n_split, D, d->H, Lq, ws_o, ws_lse, o, d->o_stride, lse,
-                              stream);
+    return launch_lse_combine((int64_t)d->B * d->H * Lq, slices, D, d->H, Lq, ws_o, ws_lse, o, d->o_stride, lse,
+                              stream, n_lists == 2 ? n_split : 0, o_first, lse_first);
 }
 
 size_t split_ws_o_bytes(const sfa_attn_desc *d, int n_split)
@@ -1060,6 +1072,46 @@ extern "C" sfa_status sfa_forward_split_noalloc(const sfa_attn_desc *d, const vo
     float *ws_lse = reinterpret_cast<float *>(static_cast<char *>(scratch) + split_ws_o_bytes(d, n_split));
     return d->d == 128 ? launch<128>(d, q, k, v, frames, counts, o, lse, dev_status, s, n_split, scratch, ws_lse)
                        : launch<64>(d, q, k, v, frames, counts, o, lse, dev_status, s, n_split, scratch, ws_lse);
+}
+
+// ------------------------------------------------------------------------------------
+// Two branches in one launch ("ISPA", §2.1 Dual-Stream Warmup): the local and the history
+// key sets of the same queries run as one grid; the partials give the local branch and,
+// merged by LSE, the full attention.
+// ------------------------------------------------------------------------------------
+extern "C" sfa_status sfa_forward_dual_workspace(const sfa_attn_desc *d, int32_t n_split, size_t *bytes)
+{
+    sfa_status st = check_desc(d);
+    if (st != SFA_OK) return st;
+    if (!bytes || n_split < 1 || 2 * n_split > d->d / 8) return SFA_ERR_INVALID_ARG;
+    *bytes = split_ws_bytes(d, 2 * n_split);
+    return SFA_OK;
+}
+
+extern "C" sfa_status sfa_forward_dual(const sfa_attn_desc *d, const void *q, const void *k, const void *v,
+                                       const int32_t *frames_local, const int32_t *counts_local,
+                                       const int32_t *frames_hist, const int32_t *counts_hist, void *o_local,
+                                       float *lse_local, void *o_full, float *lse_full, int32_t n_split,
+                                       void *workspace, size_t workspace_bytes, int32_t *dev_status,
+                                       sfa_stream_t stream)
+{
+    sfa_status st = check_desc(d);
+    if (st != SFA_OK) return st;
+    if (n_split < 1 || 2 * n_split > d->d / 8) return SFA_ERR_INVALID_ARG;
+    if (d->B == 0) return SFA_OK;
+    st = check_buffers(d, q, k, v, frames_local, counts_local, o_full, lse_full);
+    if (st != SFA_OK) return st;
+    if (!frames_hist || !counts_hist || !o_local || !lse_local || reinterpret_cast<uintptr_t>(o_local) % 16)
+        return SFA_ERR_INVALID_ARG;
+    const size_t need = split_ws_bytes(d, 2 * n_split);
+    if (!workspace || workspace_bytes < need || reinterpret_cast<uintptr_t>(workspace) % 256)
+        return SFA_ERR_INVALID_ARG;
+    cudaStream_t s = as_cuda(stream);
+    float *ws_lse = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + split_ws_o_bytes(d, 2 * n_split));
+    return d->d == 128 ? launch<128>(d, q, k, v, frames_local, counts_local, o_full, lse_full, dev_status, s, n_split,
+                                     workspace, ws_lse, nullptr, 0, 0, frames_hist, counts_hist, o_local, lse_local)
+                       : launch<64>(d, q, k, v, frames_local, counts_local, o_full, lse_full, dev_status, s, n_split,
+                                    workspace, ws_lse, nullptr, 0, 0, frames_hist, counts_hist, o_local, lse_local);
 }
 
 // ------------------------------------------------------------------------------------

@@ -13,8 +13,10 @@
 //     HBM-bound: every K and Q element is read once.  hsa_frame_mean_kernel then forms
 //     each frame's mean as the token-weighted average of its block means.
 //   * hsa_select_kernel: one CTA per (b, h, t, query block): scores of the history
-//     frames, top k_frames, scores of their blocks, top k_blocks, then the sorted union
-//     with the always-attended blocks, compacted with a block-wide prefix count.
+//     frames, top k_frames, scores of their blocks, top k_blocks (a candidate is kept
+//     when fewer than k candidates rank before it: one pass, no serial rounds), then the
+//     sorted union with the always-attended blocks, compacted with a block-wide prefix
+//     count.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -106,32 +108,13 @@ __device__ __forceinline__ bool ranks_before(float sa, int ia, float sb, int ib)
     return sa > sb || (sa == sb && ia < ib);
 }
 
-// One warp: the index (into ids/scores[0, n)) of the best entry not yet taken, or -1.
-__device__ int warp_best(const float *scores, const int *ids, const uint8_t *taken, int n)
+// Number of the n candidates that rank before candidate (s, id): its position in the
+// selection order (top-k keeps the candidates whose position is below k).
+__device__ __forceinline__ int rank_of(const float *scores, const int *ids, int n, float s, int id)
 {
-    const int lane = threadIdx.x & 31;
-    float bs = -INFINITY;
-    int bi = -1, bid = 0x7fffffff;
-    for (int i = lane; i < n; i += 32) {
-        if (taken[i]) continue;
-        if (bi < 0 || ranks_before(scores[i], ids[i], bs, bid)) {
-            bs = scores[i];
-            bi = i;
-            bid = ids[i];
-        }
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        const float os = __shfl_xor_sync(0xffffffffu, bs, off);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-        const int oid = __shfl_xor_sync(0xffffffffu, bid, off);
-        if (oi >= 0 && (bi < 0 || ranks_before(os, oid, bs, bid))) {
-            bs = os;
-            bi = oi;
-            bid = oid;
-        }
-    }
-    return bi;
+    int r = 0;
+    for (int j = 0; j < n; ++j) r += ranks_before(scores[j], ids[j], s, id) ? 1 : 0;
+    return r;
 }
 
 // dot(q, key) of D floats by one warp
@@ -147,8 +130,8 @@ __device__ __forceinline__ float warp_dot(const float *q, const float *key)
     return s;
 }
 
-// Dynamic shared memory: frame scores/ids/taken [T_kv], block scores/ids/taken
-// [k_frames' * nblk], entry flags [T_kv * nblk], warp totals.
+// Dynamic shared memory: frame scores/ids [T_kv], block scores/ids [k_frames' * nblk],
+// selected frames, frame flags [T_kv], entry flags [T_kv * nblk].
 template <int D>
 __global__ void __launch_bounds__(SELECT_THREADS) hsa_select_kernel(const __grid_constant__ SelectArgs a)
 {
@@ -173,8 +156,7 @@ __global__ void __launch_bounds__(SELECT_THREADS) hsa_select_kernel(const __grid
     int *b_id = reinterpret_cast<int *>(b_score + n_bc_max);
     int *sel = b_id + n_bc_max;                                         // [n_sel_max]
     uint8_t *f_taken = reinterpret_cast<uint8_t *>(sel + n_sel_max);   // [T_kv]
-    uint8_t *b_taken = f_taken + a.T_kv;                                // [n_bc_max]
-    uint8_t *flag = b_taken + n_bc_max;                                 // [n_entries]
+    uint8_t *flag = f_taken + a.T_kv;                                   // [n_entries]
 
     const int c = t + a.q_off;
     const int c0 = c - c % a.chunk_len;
@@ -197,22 +179,18 @@ __global__ void __launch_bounds__(SELECT_THREADS) hsa_select_kernel(const __grid
         const float s = warp_dot<D>(qv, a.kf + (bh * a.T_kv + f_id[i]) * D);
         if (lane == 0) {
             f_score[i] = s;
-            f_taken[i] = 0;
         }
     }
     __syncthreads();
-    // top k_frames (warp 0)
-    if (warp == 0) {
-        const int n_sel = min(a.k_frames, n_hist);
-        for (int k = 0; k < n_sel; ++k) {
-            const int bi = warp_best(f_score, f_id, f_taken, n_hist);
-            if (lane == 0) {
-                f_taken[bi] = 1;
-                sel[k] = f_id[bi];
-            }
-            __syncwarp();
-        }
-        if (lane == 0) n_sel_s = n_sel;
+    // top k_frames: a candidate is kept when fewer than k_frames others rank before it
+    for (int i = threadIdx.x; i < n_hist; i += SELECT_THREADS)
+        f_taken[i] = rank_of(f_score, f_id, n_hist, f_score[i], f_id[i]) < a.k_frames ? 1 : 0;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int n = 0;
+        for (int i = 0; i < n_hist; ++i)
+            if (f_taken[i]) sel[n++] = f_id[i];
+        n_sel_s = n;
     }
     __syncthreads();
     const int n_sel = n_sel_s;
@@ -224,21 +202,12 @@ __global__ void __launch_bounds__(SELECT_THREADS) hsa_select_kernel(const __grid
         if (lane == 0) {
             b_score[i] = s;
             b_id[i] = f * a.nblk + bb;
-            b_taken[i] = 0;
         }
     }
     __syncthreads();
-    if (warp == 0) {
-        const int n_pick = min(a.k_blocks, n_bc);
-        for (int k = 0; k < n_pick; ++k) {
-            const int bi = warp_best(b_score, b_id, b_taken, n_bc);
-            if (lane == 0) {
-                b_taken[bi] = 1;
-                flag[b_id[bi]] = 1;
-            }
-            __syncwarp();
-        }
-    }
+    // top k_blocks of the selected frames' blocks
+    for (int i = threadIdx.x; i < n_bc; i += SELECT_THREADS)
+        if (rank_of(b_score, b_id, n_bc, b_score[i], b_id[i]) < a.k_blocks) flag[b_id[i]] = 1;
     // always-attended frames: every block
     for (int i = threadIdx.x; i < n_entries; i += SELECT_THREADS) {
         const int f = i / a.nblk;
@@ -352,7 +321,7 @@ sfa_status run_select(const sfa_attn_desc *d, const sfa_set_params *p, int k_fra
     a.counts = counts;
     const int n_sel_max = std::min(k_frames, d->T_kv);
     const size_t n_bc_max = (size_t)n_sel_max * a.nblk;
-    const size_t smem = (size_t)d->T_kv * 8 + n_bc_max * 8 + (size_t)n_sel_max * 4 + d->T_kv + n_bc_max +
+    const size_t smem = (size_t)d->T_kv * 8 + n_bc_max * 8 + (size_t)n_sel_max * 4 + d->T_kv +
                         (size_t)d->T_kv * a.nblk;
     if (smem > 200 * 1024) return SFA_ERR_UNSUPPORTED;
     if (cudaFuncSetAttribute(hsa_select_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=

@@ -77,11 +77,15 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(int64_t rows, const uint
 // order) -> O at o + b*os0 + h*os1 + i*os2 and LSE [rows].  D/8 threads per row, the
 // lane s of a row's group holds branch s's weight (S <= D/8).
 template <int D>
-__global__ void __launch_bounds__(256) lse_combine_kernel(int64_t rows, int S, int H, int64_t Lq,
+__global__ void __launch_bounds__(256) lse_combine_kernel(int64_t rows, int S, int S1, int H, int64_t Lq,
                                                           const uint4 *__restrict__ o_part,
                                                           const float *__restrict__ lse_part, uint16_t *o,
-                                                          int64_t os0, int64_t os1, int64_t os2, float *lse)
+                                                          int64_t os0, int64_t os1, int64_t os2, float *lse,
+                                                          uint16_t *o1, float *lse1)
 {
+    // Merges slices [0, S) of the partials into (o, lse) and, when o1 is set, slices
+    // [0, S1) into (o1, lse1) (same strides): one group of D/8 threads per row, lane `sub`
+    // of the group holds slice `sub`'s LSE.
     constexpr int G = D / 8;
     const int64_t gtid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int sub = threadIdx.x % G;
@@ -89,43 +93,70 @@ __global__ void __launch_bounds__(256) lse_combine_kernel(int64_t rows, int S, i
     const int64_t row_stride = (int64_t)gridDim.x * blockDim.x / G;
     for (int64_t r = gtid / G; r < rows; r += row_stride) {
         const float ls = sub < S ? lse_part[(int64_t)sub * rows + r] : -INFINITY;
-        float m = ls;
+        const float ls1 = sub < S1 ? ls : -INFINITY;
+        float m = ls, m1 = ls1;
 #pragma unroll
-        for (int off = G / 2; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(group, m, off, G));
+        for (int off = G / 2; off > 0; off >>= 1) {
+            m = fmaxf(m, __shfl_xor_sync(group, m, off, G));
+            m1 = fmaxf(m1, __shfl_xor_sync(group, m1, off, G));
+        }
         const float w = (ls == -INFINITY) ? 0.f : expf(ls - m);
-        float tot = w;
+        const float w1 = (ls1 == -INFINITY) ? 0.f : expf(ls1 - m1);
+        float tot = w, tot1 = w1;
 #pragma unroll
-        for (int off = G / 2; off > 0; off >>= 1) tot += __shfl_xor_sync(group, tot, off, G);
+        for (int off = G / 2; off > 0; off >>= 1) {
+            tot += __shfl_xor_sync(group, tot, off, G);
+            tot1 += __shfl_xor_sync(group, tot1, off, G);
+        }
         float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        float acc1[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         for (int sidx = 0; sidx < S; ++sidx) {
             const float ws = __shfl_sync(group, w, sidx, G);
-            if (ws != 0.f) {
+            const float ws1 = __shfl_sync(group, w1, sidx, G);
+            if (ws != 0.f || ws1 != 0.f) {
                 const uint4 v = o_part[((int64_t)sidx * rows + r) * G + sub];
                 const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     acc[2 * i] += ws * bf16_lo(vv[i]);
                     acc[2 * i + 1] += ws * bf16_hi(vv[i]);
+                    acc1[2 * i] += ws1 * bf16_lo(vv[i]);
+                    acc1[2 * i + 1] += ws1 * bf16_hi(vv[i]);
                 }
             }
         }
-        const bool empty = (m == -INFINITY);
-        const float inv = empty ? 0.f : 1.f / tot;
         const int64_t b = r / ((int64_t)H * Lq), h = (r / Lq) % H, i = r % Lq;
-        uint4 out;
-        out.x = to_bf16x2(acc[0] * inv, acc[1] * inv);
-        out.y = to_bf16x2(acc[2] * inv, acc[3] * inv);
-        out.z = to_bf16x2(acc[4] * inv, acc[5] * inv);
-        out.w = to_bf16x2(acc[6] * inv, acc[7] * inv);
-        *reinterpret_cast<uint4 *>(o + b * os0 + h * os1 + i * os2 + sub * 8) = out;
-        if (sub == 0) lse[r] = empty ? -INFINITY : m + logf(tot);
+        const int64_t off = b * os0 + h * os1 + i * os2 + sub * 8;
+        {
+            const bool empty = (m == -INFINITY);
+            const float inv = empty ? 0.f : 1.f / tot;
+            uint4 out;
+            out.x = to_bf16x2(acc[0] * inv, acc[1] * inv);
+            out.y = to_bf16x2(acc[2] * inv, acc[3] * inv);
+            out.z = to_bf16x2(acc[4] * inv, acc[5] * inv);
+            out.w = to_bf16x2(acc[6] * inv, acc[7] * inv);
+            *reinterpret_cast<uint4 *>(o + off) = out;
+            if (sub == 0) lse[r] = empty ? -INFINITY : m + logf(tot);
+        }
+        if (o1) {
+            const bool empty = (m1 == -INFINITY);
+            const float inv = empty ? 0.f : 1.f / tot1;
+            uint4 out;
+            out.x = to_bf16x2(acc1[0] * inv, acc1[1] * inv);
+            out.y = to_bf16x2(acc1[2] * inv, acc1[3] * inv);
+            out.z = to_bf16x2(acc1[4] * inv, acc1[5] * inv);
+            out.w = to_bf16x2(acc1[6] * inv, acc1[7] * inv);
+            *reinterpret_cast<uint4 *>(o1 + off) = out;
+            if (sub == 0) lse1[r] = empty ? -INFINITY : m1 + logf(tot1);
+        }
     }
 }
 
 }  // namespace
 
 sfa_status launch_lse_combine(int64_t rows, int S, int d, int H, int64_t Lq, const void *o_part,
-                              const float *lse_part, void *o, const int64_t *o_stride, float *lse, cudaStream_t s)
+                              const float *lse_part, void *o, const int64_t *o_stride, float *lse, cudaStream_t s,
+                              int S1, void *o1, float *lse1)
 {
     if (rows == 0) return SFA_OK;
     int dev = 0, sms = 148;
@@ -135,11 +166,13 @@ sfa_status launch_lse_combine(int64_t rows, int S, int d, int H, int64_t Lq, con
     const int64_t cap = (int64_t)sms * 8;
     const int blocks = (int)(need < cap ? need : cap);
     if (d == 128)
-        lse_combine_kernel<128><<<blocks, threads, 0, s>>>(rows, S, H, Lq, (const uint4 *)o_part, lse_part,
-                                                           (uint16_t *)o, o_stride[0], o_stride[1], o_stride[2], lse);
+        lse_combine_kernel<128><<<blocks, threads, 0, s>>>(rows, S, S1, H, Lq, (const uint4 *)o_part, lse_part,
+                                                           (uint16_t *)o, o_stride[0], o_stride[1], o_stride[2], lse,
+                                                           (uint16_t *)o1, lse1);
     else
-        lse_combine_kernel<64><<<blocks, threads, 0, s>>>(rows, S, H, Lq, (const uint4 *)o_part, lse_part,
-                                                          (uint16_t *)o, o_stride[0], o_stride[1], o_stride[2], lse);
+        lse_combine_kernel<64><<<blocks, threads, 0, s>>>(rows, S, S1, H, Lq, (const uint4 *)o_part, lse_part,
+                                                          (uint16_t *)o, o_stride[0], o_stride[1], o_stride[2], lse,
+                                                          (uint16_t *)o1, lse1);
     return launch_status();
 }
 

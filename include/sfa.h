@@ -9,8 +9,8 @@
  *                   only, writing O (bf16) and the per-row log-sum-exp (fp32)
  *   sfa_lse_merge   merge of two partial attentions (e.g. local + history branch)
  *
- * plus variants of the forward (paged caches, split-KV) and the hierarchical block
- * selection of Light Forcing (sfa_hsa_select + sfa_forward_blocks).
+ * plus variants of the forward (paged caches, split-KV, two branches in one launch) and
+ * the hierarchical block selection of Light Forcing (sfa_hsa_select + sfa_forward_blocks).
  *
  * Conventions
  *   - A video has T latent frames of P tokens each; token i belongs to frame i / P.
@@ -247,6 +247,31 @@ sfa_status sfa_forward_split(const sfa_attn_desc *desc, const void *q, const voi
 sfa_status sfa_forward_split_noalloc(const sfa_attn_desc *desc, const void *q, const void *k, const void *v,
                                      const int32_t *frames, const int32_t *counts, void *o, float *lse,
                                      int32_t n_split, int32_t *dev_status, sfa_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
+ * Two branches in one launch
+ * ------------------------------------------------------------------------------------
+ * ("ISPA", §2.1 Dual-Stream Warmup: the local branch — current frame and sink — and the
+ *  full attention are both needed; with disjoint local and history key sets the full
+ *  attention is the LSE merge of the two branches.)  One grid runs the local lists and
+ * the history lists of the same queries (each cut into n_split key-tile ranges as in
+ * sfa_forward_split); one merge pass then writes
+ *   o_local, lse_local = attention over the local lists, and
+ *   o_full,  lse_full  = the LSE merge of both branches (attention over the union when
+ *                        the two lists of a (h, t) are disjoint).
+ * frames_local / counts_local and frames_hist / counts_hist: [H][Tq][Amax] / [H][Tq] as
+ * sfa_build_sets writes them (the same Amax).  o_local and o_full use desc->o_stride.
+ * sfa_forward_dual_workspace: bytes of workspace for n_split (1 <= 2 n_split <= d/8).
+ * The workspace must be 256-byte aligned; partial O is rounded to bf16 before the merge.
+ */
+sfa_status sfa_forward_dual_workspace(const sfa_attn_desc *desc, int32_t n_split, size_t *bytes);
+
+sfa_status sfa_forward_dual(const sfa_attn_desc *desc, const void *q, const void *k, const void *v,
+                            const int32_t *frames_local, const int32_t *counts_local,
+                            const int32_t *frames_hist, const int32_t *counts_hist, void *o_local,
+                            float *lse_local, void *o_full, float *lse_full, int32_t n_split,
+                            void *workspace, size_t workspace_bytes, int32_t *dev_status,
+                            sfa_stream_t stream);
 
 /* ------------------------------------------------------------------------------------
  * Hierarchical sparse attention (HSA): selection of key blocks, and attention over them

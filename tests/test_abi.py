@@ -187,3 +187,18 @@ def test_hsa_host_checks(sfa):
     assert lib.sfa_forward_blocks(ctypes.byref(d), good, good, good, good, good, good, good, None, None) == 2
     d = _desc(sfa)
     assert lib.sfa_forward_blocks(ctypes.byref(d), good, good, good, None, good, good, good, None, None) == 1
+
+
+def test_dual_host_checks(sfa):
+    lib = sfa.load()
+    d = _desc(sfa)  # d = 64: 2 * n_split <= 8
+    out = ctypes.c_size_t(0)
+    assert lib.sfa_forward_dual_workspace(ctypes.byref(d), 2, ctypes.byref(out)) == 0
+    assert out.value == 4 * 512 * 64 * 2 + 4 * 512 * 4
+    assert lib.sfa_forward_dual_workspace(ctypes.byref(d), 5, ctypes.byref(out)) == 1
+    good = 1 << 20
+    # history lists missing, workspace too small: refused before any launch
+    assert lib.sfa_forward_dual(ctypes.byref(d), good, good, good, good, good, None, good, good, good, good, good,
+                                1, good, 1 << 20, None, None) == 1
+    assert lib.sfa_forward_dual(ctypes.byref(d), good, good, good, good, good, good, good, good, good, good, good,
+                                1, good, 1024, None, None) == 1
