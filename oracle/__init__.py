@@ -9,6 +9,8 @@ its binding) never imports it, and it shares no code with that path.
 * ``lse_merge``  - merge of two partial attentions by LSE (numpy, ``merge.py``)
 * ``hsa``        - hierarchical frame/block selection and block-list attention
                    (numpy float64, ``hsa.py``)
+* ``gdn``        - ARL2 inter-frame gated delta rule over frames (numpy float64,
+                   ``gdn.py``)
 """
 from __future__ import annotations
 
@@ -21,6 +23,7 @@ import numpy as np
 from . import sets  # noqa: F401
 from .merge import lse_merge  # noqa: F401
 from . import hsa  # noqa: F401
+from . import gdn  # noqa: F401
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "sfa_oracle.c")

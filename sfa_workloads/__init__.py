@@ -12,6 +12,8 @@ Shapes follow the video-DiT workloads the method is described on:
   * "ISPA", §2.1 Dual-Stream Warmup: local (current + sink) and history branches.
   * "Resumen Técnico: LIGHT FORCING", §2.2 (HSA): an autoregressive chunk that
     selects history frames, then blocks, by mean-pooled keys.
+  * "Asistir Localmente, Recordar Linealmente (ARL2)", §2.1-2.2: the inter-frame branch
+    (a gated delta rule over frames), with synthetic feature-mapped inputs and gates.
 
 The real activations of those models are not available; Q, K and V are drawn
 i.i.d. N(0, 1) in fp32 and rounded to bf16, which has the right shapes, dtype
@@ -116,6 +118,8 @@ WORKLOADS = {
                               d=128, heads=(SetSpec("dense"),) * 12),
     # HSA: the streaming chunk of "stream"; sink + local window always, plus the 24 best
     # 128-token blocks of the 4 best history frames (of 17) per 256-row query block
+    # ARL2 inter-frame branch: 24 frames of the 30x52-patch shape, one state per head
+    "gdn": Workload("gdn", B=1, H=12, Tq=24, Tkv=24, q_off=0, P=1560, d=128, heads=(SetSpec("gdn"),) * 12),
     "hsa": Workload("hsa", B=1, H=12, Tq=3, Tkv=24, q_off=21, P=1560, d=128,
                     n_sink=1, n_prev=3, chunk_len=3, k_frames=4, k_blocks=24,
                     heads=(SetSpec("hsa"),) * 12),
@@ -188,3 +192,25 @@ def sample_rows(w: Workload, n_per_head: int, seed: int = 0, frames=()):
     if not rows:
         return np.zeros(0, dtype=np.int64)
     return np.unique(np.concatenate(rows)).astype(np.int64)
+
+
+def gdn_inputs(B: int, H: int, T: int, P: int, d: int, seed: int = 0):
+    """Inputs of the ARL2 inter-frame branch: Q', K' [B, H, T*P, d] bf16 with unit-norm
+    rows, V' [B, H, T*P, d] bf16, alpha [B, H, T] fp32, beta [B, H, T*P] fp32.
+
+    The page's feature maps, gates and step sizes are learned; a seeded stand-in keeps
+    the recurrence well conditioned the way a trained one is: one
+    ``torch.Generator('cpu')`` draws, in this order, Q', K', V' ~ N(0, 1) (Q', K' rows
+    then divided by their norm, in fp32, before the rounding to bf16), alpha =
+    sigmoid(N(2, 1)) per frame and beta = sigmoid(N(0, 1)) * d / P per token (a frame's
+    P unit keys act as one step of size about beta * P / d on the state).
+    """
+    g = torch.Generator("cpu").manual_seed(seed)
+    q = torch.randn(B, H, T * P, d, generator=g, dtype=torch.float32)
+    k = torch.randn(B, H, T * P, d, generator=g, dtype=torch.float32)
+    v = torch.randn(B, H, T * P, d, generator=g, dtype=torch.float32)
+    q = q / q.norm(dim=-1, keepdim=True)
+    k = k / k.norm(dim=-1, keepdim=True)
+    alpha = torch.sigmoid(torch.randn(B, H, T, generator=g, dtype=torch.float32) + 2.0)
+    beta = torch.sigmoid(torch.randn(B, H, T * P, generator=g, dtype=torch.float32)) * (d / P)
+    return q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16), alpha, beta
