@@ -377,6 +377,38 @@ def bench_hsa(sfa, dev, stream, flush, reps=20):
             "mean_blocks_per_list": round(float(counts.float().mean().item()), 2)}
 
 
+def bench_gdn(sfa, dev, stream, flush, reps=20):
+    """ARL2 inter-frame branch on the gdn workload (24 frames, 12 heads, P=1560, d=128)."""
+    from sfa_workloads import gdn_inputs
+    w = WORKLOADS["gdn"]
+    q, k, v, a, b = (x.to(dev) for x in gdn_inputs(w.B, w.H, w.Tq, w.P, w.d, seed=0))
+    o = torch.empty_like(q)
+    s = torch.empty((w.B, w.H, w.d, w.d), dtype=torch.float32, device=dev)
+
+    def run():
+        sfa.gdn_forward(q, k, v, a, b, w.P, out=o, state_out=s, stream=stream)
+
+    for _ in range(3):
+        run()
+    ts = []
+    for _ in range(reps):
+        flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        run()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ts.append(e0.elapsed_time(e1))
+    ms = float(np.median(ts))
+    flop = 3 * 2.0 * w.P * w.d * w.d * w.Tq * w.H * w.B
+    peak = float(measured_peaks()["bf16_tflops"])
+    return {"workload": "gdn: ARL2 inter-frame gated delta rule, 24 frames x 1560 tokens, H=12, d=128",
+            "ms": round(ms, 4), "gflop": round(flop / 1e9, 3), "tflops": round(flop / (ms * 1e-3) / 1e12, 2),
+            "frac": round(flop / (ms * 1e-3) / 1e12 / peak, 4), "ctas": w.B * w.H,
+            "note": "one CTA per (batch, head): the recurrence over frames is sequential"}
+
+
 # ----------------------------------------------------------------------------- oracle timing
 def cpu_baseline(seconds: float = 15.0, inputs=None):
     """Time the float64 oracle on host cores for about `seconds` on sampled query rows."""
@@ -559,7 +591,8 @@ def main():
                     help="run the workload with this many heads instead of 12 (smaller profiling case)")
     ap.add_argument("--skip-extras", action="store_true",
                     help="time the device step only: no end-to-end, merge or CPU-baseline legs")
-    ap.add_argument("--workload", choices=["lvsa41", "long121", "stream", "lsemerge", "hsa"], default="lvsa41",
+    ap.add_argument("--workload", choices=["lvsa41", "long121", "stream", "lsemerge", "hsa", "gdn"],
+                    default="lvsa41",
                     help="other workloads are timed on the device only (one JSON line, not the bench line)")
     ap.add_argument("--dual", action="store_true",
                     help="--workload lsemerge: both branches in one launch (sfa_forward_dual)")
@@ -575,12 +608,13 @@ def main():
 
     if args.workload != "lvsa41":
         if rank == 0:
-            if args.workload == "hsa":
+            if args.workload in ("hsa", "gdn"):
                 import frame_sparse_attention_b200 as sfa
                 sfa.load()
                 dev = torch.device("cuda", 0)
                 flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
-                rec = bench_hsa(sfa, dev, torch.cuda.current_stream(dev), flush, reps=args.steps)
+                fn = bench_hsa if args.workload == "hsa" else bench_gdn
+                rec = fn(sfa, dev, torch.cuda.current_stream(dev), flush, reps=args.steps)
             else:
                 rec = run_other_workload(args)
             print(json.dumps(rec), flush=True)

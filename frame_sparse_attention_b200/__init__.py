@@ -14,18 +14,20 @@ Python face of libsfa.so (C ABI in include/sfa.h):
 * ``hsa_select``  - hierarchical selection (Light Forcing HSA): pooled keys, top history
                     frames, then top 128-token key blocks, per 256-row query block
 * ``forward_blocks`` - attention of every query block over its key-block list
+* ``gdn_forward`` - ARL2's inter-frame branch: gated delta rule over frames (fp32 state)
 
 Tensors are PyTorch CUDA tensors; calls run on the current CUDA stream.
 """
 from ._lib import (SET_KINDS, SFA_DEBUG_STALL_SOFTMAX, SFA_ERR_BAD_SET, SFA_ERR_CUDA,
                    SFA_ERR_INVALID_ARG, SFA_ERR_TIMEOUT, SFA_ERR_UNSUPPORTED, SFA_OK, AttnDesc,
                    SetParams, SfaError, attn_desc, build_sets, error_string, forward, forward_blocks, forward_dual,
-                   forward_paged, forward_split, hsa_max_count, hsa_select, load, lse_merge, set_max_count,
+                   forward_paged, forward_split, gdn_forward, GdnDesc, hsa_max_count, hsa_select, load, lse_merge,
+                   set_max_count,
                    set_params, split_workspace_bytes, version)
 
 __all__ = ["SET_KINDS", "SFA_DEBUG_STALL_SOFTMAX", "SFA_ERR_BAD_SET", "SFA_ERR_CUDA",
            "SFA_ERR_INVALID_ARG", "SFA_ERR_TIMEOUT", "SFA_ERR_UNSUPPORTED", "SFA_OK", "AttnDesc",
            "SetParams", "SfaError", "attn_desc", "build_sets", "error_string", "forward", "forward_blocks",
            "forward_dual",
-           "forward_paged", "forward_split", "hsa_max_count", "hsa_select",
+           "forward_paged", "forward_split", "gdn_forward", "GdnDesc", "hsa_max_count", "hsa_select",
            "load", "lse_merge", "set_max_count", "set_params", "split_workspace_bytes", "version"]

@@ -50,10 +50,16 @@ class AttnDesc(ctypes.Structure):
 
 
 _lib = None
+class GdnDesc(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("T", ctypes.c_int32), ("P", ctypes.c_int32),
+                ("d", ctypes.c_int32), ("q_stride", ctypes.c_int64 * 3), ("k_stride", ctypes.c_int64 * 3),
+                ("v_stride", ctypes.c_int64 * 3), ("o_stride", ctypes.c_int64 * 3), ("timeout_us", ctypes.c_uint32)]
+
+
 EXPORTS = ("sfa_error_string", "sfa_version", "sfa_set_max_count", "sfa_build_sets", "sfa_forward",
            "sfa_forward_split_workspace", "sfa_forward_split", "sfa_forward_split_noalloc", "sfa_forward_paged",
            "sfa_lse_merge", "sfa_hsa_max_count", "sfa_hsa_workspace", "sfa_hsa_select", "sfa_forward_blocks",
-           "sfa_forward_dual_workspace", "sfa_forward_dual")
+           "sfa_forward_dual_workspace", "sfa_forward_dual", "sfa_gdn_forward")
 
 
 def load():
@@ -101,6 +107,8 @@ def load():
     lib.sfa_forward_dual.restype = st
     lib.sfa_forward_dual.argtypes = [ctypes.POINTER(AttnDesc), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp,
                                      ctypes.c_size_t, vp, vp]
+    lib.sfa_gdn_forward.restype = st
+    lib.sfa_gdn_forward.argtypes = [ctypes.POINTER(GdnDesc), vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp]
     lib.sfa_forward_blocks.restype = st
     lib.sfa_forward_blocks.argtypes = [ctypes.POINTER(AttnDesc), vp, vp, vp, vp, vp, vp, vp, vp, vp]
     _lib = lib
@@ -365,3 +373,34 @@ def forward_dual(q, k, v, frames_local, counts_local, frames_hist, counts_hist, 
                                    out_full.data_ptr(), lse_full.data_ptr(), n_split, workspace.data_ptr(),
                                    workspace.numel(), _ptr(dev_status), _stream(stream)), "sfa_forward_dual")
     return out_local, lse_local, out_full, lse_full
+
+
+def gdn_forward(q, k, v, alpha, beta, P: int, state_in=None, state_out=None, out=None, update: bool = True,
+                dev_status=None, stream=None, timeout_us: int = 0):
+    """ARL2 inter-frame branch over the T = L / P frames of q, k, v [B, H, L, d]: (O bf16
+    like q, final state fp32 [B, H, d, d]).  alpha fp32 [B, H, T], beta fp32 [B, H, L];
+    state_in fp32 [B, H, d, d] or None (zeros)."""
+    B, H, L, d = q.shape
+    if L % P:
+        raise ValueError(f"sequence length {L} is not a multiple of P = {P}")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or t.stride(3) != 1:
+            raise ValueError(f"{name} must be a bf16 CUDA tensor [B, H, L, d] with d contiguous")
+    out = torch.empty_like(q) if out is None else out
+    if state_out is None:
+        state_out = torch.empty((B, H, d, d), dtype=torch.float32, device=q.device)
+    for name, t in (("alpha", alpha), ("beta", beta), ("state_out", state_out)):
+        assert t.dtype == torch.float32 and t.is_contiguous(), name
+    assert tuple(alpha.shape) == (B, H, L // P) and tuple(beta.shape) == (B, H, L)
+    if state_in is not None:
+        assert state_in.dtype == torch.float32 and state_in.is_contiguous() and tuple(state_in.shape) == (B, H, d, d)
+    desc = GdnDesc()
+    desc.B, desc.H, desc.T, desc.P, desc.d = B, H, L // P, P, d
+    for field, t in (("q_stride", q), ("k_stride", k), ("v_stride", v), ("o_stride", out)):
+        arr = getattr(desc, field)
+        arr[0], arr[1], arr[2] = t.stride(0), t.stride(1), t.stride(2)
+    desc.timeout_us = timeout_us
+    _check(load().sfa_gdn_forward(ctypes.byref(desc), q.data_ptr(), k.data_ptr(), v.data_ptr(), alpha.data_ptr(),
+                                  beta.data_ptr(), _ptr(state_in), state_out.data_ptr(), out.data_ptr(),
+                                  1 if update else 0, _ptr(dev_status), _stream(stream)), "sfa_gdn_forward")
+    return out, state_out

@@ -1,0 +1,427 @@
+// ARL2 inter-frame branch: gated delta rule with frame-level state access, sm_100a.
+//
+// "Resumen Técnico: Asistir Localmente, Recordar Linealmente (ARL2)", §2.1 (Rama
+// Inter-Cuadro): a fixed-size state S [d x d] per (batch, head) replaces the KV cache;
+// frame N reads it as O_N = Q'_N S_{N-1} and then updates it as
+//   S_N = alpha_N S_{N-1} + K'_N^T diag(beta_N) (V'_N - K'_N S_{N-1});
+// §2.2: every token of a frame reads the same pre-update state (frame-level access), and
+// intermediate denoising steps read without writing (update = 0).
+//
+// Because the state changes once per frame, a frame is three dense contractions on the
+// tensor cores, tile by tile (128 tokens):
+//   O  = Q_i S           (M = 128 tokens, N = d, K = d; S as the B operand, bf16)
+//   KS = K_i S           (same)
+//   S_acc += K_i^T U_i   (M = d, N = d, K = 128 tokens), U_i = diag(beta) (V_i - KS)
+// One CTA per (batch, head) runs the frames in order (the recurrence is sequential);
+// warps 0-3 (one thread per TMEM lane) read O and KS out of tensor memory, write O, form
+// U in shared memory and update the fp32 state; warp 4 issues the TMA copies and MMAs.
+// Tensor memory: O, KS, S_acc and the fp32 state, 128 columns each.  Every wait is
+// bounded; a wait that runs out stores SFA_ERR_TIMEOUT and the CTA drains and exits.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "sfa.h"
+#include "sfa_internal.h"
+#include "sfa_ptx.cuh"
+
+namespace sfa {
+namespace {
+
+constexpr int GD = 128;          // d_k = d_v
+constexpr int GBM = 128;         // tokens per tile
+constexpr int GTHREADS = 160;    // warps 0-3 epilogue, warp 4 TMA + MMA
+constexpr int G_BOX = 128 * 128; // one 128-row x 64-column bf16 box (128-byte swizzle)
+constexpr int G_TILE = 2 * G_BOX;
+constexpr int G_S = 0, G_Q = G_TILE, G_K = 2 * G_TILE, G_V = 3 * G_TILE, G_U = 4 * G_TILE, G_BAR = 5 * G_TILE;
+constexpr int G_SMEM = G_BAR + 128 + 1024;
+constexpr uint32_t T_O = 0, T_KS = 128, T_SACC = 256, T_SST = 384;  // tensor-memory columns
+
+struct GdnArgs {
+    int32_t B, H, T, P, n_tiles, update;
+    const float *alpha;  // [B][H][T]
+    const float *beta;   // [B][H][T*P]
+    const float *s_in;   // [B][H][d][d] or null (zeros)
+    float *s_out;        // [B][H][d][d]
+    uint16_t *o;         // bf16, strided
+    int64_t os0, os1, os2;
+    int32_t *status;
+    uint64_t timeout_ns;
+};
+
+struct GBars {
+    uint32_t base;
+    __device__ uint32_t full() const { return base; }      // Q, K, V of a tile landed
+    __device__ uint32_t mma1() const { return base + 8; }  // O and KS of a tile in TMEM
+    __device__ uint32_t u_full() const { return base + 16; }  // U in smem, O/KS read (128 arrivals)
+    __device__ uint32_t sacc() const { return base + 24; }    // S_acc MMA of a tile done
+    __device__ uint32_t s_ready() const { return base + 32; } // state for the next frame (128 arrivals)
+    __device__ uint32_t drain() const { return base + 40; }
+};
+
+__device__ __forceinline__ uint64_t gns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// bounded wait; false (and the abort flag set, status written) when it runs out
+__device__ __noinline__ bool gwait(uint32_t bar, uint32_t parity, volatile int32_t *abort, int32_t *status,
+                                   uint64_t limit)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = gns();
+    for (uint32_t spins = 1;; ++spins) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort) return false;
+        if ((spins & 63) == 0 && (gns() - t0 > limit || spins > (1u << 30))) {
+            *abort = 1;
+            if (status) atomicCAS(status, 0, SFA_ERR_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ uint32_t swz(int row, int col)  // byte offset of (row, col) in a swizzled tile
+{
+    const int box = col >> 6, chunk = (col & 63) >> 3;
+    return (uint32_t)(box * G_BOX + row * 128 + ((chunk ^ (row & 7)) << 4) + (col & 7) * 2);
+}
+
+__device__ __forceinline__ float bf16f(uint16_t x) { return __uint_as_float((uint32_t)x << 16); }
+
+__global__ void __launch_bounds__(GTHREADS, 1)
+    gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ GdnArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const GBars bar{sbase + G_BAR};
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + G_BAR + 64);
+    volatile int32_t *abort = reinterpret_cast<volatile int32_t *>(smem + G_BAR + 68);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < 6; ++i) mbar_init(sbase + G_BAR + 8 * i, 1);
+        mbar_init(bar.u_full(), 128);
+        mbar_init(bar.s_ready(), 128);
+        *abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 4) {
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_q);
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+        }
+        tmem_alloc(smem_u32(tmem_slot), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 4) {
+        // ---------------------------------------------------------------- TMA + MMA
+        const uint64_t ds = sdesc_sw128(sbase + G_S, G_BOX, 1024);    // S: [d_k rows][d_v], MN-major B
+        const uint64_t dq = sdesc_sw128(sbase + G_Q, 16, 1024);       // Q tile, K-major A
+        const uint64_t dk = sdesc_sw128(sbase + G_K, 16, 1024);       // K tile, K-major A
+        const uint64_t dkt = sdesc_sw128(sbase + G_K, G_BOX, 1024);   // K tile read as K^T: MN-major A
+        const uint64_t du = sdesc_sw128(sbase + G_U, G_BOX, 1024);    // U tile, MN-major B
+        constexpr uint32_t id_qs = idesc_bf16_f32(GBM, GD, true);
+        constexpr uint32_t id_kt = idesc_bf16_f32(GD, GD, true) | (1u << 15);  // A MN-major
+        bool ok = true, issued = false, pending = false;  // pending: a tile's copies are in flight
+        uint32_t it = 0;
+        for (int n = 0; n < a.T && ok; ++n) {
+            ok = __all_sync(0xffffffffu, gwait(bar.s_ready(), n & 1, abort, a.status, a.timeout_ns));
+            for (int i = 0; i < a.n_tiles && ok; ++i, ++it) {
+                if (elect_one()) {
+                    mbar_arrive_expect_tx(bar.full(), 3 * G_TILE);
+#pragma unroll
+                    for (int kb = 0; kb < 2; ++kb) {
+                        tma_load_5d(sbase + G_Q + kb * G_BOX, &tm_q, bar.full(), kb * 64, i * GBM, n, h, b);
+                        tma_load_5d(sbase + G_K + kb * G_BOX, &tm_k, bar.full(), kb * 64, i * GBM, n, h, b);
+                        tma_load_5d(sbase + G_V + kb * G_BOX, &tm_v, bar.full(), kb * 64, i * GBM, n, h, b);
+                    }
+                }
+                __syncwarp();
+                pending = true;
+                if (!(ok = __all_sync(0xffffffffu, gwait(bar.full(), it & 1, abort, a.status, a.timeout_ns)))) break;
+                pending = false;
+                tc_fence_after();
+                if (elect_one()) {
+#pragma unroll
+                    for (uint32_t kk = 0; kk < GD / 16; ++kk) {
+                        const uint32_t ka = (kk >> 2) * G_BOX + (kk & 3) * 32;
+                        mma_ss(tmem + T_O, dq + (ka >> 4), ds + ((kk * 2048) >> 4), id_qs, kk > 0);
+                        mma_ss(tmem + T_KS, dk + (ka >> 4), ds + ((kk * 2048) >> 4), id_qs, kk > 0);
+                    }
+                    tc_commit(bar.mma1());
+                }
+                __syncwarp();
+                issued = true;
+                if (!(ok = __all_sync(0xffffffffu, gwait(bar.u_full(), it & 1, abort, a.status, a.timeout_ns)))) break;
+                tc_fence_after();
+                if (elect_one()) {
+                    // S_acc += K^T U over the tile's 128 tokens, 16 per step
+#pragma unroll
+                    for (uint32_t kk = 0; kk < GBM / 16; ++kk)
+                        mma_ss(tmem + T_SACC, dkt + ((kk * 2048) >> 4), du + ((kk * 2048) >> 4), id_kt,
+                               (i > 0 || kk > 0) ? 1u : 0u);
+                    tc_commit(bar.sacc());
+                }
+                __syncwarp();
+                ok = __all_sync(0xffffffffu, gwait(bar.sacc(), it & 1, abort, a.status, a.timeout_ns));
+            }
+        }
+        if (__any_sync(0xffffffffu, *abort != 0)) {
+            const uint64_t t0 = gns();
+            if (issued) {  // tensor cores idle before TMEM is freed
+                if (elect_one()) tc_commit(bar.drain());
+                __syncwarp();
+                while (!mbar_try_wait(bar.drain(), 0) && gns() - t0 < 2000000000ull) {
+                }
+            }
+            // copies still in flight land before the CTA exits
+            while (pending && !mbar_try_wait(bar.full(), it & 1) && gns() - t0 < 2000000000ull) {
+            }
+        }
+        __syncwarp();
+    } else {
+        // ---------------------------------------------------------------- epilogue, row r
+        const int r = threadIdx.x;  // TMEM lane = tile row = state row (d_k index)
+        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+        const int64_t bhi = (int64_t)b * a.H + h;
+        // state in: fp32 row r into TMEM, bf16 row r into the B-operand tile
+        {
+            float srow[GD];
+#pragma unroll
+            for (int c = 0; c < GD; ++c) srow[c] = a.s_in ? a.s_in[(bhi * GD + r) * GD + c] : 0.f;
+#pragma unroll
+            for (int c = 0; c < GD / 32; ++c) {
+                uint32_t w[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(srow[c * 32 + j]);
+                tmem_st32(lane_base + T_SST + c * 32, w);
+            }
+#pragma unroll
+            for (int c = 0; c < GD; c += 8) {
+                uint32_t pk[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) pk[j] = pack_bf16x2(srow[c + 2 * j], srow[c + 2 * j + 1]);
+                st_shared_v4(sbase + G_S + swz(r, c), pk);
+            }
+        }
+        tmem_wait_st();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(bar.s_ready());
+        bool ok = true;
+        uint32_t it = 0;
+        for (int n = 0; n < a.T && ok; ++n) {
+            for (int i = 0; i < a.n_tiles; ++i, ++it) {
+                ok = __all_sync(0xffffffffu, gwait(bar.mma1(), it & 1, abort, a.status, a.timeout_ns)) &&
+                     __all_sync(0xffffffffu, gwait(bar.full(), it & 1, abort, a.status, a.timeout_ns));
+                if (!ok) break;
+                tc_fence_after();
+                const int row = i * GBM + r;
+                const bool valid = row < a.P;
+                // O row -> global bf16
+                uint16_t *orow = a.o + b * a.os0 + h * a.os1 + ((int64_t)n * a.P + row) * a.os2;
+#pragma unroll
+                for (int c = 0; c < GD / 32; ++c) {
+                    uint32_t v[32];
+                    tmem_ld32(lane_base + T_O + c * 32, v);
+                    tmem_wait_ld_regs(v);
+                    if (valid) {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            uint4 w;
+                            w.x = pack_bf16x2(__uint_as_float(v[8 * q]), __uint_as_float(v[8 * q + 1]));
+                            w.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3]));
+                            w.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5]));
+                            w.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7]));
+                            *reinterpret_cast<uint4 *>(orow + c * 32 + q * 8) = w;
+                        }
+                    }
+                }
+                // U row = beta_row (V row - KS row) -> bf16, same swizzled layout as V
+                const float bt = valid ? a.beta[(bhi * a.T + n) * a.P + row] : 0.f;
+#pragma unroll
+                for (int c = 0; c < GD / 32; ++c) {
+                    uint32_t ks[32];
+                    tmem_ld32(lane_base + T_KS + c * 32, ks);
+                    tmem_wait_ld_regs(ks);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int col = c * 32 + q * 8;
+                        const uint4 vv = *reinterpret_cast<const uint4 *>(smem + G_V + swz(r, col));
+                        const uint32_t vw[4] = {vv.x, vv.y, vv.z, vv.w};
+                        uint32_t pk[4];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const float v0 = bf16f((uint16_t)(vw[j] & 0xffffu)), v1 = bf16f((uint16_t)(vw[j] >> 16));
+                            pk[j] = pack_bf16x2(bt * (v0 - __uint_as_float(ks[8 * q + 2 * j])),
+                                                bt * (v1 - __uint_as_float(ks[8 * q + 2 * j + 1])));
+                        }
+                        st_shared_v4(sbase + G_U + swz(r, col), pk);
+                    }
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(bar.u_full());
+            }
+            if (!ok) break;
+            // frame end: S <- alpha S + S_acc, fp32 in TMEM, bf16 copy for the next frame
+            ok = __all_sync(0xffffffffu, gwait(bar.sacc(), (it - 1) & 1, abort, a.status, a.timeout_ns));
+            if (!ok) break;
+            tc_fence_after();
+            if (a.update) {
+                const float al = a.alpha[bhi * a.T + n];
+#pragma unroll
+                for (int c = 0; c < GD / 32; ++c) {
+                    uint32_t s[32], acc[32];
+                    tmem_ld32(lane_base + T_SST + c * 32, s);
+                    tmem_wait_ld_regs(s);
+                    tmem_ld32(lane_base + T_SACC + c * 32, acc);
+                    tmem_wait_ld_regs(acc);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        s[j] = __float_as_uint(fmaf(al, __uint_as_float(s[j]), __uint_as_float(acc[j])));
+                    tmem_st32(lane_base + T_SST + c * 32, s);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint32_t pk[4];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            pk[j] = pack_bf16x2(__uint_as_float(s[8 * q + 2 * j]), __uint_as_float(s[8 * q + 2 * j + 1]));
+                        st_shared_v4(sbase + G_S + swz(r, c * 32 + q * 8), pk);
+                    }
+                }
+            }
+            tmem_wait_st();
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(bar.s_ready());
+        }
+        // state out
+        if (ok && a.s_out) {
+            tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < GD / 32; ++c) {
+                uint32_t s[32];
+                tmem_ld32(lane_base + T_SST + c * 32, s);
+                tmem_wait_ld_regs(s);
+#pragma unroll
+                for (int j = 0; j < 32; j += 4) {
+                    float4 w = make_float4(__uint_as_float(s[j]), __uint_as_float(s[j + 1]), __uint_as_float(s[j + 2]),
+                                           __uint_as_float(s[j + 3]));
+                    *reinterpret_cast<float4 *>(a.s_out + (bhi * GD + r) * GD + c * 32 + j) = w;
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 4) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ---------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// bf16 [B][H][T*P][d] as a 5-D map (d, P, T, H, B), box 64 x 128 x 1 x 1 x 1, 128-byte
+// swizzle: a tile never crosses its frame; rows past the frame read as zero
+bool encode_frames(CUtensorMap *m, const void *base, int B, int H, int T, int P, const int64_t *stride)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t gd[5] = {(cuuint64_t)GD, (cuuint64_t)P, (cuuint64_t)T, (cuuint64_t)H, (cuuint64_t)B};
+    const cuuint64_t gs[4] = {(cuuint64_t)stride[2] * 2, (cuuint64_t)P * stride[2] * 2, (cuuint64_t)stride[1] * 2,
+                              (cuuint64_t)stride[0] * 2};
+    const cuuint32_t box[5] = {64, (cuuint32_t)GBM, 1, 1, 1}, es[5] = {1, 1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), gd, gs, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool gdn_stride_ok(const int64_t *s)
+{
+    return s[2] >= GD && s[0] >= 0 && s[1] >= 0 && s[0] % 8 == 0 && s[1] % 8 == 0 && s[2] % 8 == 0;
+}
+
+}  // namespace
+}  // namespace sfa
+
+using namespace sfa;
+
+extern "C" sfa_status sfa_gdn_forward(const sfa_gdn_desc *d, const void *q, const void *k, const void *v,
+                                      const float *alpha, const float *beta, const float *state_in,
+                                      float *state_out, void *o, int32_t update, int32_t *dev_status,
+                                      sfa_stream_t stream)
+{
+    if (!d || d->B < 0 || d->H < 1 || d->T < 1 || d->P < 1) return SFA_ERR_INVALID_ARG;
+    if (d->d != GD) return SFA_ERR_UNSUPPORTED;
+    if ((int64_t)d->T * d->P >= ((int64_t)1 << 31) || (int64_t)d->B * d->H >= ((int64_t)1 << 31))
+        return SFA_ERR_INVALID_ARG;
+    if (d->B == 0) return SFA_OK;
+    if (!q || !k || !v || !o || !alpha || !beta || !state_out) return SFA_ERR_INVALID_ARG;
+    const void *ptrs[5] = {q, k, v, o, state_out};
+    for (const void *p : ptrs)
+        if (reinterpret_cast<uintptr_t>(p) % 16) return SFA_ERR_INVALID_ARG;
+    if (state_in && reinterpret_cast<uintptr_t>(state_in) % 16) return SFA_ERR_INVALID_ARG;
+    if (!gdn_stride_ok(d->q_stride) || !gdn_stride_ok(d->k_stride) || !gdn_stride_ok(d->v_stride) ||
+        !gdn_stride_ok(d->o_stride))
+        return SFA_ERR_INVALID_ARG;
+    CUtensorMap tq, tk, tv;
+    if (!encode_frames(&tq, q, d->B, d->H, d->T, d->P, d->q_stride) ||
+        !encode_frames(&tk, k, d->B, d->H, d->T, d->P, d->k_stride) ||
+        !encode_frames(&tv, v, d->B, d->H, d->T, d->P, d->v_stride))
+        return SFA_ERR_UNSUPPORTED;
+    GdnArgs a;
+    a.B = d->B;
+    a.H = d->H;
+    a.T = d->T;
+    a.P = d->P;
+    a.n_tiles = (d->P + GBM - 1) / GBM;
+    a.update = update ? 1 : 0;
+    a.alpha = alpha;
+    a.beta = beta;
+    a.s_in = state_in;
+    a.s_out = state_out;
+    a.o = static_cast<uint16_t *>(o);
+    a.os0 = d->o_stride[0];
+    a.os1 = d->o_stride[1];
+    a.os2 = d->o_stride[2];
+    a.status = dev_status;
+    a.timeout_ns = (uint64_t)(d->timeout_us ? d->timeout_us : 2000000u) * 1000;
+    if (cudaFuncSetAttribute(gdn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, G_SMEM) != cudaSuccess)
+        return SFA_ERR_CUDA;
+    gdn_kernel<<<(unsigned)(d->B * d->H), GTHREADS, G_SMEM, as_cuda(stream)>>>(tq, tk, tv, a);
+    return launch_status();
+}

@@ -9,8 +9,9 @@
  *                   only, writing O (bf16) and the per-row log-sum-exp (fp32)
  *   sfa_lse_merge   merge of two partial attentions (e.g. local + history branch)
  *
- * plus variants of the forward (paged caches, split-KV, two branches in one launch) and
- * the hierarchical block selection of Light Forcing (sfa_hsa_select + sfa_forward_blocks).
+ * plus variants of the forward (paged caches, split-KV, two branches in one launch), the
+ * hierarchical block selection of Light Forcing (sfa_hsa_select + sfa_forward_blocks) and
+ * ARL2's inter-frame gated-delta branch (sfa_gdn_forward).
  *
  * Conventions
  *   - A video has T latent frames of P tokens each; token i belongs to frame i / P.
@@ -332,6 +333,40 @@ sfa_status sfa_hsa_select(const sfa_attn_desc *desc, const sfa_set_params *p, in
 sfa_status sfa_forward_blocks(const sfa_attn_desc *desc, const void *q, const void *k, const void *v,
                               const int32_t *blocks, const int32_t *counts, void *o, float *lse,
                               int32_t *dev_status, sfa_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
+ * ARL2 inter-frame branch: gated delta rule over frames
+ * ------------------------------------------------------------------------------------
+ * ("Resumen Técnico: Asistir Localmente, Recordar Linealmente (ARL2)", §2.1 Rama
+ *  Inter-Cuadro and §2.2 Gestión del Estado de Memoria.)  Per (batch b, head h) a state
+ * S [d][d] (fp32) replaces the KV cache.  For frames N = 0 .. T-1 in order:
+ *     O_N = Q'_N S_{N-1}                       (every token of the frame reads the same,
+ *                                              pre-update state: frame-level access)
+ *     S_N = alpha_N S_{N-1} + K'_N^T diag(beta_N) (V'_N - K'_N S_{N-1})   if update != 0
+ *     S_N = S_{N-1}                                                        if update == 0
+ * (update == 0 is the read-only access of the intermediate denoising steps).
+ *   q, k, v, o  bf16 [B][H][T*P][d] with the strides in the descriptor (d contiguous; 16-byte
+ *               aligned bases, strides multiples of 8 elements); q, k, v are the
+ *               feature-mapped projections Q', K', V'.
+ *   alpha       fp32 [B][H][T] (one forget factor per frame), contiguous.
+ *   beta        fp32 [B][H][T*P] (one step size per token), contiguous.
+ *   state_in    fp32 [B][H][d][d] (row = key dimension), contiguous, or NULL for zeros.
+ *   state_out   fp32 [B][H][d][d]; may be the same buffer as state_in.
+ * The tensor cores read S and the per-token corrections as bf16; the state itself is kept
+ * and updated in fp32.  Supported: d = 128, any P >= 1, any T >= 1.
+ */
+typedef struct {
+    int32_t B, H, T, P, d;
+    int64_t q_stride[3]; /* batch, head, token (elements) */
+    int64_t k_stride[3];
+    int64_t v_stride[3];
+    int64_t o_stride[3];
+    uint32_t timeout_us; /* limit of every wait inside the kernel; 0 = 2 s */
+} sfa_gdn_desc;
+
+sfa_status sfa_gdn_forward(const sfa_gdn_desc *desc, const void *q, const void *k, const void *v,
+                           const float *alpha, const float *beta, const float *state_in, float *state_out,
+                           void *o, int32_t update, int32_t *dev_status, sfa_stream_t stream);
 
 /* ------------------------------------------------------------------------------------
  * LSE merge
