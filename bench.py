@@ -368,13 +368,37 @@ def bench_hsa(sfa, dev, stream, flush, reps=20):
     peak = float(measured_peaks()["bf16_tflops"])
     tf = flops / (fwd_ms * 1e-3) / 1e12
     pool_bytes = (k.numel() + q.numel()) * 2
+    hbm = float(measured_peaks()["hbm_gbs"])
+    # the oracle on a bounded sample: one query block per (head, frame), its selection and
+    # its rows' attention (float64 numpy), about a few seconds of host work
+    import time
+    from oracle import hsa as ohsa
+    qf, kf_, vf = q_h.float().numpy(), k_h.float().numpy(), v_h.float().numpy()
+    t0 = time.perf_counter()
+    kw = dict(P=w.P, T_kv=w.Tkv, q_off=w.q_off, chunk_len=w.chunk_len, n_prev=w.n_prev, n_sink=w.n_sink,
+              k_frames=w.k_frames, k_blocks=w.k_blocks)
+    o_lists, o_counts = ohsa.build_block_lists(qf, kf_, Bmax=blocks.shape[-1], **kw)
+    rows = np.asarray([(h * w.Lq) + t * w.P + r for h in range(w.H) for t in range(w.Tq) for r in range(0, 256, 8)])
+    ohsa.attention_blocks(qf, kf_, vf, o_lists, o_counts, w.P, 1 / math.sqrt(w.d), rows=rows)
+    dt = time.perf_counter() - t0
+    keys_per_row = float(np.mean([o_counts[0, h, t, 0] for h in range(w.H) for t in range(w.Tq)])) * 128
     return {"workload": "hsa: 3 query frames after 21 history frames, P=1560, H=12, d=128; sink 1 + "
                         "local 6 frames always, 24 blocks of the 4 best history frames per 256-row query block",
             "select_ms": round(sel_ms, 4), "select_pool_bytes": pool_bytes,
             "forward_blocks_ms": round(fwd_ms, 4), "attended_tflop": round(flops / 1e12, 4),
             "forward_tflops": round(tf, 1), "forward_frac": round(tf / peak, 4),
             "step_tflops": round(flops / ((sel_ms + fwd_ms) * 1e-3) / 1e12, 1),
-            "mean_blocks_per_list": round(float(counts.float().mean().item()), 2)}
+            "mean_blocks_per_list": round(float(counts.float().mean().item()), 2),
+            "roofline": {"forward_blocks": {"bound": "tensor", "achieved": round(tf, 1), "peak": peak,
+                                            "unit": "TFLOP/s", "frac": round(tf / peak, 4)},
+                         "select": {"bound": "hbm", "achieved": round(pool_bytes / (sel_ms * 1e-3) / 1e9, 1),
+                                    "peak": hbm, "unit": "GB/s",
+                                    "frac": round(pool_bytes / (sel_ms * 1e-3) / 1e9 / hbm, 4),
+                                    "note": "bytes = K and Q read once by the pooling"}},
+            "cpu_baseline": {"value": round(4.0 * w.d * keys_per_row * len(rows) / dt / 1e12, 8), "unit": "TFLOP/s",
+                             "cores": os.cpu_count() or 1, "kind": "oracle",
+                             "sample": f"selection of every list + attention of {len(rows)} query rows "
+                                       f"(float64 numpy, {dt:.1f} s; value counts the attention rows only)"}}
 
 
 def bench_gdn(sfa, dev, stream, flush, reps=20):
@@ -403,7 +427,20 @@ def bench_gdn(sfa, dev, stream, flush, reps=20):
     ms = float(np.median(ts))
     flop = 3 * 2.0 * w.P * w.d * w.d * w.Tq * w.H * w.B
     peak = float(measured_peaks()["bf16_tflops"])
+    # the oracle on a bounded sample: one head, all 24 frames (float64 numpy)
+    import time
+    from oracle import gdn as ogdn
+    qh, kh, vh, ah, bh = gdn_inputs(w.B, w.H, w.Tq, w.P, w.d, seed=0)
+    t0 = time.perf_counter()
+    ogdn.gdn_frames(qh[:, :1].float().numpy(), kh[:, :1].float().numpy(), vh[:, :1].float().numpy(),
+                    ah[:, :1].numpy(), bh[:, :1].numpy(), w.P)
+    dt = time.perf_counter() - t0
     return {"workload": "gdn: ARL2 inter-frame gated delta rule, 24 frames x 1560 tokens, H=12, d=128",
+            "roofline": {"bound": "tensor", "achieved": round(flop / (ms * 1e-3) / 1e12, 2), "peak": peak,
+                         "unit": "TFLOP/s", "frac": round(flop / (ms * 1e-3) / 1e12 / peak, 4)},
+            "cpu_baseline": {"value": round(flop / w.H / dt / 1e12, 8), "unit": "TFLOP/s",
+                             "cores": os.cpu_count() or 1, "kind": "oracle",
+                             "sample": f"one head of the workload, all 24 frames (float64 numpy, {dt:.2f} s)"},
             "ms": round(ms, 4), "gflop": round(flop / 1e9, 3), "tflops": round(flop / (ms * 1e-3) / 1e12, 2),
             "frac": round(flop / (ms * 1e-3) / 1e12 / peak, 4), "ctas": w.B * w.H,
             "note": "one CTA per (batch, head): the recurrence over frames is sequential"}
