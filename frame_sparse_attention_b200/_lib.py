@@ -59,7 +59,7 @@ class GdnDesc(ctypes.Structure):
 EXPORTS = ("sfa_error_string", "sfa_version", "sfa_set_max_count", "sfa_build_sets", "sfa_forward",
            "sfa_forward_split_workspace", "sfa_forward_split", "sfa_forward_split_noalloc", "sfa_forward_paged",
            "sfa_lse_merge", "sfa_hsa_max_count", "sfa_hsa_workspace", "sfa_hsa_select", "sfa_forward_blocks",
-           "sfa_forward_dual_workspace", "sfa_forward_dual", "sfa_gdn_forward")
+           "sfa_forward_dual_workspace", "sfa_forward_dual", "sfa_gdn_workspace", "sfa_gdn_forward")
 
 
 def load():
@@ -108,7 +108,10 @@ def load():
     lib.sfa_forward_dual.argtypes = [ctypes.POINTER(AttnDesc), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp,
                                      ctypes.c_size_t, vp, vp]
     lib.sfa_gdn_forward.restype = st
-    lib.sfa_gdn_forward.argtypes = [ctypes.POINTER(GdnDesc), vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp]
+    lib.sfa_gdn_workspace.restype = st
+    lib.sfa_gdn_workspace.argtypes = [ctypes.POINTER(GdnDesc), ctypes.POINTER(ctypes.c_size_t)]
+    lib.sfa_gdn_forward.argtypes = [ctypes.POINTER(GdnDesc), vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, ctypes.c_size_t,
+                                    vp, vp]
     lib.sfa_forward_blocks.restype = st
     lib.sfa_forward_blocks.argtypes = [ctypes.POINTER(AttnDesc), vp, vp, vp, vp, vp, vp, vp, vp, vp]
     _lib = lib
@@ -376,10 +379,12 @@ def forward_dual(q, k, v, frames_local, counts_local, frames_hist, counts_hist, 
 
 
 def gdn_forward(q, k, v, alpha, beta, P: int, state_in=None, state_out=None, out=None, update: bool = True,
-                dev_status=None, stream=None, timeout_us: int = 0):
+                workspace="auto", dev_status=None, stream=None, timeout_us: int = 0):
     """ARL2 inter-frame branch over the T = L / P frames of q, k, v [B, H, L, d]: (O bf16
     like q, final state fp32 [B, H, d, d]).  alpha fp32 [B, H, T], beta fp32 [B, H, L];
-    state_in fp32 [B, H, d, d] or None (zeros)."""
+    state_in fp32 [B, H, d, d] or None (zeros).  workspace: "auto" (allocated here: the
+    frame's tiles spread over several CTAs per head), a uint8 CUDA tensor, or None (one CTA
+    per head)."""
     B, H, L, d = q.shape
     if L % P:
         raise ValueError(f"sequence length {L} is not a multiple of P = {P}")
@@ -400,7 +405,13 @@ def gdn_forward(q, k, v, alpha, beta, P: int, state_in=None, state_out=None, out
         arr = getattr(desc, field)
         arr[0], arr[1], arr[2] = t.stride(0), t.stride(1), t.stride(2)
     desc.timeout_us = timeout_us
+    if isinstance(workspace, str):
+        nbytes = ctypes.c_size_t(0)
+        _check(load().sfa_gdn_workspace(ctypes.byref(desc), ctypes.byref(nbytes)), "sfa_gdn_workspace")
+        workspace = torch.empty(nbytes.value, dtype=torch.uint8, device=q.device) if nbytes.value else None
+    ws_ptr, ws_bytes = (workspace.data_ptr(), workspace.numel()) if workspace is not None else (None, 0)
     _check(load().sfa_gdn_forward(ctypes.byref(desc), q.data_ptr(), k.data_ptr(), v.data_ptr(), alpha.data_ptr(),
                                   beta.data_ptr(), _ptr(state_in), state_out.data_ptr(), out.data_ptr(),
-                                  1 if update else 0, _ptr(dev_status), _stream(stream)), "sfa_gdn_forward")
+                                  1 if update else 0, ws_ptr, ws_bytes, _ptr(dev_status), _stream(stream)),
+           "sfa_gdn_forward")
     return out, state_out

@@ -12,14 +12,20 @@
 //   O  = Q_i S           (M = 128 tokens, N = d, K = d; S as the B operand, bf16)
 //   KS = K_i S           (same)
 //   S_acc += K_i^T U_i   (M = d, N = d, K = 128 tokens), U_i = diag(beta) (V_i - KS)
-// One CTA per (batch, head) runs the frames in order (the recurrence is sequential);
-// warps 0-3 (one thread per TMEM lane) read O and KS out of tensor memory, write O, form
-// U in shared memory and update the fp32 state; warp 4 issues the TMA copies and MMAs.
+// G CTAs per (batch, head) run the frames in order (the recurrence is sequential); CTA g
+// takes tiles g, g + G, ... of every frame.  With G > 1 each CTA writes its partial
+// S_acc to a workspace, the G CTAs of a head meet at a counter in global memory (one
+// cooperative launch, so all CTAs are resident; the wait is bounded), and each CTA adds
+// the G partials itself (double-buffered by frame parity, so one meeting per frame is
+// enough).  Warps 0-3 (one thread per TMEM lane) read O and KS out of tensor memory,
+// write O, form U in shared memory and update the fp32 state; warp 4 issues the TMA
+// copies and MMAs.
 // Tensor memory: O, KS, S_acc and the fp32 state, 128 columns each.  Every wait is
 // bounded; a wait that runs out stores SFA_ERR_TIMEOUT and the CTA drains and exits.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <mutex>
@@ -42,6 +48,9 @@ constexpr uint32_t T_O = 0, T_KS = 128, T_SACC = 256, T_SST = 384;  // tensor-me
 
 struct GdnArgs {
     int32_t B, H, T, P, n_tiles, update;
+    int32_t G;           // CTAs per (batch, head)
+    float *part;         // [2][B*H][G][d][d] partial S_acc (G > 1)
+    uint32_t *count;     // [B*H] arrivals (G > 1), zero at launch
     const float *alpha;  // [B][H][T]
     const float *beta;   // [B][H][T*P]
     const float *s_in;   // [B][H][d][d] or null (zeros)
@@ -105,7 +114,7 @@ __global__ void __launch_bounds__(GTHREADS, 1)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + G_BAR + 64);
     volatile int32_t *abort = reinterpret_cast<volatile int32_t *>(smem + G_BAR + 68);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
+    const int bh = blockIdx.x / a.G, g = blockIdx.x % a.G, b = bh / a.H, h = bh % a.H;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < 6; ++i) mbar_init(sbase + G_BAR + 8 * i, 1);
@@ -141,7 +150,7 @@ __global__ void __launch_bounds__(GTHREADS, 1)
         uint32_t it = 0;
         for (int n = 0; n < a.T && ok; ++n) {
             ok = __all_sync(0xffffffffu, gwait(bar.s_ready(), n & 1, abort, a.status, a.timeout_ns));
-            for (int i = 0; i < a.n_tiles && ok; ++i, ++it) {
+            for (int i = g; i < a.n_tiles && ok; i += a.G, ++it) {
                 if (elect_one()) {
                     mbar_arrive_expect_tx(bar.full(), 3 * G_TILE);
 #pragma unroll
@@ -174,7 +183,7 @@ __global__ void __launch_bounds__(GTHREADS, 1)
 #pragma unroll
                     for (uint32_t kk = 0; kk < GBM / 16; ++kk)
                         mma_ss(tmem + T_SACC, dkt + ((kk * 2048) >> 4), du + ((kk * 2048) >> 4), id_kt,
-                               (i > 0 || kk > 0) ? 1u : 0u);
+                               (i > g || kk > 0) ? 1u : 0u);
                     tc_commit(bar.sacc());
                 }
                 __syncwarp();
@@ -226,7 +235,7 @@ __global__ void __launch_bounds__(GTHREADS, 1)
         bool ok = true;
         uint32_t it = 0;
         for (int n = 0; n < a.T && ok; ++n) {
-            for (int i = 0; i < a.n_tiles; ++i, ++it) {
+            for (int i = g; i < a.n_tiles; i += a.G, ++it) {
                 ok = __all_sync(0xffffffffu, gwait(bar.mma1(), it & 1, abort, a.status, a.timeout_ns)) &&
                      __all_sync(0xffffffffu, gwait(bar.full(), it & 1, abort, a.status, a.timeout_ns));
                 if (!ok) break;
@@ -283,15 +292,68 @@ __global__ void __launch_bounds__(GTHREADS, 1)
             ok = __all_sync(0xffffffffu, gwait(bar.sacc(), (it - 1) & 1, abort, a.status, a.timeout_ns));
             if (!ok) break;
             tc_fence_after();
+            if (a.update && a.G > 1) {
+                // this CTA's partial out, meet the head's other CTAs, then add all partials
+                float *mine = a.part + ((((int64_t)(n & 1) * a.B * a.H + bh) * a.G + g) * GD + r) * GD;
+#pragma unroll
+                for (int c = 0; c < GD / 32; ++c) {
+                    uint32_t acc[32];
+                    tmem_ld32(lane_base + T_SACC + c * 32, acc);
+                    tmem_wait_ld_regs(acc);
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4)
+                        __stcg(reinterpret_cast<float4 *>(mine + c * 32 + j),
+                               make_float4(__uint_as_float(acc[j]), __uint_as_float(acc[j + 1]),
+                                           __uint_as_float(acc[j + 2]), __uint_as_float(acc[j + 3])));
+                }
+                __threadfence();
+                named_bar_sync(1, 128);
+                if (r == 0) {
+                    atomicAdd(a.count + bh, 1u);
+                    const uint32_t want = (uint32_t)a.G * (uint32_t)(n + 1);
+                    const uint64_t t0 = gns();
+                    for (uint32_t spins = 0; *reinterpret_cast<volatile uint32_t *>(a.count + bh) < want; ++spins) {
+                        if (*abort) break;
+                        if ((spins & 63) == 63 && gns() - t0 > a.timeout_ns) {
+                            *abort = 1;
+                            if (a.status) atomicCAS(a.status, 0, SFA_ERR_TIMEOUT);
+                            break;
+                        }
+                    }
+                    __threadfence();
+                }
+                named_bar_sync(1, 128);
+                if (*abort) {
+                    ok = false;
+                    break;
+                }
+            }
             if (a.update) {
                 const float al = a.alpha[bhi * a.T + n];
+                const float *parts = a.part + (((int64_t)(n & 1) * a.B * a.H + bh) * a.G * GD + r) * GD;
 #pragma unroll
                 for (int c = 0; c < GD / 32; ++c) {
                     uint32_t s[32], acc[32];
                     tmem_ld32(lane_base + T_SST + c * 32, s);
                     tmem_wait_ld_regs(s);
-                    tmem_ld32(lane_base + T_SACC + c * 32, acc);
-                    tmem_wait_ld_regs(acc);
+                    if (a.G > 1) {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) acc[j] = 0u;
+                        for (int gg = 0; gg < a.G; ++gg) {
+                            const float *src = parts + (int64_t)gg * GD * GD + c * 32;
+#pragma unroll
+                            for (int j = 0; j < 32; j += 4) {
+                                const float4 v4 = __ldcg(reinterpret_cast<const float4 *>(src + j));
+                                acc[j] = __float_as_uint(__uint_as_float(acc[j]) + v4.x);
+                                acc[j + 1] = __float_as_uint(__uint_as_float(acc[j + 1]) + v4.y);
+                                acc[j + 2] = __float_as_uint(__uint_as_float(acc[j + 2]) + v4.z);
+                                acc[j + 3] = __float_as_uint(__uint_as_float(acc[j + 3]) + v4.w);
+                            }
+                        }
+                    } else {
+                        tmem_ld32(lane_base + T_SACC + c * 32, acc);
+                        tmem_wait_ld_regs(acc);
+                    }
 #pragma unroll
                     for (int j = 0; j < 32; ++j)
                         s[j] = __float_as_uint(fmaf(al, __uint_as_float(s[j]), __uint_as_float(acc[j])));
@@ -311,8 +373,8 @@ __global__ void __launch_bounds__(GTHREADS, 1)
             tc_fence_before();
             mbar_arrive(bar.s_ready());
         }
-        // state out
-        if (ok && a.s_out) {
+        // state out (CTA 0 of the head; all hold the same state)
+        if (ok && a.s_out && g == 0) {
             tc_fence_after();
 #pragma unroll
             for (int c = 0; c < GD / 32; ++c) {
@@ -375,15 +437,42 @@ bool gdn_stride_ok(const int64_t *s)
     return s[2] >= GD && s[0] >= 0 && s[1] >= 0 && s[0] % 8 == 0 && s[1] % 8 == 0 && s[2] % 8 == 0;
 }
 
+// CTAs per (batch, head): about two tiles of a frame each, all resident at once (one CTA
+// per SM: the kernel's shared memory allows no second one)
+int gdn_split(const sfa_gdn_desc *d)
+{
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int n_tiles = (d->P + GBM - 1) / GBM;
+    const int64_t heads = (int64_t)d->B * d->H;
+    int G = (n_tiles + 1) / 2;
+    if (heads * G > sms) G = (int)std::max<int64_t>(1, sms / heads);
+    return std::max(G, 1);
+}
+
+size_t gdn_part_bytes(const sfa_gdn_desc *d, int G)
+{
+    return ((size_t)2 * d->B * d->H * G * GD * GD * 4 + 255) / 256 * 256;
+}
+
 }  // namespace
 }  // namespace sfa
 
 using namespace sfa;
 
+extern "C" sfa_status sfa_gdn_workspace(const sfa_gdn_desc *d, size_t *bytes)
+{
+    if (!d || !bytes || d->B < 0 || d->H < 1 || d->T < 1 || d->P < 1) return SFA_ERR_INVALID_ARG;
+    if (d->d != GD) return SFA_ERR_UNSUPPORTED;
+    const int G = gdn_split(d);
+    *bytes = G > 1 ? gdn_part_bytes(d, G) + ((size_t)d->B * d->H * 4 + 255) / 256 * 256 : 0;
+    return SFA_OK;
+}
+
 extern "C" sfa_status sfa_gdn_forward(const sfa_gdn_desc *d, const void *q, const void *k, const void *v,
                                       const float *alpha, const float *beta, const float *state_in,
-                                      float *state_out, void *o, int32_t update, int32_t *dev_status,
-                                      sfa_stream_t stream)
+                                      float *state_out, void *o, int32_t update, void *workspace,
+                                      size_t workspace_bytes, int32_t *dev_status, sfa_stream_t stream)
 {
     if (!d || d->B < 0 || d->H < 1 || d->T < 1 || d->P < 1) return SFA_ERR_INVALID_ARG;
     if (d->d != GD) return SFA_ERR_UNSUPPORTED;
@@ -420,8 +509,27 @@ extern "C" sfa_status sfa_gdn_forward(const sfa_gdn_desc *d, const void *q, cons
     a.os2 = d->o_stride[2];
     a.status = dev_status;
     a.timeout_ns = (uint64_t)(d->timeout_us ? d->timeout_us : 2000000u) * 1000;
+    // several CTAs per head need the workspace (and a read-write frame loop); otherwise one
+    int G = (workspace && update) ? gdn_split(d) : 1;
+    a.G = G;
+    a.part = nullptr;
+    a.count = nullptr;
+    cudaStream_t s = as_cuda(stream);
     if (cudaFuncSetAttribute(gdn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, G_SMEM) != cudaSuccess)
         return SFA_ERR_CUDA;
-    gdn_kernel<<<(unsigned)(d->B * d->H), GTHREADS, G_SMEM, as_cuda(stream)>>>(tq, tk, tv, a);
+    if (G > 1) {
+        const size_t pb = gdn_part_bytes(d, G), need = pb + ((size_t)d->B * d->H * 4 + 255) / 256 * 256;
+        if (workspace_bytes < need || reinterpret_cast<uintptr_t>(workspace) % 256) return SFA_ERR_INVALID_ARG;
+        a.part = static_cast<float *>(workspace);
+        a.count = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(workspace) + pb);
+        if (cudaMemsetAsync(a.count, 0, (size_t)d->B * d->H * 4, s) != cudaSuccess) return SFA_ERR_CUDA;
+        // the G CTAs of a head wait for one another: one cooperative launch keeps them all resident
+        void *args[] = {&tq, &tk, &tv, &a};
+        const cudaError_t e = cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(gdn_kernel),
+                                                          dim3((unsigned)(d->B * d->H * G)), dim3(GTHREADS), args,
+                                                          G_SMEM, s);
+        return e == cudaSuccess ? launch_status() : SFA_ERR_CUDA;
+    }
+    gdn_kernel<<<(unsigned)(d->B * d->H), GTHREADS, G_SMEM, s>>>(tq, tk, tv, a);
     return launch_status();
 }

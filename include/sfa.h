@@ -354,6 +354,11 @@ sfa_status sfa_forward_blocks(const sfa_attn_desc *desc, const void *q, const vo
  *   state_out   fp32 [B][H][d][d]; may be the same buffer as state_in.
  * The tensor cores read S and the per-token corrections as bf16; the state itself is kept
  * and updated in fp32.  Supported: d = 128, any P >= 1, any T >= 1.
+ * workspace: with a device workspace of sfa_gdn_workspace bytes (256-byte aligned;
+ *   scratch, overwritten) and update != 0, the token tiles of every frame are spread over
+ *   several CTAs per (batch, head) that exchange their partial updates through it (one
+ *   cooperative launch; every wait is bounded); with NULL, one CTA per (batch, head).
+ *   The result is the same up to the order of the fp32 sums.
  */
 typedef struct {
     int32_t B, H, T, P, d;
@@ -364,9 +369,12 @@ typedef struct {
     uint32_t timeout_us; /* limit of every wait inside the kernel; 0 = 2 s */
 } sfa_gdn_desc;
 
+sfa_status sfa_gdn_workspace(const sfa_gdn_desc *desc, size_t *bytes);
+
 sfa_status sfa_gdn_forward(const sfa_gdn_desc *desc, const void *q, const void *k, const void *v,
                            const float *alpha, const float *beta, const float *state_in, float *state_out,
-                           void *o, int32_t update, int32_t *dev_status, sfa_stream_t stream);
+                           void *o, int32_t update, void *workspace, size_t workspace_bytes,
+                           int32_t *dev_status, sfa_stream_t stream);
 
 /* ------------------------------------------------------------------------------------
  * LSE merge

@@ -111,3 +111,25 @@ def test_gdn_rejects_bad_arguments():
     d64 = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(m.SfaError):
         m.gdn_forward(d64, d64, d64, a, b, 64, state_out=torch.empty(1, 1, 64, 64, device="cuda"))
+
+
+def test_gdn_tiles_spread_over_ctas_match_one_cta_per_head():
+    # 8 tiles per frame: with the workspace, 4 CTAs per head exchange partial updates every
+    # frame.  The fp32 sums run in another order, and the state is rounded to bf16 for the
+    # tensor cores every frame, so a last-bit difference can flip a bf16 rounding: both runs
+    # are held to the oracle bound, and to each other by the same bound
+    B, H, T, P = 2, 3, 4, 1000
+    q, k, v, a, b, s0 = (x.cuda() for x in _inputs(B, H, T, P, seed=11))
+    m = sfa()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o1, s1 = m.gdn_forward(q, k, v, a, b, P, state_in=s0, workspace=None)
+    o2, s2 = m.gdn_forward(q, k, v, a, b, P, state_in=s0, dev_status=status)   # several CTAs per head
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    o_ref, s_ref = _oracle(q.cpu(), k.cpu(), v.cpu(), a.cpu(), b.cpu(), P, s0.cpu())
+    tol = T * 2.0 ** -8
+    for o, s in ((o1, s1), (o2, s2)):
+        assert _rel(s.cpu().numpy(), s_ref) <= tol
+        assert _rel(o.float().cpu().numpy(), o_ref) <= tol
+    assert _rel(s2.cpu().numpy(), s1.cpu().numpy()) <= tol
+    assert _rel(o2.float().cpu().numpy(), o1.float().cpu().numpy()) <= tol
