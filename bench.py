@@ -442,8 +442,9 @@ def bench_gdn(sfa, dev, stream, flush, reps=20):
                              "cores": os.cpu_count() or 1, "kind": "oracle",
                              "sample": f"one head of the workload, all 24 frames (float64 numpy, {dt:.2f} s)"},
             "ms": round(ms, 4), "gflop": round(flop / 1e9, 3), "tflops": round(flop / (ms * 1e-3) / 1e12, 2),
-            "frac": round(flop / (ms * 1e-3) / 1e12 / peak, 4), "ctas": w.B * w.H,
-            "note": "one CTA per (batch, head): the recurrence over frames is sequential"}
+            "frac": round(flop / (ms * 1e-3) / 1e12 / peak, 4),
+            "note": "frames in order per (batch, head); each frame's tiles spread over several CTAs "
+                    "per head that exchange partial state updates (sfa_gdn_forward with a workspace)"}
 
 
 # ----------------------------------------------------------------------------- oracle timing
