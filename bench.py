@@ -210,17 +210,17 @@ def run_ours(args, rank, world, local_rank):
 
     # end to end through the public API with host buffers: H2D of Q, K, V from pinned
     # memory, sets + attention, D2H of O and LSE into pinned memory, every step
+    # (sfa.forward_host overlaps the copies of one head group with the attention of another)
     q_p, k_p, v_p = (x.pin_memory() for x in (q_h, k_h, v_h))
     o_p = torch.empty(q_h.shape, dtype=torch.bfloat16).pin_memory()
     lse_p = torch.empty((w.B, w.H, w.Lq), dtype=torch.float32).pin_memory()
 
     def e2e_step():
-        q.copy_(q_p, non_blocking=True)
-        k.copy_(k_p, non_blocking=True)
-        v.copy_(v_p, non_blocking=True)
-        step()
-        o_p.copy_(out, non_blocking=True)
-        lse_p.copy_(lse, non_blocking=True)
+        # sets on the device, then the host-to-host forward: per (batch, head-group) chunk,
+        # the copy in, the attention and the copy out run on three streams as a pipeline
+        sfa.build_sets(params, kinds, None, Amax, frames, counts, stream=stream)
+        sfa.forward_host(q_p, k_p, v_p, frames, counts, w.P, out_host=o_p, lse_host=lse_p,
+                         buffers=(q, k, v, out, lse), dev_status=status, stream=stream)
 
     e2e_step()
     torch.cuda.synchronize(dev)

@@ -415,3 +415,62 @@ def gdn_forward(q, k, v, alpha, beta, P: int, state_in=None, state_out=None, out
                                   1 if update else 0, ws_ptr, ws_bytes, _ptr(dev_status), _stream(stream)),
            "sfa_gdn_forward")
     return out, state_out
+
+
+def forward_host(q_host, k_host, v_host, frames, counts, P: int, out_host=None, lse_host=None, n_chunks: int = 6,
+                 scale: float | None = None, device=None, buffers=None, dev_status=None, stream=None):
+    """Frame-sparse attention of host tensors: (O, LSE) back in pinned host memory.
+
+    q_host, k_host, v_host: pinned bf16 CPU tensors [B, H, L, d]; frames / counts as for
+    ``forward`` (device).  The (batch, head-group) chunks run as a pipeline on three
+    streams: the copy of chunk i+1 to the GPU and of chunk i-1 back overlap the attention
+    of chunk i.  The whole call is ordered after the work already queued on ``stream``
+    and ``stream`` waits for it to finish, like a single kernel on that stream.
+    ``buffers``: optional device tensors (q, k, v, out, lse) to reuse between calls."""
+    B, H, Lq, d = q_host.shape
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    if out_host is None:
+        out_host = torch.empty(q_host.shape, dtype=torch.bfloat16).pin_memory()
+    if lse_host is None:
+        lse_host = torch.empty((B, H, Lq), dtype=torch.float32).pin_memory()
+    own = buffers is None
+    if own:
+        buffers = (torch.empty(q_host.shape, dtype=torch.bfloat16, device=device),
+                   torch.empty(k_host.shape, dtype=torch.bfloat16, device=device),
+                   torch.empty(v_host.shape, dtype=torch.bfloat16, device=device),
+                   torch.empty(q_host.shape, dtype=torch.bfloat16, device=device),
+                   torch.empty((B, H, Lq), dtype=torch.float32, device=device))
+    q, k, v, out, lse = buffers
+    main = torch.cuda.current_stream(device) if stream is None else stream
+    per_b = max(1, min(H, n_chunks // B if n_chunks >= B else 1))
+    bounds = [(b, (H * i) // per_b, (H * (i + 1)) // per_b) for b in range(B) for i in range(per_b)]
+    s_in, s_run, s_out = (torch.cuda.Stream(device) for _ in range(3))
+    start = torch.cuda.Event()
+    start.record(main)
+    for s in (s_in, s_run, s_out):
+        s.wait_event(start)
+    if own:  # the side streams use these buffers after this call returns
+        for t in buffers:
+            for s in (s_in, s_run, s_out):
+                t.record_stream(s)
+    for b, h0, h1 in bounds:
+        sl = (slice(b, b + 1), slice(h0, h1))
+        with torch.cuda.stream(s_in):
+            for dst, src in ((q, q_host), (k, k_host), (v, v_host)):
+                dst[sl].copy_(src[sl], non_blocking=True)
+            e_in = torch.cuda.Event()
+            e_in.record(s_in)
+        s_run.wait_event(e_in)
+        forward(q[sl], k[sl], v[sl], frames[h0:h1], counts[h0:h1], P, scale=scale, out=out[sl], lse=lse[sl],
+                dev_status=dev_status, stream=s_run)
+        e_run = torch.cuda.Event()
+        e_run.record(s_run)
+        s_out.wait_event(e_run)
+        with torch.cuda.stream(s_out):
+            out_host[sl].copy_(out[sl], non_blocking=True)
+            lse_host[sl].copy_(lse[sl], non_blocking=True)
+    for s in (s_in, s_run, s_out):
+        end = torch.cuda.Event()
+        end.record(s)
+        main.wait_event(end)
+    return out_host, lse_host

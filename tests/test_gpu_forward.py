@@ -175,3 +175,18 @@ def test_stream_sampled():
         rows.append(h * w.Lq + 1 * w.P + np.arange(w.P))
     rows = np.unique(np.concatenate(rows)).astype(np.int64)
     run_and_check(w, q, k, v, rows=rows)
+
+
+def test_forward_host_pipeline_equals_device_forward():
+    # the host-to-host call (copies pipelined with the attention over head groups) gives
+    # exactly the device call's result
+    w = Workload("host", B=2, H=5, Tq=3, Tkv=5, q_off=2, P=200, d=128, n_sink=1, n_prev=1, chunk_len=1,
+                 heads=(SetSpec("anchor"),) * 5)
+    q, k, v = workload_qkv(w, seed=12)
+    fr, cn = gpu_sets(w)
+    o_ref, l_ref = sfa().forward(q.cuda(), k.cuda(), v.cuda(), fr, cn, w.P)
+    qp, kp, vp = (x.pin_memory() for x in (q, k, v))
+    for n_chunks in (1, 3, 7):
+        o, l = sfa().forward_host(qp, kp, vp, fr, cn, w.P, n_chunks=n_chunks)
+        torch.cuda.synchronize()
+        assert torch.equal(o, o_ref.cpu()) and torch.equal(l, l_ref.cpu())
