@@ -13,11 +13,14 @@
 //   KS = K_i S           (same)
 //   S_acc += K_i^T U_i   (M = d, N = d, K = 128 tokens), U_i = diag(beta) (V_i - KS)
 // G CTAs per (batch, head) run the frames in order (the recurrence is sequential); CTA g
-// takes tiles g, g + G, ... of every frame.  With G > 1 each CTA writes its partial
-// S_acc to a workspace, the G CTAs of a head meet at a counter in global memory (one
-// cooperative launch, so all CTAs are resident; the wait is bounded), and each CTA adds
-// the G partials itself (double-buffered by frame parity, so one meeting per frame is
-// enough).  Warps 0-3 (one thread per TMEM lane) read O and KS out of tensor memory,
+// takes tiles g, g + G, ... of every frame.  With G > 1 each CTA adds its partial S_acc
+// into one fp32 sum per head with a bulk reduce-add (cp.reduce.async.bulk, performed in
+// L2), the G CTAs of a head meet at a counter in global memory (one cooperative launch,
+// so all CTAs are resident; the wait is bounded), and each reads the sum back.  The sums
+// rotate over three buffers by frame: buffer n mod 3 is summed into in frame n, and CTA 0
+// zeroes buffer (n + 2) mod 3 after the meeting of frame n, when every CTA has finished
+// reading it (frame n - 1) and none can add into it yet (frame n + 2 comes after the next
+// meeting); one meeting per frame is enough.  Warps 0-3 (one thread per TMEM lane) read O and KS out of tensor memory,
 // write O, form U in shared memory and update the fp32 state; warp 4 issues the TMA
 // copies and MMAs.
 // Tensor memory: O, KS, S_acc and the fp32 state, 128 columns each.  Every wait is
@@ -49,7 +52,7 @@ constexpr uint32_t T_O = 0, T_KS = 128, T_SACC = 256, T_SST = 384;  // tensor-me
 struct GdnArgs {
     int32_t B, H, T, P, n_tiles, update;
     int32_t G;           // CTAs per (batch, head)
-    float *part;         // [2][B*H][G][d][d] partial S_acc (G > 1)
+    float *part;         // [3][B*H][d][d] sums of the partial S_acc (G > 1), zero at launch
     uint32_t *count;     // [B*H] arrivals (G > 1), zero at launch
     const float *alpha;  // [B][H][T]
     const float *beta;   // [B][H][T*P]
@@ -293,8 +296,10 @@ __global__ void __launch_bounds__(GTHREADS, 1)
             if (!ok) break;
             tc_fence_after();
             if (a.update && a.G > 1) {
-                // this CTA's partial out, meet the head's other CTAs, then add all partials
-                float *mine = a.part + ((((int64_t)(n & 1) * a.B * a.H + bh) * a.G + g) * GD + r) * GD;
+                // this CTA's partial, staged row-major in the free Q/K tiles, added into the
+                // head's sum in L2; then meet the head's other CTAs
+                float *stage = reinterpret_cast<float *>(smem + G_Q);
+                float *sum = a.part + ((int64_t)(n % 3) * a.B * a.H + bh) * GD * GD;
 #pragma unroll
                 for (int c = 0; c < GD / 32; ++c) {
                     uint32_t acc[32];
@@ -302,13 +307,16 @@ __global__ void __launch_bounds__(GTHREADS, 1)
                     tmem_wait_ld_regs(acc);
 #pragma unroll
                     for (int j = 0; j < 32; j += 4)
-                        __stcg(reinterpret_cast<float4 *>(mine + c * 32 + j),
-                               make_float4(__uint_as_float(acc[j]), __uint_as_float(acc[j + 1]),
-                                           __uint_as_float(acc[j + 2]), __uint_as_float(acc[j + 3])));
+                        *reinterpret_cast<float4 *>(stage + r * GD + c * 32 + j) =
+                            make_float4(__uint_as_float(acc[j]), __uint_as_float(acc[j + 1]),
+                                        __uint_as_float(acc[j + 2]), __uint_as_float(acc[j + 3]));
                 }
-                __threadfence();
+                fence_proxy_async_smem();
                 named_bar_sync(1, 128);
                 if (r == 0) {
+                    bulk_reduce_add_f32(sum, sbase + G_Q, GD * GD * 4);
+                    bulk_commit_and_wait_all();
+                    __threadfence();
                     atomicAdd(a.count + bh, 1u);
                     const uint32_t want = (uint32_t)a.G * (uint32_t)(n + 1);
                     const uint64_t t0 = gns();
@@ -327,10 +335,16 @@ __global__ void __launch_bounds__(GTHREADS, 1)
                     ok = false;
                     break;
                 }
+                if (g == 0) {  // buffer (n + 2) mod 3: read by every CTA in frame n - 1, next summed into in frame n + 2
+                    float *z = a.part + ((int64_t)((n + 2) % 3) * a.B * a.H + bh) * GD * GD + r * GD;
+#pragma unroll
+                    for (int j = 0; j < GD; j += 4) __stcg(reinterpret_cast<float4 *>(z + j), make_float4(0.f, 0.f, 0.f, 0.f));
+                    __threadfence();  // visible before this CTA's next arrival
+                }
             }
             if (a.update) {
                 const float al = a.alpha[bhi * a.T + n];
-                const float *parts = a.part + (((int64_t)(n & 1) * a.B * a.H + bh) * a.G * GD + r) * GD;
+                const float *sumrow = a.part + (((int64_t)(n % 3) * a.B * a.H + bh) * GD + r) * GD;
 #pragma unroll
                 for (int c = 0; c < GD / 32; ++c) {
                     uint32_t s[32], acc[32];
@@ -338,17 +352,12 @@ __global__ void __launch_bounds__(GTHREADS, 1)
                     tmem_wait_ld_regs(s);
                     if (a.G > 1) {
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) acc[j] = 0u;
-                        for (int gg = 0; gg < a.G; ++gg) {
-                            const float *src = parts + (int64_t)gg * GD * GD + c * 32;
-#pragma unroll
-                            for (int j = 0; j < 32; j += 4) {
-                                const float4 v4 = __ldcg(reinterpret_cast<const float4 *>(src + j));
-                                acc[j] = __float_as_uint(__uint_as_float(acc[j]) + v4.x);
-                                acc[j + 1] = __float_as_uint(__uint_as_float(acc[j + 1]) + v4.y);
-                                acc[j + 2] = __float_as_uint(__uint_as_float(acc[j + 2]) + v4.z);
-                                acc[j + 3] = __float_as_uint(__uint_as_float(acc[j + 3]) + v4.w);
-                            }
+                        for (int j = 0; j < 32; j += 4) {
+                            const float4 v4 = __ldcg(reinterpret_cast<const float4 *>(sumrow + c * 32 + j));
+                            acc[j] = __float_as_uint(v4.x);
+                            acc[j + 1] = __float_as_uint(v4.y);
+                            acc[j + 2] = __float_as_uint(v4.z);
+                            acc[j + 3] = __float_as_uint(v4.w);
                         }
                     } else {
                         tmem_ld32(lane_base + T_SACC + c * 32, acc);
@@ -450,9 +459,9 @@ int gdn_split(const sfa_gdn_desc *d)
     return std::max(G, 1);
 }
 
-size_t gdn_part_bytes(const sfa_gdn_desc *d, int G)
+size_t gdn_part_bytes(const sfa_gdn_desc *d, int)
 {
-    return ((size_t)2 * d->B * d->H * G * GD * GD * 4 + 255) / 256 * 256;
+    return ((size_t)3 * d->B * d->H * GD * GD * 4 + 255) / 256 * 256;
 }
 
 }  // namespace
@@ -522,7 +531,7 @@ extern "C" sfa_status sfa_gdn_forward(const sfa_gdn_desc *d, const void *q, cons
         if (workspace_bytes < need || reinterpret_cast<uintptr_t>(workspace) % 256) return SFA_ERR_INVALID_ARG;
         a.part = static_cast<float *>(workspace);
         a.count = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(workspace) + pb);
-        if (cudaMemsetAsync(a.count, 0, (size_t)d->B * d->H * 4, s) != cudaSuccess) return SFA_ERR_CUDA;
+        if (cudaMemsetAsync(workspace, 0, need, s) != cudaSuccess) return SFA_ERR_CUDA;  // sums and counters
         // the G CTAs of a head wait for one another: one cooperative launch keeps them all resident
         void *args[] = {&tq, &tk, &tv, &a};
         const cudaError_t e = cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(gdn_kernel),

@@ -98,6 +98,24 @@ __device__ __forceinline__ void tma_store_5d(const void *tmap, uint32_t src, int
 
 __device__ __forceinline__ void tma_store_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 
+// dst[i] += src[i] for `bytes` / 4 floats (global dst, shared src; 16-byte aligned, a
+// multiple of 16 bytes), performed by the async proxy in L2
+__device__ __forceinline__ void bulk_reduce_add_f32(float *dst, uint32_t src, uint32_t bytes)
+{
+    asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(dst), "r"(src),
+                 "r"(bytes)
+                 : "memory");
+}
+
+// commit the pending bulk operations and wait until they are complete, writes included,
+// then order them before this thread's later global accesses
+__device__ __forceinline__ void bulk_commit_and_wait_all()
+{
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 __device__ __forceinline__ void tma_store_wait_read_all()
 {
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
