@@ -19,7 +19,9 @@
 //     tile), O += P V with P read from shared memory (both operands in shared memory: the
 //     tensor-memory-A form of this MMA runs at ~0.6x the rate on sm_100); a partial last
 //     tile uses an MMA N (for S) and K (for P V) rounded up to 16 only.  While the
-//     softmax of one tile runs, the tensor cores work on the other;
+//     softmax of one tile runs, the tensor cores work on the other.  A CTA with a single
+//     query tile (the last tile of a frame with an odd tile count) uses the idle tile's S
+//     and P buffers as second buffers and runs S two key tiles ahead instead;
 //   * warps 0-3 (tile A) and 4-7 (tile B), one thread per query row = TMEM lane, run the
 //     online softmax in fp32 (exp2 with the scale folded into one FMA; O is rescaled only
 //     when a row's running max grows by more than 2^8, otherwise the stale max is kept),
@@ -78,7 +80,7 @@ struct Cfg {
     static constexpr int SMEM_V = SMEM_K + NSK * TILE_BYTES;
     static constexpr int SMEM_BAR = SMEM_V + NSV * TILE_BYTES;
     static constexpr int SMEM_BYTES = SMEM_BAR + 256 + 1024;  // + barriers, + alignment slack
-    static_assert(2 * NSK + 2 * NSV + 7 <= 20, "mbarriers must fit in 160 bytes");
+    static_assert(2 * NSK + 2 * NSV + 8 <= 20, "mbarriers must fit in 160 bytes");
     static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 };
 
@@ -95,7 +97,8 @@ struct Bars {
     __device__ uint32_t p_full(int x) const { return q_full() + 24 + 8 * x; }  // P of query tile x in smem
     __device__ uint32_t o_final() const { return q_full() + 40; }              // after the last P V
     __device__ uint32_t drain() const { return q_full() + 48; }
-    static constexpr int COUNT = 2 * Cfg<D>::NSK + 2 * Cfg<D>::NSV + 7;
+    __device__ uint32_t pv_done() const { return q_full() + 56; }  // one-tile CTAs: a P V complete
+    static constexpr int COUNT = 2 * Cfg<D>::NSK + 2 * Cfg<D>::NSV + 8;
 };
 
 struct FwdArgs {
@@ -464,6 +467,88 @@ done:
     __syncwarp();
 }
 
+// The tensor-core schedule of a CTA with one query tile (the last, partial tile of a frame
+// with an odd number of tiles): the other tile's S and P buffers serve as second buffers,
+// S runs two key tiles ahead of the softmax,
+//   S(0) S(1) | P V(j) S(j+2) | ...
+// so the softmax of tile j+1 starts as soon as it has finished tile j.  S(j+2) goes into
+// the buffer the softmax of tile j has read out; P of tile j+2 is written only after
+// S(j+2) completes, hence after P V(j).  The softmax rescales O only after P V of the
+// previous tile is complete (pv_done).
+template <int D>
+__device__ void mma_single(const FwdArgs &a, uint32_t sbase, uint32_t tmem, int h, const int32_t *fl, int cnt,
+                           int t_off, int n_tiles, const Ctl &ctl)
+{
+    using C = Cfg<D>;
+    const Bars<D> bar{sbase + C::SMEM_BAR};
+    if (n_tiles <= 0) return;
+    const uint64_t dq = sdesc_sw128(sbase + C::SMEM_Q, 16, 1024);
+    const uint64_t dk = sdesc_sw128(sbase + C::SMEM_K, 16, 1024);
+    const uint64_t dv = sdesc_sw128(sbase + C::SMEM_V, C::BOX_BYTES, 1024);
+    const uint64_t dp = sdesc_sw128(sbase + C::SMEM_P, 16, 1024);
+    bool issued = false;
+    KvIter it;
+    it.init(fl, cnt, a.P, a.slots ? a.slots + (int64_t)h * a.T_kv : nullptr, a.nblk);
+    it.skip(t_off);
+    int st, nv_j = 0, nv_j1 = 0, nv_j2 = 0;  // valid keys of tiles j, j+1, j+2
+    it.next(st, nv_j);
+    if (n_tiles > 1) it.next(st, nv_j1);
+    if (!__all_sync(0xffffffffu, wait_bar(bar.q_full(), 0, ctl))) goto done;
+    for (int j = 0; j < 2 && j < n_tiles; ++j) {
+        const int sk = j % C::NSK;
+        if (!__all_sync(0xffffffffu, wait_bar(bar.k_full(sk), (j / C::NSK) & 1, ctl))) goto done;
+        tc_fence_after();
+        issue_s<D>(tmem + tcol_s(j), dq, desc_add(dk, sk * C::TILE_BYTES),
+                   idesc_bf16_f32(BM, mma_n(j ? nv_j1 : nv_j), false));
+        commit_one(bar.s_full(j));
+        commit_one(bar.k_free(sk));
+        issued = true;
+    }
+    for (int j = 0; j < n_tiles; ++j) {
+        const int bj = j & 1, sv = j % C::NSV, nvj = nv_j;
+        nv_j2 = 0;
+        if (j + 2 < n_tiles) it.next(st, nv_j2);
+        if (!__all_sync(0xffffffffu, wait_bar(bar.p_full(bj), (j >> 1) & 1, ctl))) goto done;
+        if (!__all_sync(0xffffffffu, wait_bar(bar.v_full(sv), (j / C::NSV) & 1, ctl))) goto done;
+        if (nvj & 15) {
+            // P V reads V up to the next multiple of 16 keys, where P is 0; those few rows
+            // hold whatever follows the run in memory, so they are zeroed first
+            const int r0 = nvj, r1 = (nvj + 15) & ~15;
+            const uint32_t vslot = sbase + C::SMEM_V + sv * C::TILE_BYTES;
+            const uint32_t zero[4] = {0u, 0u, 0u, 0u};
+            for (int idx = (int)(threadIdx.x & 31); idx < (r1 - r0) * C::KBOX * 8; idx += 32) {
+                const int r = r0 + idx / (C::KBOX * 8), kb = (idx / 8) % C::KBOX, ch = idx % 8;
+                st_shared_v4(vslot + kb * C::BOX_BYTES + r * 128 + ch * 16, zero);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+        }
+        tc_fence_after();
+        issue_pv<D>(tmem + tcol_o(0), desc_add(dp, bj * C::P_BYTES), desc_add(dv, sv * C::TILE_BYTES), mma_n(nvj),
+                    j > 0);
+        commit_one(bar.pv_done());
+        commit_one(bar.v_free(sv));
+        if (j == n_tiles - 1) commit_one(bar.o_final());
+        if (j + 2 < n_tiles) {
+            const int sk = (j + 2) % C::NSK;
+            if (!__all_sync(0xffffffffu, wait_bar(bar.k_full(sk), ((j + 2) / C::NSK) & 1, ctl))) goto done;
+            tc_fence_after();
+            issue_s<D>(tmem + tcol_s(bj), dq, desc_add(dk, sk * C::TILE_BYTES),
+                       idesc_bf16_f32(BM, mma_n(nv_j2), false));
+            commit_one(bar.s_full(bj));
+            commit_one(bar.k_free(sk));
+        }
+        nv_j = nv_j1;
+        nv_j1 = nv_j2;
+    }
+done:
+    if (__any_sync(0xffffffffu, *ctl.abort != 0) && issued) {  // wait for the tensor cores before TMEM is released
+        commit_one(bar.drain());
+        wait_drain(bar.drain(), 0);
+    }
+    __syncwarp();
+}
+
 // Max of 32 values with 3-input max in a tree (depth 4).
 __device__ __forceinline__ float max32(const uint32_t (&r)[32])
 {
@@ -536,8 +621,8 @@ __device__ __forceinline__ float sum8(const float (&acc)[8])
 // take the exact two-pass path: row max first, then P (S is re-read from TMEM; P lives
 // in shared memory), and O is rescaled in place.  FULL: all 128 keys valid.
 template <int D, bool FULL>
-__device__ __forceinline__ void softmax_tile(uint32_t t_s, uint32_t p_row, int row, uint32_t t_o, int nv, float sl2,
-                                             float &m_used, float &l, int j)
+__device__ __forceinline__ bool softmax_tile(uint32_t t_s, uint32_t p_row, int row, uint32_t t_o, int nv, float sl2,
+                                             float &m_used, float &l, int j, uint32_t pv_done, const Ctl &ctl)
 {
     const int nch = FULL ? 4 : (nv + 31) >> 5;
     if (j > 0) {  // streaming pass against the current max
@@ -561,7 +646,7 @@ __device__ __forceinline__ void softmax_tile(uint32_t t_s, uint32_t p_row, int r
         }
         if (!__any_sync(0xffffffffu, grow)) {
             l += sum8(acc);
-            return;
+            return true;
         }
     }
     // exact pass: row max over the tile, then P against the new max
@@ -591,6 +676,11 @@ __device__ __forceinline__ void softmax_tile(uint32_t t_s, uint32_t p_row, int r
     // together (tcgen05.ld/st are warp-wide).  P V of the previous tile is already done:
     // S of this tile was issued after it, and its completion was waited for.
     if (j > 0 && __any_sync(0xffffffffu, resc)) {
+        // (one-tile CTAs run S two tiles ahead: P V of the previous tile may still run)
+        if (pv_done) {
+            if (!__all_sync(0xffffffffu, wait_bar(pv_done, (j - 1) & 1, ctl))) return false;
+            tc_fence_after();
+        }
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
@@ -603,6 +693,7 @@ __device__ __forceinline__ void softmax_tile(uint32_t t_s, uint32_t p_row, int r
     }
     l = l * alpha + sum8(acc);
     m_used = m_new;
+    return true;
 }
 
 // Softmax and epilogue of query tile x (0: warps 0-3, 1: warps 4-7), one thread per
@@ -610,7 +701,7 @@ __device__ __forceinline__ void softmax_tile(uint32_t t_s, uint32_t p_row, int r
 template <int D>
 __device__ void softmax_role(const CUtensorMap *tm_o, const FwdArgs &a, uint8_t *smem, uint32_t sbase,
                              uint32_t tmem, int x, int b, int b_out, int h, int t, int qt, const int32_t *fl,
-                             int cnt, int t_off, int n_tiles, bool bad_set, const Ctl &ctl)
+                             int cnt, int t_off, int n_tiles, bool bad_set, bool one_tile, const Ctl &ctl)
 {
     using C = Cfg<D>;
     const Bars<D> bar{sbase + C::SMEM_BAR};
@@ -619,8 +710,7 @@ __device__ void softmax_role(const CUtensorMap *tm_o, const FwdArgs &a, uint8_t 
     const int row = threadIdx.x & 127;  // query row inside the tile == TMEM lane
     const int warp = (threadIdx.x >> 5) & 3;
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-    const uint32_t t_s = lane_base + tcol_s(x), t_o = lane_base + tcol_o(x);
-    const uint32_t p_row = sbase + C::SMEM_P + x * C::P_BYTES + row * 128;
+    const uint32_t t_o = lane_base + tcol_o(x);
     const float sl2 = a.scale_log2;
 
     float m_used = -INFINITY;  // running row max (log2 units, scale folded in)
@@ -632,19 +722,29 @@ __device__ void softmax_role(const CUtensorMap *tm_o, const FwdArgs &a, uint8_t 
     for (int j = 0; j < n_tiles; ++j) {
         int st, nv;
         it.next(st, nv);
-        // S of tile j has one pending phase: S of tile j+1 waits for P of tile j
-        const bool got = wait_bar(bar.s_full(x), j & 1, ctl);
+        // S and P buffers: the tile's own, or (a CTA with one query tile) both tiles'
+        // buffers in turn, S two tiles ahead.  Either way one pending phase per buffer.
+        const int xb = one_tile ? (j & 1) : x;
+        const uint32_t par = one_tile ? (uint32_t)(j >> 1) & 1 : (uint32_t)j & 1;
+        const uint32_t t_s = lane_base + tcol_s(xb);
+        const uint32_t p_row = sbase + C::SMEM_P + xb * C::P_BYTES + row * 128;
+        const bool got = wait_bar(bar.s_full(xb), par, ctl);
         if (!__all_sync(0xffffffffu, got)) {
             alive = false;
             break;
         }
         tc_fence_after();
-        if (nv >= BN) softmax_tile<D, true>(t_s, p_row, row, t_o, nv, sl2, m_used, l, j);
-        else softmax_tile<D, false>(t_s, p_row, row, t_o, nv, sl2, m_used, l, j);
+        const uint32_t pvw = one_tile ? bar.pv_done() : 0u;
+        const bool ok = nv >= BN ? softmax_tile<D, true>(t_s, p_row, row, t_o, nv, sl2, m_used, l, j, pvw, ctl)
+                                 : softmax_tile<D, false>(t_s, p_row, row, t_o, nv, sl2, m_used, l, j, pvw, ctl);
+        if (!ok) {
+            alive = false;
+            break;
+        }
         tmem_wait_st();            // O rescale stores, if any
         fence_proxy_async_smem();  // P written with st.shared is read by the tensor cores
         tc_fence_before();
-        if (!((a.debug_flags & SFA_DEBUG_STALL_SOFTMAX) && j == 0)) mbar_arrive(bar.p_full(x));
+        if (!((a.debug_flags & SFA_DEBUG_STALL_SOFTMAX) && j == 0)) mbar_arrive(bar.p_full(xb));
     }
 
     // ---- epilogue: O / l -> bf16 -> swizzled smem (this tile's Q space) -> TMA store
@@ -785,12 +885,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     } else if (warp == V_LOAD_WARP) {
         loader_role<D, false>(&tm_q, &tm_v, a, sbase, b, h, t, qt_a, has_b, fl, cnt, t_off, n_tiles, ctl);
     } else if (warp == MMA_WARP) {
-        mma_role<D>(a, sbase, tmem, h, has_b, fl, cnt, t_off, n_tiles, ctl);
+        if (has_b) mma_role<D>(a, sbase, tmem, h, has_b, fl, cnt, t_off, n_tiles, ctl);
+        else mma_single<D>(a, sbase, tmem, h, fl, cnt, t_off, n_tiles, ctl);
     } else if (warp < 8) {
         const int xt = warp >> 2;  // query tile of this softmax warpgroup
         if (!skipped && (xt == 0 || has_b))
             softmax_role<D>(&tm_o, a, smem, sbase, tmem, xt, b, b_out, h, t, qt_a + xt, fl, cnt, t_off, n_tiles,
-                            bad_set, ctl);
+                            bad_set, !has_b, ctl);
     }
 
     tc_fence_before();
