@@ -417,14 +417,16 @@ def gdn_forward(q, k, v, alpha, beta, P: int, state_in=None, state_out=None, out
     return out, state_out
 
 
-def forward_host(q_host, k_host, v_host, frames, counts, P: int, out_host=None, lse_host=None, n_chunks: int = 6,
-                 scale: float | None = None, device=None, buffers=None, dev_status=None, stream=None):
+def forward_host(q_host, k_host, v_host, frames, counts, P: int, out_host=None, lse_host=None, n_chunks: int = 12,
+                 scale: float | None = None, device=None, buffers=None, dev_status=None, stream=None,
+                 compute_streams: int = 2):
     """Frame-sparse attention of host tensors: (O, LSE) back in pinned host memory.
 
     q_host, k_host, v_host: pinned bf16 CPU tensors [B, H, L, d]; frames / counts as for
-    ``forward`` (device).  The (batch, head-group) chunks run as a pipeline on three
-    streams: the copy of chunk i+1 to the GPU and of chunk i-1 back overlap the attention
-    of chunk i.  The whole call is ordered after the work already queued on ``stream``
+    ``forward`` (device).  The (batch, head-group) chunks run as a pipeline: the copy of
+    chunk i+1 to the GPU and of chunk i-1 back overlap the attention of chunk i, and the
+    attention of consecutive chunks alternates between ``compute_streams`` streams so
+    that the last wave of one kernel overlaps the first of the next.  The whole call is ordered after the work already queued on ``stream``
     and ``stream`` waits for it to finish, like a single kernel on that stream.
     ``buffers``: optional device tensors (q, k, v, out, lse) to reuse between calls."""
     B, H, Lq, d = q_host.shape
@@ -444,16 +446,18 @@ def forward_host(q_host, k_host, v_host, frames, counts, P: int, out_host=None, 
     main = torch.cuda.current_stream(device) if stream is None else stream
     per_b = max(1, min(H, n_chunks // B if n_chunks >= B else 1))
     bounds = [(b, (H * i) // per_b, (H * (i + 1)) // per_b) for b in range(B) for i in range(per_b)]
-    s_in, s_run, s_out = (torch.cuda.Stream(device) for _ in range(3))
+    s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    s_runs = [torch.cuda.Stream(device) for _ in range(max(1, compute_streams))]
     start = torch.cuda.Event()
     start.record(main)
-    for s in (s_in, s_run, s_out):
+    for s in [s_in, s_out] + s_runs:
         s.wait_event(start)
     if own:  # the side streams use these buffers after this call returns
         for t in buffers:
-            for s in (s_in, s_run, s_out):
+            for s in [s_in, s_out] + s_runs:
                 t.record_stream(s)
-    for b, h0, h1 in bounds:
+    for c, (b, h0, h1) in enumerate(bounds):
+        s_run = s_runs[c % len(s_runs)]
         sl = (slice(b, b + 1), slice(h0, h1))
         with torch.cuda.stream(s_in):
             for dst, src in ((q, q_host), (k, k_host), (v, v_host)):
@@ -469,7 +473,7 @@ def forward_host(q_host, k_host, v_host, frames, counts, P: int, out_host=None, 
         with torch.cuda.stream(s_out):
             out_host[sl].copy_(out[sl], non_blocking=True)
             lse_host[sl].copy_(lse[sl], non_blocking=True)
-    for s in (s_in, s_run, s_out):
+    for s in [s_in, s_out] + s_runs:
         end = torch.cuda.Event()
         end.record(s)
         main.wait_event(end)
