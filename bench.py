@@ -364,6 +364,10 @@ def bench_hsa(sfa, dev, stream, flush, reps=20):
 
     sel_ms = timed(lambda: sfa.hsa_select(q, k, params, w.k_frames, w.k_blocks, workspace=wsp, stream=stream))
     fwd_ms = timed(lambda: sfa.forward_blocks(q, k, v, blocks, counts, w.P, out=o, lse=lse, stream=stream))
+    # 252 CTAs are 1.7 waves of 148 SMs: the split form balances them
+    split_ws = torch.empty(max(sfa.split_workspace_bytes(desc, 2), 1), dtype=torch.uint8, device=dev)
+    fwd2_ms = timed(lambda: sfa.forward_blocks(q, k, v, blocks, counts, w.P, out=o, lse=lse, stream=stream,
+                                               n_split=2, workspace=split_ws))
     flops = block_list_flops(blocks.cpu().numpy(), counts.cpu().numpy(), w.P, w.d)
     peak = float(measured_peaks()["bf16_tflops"])
     tf = flops / (fwd_ms * 1e-3) / 1e12
@@ -387,6 +391,8 @@ def bench_hsa(sfa, dev, stream, flush, reps=20):
             "select_ms": round(sel_ms, 4), "select_pool_bytes": pool_bytes,
             "forward_blocks_ms": round(fwd_ms, 4), "attended_tflop": round(flops / 1e12, 4),
             "forward_tflops": round(tf, 1), "forward_frac": round(tf / peak, 4),
+            "forward_blocks_split2_ms": round(fwd2_ms, 4),
+            "forward_split2_tflops": round(flops / (fwd2_ms * 1e-3) / 1e12, 1),
             "step_tflops": round(flops / ((sel_ms + fwd_ms) * 1e-3) / 1e12, 1),
             "mean_blocks_per_list": round(float(counts.float().mean().item()), 2),
             "roofline": {"forward_blocks": {"bound": "tensor", "achieved": round(tf, 1), "peak": peak,

@@ -59,6 +59,7 @@ class GdnDesc(ctypes.Structure):
 EXPORTS = ("sfa_error_string", "sfa_version", "sfa_set_max_count", "sfa_build_sets", "sfa_forward",
            "sfa_forward_split_workspace", "sfa_forward_split", "sfa_forward_split_noalloc", "sfa_forward_paged",
            "sfa_lse_merge", "sfa_hsa_max_count", "sfa_hsa_workspace", "sfa_hsa_select", "sfa_forward_blocks",
+           "sfa_forward_blocks_split",
            "sfa_forward_dual_workspace", "sfa_forward_dual", "sfa_gdn_workspace", "sfa_gdn_forward")
 
 
@@ -112,6 +113,9 @@ def load():
     lib.sfa_gdn_workspace.argtypes = [ctypes.POINTER(GdnDesc), ctypes.POINTER(ctypes.c_size_t)]
     lib.sfa_gdn_forward.argtypes = [ctypes.POINTER(GdnDesc), vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, ctypes.c_size_t,
                                     vp, vp]
+    lib.sfa_forward_blocks_split.restype = st
+    lib.sfa_forward_blocks_split.argtypes = [ctypes.POINTER(AttnDesc), vp, vp, vp, vp, vp, vp, vp, i32, vp,
+                                             ctypes.c_size_t, vp, vp]
     lib.sfa_forward_blocks.restype = st
     lib.sfa_forward_blocks.argtypes = [ctypes.POINTER(AttnDesc), vp, vp, vp, vp, vp, vp, vp, vp, vp]
     _lib = lib
@@ -329,7 +333,7 @@ def hsa_select(q, k, params: SetParams, k_frames: int, k_blocks: int, Amax: int 
 
 
 def forward_blocks(q, k, v, blocks, counts, P: int, scale: float | None = None, out=None, lse=None,
-                   dev_status=None, stream=None, timeout_us: int = 0):
+                   dev_status=None, stream=None, timeout_us: int = 0, n_split: int = 1, workspace=None):
     """Attention of every query block over its key-block list: (O bf16 like q, LSE fp32)."""
     B, H, Lq, d = q.shape
     if out is None:
@@ -342,9 +346,17 @@ def forward_blocks(q, k, v, blocks, counts, P: int, scale: float | None = None, 
     desc = attn_desc(q, k, v, out, P, blocks.shape[-1], scale, timeout_us)
     nqb = (P + QUERY_BLOCK - 1) // QUERY_BLOCK
     assert tuple(blocks.shape[:4]) == (B, H, desc.Tq, nqb) and tuple(counts.shape) == (B, H, desc.Tq, nqb)
-    _check(load().sfa_forward_blocks(ctypes.byref(desc), q.data_ptr(), k.data_ptr(), v.data_ptr(),
-                                     blocks.data_ptr(), counts.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                                     _ptr(dev_status), _stream(stream)), "sfa_forward_blocks")
+    if n_split == 1:
+        _check(load().sfa_forward_blocks(ctypes.byref(desc), q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                         blocks.data_ptr(), counts.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                         _ptr(dev_status), _stream(stream)), "sfa_forward_blocks")
+        return out, lse
+    if workspace is None:
+        workspace = torch.empty(max(split_workspace_bytes(desc, n_split), 1), dtype=torch.uint8, device=q.device)
+    _check(load().sfa_forward_blocks_split(ctypes.byref(desc), q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                           blocks.data_ptr(), counts.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                           n_split, workspace.data_ptr(), workspace.numel(), _ptr(dev_status),
+                                           _stream(stream)), "sfa_forward_blocks_split")
     return out, lse
 
 

@@ -1219,6 +1219,35 @@ extern "C" sfa_status sfa_forward_dual(const sfa_attn_desc *d, const void *q, co
 // Key-block lists (hierarchical selection): each (b, h, t, query block of 256 rows) has
 // its own sorted list of 128-token key blocks.
 // ------------------------------------------------------------------------------------
+extern "C" sfa_status sfa_forward_blocks_split(const sfa_attn_desc *d, const void *q, const void *k, const void *v,
+                                               const int32_t *blocks, const int32_t *counts, void *o, float *lse,
+                                               int32_t n_split, void *workspace, size_t workspace_bytes,
+                                               int32_t *dev_status, sfa_stream_t stream)
+{
+    sfa_status st = check_desc(d);
+    if (st != SFA_OK) return st;
+    if ((int64_t)d->T_kv * ((d->P + KEY_BLOCK - 1) / KEY_BLOCK) >= ((int64_t)1 << 31)) return SFA_ERR_INVALID_ARG;
+    if (n_split < 1 || n_split > d->d / 8) return SFA_ERR_INVALID_ARG;
+    if (d->B == 0) return SFA_OK;
+    st = check_buffers(d, q, k, v, blocks, counts, o, lse);
+    if (st != SFA_OK) return st;
+    cudaStream_t s = as_cuda(stream);
+    const int nblk = (d->P + KEY_BLOCK - 1) / KEY_BLOCK;
+    if (n_split == 1)
+        return d->d == 128 ? launch<128>(d, q, k, v, blocks, counts, o, lse, dev_status, s, 1, nullptr, nullptr, nullptr,
+                                         0, nblk)
+                           : launch<64>(d, q, k, v, blocks, counts, o, lse, dev_status, s, 1, nullptr, nullptr, nullptr,
+                                        0, nblk);
+    const size_t need = split_ws_bytes(d, n_split);
+    if (!workspace || workspace_bytes < need || reinterpret_cast<uintptr_t>(workspace) % 256)
+        return SFA_ERR_INVALID_ARG;
+    float *ws_lse = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + split_ws_o_bytes(d, n_split));
+    return d->d == 128 ? launch<128>(d, q, k, v, blocks, counts, o, lse, dev_status, s, n_split, workspace, ws_lse,
+                                     nullptr, 0, nblk)
+                       : launch<64>(d, q, k, v, blocks, counts, o, lse, dev_status, s, n_split, workspace, ws_lse,
+                                    nullptr, 0, nblk);
+}
+
 extern "C" sfa_status sfa_forward_blocks(const sfa_attn_desc *d, const void *q, const void *k, const void *v,
                                          const int32_t *blocks, const int32_t *counts, void *o, float *lse,
                                          int32_t *dev_status, sfa_stream_t stream)

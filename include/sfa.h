@@ -334,6 +334,14 @@ sfa_status sfa_forward_blocks(const sfa_attn_desc *desc, const void *q, const vo
                               const int32_t *blocks, const int32_t *counts, void *o, float *lse,
                               int32_t *dev_status, sfa_stream_t stream);
 
+/* sfa_forward_blocks with the key tiles of every unit cut into n_split ranges and merged
+ * by LSE, as sfa_forward_split does for frame lists (workspace: the size
+ * sfa_forward_split_workspace gives for the same descriptor and n_split). */
+sfa_status sfa_forward_blocks_split(const sfa_attn_desc *desc, const void *q, const void *k, const void *v,
+                                    const int32_t *blocks, const int32_t *counts, void *o, float *lse,
+                                    int32_t n_split, void *workspace, size_t workspace_bytes,
+                                    int32_t *dev_status, sfa_stream_t stream);
+
 /* ------------------------------------------------------------------------------------
  * ARL2 inter-frame branch: gated delta rule over frames
  * ------------------------------------------------------------------------------------

@@ -165,3 +165,18 @@ def test_hsa_workload_selection_and_sampled_attention():
     o_ref, l_ref = hsa.attention_blocks(q.float().numpy(), k.float().numpy(), v.float().numpy(), lists, cnts,
                                         w.P, 1 / math.sqrt(w.d), rows=rows)
     compare(o.float().cpu().reshape(-1, w.d).numpy()[rows], lse.cpu().reshape(-1).numpy()[rows], o_ref, l_ref)
+
+
+@pytest.mark.parametrize("n_split", [2, 4])
+def test_forward_blocks_split_matches_oracle(n_split):
+    w = SMALL[0]
+    q, k, v = workload_qkv(w, seed=5)
+    Amax = sfa().hsa_max_count(_params(w), w.P, w.k_frames, w.k_blocks)
+    lists, counts = hsa.build_block_lists(q.float().numpy(), k.float().numpy(), Bmax=Amax, **_kw(w))
+    o, lse = sfa().forward_blocks(q.cuda(), k.cuda(), v.cuda(), torch.from_numpy(lists).cuda(),
+                                  torch.from_numpy(counts).cuda(), w.P, n_split=n_split)
+    torch.cuda.synchronize()
+    o_ref, l_ref = hsa.attention_blocks(q.float().numpy(), k.float().numpy(), v.float().numpy(), lists, counts,
+                                        w.P, 1 / math.sqrt(w.d))
+    compare(o.float().cpu().reshape(-1, w.d).numpy(), lse.cpu().reshape(-1).numpy(), o_ref.reshape(-1, w.d),
+            l_ref.reshape(-1))
