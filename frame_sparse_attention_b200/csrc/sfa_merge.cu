@@ -39,6 +39,8 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(int64_t rows, const uint
         // the row's first lane reads both LSEs and hands them to its group, so an
         // in-place lse write below cannot overtake another lane's read
         const unsigned group = ((1u << G) - 1u) << ((threadIdx.x % 32) & ~(G - 1));
+        const uint4 a = o1[r * G + sub];  // issued first: independent of the LSEs
+        const uint4 b = o2[r * G + sub];
         float l1 = 0.f, l2 = 0.f;
         if (sub == 0) {
             l1 = lse1[r];
@@ -46,8 +48,6 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(int64_t rows, const uint
         }
         l1 = __shfl_sync(group, l1, 0, G);
         l2 = __shfl_sync(group, l2, 0, G);
-        const uint4 a = o1[r * G + sub];
-        const uint4 b = o2[r * G + sub];
         const float m = fmaxf(l1, l2);
         float w1 = 0.f, w2 = 0.f, L = -INFINITY;
         if (m != -INFINITY) {
