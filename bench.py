@@ -59,9 +59,9 @@ def measured_peaks():
 
 # DRAM bytes (read + write) of one forward launch on this workload, from one ncu capture
 # of the same kernel on the 4-head version of the workload scaled by 3 to 12 heads (the
-# traffic is per (head, frame, query tile) unit): 3 x (197.487872 + 53.305344) MB.  Set
+# traffic is per (head, frame, query tile) unit): 3 x (196.734208 + 52.413696) MB.  Set
 # back to None whenever the forward kernel changes, until it is re-measured.
-NCU_TRAFFIC_BYTES = 752_379_648
+NCU_TRAFFIC_BYTES = 747_443_712
 
 
 def max_over_ranks(x: float, device) -> float:
