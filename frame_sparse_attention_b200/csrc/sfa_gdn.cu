@@ -13,16 +13,19 @@
 //   KS = K_i S           (same)
 //   S_acc += K_i^T U_i   (M = d, N = d, K = 128 tokens), U_i = diag(beta) (V_i - KS)
 // G CTAs per (batch, head) run the frames in order (the recurrence is sequential); CTA g
-// takes tiles g, g + G, ... of every frame.  With G > 1 each CTA adds its partial S_acc
-// into one fp32 sum per head with a bulk reduce-add (cp.reduce.async.bulk, performed in
-// L2), the G CTAs of a head meet at a counter in global memory (one cooperative launch,
-// so all CTAs are resident; the wait is bounded), and each reads the sum back.  The sums
-// rotate over three buffers by frame: buffer n mod 3 is summed into in frame n, and CTA 0
-// zeroes buffer (n + 2) mod 3 after the meeting of frame n, when every CTA has finished
-// reading it (frame n - 1) and none can add into it yet (frame n + 2 comes after the next
-// meeting); one meeting per frame is enough.  Warps 0-3 (one thread per TMEM lane) read O and KS out of tensor memory,
-// write O, form U in shared memory and update the fp32 state; warp 4 issues the TMA
-// copies and MMAs.
+// takes tiles g, g + G, ... of every frame, and its tiles form one sequence over the frames
+// through two shared-memory slots, so the copies of the next tile are in flight while the
+// current one computes.  With G > 1 each CTA adds its partial S_acc into one fp32 sum per
+// head with a TMA reduce-add (performed in L2), the G CTAs of a head meet at a counter in
+// global memory (one cooperative launch, so all CTAs are resident; the wait is bounded),
+// and each copies the sum back with one TMA load.  The sums rotate over three buffers by
+// frame: buffer n mod 3 is summed into in frame n, and CTA 0 zeroes buffer (n + 2) mod 3
+// after the meeting of frame n, when every CTA has finished reading it (frame n - 1) and
+// none can add into it yet (frame n + 2 comes after the next meeting); one meeting per
+// frame is enough.  Per tile the MMAs run KS first, then O, then (once U is in shared
+// memory) S_acc.  Warps 0-3 (one thread per TMEM lane) form U over V, read O out to
+// global memory and update the fp32 state; warp 4 issues the TMA copies and MMAs.
+// Read-only steps (update = 0) leave the state alone, so their frames are independent.
 // Tensor memory: O, KS, S_acc and the fp32 state, 128 columns each.  Every wait is
 // bounded; a wait that runs out stores SFA_ERR_TIMEOUT and the CTA drains and exits.
 #include <cuda.h>
@@ -31,6 +34,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdint>
+#include <cstring>
 #include <mutex>
 
 #include "sfa.h"
@@ -45,33 +49,43 @@ constexpr int GBM = 128;         // tokens per tile
 constexpr int GTHREADS = 160;    // warps 0-3 epilogue, warp 4 TMA + MMA
 constexpr int G_BOX = 128 * 128; // one 128-row x 64-column bf16 box (128-byte swizzle)
 constexpr int G_TILE = 2 * G_BOX;
-constexpr int G_S = 0, G_Q = G_TILE, G_K = 2 * G_TILE, G_V = 3 * G_TILE, G_U = 4 * G_TILE, G_BAR = 5 * G_TILE;
+constexpr int F_BOX = 128 * 128; // one 128-row x 32-column fp32 box (128-byte swizzle)
+// shared memory: the bf16 state (B operand of O and KS), then two slots of Q, K, V for
+// consecutive tiles (U is written over V); at a frame end the Q and K of the slot of the
+// frame's last tile stage the partial S_acc and then the head's sum (64 KB fp32)
+constexpr int G_S = 0, G_SLOT0 = G_TILE, G_SLOT_BYTES = 3 * G_TILE;
+constexpr int SL_Q = 0, SL_K = G_TILE, SL_V = 2 * G_TILE;
+constexpr int G_BAR = G_SLOT0 + 2 * G_SLOT_BYTES;
 constexpr int G_SMEM = G_BAR + 128 + 1024;
 constexpr uint32_t T_O = 0, T_KS = 128, T_SACC = 256, T_SST = 384;  // tensor-memory columns
 
 struct GdnArgs {
     int32_t B, H, T, P, n_tiles, update;
     int32_t G;           // CTAs per (batch, head)
-    float *part;         // [3][B*H][d][d] sums of the partial S_acc (G > 1), zero at launch
-    uint32_t *count;     // [B*H] arrivals (G > 1), zero at launch
+    float *part;         // [3][B*H][d][d] sums of the partial S_acc (G > 1 with update), zero at launch
+    uint32_t *count;     // [B*H] arrivals (G > 1 with update), zero at launch
     const float *alpha;  // [B][H][T]
     const float *beta;   // [B][H][T*P]
     const float *s_in;   // [B][H][d][d] or null (zeros)
     float *s_out;        // [B][H][d][d]
-    uint16_t *o;         // bf16, strided
-    int64_t os0, os1, os2;
     int32_t *status;
     uint64_t timeout_ns;
 };
 
 struct GBars {
     uint32_t base;
-    __device__ uint32_t full() const { return base; }      // Q, K, V of a tile landed
-    __device__ uint32_t mma1() const { return base + 8; }  // O and KS of a tile in TMEM
-    __device__ uint32_t u_full() const { return base + 16; }  // U in smem, O/KS read (128 arrivals)
-    __device__ uint32_t sacc() const { return base + 24; }    // S_acc MMA of a tile done
-    __device__ uint32_t s_ready() const { return base + 32; } // state for the next frame (128 arrivals)
-    __device__ uint32_t drain() const { return base + 40; }
+    __device__ uint32_t full(uint32_t s) const { return base + 8 * s; }  // Q, K, V of slot s landed
+    __device__ uint32_t ks() const { return base + 16; }       // KS of a tile in TMEM
+    __device__ uint32_t o() const { return base + 24; }        // O of a tile in TMEM
+    __device__ uint32_t u_full() const { return base + 32; }   // U in smem, KS read (128 arrivals)
+    __device__ uint32_t o_free() const { return base + 40; }   // O read out of TMEM (128 arrivals)
+    __device__ uint32_t sacc() const { return base + 48; }     // S_acc MMA of a tile done
+    __device__ uint32_t s_ready() const { return base + 56; }  // state for the next frame (128 arrivals)
+    __device__ uint32_t sum() const { return base + 64; }      // the head's summed S_acc landed
+    __device__ uint32_t drain() const { return base + 72; }
+    __device__ uint32_t staged() const { return base + 80; }   // partial S_acc staged (128 arrivals)
+    __device__ uint32_t o_staged() const { return base + 88; } // O tile in shared memory (128 arrivals)
+    __device__ uint32_t o_sent() const { return base + 96; }   // O tile's store has read shared memory
 };
 
 __device__ __forceinline__ uint64_t gns()
@@ -82,10 +96,9 @@ __device__ __forceinline__ uint64_t gns()
 }
 
 // bounded wait; false (and the abort flag set, status written) when it runs out
-__device__ __noinline__ bool gwait(uint32_t bar, uint32_t parity, volatile int32_t *abort, int32_t *status,
-                                   uint64_t limit)
+__device__ __noinline__ bool gwait_slow(uint32_t bar, uint32_t parity, volatile int32_t *abort, int32_t *status,
+                                        uint64_t limit)
 {
-    if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = gns();
     for (uint32_t spins = 1;; ++spins) {
         if (mbar_try_wait(bar, parity)) return true;
@@ -98,31 +111,58 @@ __device__ __noinline__ bool gwait(uint32_t bar, uint32_t parity, volatile int32
     }
 }
 
-__device__ __forceinline__ uint32_t swz(int row, int col)  // byte offset of (row, col) in a swizzled tile
+// the first test inline (no call: loads this thread has in flight stay in flight)
+__device__ __forceinline__ bool gwait(uint32_t bar, uint32_t parity, volatile int32_t *abort, int32_t *status,
+                                      uint64_t limit)
+{
+    return mbar_try_wait(bar, parity) || gwait_slow(bar, parity, abort, status, limit);
+}
+
+// wait for copies already in flight, whatever the abort flag says, for at most 2 s
+__device__ __forceinline__ void gdrain(uint32_t bar, uint32_t parity)
+{
+    const uint64_t t0 = gns();
+    while (!mbar_try_wait(bar, parity) && gns() - t0 < 2000000000ull) {
+    }
+}
+
+__device__ __forceinline__ uint32_t swz(int row, int col)  // byte offset of bf16 (row, col) in a swizzled tile
 {
     const int box = col >> 6, chunk = (col & 63) >> 3;
     return (uint32_t)(box * G_BOX + row * 128 + ((chunk ^ (row & 7)) << 4) + (col & 7) * 2);
+}
+
+// byte offset of fp32 columns 32 c + 4 j .. + 3 of row r in four swizzled 32-column boxes
+// (the layout a 128-byte-swizzle TMA copy of a 32 x 128 fp32 box uses)
+__device__ __forceinline__ uint32_t fswz(int r, int c, int j)
+{
+    return (uint32_t)(c * F_BOX + r * 128 + ((j ^ (r & 7)) << 4));
 }
 
 __device__ __forceinline__ float bf16f(uint16_t x) { return __uint_as_float((uint32_t)x << 16); }
 
 __global__ void __launch_bounds__(GTHREADS, 1)
     gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ GdnArgs a)
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+               const __grid_constant__ CUtensorMap tm_part, const __grid_constant__ GdnArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
     const GBars bar{sbase + G_BAR};
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + G_BAR + 64);
-    volatile int32_t *abort = reinterpret_cast<volatile int32_t *>(smem + G_BAR + 68);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + G_BAR + 112);
+    volatile int32_t *abort = reinterpret_cast<volatile int32_t *>(smem + G_BAR + 116);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int bh = blockIdx.x / a.G, g = blockIdx.x % a.G, b = bh / a.H, h = bh % a.H;
+    const bool upd = a.update != 0, spread = upd && a.G > 1;  // spread: partial updates summed over the head's CTAs
+    const int per = (a.n_tiles - g + a.G - 1) / a.G;          // tiles of a frame this CTA takes: g, g + G, ...
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < 6; ++i) mbar_init(sbase + G_BAR + 8 * i, 1);
-        mbar_init(bar.u_full(), 128);
-        mbar_init(bar.s_ready(), 128);
+        const uint32_t single[8] = {bar.full(0), bar.full(1), bar.ks(),  bar.o(),
+                                    bar.sacc(),    bar.sum(),     bar.drain(), bar.o_sent()};
+        for (uint32_t x : single) mbar_init(x, 1);
+        const uint32_t all[5] = {bar.u_full(), bar.o_free(), bar.s_ready(), bar.staged(), bar.o_staged()};
+        for (uint32_t x : all) mbar_init(x, 128);
         *abort = 0;
         fence_mbar_init();
     }
@@ -131,6 +171,8 @@ __global__ void __launch_bounds__(GTHREADS, 1)
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
+            tma_prefetch_desc(&tm_o);
+            if (spread) tma_prefetch_desc(&tm_part);
         }
         tmem_alloc(smem_u32(tmem_slot), 512);
         tmem_relinquish();
@@ -142,68 +184,107 @@ __global__ void __launch_bounds__(GTHREADS, 1)
 
     if (warp == 4) {
         // ---------------------------------------------------------------- TMA + MMA
+        // The CTA's tiles form one sequence over the frames (tile t: frame t / per); tile t
+        // uses slot t & 1, and its copies are issued while tile t - 1 is in flight.
         const uint64_t ds = sdesc_sw128(sbase + G_S, G_BOX, 1024);    // S: [d_k rows][d_v], MN-major B
-        const uint64_t dq = sdesc_sw128(sbase + G_Q, 16, 1024);       // Q tile, K-major A
-        const uint64_t dk = sdesc_sw128(sbase + G_K, 16, 1024);       // K tile, K-major A
-        const uint64_t dkt = sdesc_sw128(sbase + G_K, G_BOX, 1024);   // K tile read as K^T: MN-major A
-        const uint64_t du = sdesc_sw128(sbase + G_U, G_BOX, 1024);    // U tile, MN-major B
         constexpr uint32_t id_qs = idesc_bf16_f32(GBM, GD, true);
         constexpr uint32_t id_kt = idesc_bf16_f32(GD, GD, true) | (1u << 15);  // A MN-major
-        bool ok = true, issued = false, pending = false;  // pending: a tile's copies are in flight
-        uint32_t it = 0;
-        for (int n = 0; n < a.T && ok; ++n) {
-            ok = __all_sync(0xffffffffu, gwait(bar.s_ready(), n & 1, abort, a.status, a.timeout_ns));
-            for (int i = g; i < a.n_tiles && ok; i += a.G, ++it) {
-                if (elect_one()) {
-                    mbar_arrive_expect_tx(bar.full(), 3 * G_TILE);
+        const uint32_t total = (uint32_t)per * (uint32_t)a.T;
+        uint32_t n_loaded = 0, n_landed = 0;  // tiles whose copies were issued / seen landed here
+        bool ok = true, issued = false;
+        auto load = [&](uint32_t t) {
+            const uint32_t dst = sbase + G_SLOT0 + (t & 1) * G_SLOT_BYTES;
+            const int n = (int)(t / per), i = g + (int)(t % per) * a.G;
+            if (elect_one()) {
+                mbar_arrive_expect_tx(bar.full(t & 1), 3 * G_TILE);
 #pragma unroll
-                    for (int kb = 0; kb < 2; ++kb) {
-                        tma_load_5d(sbase + G_Q + kb * G_BOX, &tm_q, bar.full(), kb * 64, i * GBM, n, h, b);
-                        tma_load_5d(sbase + G_K + kb * G_BOX, &tm_k, bar.full(), kb * 64, i * GBM, n, h, b);
-                        tma_load_5d(sbase + G_V + kb * G_BOX, &tm_v, bar.full(), kb * 64, i * GBM, n, h, b);
-                    }
+                for (int kb = 0; kb < 2; ++kb) {
+                    tma_load_5d(dst + SL_K + kb * G_BOX, &tm_k, bar.full(t & 1), kb * 64, i * GBM, n, h, b);
+                    tma_load_5d(dst + SL_Q + kb * G_BOX, &tm_q, bar.full(t & 1), kb * 64, i * GBM, n, h, b);
+                    tma_load_5d(dst + SL_V + kb * G_BOX, &tm_v, bar.full(t & 1), kb * 64, i * GBM, n, h, b);
                 }
-                __syncwarp();
-                pending = true;
-                if (!(ok = __all_sync(0xffffffffu, gwait(bar.full(), it & 1, abort, a.status, a.timeout_ns)))) break;
-                pending = false;
-                tc_fence_after();
+            }
+            __syncwarp();
+            n_loaded = t + 1;
+        };
+        if (total > 0) load(0);
+        for (uint32_t it = 0; it < total && ok; ++it) {
+            const uint32_t n = it / per, ii = it % per, slot = it & 1;
+            // a frame starts from the state of the previous one (read-only steps: the input state)
+            if (ii == 0 && (upd || n == 0) &&
+                !(ok = __all_sync(0xffffffffu, gwait(bar.s_ready(), n & 1, abort, a.status, a.timeout_ns))))
+                break;
+            if (!(ok = __all_sync(0xffffffffu, gwait(bar.full(slot), (it >> 1) & 1, abort, a.status, a.timeout_ns))))
+                break;
+            n_landed = it + 1;
+            tc_fence_after();
+            const uint32_t sl = sbase + G_SLOT0 + slot * G_SLOT_BYTES;
+            const uint64_t dq = sdesc_sw128(sl + SL_Q, 16, 1024);   // Q tile, K-major A
+            const uint64_t dk = sdesc_sw128(sl + SL_K, 16, 1024);   // K tile, K-major A
+            if (upd) {  // KS first: U waits for it (KS of the previous tile was read before its U)
                 if (elect_one()) {
 #pragma unroll
                     for (uint32_t kk = 0; kk < GD / 16; ++kk) {
                         const uint32_t ka = (kk >> 2) * G_BOX + (kk & 3) * 32;
-                        mma_ss(tmem + T_O, dq + (ka >> 4), ds + ((kk * 2048) >> 4), id_qs, kk > 0);
                         mma_ss(tmem + T_KS, dk + (ka >> 4), ds + ((kk * 2048) >> 4), id_qs, kk > 0);
                     }
-                    tc_commit(bar.mma1());
+                    tc_commit(bar.ks());
                 }
                 __syncwarp();
                 issued = true;
-                if (!(ok = __all_sync(0xffffffffu, gwait(bar.u_full(), it & 1, abort, a.status, a.timeout_ns)))) break;
+            }
+            // O of the previous tile read out of TMEM
+            if (it > 0 &&
+                !(ok = __all_sync(0xffffffffu, gwait(bar.o_free(), (it - 1) & 1, abort, a.status, a.timeout_ns))))
+                break;
+            tc_fence_after();
+            if (elect_one()) {
+#pragma unroll
+                for (uint32_t kk = 0; kk < GD / 16; ++kk) {
+                    const uint32_t ka = (kk >> 2) * G_BOX + (kk & 3) * 32;
+                    mma_ss(tmem + T_O, dq + (ka >> 4), ds + ((kk * 2048) >> 4), id_qs, kk > 0);
+                }
+                tc_commit(bar.o());
+            }
+            __syncwarp();
+            issued = true;
+            if (it + 1 < total) {
+                // the other slot last held tile it - 1: its S_acc MMA is done, its O tile has
+                // left through the Q buffer, and (at a frame start) the staged sums of the frame
+                // before were read by the time the state was ready
+                if (upd && it > 0 &&
+                    !(ok = __all_sync(0xffffffffu, gwait(bar.sacc(), (it - 1) & 1, abort, a.status, a.timeout_ns))))
+                    break;
+                if (it > 0 &&
+                    !(ok = __all_sync(0xffffffffu, gwait(bar.o_sent(), (it - 1) & 1, abort, a.status, a.timeout_ns))))
+                    break;
+                load(it + 1);
+            }
+            if (upd) {
+                if (!(ok = __all_sync(0xffffffffu, gwait(bar.u_full(), it & 1, abort, a.status, a.timeout_ns))))
+                    break;
                 tc_fence_after();
+                const uint64_t dkt = sdesc_sw128(sl + SL_K, G_BOX, 1024);  // K tile read as K^T: MN-major A
+                const uint64_t du = sdesc_sw128(sl + SL_V, G_BOX, 1024);   // U tile, MN-major B
                 if (elect_one()) {
                     // S_acc += K^T U over the tile's 128 tokens, 16 per step
 #pragma unroll
                     for (uint32_t kk = 0; kk < GBM / 16; ++kk)
                         mma_ss(tmem + T_SACC, dkt + ((kk * 2048) >> 4), du + ((kk * 2048) >> 4), id_kt,
-                               (i > g || kk > 0) ? 1u : 0u);
+                               (ii > 0 || kk > 0) ? 1u : 0u);
                     tc_commit(bar.sacc());
                 }
                 __syncwarp();
-                ok = __all_sync(0xffffffffu, gwait(bar.sacc(), it & 1, abort, a.status, a.timeout_ns));
             }
         }
         if (__any_sync(0xffffffffu, *abort != 0)) {
-            const uint64_t t0 = gns();
             if (issued) {  // tensor cores idle before TMEM is freed
                 if (elect_one()) tc_commit(bar.drain());
                 __syncwarp();
-                while (!mbar_try_wait(bar.drain(), 0) && gns() - t0 < 2000000000ull) {
-                }
+                gdrain(bar.drain(), 0);
             }
             // copies still in flight land before the CTA exits
-            while (pending && !mbar_try_wait(bar.full(), it & 1) && gns() - t0 < 2000000000ull) {
-            }
+            for (uint32_t t = n_landed; t < n_loaded; ++t) gdrain(bar.full(t & 1), (t >> 1) & 1);
         }
         __syncwarp();
     } else {
@@ -236,91 +317,113 @@ __global__ void __launch_bounds__(GTHREADS, 1)
         tc_fence_before();
         mbar_arrive(bar.s_ready());
         bool ok = true;
+        int sum_n = -1;  // thread 0: the frame whose sum is being copied in, or -1
         uint32_t it = 0;
         for (int n = 0; n < a.T && ok; ++n) {
-            for (int i = g; i < a.n_tiles; i += a.G, ++it) {
-                ok = __all_sync(0xffffffffu, gwait(bar.mma1(), it & 1, abort, a.status, a.timeout_ns)) &&
-                     __all_sync(0xffffffffu, gwait(bar.full(), it & 1, abort, a.status, a.timeout_ns));
-                if (!ok) break;
-                tc_fence_after();
+            const float al = upd ? a.alpha[bhi * a.T + n] : 0.f;
+            for (int ii = 0; ii < per; ++ii, ++it) {
+                const int i = g + ii * a.G;
+                const uint32_t sl = G_SLOT0 + (it & 1) * G_SLOT_BYTES;
                 const int row = i * GBM + r;
                 const bool valid = row < a.P;
-                // O row -> global bf16
-                uint16_t *orow = a.o + b * a.os0 + h * a.os1 + ((int64_t)n * a.P + row) * a.os2;
+                if (upd) {
+                    const float bt = valid ? a.beta[(bhi * a.T + n) * a.P + row] : 0.f;
+                    ok = __all_sync(0xffffffffu, gwait(bar.ks(), it & 1, abort, a.status, a.timeout_ns)) &&
+                         __all_sync(0xffffffffu, gwait(bar.full(it & 1), (it >> 1) & 1, abort, a.status, a.timeout_ns));
+                    if (!ok) break;
+                    tc_fence_after();
+                    // U row = beta_row (V row - KS row) -> bf16, written over the V row
+#pragma unroll
+                    for (int c = 0; c < GD / 32; ++c) {
+                        uint32_t ks[32];
+                        tmem_ld32(lane_base + T_KS + c * 32, ks);
+                        tmem_wait_ld_regs(ks);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const uint32_t off = sl + SL_V + swz(r, c * 32 + q * 8);
+                            const uint4 vv = *reinterpret_cast<const uint4 *>(smem + off);
+                            const uint32_t vw[4] = {vv.x, vv.y, vv.z, vv.w};
+                            uint32_t pk[4];
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                const float v0 = bf16f((uint16_t)(vw[j] & 0xffffu)), v1 = bf16f((uint16_t)(vw[j] >> 16));
+                                pk[j] = pack_bf16x2(bt * (v0 - __uint_as_float(ks[8 * q + 2 * j])),
+                                                    bt * (v1 - __uint_as_float(ks[8 * q + 2 * j + 1])));
+                            }
+                            st_shared_v4(sbase + off, pk);
+                        }
+                    }
+                    fence_proxy_async_smem();
+                    tc_fence_before();
+                    mbar_arrive(bar.u_full());
+                }
+                if (!(ok = __all_sync(0xffffffffu, gwait(bar.o(), it & 1, abort, a.status, a.timeout_ns)))) break;
+                tc_fence_after();
+                // O row -> bf16 into the Q buffer (read by the finished O MMA), in the layout of
+                // the output's tensor map; one TMA store writes the tile (rows past the frame
+                // are not written)
 #pragma unroll
                 for (int c = 0; c < GD / 32; ++c) {
                     uint32_t v[32];
                     tmem_ld32(lane_base + T_O + c * 32, v);
                     tmem_wait_ld_regs(v);
-                    if (valid) {
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            uint4 w;
-                            w.x = pack_bf16x2(__uint_as_float(v[8 * q]), __uint_as_float(v[8 * q + 1]));
-                            w.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3]));
-                            w.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5]));
-                            w.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7]));
-                            *reinterpret_cast<uint4 *>(orow + c * 32 + q * 8) = w;
-                        }
-                    }
-                }
-                // U row = beta_row (V row - KS row) -> bf16, same swizzled layout as V
-                const float bt = valid ? a.beta[(bhi * a.T + n) * a.P + row] : 0.f;
-#pragma unroll
-                for (int c = 0; c < GD / 32; ++c) {
-                    uint32_t ks[32];
-                    tmem_ld32(lane_base + T_KS + c * 32, ks);
-                    tmem_wait_ld_regs(ks);
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
-                        const int col = c * 32 + q * 8;
-                        const uint4 vv = *reinterpret_cast<const uint4 *>(smem + G_V + swz(r, col));
-                        const uint32_t vw[4] = {vv.x, vv.y, vv.z, vv.w};
-                        uint32_t pk[4];
+                        uint32_t w[4];
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const float v0 = bf16f((uint16_t)(vw[j] & 0xffffu)), v1 = bf16f((uint16_t)(vw[j] >> 16));
-                            pk[j] = pack_bf16x2(bt * (v0 - __uint_as_float(ks[8 * q + 2 * j])),
-                                                bt * (v1 - __uint_as_float(ks[8 * q + 2 * j + 1])));
-                        }
-                        st_shared_v4(sbase + G_U + swz(r, col), pk);
+                        for (int j = 0; j < 4; ++j)
+                            w[j] = pack_bf16x2(__uint_as_float(v[8 * q + 2 * j]), __uint_as_float(v[8 * q + 2 * j + 1]));
+                        st_shared_v4(sbase + sl + SL_Q + swz(r, c * 32 + q * 8), w);
                     }
                 }
                 fence_proxy_async_smem();
                 tc_fence_before();
-                mbar_arrive(bar.u_full());
+                mbar_arrive(bar.o_free());
+                mbar_arrive(bar.o_staged());
+                bool sent = true;
+                if (r == 0 && (sent = gwait(bar.o_staged(), it & 1, abort, a.status, a.timeout_ns))) {
+#pragma unroll
+                    for (int kb = 0; kb < 2; ++kb)
+                        tma_store_5d(&tm_o, sbase + sl + SL_Q + kb * G_BOX, kb * 64, i * GBM, n, h, b);
+                    tma_store_commit();
+                    tma_store_wait_read_all();
+                    mbar_arrive(bar.o_sent());
+                }
+                if (!(ok = __all_sync(0xffffffffu, sent))) break;
             }
-            if (!ok) break;
-            // frame end: S <- alpha S + S_acc, fp32 in TMEM, bf16 copy for the next frame
+            if (!ok || !upd) continue;
+            // frame end: S <- alpha S + S_acc (summed over the head's CTAs), fp32 in TMEM,
+            // bf16 copy for the next frame
             ok = __all_sync(0xffffffffu, gwait(bar.sacc(), (it - 1) & 1, abort, a.status, a.timeout_ns));
             if (!ok) break;
             tc_fence_after();
-            if (a.update && a.G > 1) {
-                // this CTA's partial, staged row-major in the free Q/K tiles, added into the
-                // head's sum in L2; then meet the head's other CTAs
-                float *stage = reinterpret_cast<float *>(smem + G_Q);
-                float *sum = a.part + ((int64_t)(n % 3) * a.B * a.H + bh) * GD * GD;
+            const uint32_t stage = G_SLOT0 + ((it - 1) & 1) * G_SLOT_BYTES + SL_K;  // K and U of the last tile
+            if (spread) {
+                // this CTA's partial, swizzled like the fp32 boxes of the sum's tensor map
 #pragma unroll
                 for (int c = 0; c < GD / 32; ++c) {
                     uint32_t acc[32];
                     tmem_ld32(lane_base + T_SACC + c * 32, acc);
                     tmem_wait_ld_regs(acc);
 #pragma unroll
-                    for (int j = 0; j < 32; j += 4)
-                        *reinterpret_cast<float4 *>(stage + r * GD + c * 32 + j) =
-                            make_float4(__uint_as_float(acc[j]), __uint_as_float(acc[j + 1]),
-                                        __uint_as_float(acc[j + 2]), __uint_as_float(acc[j + 3]));
+                    for (int j = 0; j < 8; ++j) {
+                        const uint32_t w[4] = {acc[4 * j], acc[4 * j + 1], acc[4 * j + 2], acc[4 * j + 3]};
+                        st_shared_v4(sbase + stage + fswz(r, c, j), w);
+                    }
                 }
                 fence_proxy_async_smem();
-                named_bar_sync(1, 128);
-                if (r == 0) {
-                    bulk_reduce_add_f32(sum, sbase + G_Q, GD * GD * 4);
+                __threadfence();  // this thread's zeroing of the frame before, ahead of the arrival
+                mbar_arrive(bar.staged());
+                if (r == 0 && gwait(bar.staged(), n & 1, abort, a.status, a.timeout_ns)) {
+                    // add it into the head's sum in L2, meet the head's other CTAs, fetch the sum
+                    const int y = ((n % 3) * a.B * a.H + bh) * GD;
+#pragma unroll
+                    for (int c = 0; c < GD / 32; ++c) tma_reduce_add_2d(&tm_part, sbase + stage + c * F_BOX, c * 32, y);
                     bulk_commit_and_wait_all();
-                    __threadfence();
-                    atomicAdd(a.count + bh, 1u);
+                    red_release_add(a.count + bh, 1u);
                     const uint32_t want = (uint32_t)a.G * (uint32_t)(n + 1);
                     const uint64_t t0 = gns();
-                    for (uint32_t spins = 0; *reinterpret_cast<volatile uint32_t *>(a.count + bh) < want; ++spins) {
+                    for (uint32_t spins = 0; ld_acquire(a.count + bh) < want; ++spins) {
                         if (*abort) break;
                         if ((spins & 63) == 63 && gns() - t0 > a.timeout_ns) {
                             *abort = 1;
@@ -328,60 +431,65 @@ __global__ void __launch_bounds__(GTHREADS, 1)
                             break;
                         }
                     }
-                    __threadfence();
-                }
-                named_bar_sync(1, 128);
-                if (*abort) {
-                    ok = false;
-                    break;
-                }
-                if (g == 0) {  // buffer (n + 2) mod 3: read by every CTA in frame n - 1, next summed into in frame n + 2
-                    float *z = a.part + ((int64_t)((n + 2) % 3) * a.B * a.H + bh) * GD * GD + r * GD;
+                    fence_proxy_async_global();
+                    if (!*abort) {
+                        mbar_arrive_expect_tx(bar.sum(), 4 * F_BOX);
 #pragma unroll
-                    for (int j = 0; j < GD; j += 4) __stcg(reinterpret_cast<float4 *>(z + j), make_float4(0.f, 0.f, 0.f, 0.f));
-                    __threadfence();  // visible before this CTA's next arrival
+                        for (int c = 0; c < GD / 32; ++c)
+                            tma_load_2d(sbase + stage + c * F_BOX, &tm_part, bar.sum(), c * 32, y);
+                        sum_n = n;
+                    }
                 }
+                // (a warp that left on an abort never arrives: every wait here is bounded)
+                if (!(ok = __all_sync(0xffffffffu, gwait(bar.sum(), n & 1, abort, a.status, a.timeout_ns)))) break;
+                sum_n = -1;
             }
-            if (a.update) {
-                const float al = a.alpha[bhi * a.T + n];
-                const float *sumrow = a.part + (((int64_t)(n % 3) * a.B * a.H + bh) * GD + r) * GD;
 #pragma unroll
-                for (int c = 0; c < GD / 32; ++c) {
-                    uint32_t s[32], acc[32];
-                    tmem_ld32(lane_base + T_SST + c * 32, s);
-                    tmem_wait_ld_regs(s);
-                    if (a.G > 1) {
+            for (int c = 0; c < GD / 32; ++c) {
+                uint32_t s[32], acc[32];
+                tmem_ld32(lane_base + T_SST + c * 32, s);
+                tmem_wait_ld_regs(s);
+                if (spread) {
 #pragma unroll
-                        for (int j = 0; j < 32; j += 4) {
-                            const float4 v4 = __ldcg(reinterpret_cast<const float4 *>(sumrow + c * 32 + j));
-                            acc[j] = __float_as_uint(v4.x);
-                            acc[j + 1] = __float_as_uint(v4.y);
-                            acc[j + 2] = __float_as_uint(v4.z);
-                            acc[j + 3] = __float_as_uint(v4.w);
-                        }
-                    } else {
-                        tmem_ld32(lane_base + T_SACC + c * 32, acc);
-                        tmem_wait_ld_regs(acc);
+                    for (int j = 0; j < 8; ++j) {
+                        const uint4 v4 = *reinterpret_cast<const uint4 *>(smem + stage + fswz(r, c, j));
+                        acc[4 * j] = v4.x;
+                        acc[4 * j + 1] = v4.y;
+                        acc[4 * j + 2] = v4.z;
+                        acc[4 * j + 3] = v4.w;
                     }
+                } else {
+                    tmem_ld32(lane_base + T_SACC + c * 32, acc);
+                    tmem_wait_ld_regs(acc);
+                }
 #pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        s[j] = __float_as_uint(fmaf(al, __uint_as_float(s[j]), __uint_as_float(acc[j])));
-                    tmem_st32(lane_base + T_SST + c * 32, s);
+                for (int j = 0; j < 32; ++j)
+                    s[j] = __float_as_uint(fmaf(al, __uint_as_float(s[j]), __uint_as_float(acc[j])));
+                tmem_st32(lane_base + T_SST + c * 32, s);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        uint32_t pk[4];
+                for (int q = 0; q < 4; ++q) {
+                    uint32_t pk[4];
 #pragma unroll
-                        for (int j = 0; j < 4; ++j)
-                            pk[j] = pack_bf16x2(__uint_as_float(s[8 * q + 2 * j]), __uint_as_float(s[8 * q + 2 * j + 1]));
-                        st_shared_v4(sbase + G_S + swz(r, c * 32 + q * 8), pk);
-                    }
+                    for (int j = 0; j < 4; ++j)
+                        pk[j] = pack_bf16x2(__uint_as_float(s[8 * q + 2 * j]), __uint_as_float(s[8 * q + 2 * j + 1]));
+                    st_shared_v4(sbase + G_S + swz(r, c * 32 + q * 8), pk);
                 }
             }
             tmem_wait_st();
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(bar.s_ready());
+            if (spread) {
+                // buffer (n + 2) mod 3 was read by every CTA in frame n - 1 and is next summed
+                // into in frame n + 2, after every CTA's arrival of frame n + 1: CTA g zeroes
+                // its share of it now (fenced before its next arrival)
+                float4 *z = reinterpret_cast<float4 *>(a.part + ((int64_t)((n + 2) % 3) * a.B * a.H + bh) * GD * GD);
+                const int z0 = g * (GD * GD / 4) / a.G, z1 = (g + 1) * (GD * GD / 4) / a.G;
+                for (int j = z0 + r; j < z1; j += 128) __stcg(z + j, make_float4(0.f, 0.f, 0.f, 0.f));
+            }
         }
+        if (sum_n >= 0) gdrain(bar.sum(), (uint32_t)sum_n & 1);
+        if (r == 0) bulk_commit_and_wait_all();  // the last O tiles written
         // state out (CTA 0 of the head; all hold the same state)
         if (ok && a.s_out && g == 0) {
             tc_fence_after();
@@ -427,7 +535,8 @@ EncodeTiledFn encode_fn()
 }
 
 // bf16 [B][H][T*P][d] as a 5-D map (d, P, T, H, B), box 64 x 128 x 1 x 1 x 1, 128-byte
-// swizzle: a tile never crosses its frame; rows past the frame read as zero
+// swizzle: a tile never crosses its frame; rows past the frame read as zero and are not
+// written by a store
 bool encode_frames(CUtensorMap *m, const void *base, int B, int H, int T, int P, const int64_t *stride)
 {
     EncodeTiledFn fn = encode_fn();
@@ -438,6 +547,20 @@ bool encode_frames(CUtensorMap *m, const void *base, int B, int H, int T, int P,
     const cuuint32_t box[5] = {64, (cuuint32_t)GBM, 1, 1, 1}, es[5] = {1, 1, 1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), gd, gs, box, es,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// the fp32 sums [3 * B * H * d rows][d] as a 2-D map, box 32 columns x 128 rows, 128-byte
+// swizzle: four boxes hold one head's d x d sum
+bool encode_part(CUtensorMap *m, float *part, int64_t rows)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t gd[2] = {(cuuint64_t)GD, (cuuint64_t)rows};
+    const cuuint64_t gs[1] = {(cuuint64_t)GD * 4};
+    const cuuint32_t box[2] = {32, 128}, es[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, part, gd, gs, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -496,10 +619,11 @@ extern "C" sfa_status sfa_gdn_forward(const sfa_gdn_desc *d, const void *q, cons
     if (!gdn_stride_ok(d->q_stride) || !gdn_stride_ok(d->k_stride) || !gdn_stride_ok(d->v_stride) ||
         !gdn_stride_ok(d->o_stride))
         return SFA_ERR_INVALID_ARG;
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
     if (!encode_frames(&tq, q, d->B, d->H, d->T, d->P, d->q_stride) ||
         !encode_frames(&tk, k, d->B, d->H, d->T, d->P, d->k_stride) ||
-        !encode_frames(&tv, v, d->B, d->H, d->T, d->P, d->v_stride))
+        !encode_frames(&tv, v, d->B, d->H, d->T, d->P, d->v_stride) ||
+        !encode_frames(&to, o, d->B, d->H, d->T, d->P, d->o_stride))
         return SFA_ERR_UNSUPPORTED;
     GdnArgs a;
     a.B = d->B;
@@ -512,33 +636,34 @@ extern "C" sfa_status sfa_gdn_forward(const sfa_gdn_desc *d, const void *q, cons
     a.beta = beta;
     a.s_in = state_in;
     a.s_out = state_out;
-    a.o = static_cast<uint16_t *>(o);
-    a.os0 = d->o_stride[0];
-    a.os1 = d->o_stride[1];
-    a.os2 = d->o_stride[2];
     a.status = dev_status;
     a.timeout_ns = (uint64_t)(d->timeout_us ? d->timeout_us : 2000000u) * 1000;
-    // several CTAs per head need the workspace (and a read-write frame loop); otherwise one
-    int G = (workspace && update) ? gdn_split(d) : 1;
+    // read-only steps: the frames are independent, so the tiles spread over several CTAs per
+    // head without meeting; updating steps spread them only with the workspace, through which
+    // the CTAs exchange their partial updates, and one CTA per head otherwise
+    const int G = (workspace || !update) ? gdn_split(d) : 1;
     a.G = G;
     a.part = nullptr;
     a.count = nullptr;
+    CUtensorMap tp;
+    std::memset(&tp, 0, sizeof(tp));  // read only by CTAs that exchange partial updates
     cudaStream_t s = as_cuda(stream);
     if (cudaFuncSetAttribute(gdn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, G_SMEM) != cudaSuccess)
         return SFA_ERR_CUDA;
-    if (G > 1) {
+    if (G > 1 && update) {
         const size_t pb = gdn_part_bytes(d, G), need = pb + ((size_t)d->B * d->H * 4 + 255) / 256 * 256;
         if (workspace_bytes < need || reinterpret_cast<uintptr_t>(workspace) % 256) return SFA_ERR_INVALID_ARG;
         a.part = static_cast<float *>(workspace);
         a.count = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(workspace) + pb);
+        if (!encode_part(&tp, a.part, (int64_t)3 * d->B * d->H * GD)) return SFA_ERR_UNSUPPORTED;
         if (cudaMemsetAsync(workspace, 0, need, s) != cudaSuccess) return SFA_ERR_CUDA;  // sums and counters
         // the G CTAs of a head wait for one another: one cooperative launch keeps them all resident
-        void *args[] = {&tq, &tk, &tv, &a};
+        void *args[] = {&tq, &tk, &tv, &to, &tp, &a};
         const cudaError_t e = cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(gdn_kernel),
                                                           dim3((unsigned)(d->B * d->H * G)), dim3(GTHREADS), args,
                                                           G_SMEM, s);
         return e == cudaSuccess ? launch_status() : SFA_ERR_CUDA;
     }
-    gdn_kernel<<<(unsigned)(d->B * d->H), GTHREADS, G_SMEM, s>>>(tq, tk, tv, a);
+    gdn_kernel<<<(unsigned)(d->B * d->H * G), GTHREADS, G_SMEM, s>>>(tq, tk, tv, to, tp, a);
     return launch_status();
 }

@@ -87,6 +87,25 @@ __device__ __forceinline__ void tma_load_5d(uint32_t dst, const void *tmap, uint
         : "memory");
 }
 
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, uint32_t bar, int c0, int c1)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar), "r"(c0), "r"(c1)
+        : "memory");
+}
+
+// global tile at (c0, c1) += the shared box at src, element-wise in the map's type,
+// performed by the async proxy in L2 (completion through the bulk group)
+__device__ __forceinline__ void tma_reduce_add_2d(const void *tmap, uint32_t src, int c0, int c1)
+{
+    asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(tmap)),
+                 "r"(src), "r"(c0), "r"(c1)
+                 : "memory");
+}
+
 __device__ __forceinline__ void tma_store_5d(const void *tmap, uint32_t src, int c0, int c1, int c2, int c3,
                                              int c4)
 {
@@ -97,15 +116,6 @@ __device__ __forceinline__ void tma_store_5d(const void *tmap, uint32_t src, int
 }
 
 __device__ __forceinline__ void tma_store_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-
-// dst[i] += src[i] for `bytes` / 4 floats (global dst, shared src; 16-byte aligned, a
-// multiple of 16 bytes), performed by the async proxy in L2
-__device__ __forceinline__ void bulk_reduce_add_f32(float *dst, uint32_t src, uint32_t bytes)
-{
-    asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(dst), "r"(src),
-                 "r"(bytes)
-                 : "memory");
-}
 
 // commit the pending bulk operations and wait until they are complete, writes included,
 // then order them before this thread's later global accesses
@@ -119,6 +129,26 @@ __device__ __forceinline__ void bulk_commit_and_wait_all()
 __device__ __forceinline__ void tma_store_wait_read_all()
 {
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// *p += v at GPU scope, ordered after this thread's earlier memory operations (release)
+__device__ __forceinline__ void red_release_add(uint32_t *p, uint32_t v)
+{
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// *p at GPU scope, ordered before this thread's later memory operations (acquire)
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t *p)
+{
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// global accesses this thread has ordered (an acquire) -> before its later async-proxy copies
+__device__ __forceinline__ void fence_proxy_async_global()
+{
+    asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 // generic-proxy shared-memory writes -> visible to the async proxy (TMA store reads)

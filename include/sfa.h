@@ -366,7 +366,8 @@ sfa_status sfa_forward_blocks_split(const sfa_attn_desc *desc, const void *q, co
  *   scratch, overwritten) and update != 0, the token tiles of every frame are spread over
  *   several CTAs per (batch, head) that exchange their partial updates through it (one
  *   cooperative launch; every wait is bounded); with NULL, one CTA per (batch, head).
- *   The result is the same up to the order of the fp32 sums.
+ *   The result is the same up to the order of the fp32 sums.  With update == 0 the
+ *   frames are independent and the tiles are always spread; the workspace is not used.
  */
 typedef struct {
     int32_t B, H, T, P, d;
