@@ -23,8 +23,9 @@
 // after the meeting of frame n, when every CTA has finished reading it (frame n - 1) and
 // none can add into it yet (frame n + 2 comes after the next meeting); one meeting per
 // frame is enough.  Per tile the MMAs run KS first, then O, then (once U is in shared
-// memory) S_acc.  Warps 0-3 (one thread per TMEM lane) form U over V, read O out to
-// global memory and update the fp32 state; warp 4 issues the TMA copies and MMAs.
+// memory) S_acc.  Warps 0-7 (two threads per TMEM lane, 64 columns each) form U over V,
+// stage O in the tile's Q buffer and update the fp32 state; warp 8 issues the TMA copies,
+// the MMAs and the TMA stores of O.
 // Read-only steps (update = 0) leave the state alone, so their frames are independent.
 // Tensor memory: O, KS, S_acc and the fp32 state, 128 columns each.  Every wait is
 // bounded; a wait that runs out stores SFA_ERR_TIMEOUT and the CTA drains and exits.
@@ -46,7 +47,9 @@ namespace {
 
 constexpr int GD = 128;          // d_k = d_v
 constexpr int GBM = 128;         // tokens per tile
-constexpr int GTHREADS = 160;    // warps 0-3 epilogue, warp 4 TMA + MMA
+constexpr int GEPI = 256;        // warps 0-7: epilogue (two threads per TMEM lane)
+constexpr int GW_MMA = 8;        // warp 8: TMA copies and MMAs
+constexpr int GTHREADS = GEPI + 32;
 constexpr int G_BOX = 128 * 128; // one 128-row x 64-column bf16 box (128-byte swizzle)
 constexpr int G_TILE = 2 * G_BOX;
 constexpr int F_BOX = 128 * 128; // one 128-row x 32-column fp32 box (128-byte swizzle)
@@ -77,15 +80,13 @@ struct GBars {
     __device__ uint32_t full(uint32_t s) const { return base + 8 * s; }  // Q, K, V of slot s landed
     __device__ uint32_t ks() const { return base + 16; }       // KS of a tile in TMEM
     __device__ uint32_t o() const { return base + 24; }        // O of a tile in TMEM
-    __device__ uint32_t u_full() const { return base + 32; }   // U in smem, KS read (128 arrivals)
-    __device__ uint32_t o_free() const { return base + 40; }   // O read out of TMEM (128 arrivals)
+    __device__ uint32_t u_full() const { return base + 32; }   // U in smem, KS read (all epilogue threads)
+    __device__ uint32_t o_free() const { return base + 40; }   // O read out of TMEM into the Q buffer (all)
     __device__ uint32_t sacc() const { return base + 48; }     // S_acc MMA of a tile done
-    __device__ uint32_t s_ready() const { return base + 56; }  // state for the next frame (128 arrivals)
+    __device__ uint32_t s_ready() const { return base + 56; }  // state for the next frame (all)
     __device__ uint32_t sum() const { return base + 64; }      // the head's summed S_acc landed
     __device__ uint32_t drain() const { return base + 72; }
-    __device__ uint32_t staged() const { return base + 80; }   // partial S_acc staged (128 arrivals)
-    __device__ uint32_t o_staged() const { return base + 88; } // O tile in shared memory (128 arrivals)
-    __device__ uint32_t o_sent() const { return base + 96; }   // O tile's store has read shared memory
+    __device__ uint32_t staged() const { return base + 80; }   // partial S_acc staged (all)
 };
 
 __device__ __forceinline__ uint64_t gns()
@@ -95,8 +96,9 @@ __device__ __forceinline__ uint64_t gns()
     return t;
 }
 
-// bounded wait; false (and the abort flag set, status written) when it runs out
-__device__ __noinline__ bool gwait_slow(uint32_t bar, uint32_t parity, volatile int32_t *abort, int32_t *status,
+// bounded wait; false (and the abort flag set, status written) when it runs out.  Inline
+// throughout: a call would make the thread first wait for the loads it has in flight.
+__device__ __forceinline__ bool gwait_slow(uint32_t bar, uint32_t parity, volatile int32_t *abort, int32_t *status,
                                         uint64_t limit)
 {
     const uint64_t t0 = gns();
@@ -111,7 +113,6 @@ __device__ __noinline__ bool gwait_slow(uint32_t bar, uint32_t parity, volatile 
     }
 }
 
-// the first test inline (no call: loads this thread has in flight stay in flight)
 __device__ __forceinline__ bool gwait(uint32_t bar, uint32_t parity, volatile int32_t *abort, int32_t *status,
                                       uint64_t limit)
 {
@@ -158,15 +159,14 @@ __global__ void __launch_bounds__(GTHREADS, 1)
     const int per = (a.n_tiles - g + a.G - 1) / a.G;          // tiles of a frame this CTA takes: g, g + G, ...
 
     if (threadIdx.x == 0) {
-        const uint32_t single[8] = {bar.full(0), bar.full(1), bar.ks(),  bar.o(),
-                                    bar.sacc(),    bar.sum(),     bar.drain(), bar.o_sent()};
+        const uint32_t single[7] = {bar.full(0), bar.full(1), bar.ks(), bar.o(), bar.sacc(), bar.sum(), bar.drain()};
         for (uint32_t x : single) mbar_init(x, 1);
-        const uint32_t all[5] = {bar.u_full(), bar.o_free(), bar.s_ready(), bar.staged(), bar.o_staged()};
-        for (uint32_t x : all) mbar_init(x, 128);
+        const uint32_t all[4] = {bar.u_full(), bar.o_free(), bar.s_ready(), bar.staged()};
+        for (uint32_t x : all) mbar_init(x, GEPI);
         *abort = 0;
         fence_mbar_init();
     }
-    if (warp == 4) {
+    if (warp == GW_MMA) {
         if (lane == 0) {
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
@@ -182,7 +182,7 @@ __global__ void __launch_bounds__(GTHREADS, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 4) {
+    if (warp == GW_MMA) {
         // ---------------------------------------------------------------- TMA + MMA
         // The CTA's tiles form one sequence over the frames (tile t: frame t / per); tile t
         // uses slot t & 1, and its copies are issued while tile t - 1 is in flight.
@@ -206,6 +206,18 @@ __global__ void __launch_bounds__(GTHREADS, 1)
             }
             __syncwarp();
             n_loaded = t + 1;
+        };
+        // O of tile t (staged by the epilogue in its Q buffer) -> global; lane 0 owns the
+        // bulk groups
+        auto store_o = [&](uint32_t t) {
+            const uint32_t src = sbase + G_SLOT0 + (t & 1) * G_SLOT_BYTES + SL_Q;
+            const int n = (int)(t / per), i = g + (int)(t % per) * a.G;
+            if (lane == 0) {
+#pragma unroll
+                for (int kb = 0; kb < 2; ++kb) tma_store_5d(&tm_o, src + kb * G_BOX, kb * 64, i * GBM, n, h, b);
+                tma_store_commit();
+            }
+            __syncwarp();
         };
         if (total > 0) load(0);
         for (uint32_t it = 0; it < total && ok; ++it) {
@@ -233,10 +245,13 @@ __global__ void __launch_bounds__(GTHREADS, 1)
                 __syncwarp();
                 issued = true;
             }
-            // O of the previous tile read out of TMEM
-            if (it > 0 &&
-                !(ok = __all_sync(0xffffffffu, gwait(bar.o_free(), (it - 1) & 1, abort, a.status, a.timeout_ns))))
-                break;
+            // O of the previous tile read out of TMEM and staged: its store goes out (a frame's
+            // last tile went out already, during the frame end)
+            if (it > 0 && ii != 0) {
+                if (!(ok = __all_sync(0xffffffffu, gwait(bar.o_free(), (it - 1) & 1, abort, a.status, a.timeout_ns))))
+                    break;
+                store_o(it - 1);
+            }
             tc_fence_after();
             if (elect_one()) {
 #pragma unroll
@@ -249,15 +264,14 @@ __global__ void __launch_bounds__(GTHREADS, 1)
             __syncwarp();
             issued = true;
             if (it + 1 < total) {
-                // the other slot last held tile it - 1: its S_acc MMA is done, its O tile has
-                // left through the Q buffer, and (at a frame start) the staged sums of the frame
-                // before were read by the time the state was ready
+                // the other slot last held tile it - 1: its S_acc MMA is done, its O tile's
+                // store has read the Q buffer, and (at a frame start) the staged sums of the
+                // frame before were read by the time the state was ready
                 if (upd && it > 0 &&
                     !(ok = __all_sync(0xffffffffu, gwait(bar.sacc(), (it - 1) & 1, abort, a.status, a.timeout_ns))))
                     break;
-                if (it > 0 &&
-                    !(ok = __all_sync(0xffffffffu, gwait(bar.o_sent(), (it - 1) & 1, abort, a.status, a.timeout_ns))))
-                    break;
+                if (lane == 0) tma_store_wait_read_all();
+                __syncwarp();
                 load(it + 1);
             }
             if (upd) {
@@ -276,7 +290,14 @@ __global__ void __launch_bounds__(GTHREADS, 1)
                 }
                 __syncwarp();
             }
+            if (ii + 1 == (uint32_t)per) {  // the frame's last tile: its O goes out now
+                if (!(ok = __all_sync(0xffffffffu, gwait(bar.o_free(), it & 1, abort, a.status, a.timeout_ns))))
+                    break;
+                store_o(it);
+            }
         }
+        if (lane == 0) bulk_commit_and_wait_all();  // every O store complete
+        __syncwarp();
         if (__any_sync(0xffffffffu, *abort != 0)) {
             if (issued) {  // tensor cores idle before TMEM is freed
                 if (elect_one()) tc_commit(bar.drain());
@@ -288,28 +309,32 @@ __global__ void __launch_bounds__(GTHREADS, 1)
         }
         __syncwarp();
     } else {
-        // ---------------------------------------------------------------- epilogue, row r
-        const int r = threadIdx.x;  // TMEM lane = tile row = state row (d_k index)
-        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+        // ---------------------------------------------------------------- epilogue, row r, half hc
+        // warps w and w + 4 share TMEM lanes 32 (w mod 4) .. + 31 (tile rows, state rows) and
+        // take 64 columns each
+        const int e = threadIdx.x, qd = warp & 3, hc = warp >> 2;
+        const int r = qd * 32 + lane;  // TMEM lane = tile row = state row (d_k index)
+        const int c0 = hc * 2;         // this thread's 32-column chunks: c0, c0 + 1
+        const uint32_t lane_base = tmem + ((uint32_t)(qd * 32) << 16);
         const int64_t bhi = (int64_t)b * a.H + h;
-        // state in: fp32 row r into TMEM, bf16 row r into the B-operand tile
+        // state in: fp32 row r into TMEM, bf16 row r into the B-operand tile (this half)
         {
-            float srow[GD];
+            float srow[64];
 #pragma unroll
-            for (int c = 0; c < GD; ++c) srow[c] = a.s_in ? a.s_in[(bhi * GD + r) * GD + c] : 0.f;
+            for (int c = 0; c < 64; ++c) srow[c] = a.s_in ? a.s_in[(bhi * GD + r) * GD + hc * 64 + c] : 0.f;
 #pragma unroll
-            for (int c = 0; c < GD / 32; ++c) {
+            for (int cc = 0; cc < 2; ++cc) {
                 uint32_t w[32];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(srow[c * 32 + j]);
-                tmem_st32(lane_base + T_SST + c * 32, w);
+                for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(srow[cc * 32 + j]);
+                tmem_st32(lane_base + T_SST + (c0 + cc) * 32, w);
             }
 #pragma unroll
-            for (int c = 0; c < GD; c += 8) {
+            for (int c = 0; c < 64; c += 8) {
                 uint32_t pk[4];
 #pragma unroll
                 for (int j = 0; j < 4; ++j) pk[j] = pack_bf16x2(srow[c + 2 * j], srow[c + 2 * j + 1]);
-                st_shared_v4(sbase + G_S + swz(r, c), pk);
+                st_shared_v4(sbase + G_S + swz(r, hc * 64 + c), pk);
             }
         }
         tmem_wait_st();
@@ -319,22 +344,27 @@ __global__ void __launch_bounds__(GTHREADS, 1)
         bool ok = true;
         int sum_n = -1;  // thread 0: the frame whose sum is being copied in, or -1
         uint32_t it = 0;
+        // beta of this thread's row in the CTA's tile t (0 past the frame), loaded a tile ahead
+        auto beta_of = [&](uint32_t t) {
+            const int n = (int)(t / per), row = (g + (int)(t % per) * a.G) * GBM + r;
+            return (upd && n < a.T && row < a.P) ? a.beta[(bhi * a.T + n) * a.P + row] : 0.f;
+        };
+        float bt_next = beta_of(0);
         for (int n = 0; n < a.T && ok; ++n) {
             const float al = upd ? a.alpha[bhi * a.T + n] : 0.f;
             for (int ii = 0; ii < per; ++ii, ++it) {
-                const int i = g + ii * a.G;
                 const uint32_t sl = G_SLOT0 + (it & 1) * G_SLOT_BYTES;
-                const int row = i * GBM + r;
-                const bool valid = row < a.P;
+                const float bt = bt_next;
+                bt_next = beta_of(it + 1);
                 if (upd) {
-                    const float bt = valid ? a.beta[(bhi * a.T + n) * a.P + row] : 0.f;
                     ok = __all_sync(0xffffffffu, gwait(bar.ks(), it & 1, abort, a.status, a.timeout_ns)) &&
                          __all_sync(0xffffffffu, gwait(bar.full(it & 1), (it >> 1) & 1, abort, a.status, a.timeout_ns));
                     if (!ok) break;
                     tc_fence_after();
                     // U row = beta_row (V row - KS row) -> bf16, written over the V row
 #pragma unroll
-                    for (int c = 0; c < GD / 32; ++c) {
+                    for (int cc = 0; cc < 2; ++cc) {
+                        const int c = c0 + cc;
                         uint32_t ks[32];
                         tmem_ld32(lane_base + T_KS + c * 32, ks);
                         tmem_wait_ld_regs(ks);
@@ -360,10 +390,10 @@ __global__ void __launch_bounds__(GTHREADS, 1)
                 if (!(ok = __all_sync(0xffffffffu, gwait(bar.o(), it & 1, abort, a.status, a.timeout_ns)))) break;
                 tc_fence_after();
                 // O row -> bf16 into the Q buffer (read by the finished O MMA), in the layout of
-                // the output's tensor map; one TMA store writes the tile (rows past the frame
-                // are not written)
+                // the output's tensor map; the MMA warp's TMA store writes the tile
 #pragma unroll
-                for (int c = 0; c < GD / 32; ++c) {
+                for (int cc = 0; cc < 2; ++cc) {
+                    const int c = c0 + cc;
                     uint32_t v[32];
                     tmem_ld32(lane_base + T_O + c * 32, v);
                     tmem_wait_ld_regs(v);
@@ -379,17 +409,6 @@ __global__ void __launch_bounds__(GTHREADS, 1)
                 fence_proxy_async_smem();
                 tc_fence_before();
                 mbar_arrive(bar.o_free());
-                mbar_arrive(bar.o_staged());
-                bool sent = true;
-                if (r == 0 && (sent = gwait(bar.o_staged(), it & 1, abort, a.status, a.timeout_ns))) {
-#pragma unroll
-                    for (int kb = 0; kb < 2; ++kb)
-                        tma_store_5d(&tm_o, sbase + sl + SL_Q + kb * G_BOX, kb * 64, i * GBM, n, h, b);
-                    tma_store_commit();
-                    tma_store_wait_read_all();
-                    mbar_arrive(bar.o_sent());
-                }
-                if (!(ok = __all_sync(0xffffffffu, sent))) break;
             }
             if (!ok || !upd) continue;
             // frame end: S <- alpha S + S_acc (summed over the head's CTAs), fp32 in TMEM,
@@ -401,7 +420,8 @@ __global__ void __launch_bounds__(GTHREADS, 1)
             if (spread) {
                 // this CTA's partial, swizzled like the fp32 boxes of the sum's tensor map
 #pragma unroll
-                for (int c = 0; c < GD / 32; ++c) {
+                for (int cc = 0; cc < 2; ++cc) {
+                    const int c = c0 + cc;
                     uint32_t acc[32];
                     tmem_ld32(lane_base + T_SACC + c * 32, acc);
                     tmem_wait_ld_regs(acc);
@@ -412,9 +432,10 @@ __global__ void __launch_bounds__(GTHREADS, 1)
                     }
                 }
                 fence_proxy_async_smem();
-                __threadfence();  // this thread's zeroing of the frame before, ahead of the arrival
+                // (the arrival also orders this thread's zeroing of the frame before ahead of
+                // thread 0's release of the CTA's next arrival at the counter)
                 mbar_arrive(bar.staged());
-                if (r == 0 && gwait(bar.staged(), n & 1, abort, a.status, a.timeout_ns)) {
+                if (e == 0 && gwait(bar.staged(), n & 1, abort, a.status, a.timeout_ns)) {
                     // add it into the head's sum in L2, meet the head's other CTAs, fetch the sum
                     const int y = ((n % 3) * a.B * a.H + bh) * GD;
 #pragma unroll
@@ -445,7 +466,8 @@ __global__ void __launch_bounds__(GTHREADS, 1)
                 sum_n = -1;
             }
 #pragma unroll
-            for (int c = 0; c < GD / 32; ++c) {
+            for (int cc = 0; cc < 2; ++cc) {
+                const int c = c0 + cc;
                 uint32_t s[32], acc[32];
                 tmem_ld32(lane_base + T_SST + c * 32, s);
                 tmem_wait_ld_regs(s);
@@ -482,19 +504,19 @@ __global__ void __launch_bounds__(GTHREADS, 1)
             if (spread) {
                 // buffer (n + 2) mod 3 was read by every CTA in frame n - 1 and is next summed
                 // into in frame n + 2, after every CTA's arrival of frame n + 1: CTA g zeroes
-                // its share of it now (fenced before its next arrival)
+                // its share of it now (released by thread 0's next arrival)
                 float4 *z = reinterpret_cast<float4 *>(a.part + ((int64_t)((n + 2) % 3) * a.B * a.H + bh) * GD * GD);
                 const int z0 = g * (GD * GD / 4) / a.G, z1 = (g + 1) * (GD * GD / 4) / a.G;
-                for (int j = z0 + r; j < z1; j += 128) __stcg(z + j, make_float4(0.f, 0.f, 0.f, 0.f));
+                for (int j = z0 + e; j < z1; j += GEPI) __stcg(z + j, make_float4(0.f, 0.f, 0.f, 0.f));
             }
         }
         if (sum_n >= 0) gdrain(bar.sum(), (uint32_t)sum_n & 1);
-        if (r == 0) bulk_commit_and_wait_all();  // the last O tiles written
         // state out (CTA 0 of the head; all hold the same state)
         if (ok && a.s_out && g == 0) {
             tc_fence_after();
 #pragma unroll
-            for (int c = 0; c < GD / 32; ++c) {
+            for (int cc = 0; cc < 2; ++cc) {
+                const int c = c0 + cc;
                 uint32_t s[32];
                 tmem_ld32(lane_base + T_SST + c * 32, s);
                 tmem_wait_ld_regs(s);
@@ -509,7 +531,7 @@ __global__ void __launch_bounds__(GTHREADS, 1)
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 4) {
+    if (warp == GW_MMA) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
