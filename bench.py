@@ -62,6 +62,10 @@ def measured_peaks():
 # traffic is per (head, frame, query tile) unit): 3 x (196.734208 + 52.413696) MB.  Set
 # back to None whenever the forward kernel changes, until it is re-measured.
 NCU_TRAFFIC_BYTES = 747_443_712
+# DRAM bytes read + written by one launch of the gated-delta kernel on the gdn workload,
+# from an ncu capture of that launch: 348.559616 + 97.579264 MB.  None once the kernel
+# changes, until it is re-measured.
+GDN_NCU_TRAFFIC_BYTES = 446_138_880
 
 
 def max_over_ranks(x: float, device) -> float:
@@ -443,7 +447,9 @@ def bench_gdn(sfa, dev, stream, flush, reps=20):
     dt = time.perf_counter() - t0
     return {"workload": "gdn: ARL2 inter-frame gated delta rule, 24 frames x 1560 tokens, H=12, d=128",
             "roofline": {"bound": "tensor", "achieved": round(flop / (ms * 1e-3) / 1e12, 2), "peak": peak,
-                         "unit": "TFLOP/s", "frac": round(flop / (ms * 1e-3) / 1e12 / peak, 4)},
+                         "unit": "TFLOP/s", "frac": round(flop / (ms * 1e-3) / 1e12 / peak, 4),
+                         "traffic": GDN_NCU_TRAFFIC_BYTES,
+                         "traffic_note": "DRAM read+write bytes per launch, ncu capture (Q', K', V' read once, O written)"},
             "cpu_baseline": {"value": round(flop / w.H / dt / 1e12, 8), "unit": "TFLOP/s",
                              "cores": os.cpu_count() or 1, "kind": "oracle",
                              "sample": f"one head of the workload, all 24 frames (float64 numpy, {dt:.2f} s)"},
