@@ -11,7 +11,7 @@ TEST INFRASTRUCTURE ONLY.
   * §2.2 (Actualizaciones de Paso Limpio): during the intermediate denoising steps the
     state is read but not written.
 
-Readings (each listed in the design doc):
+Readings of the page (where it leaves a step open):
   * shapes: Q'_N, K'_N are [P, d_k] and V'_N is [P, d_v] (the frame's tokens as rows);
     S is [d_k, d_v]; the update's correction term is K'_N^T diag(β_N) (V'_N - K'_N S_{N-1})
     (the transpose makes the product [d_k, d_v]);

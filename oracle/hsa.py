@@ -9,7 +9,7 @@ the page's order:
      block-level pooled keys;
   4. attention is computed over the selected frame-block pairs only.
 
-Readings where the page is silent (each listed in the design doc):
+Readings where the page is silent:
   * a key block is 128 consecutive tokens of one frame (block b of frame f holds tokens
     [f*P + 128*b, f*P + min(128*(b+1), P))), numbered g = f * nblk + b with
     nblk = ceil(P / 128); a query block is 256 consecutive query rows of one frame
