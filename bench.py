@@ -460,6 +460,18 @@ def bench_gdn(sfa, dev, stream, flush, reps=20):
 
 
 # ----------------------------------------------------------------------------- oracle timing
+def cpu_model() -> str:
+    """The host CPU's model name (Linux /proc/cpuinfo), or "unknown"."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_baseline(seconds: float = 15.0, inputs=None):
     """Time the float64 oracle on host cores for about `seconds` on sampled query rows."""
     import oracle
@@ -485,9 +497,12 @@ def cpu_baseline(seconds: float = 15.0, inputs=None):
     per_row = dt / max(n, 1)
     n_per_head = max(1, int(seconds / per_row / w.H))
     n, fl, dt = run(n_per_head, seed=101)
-    return {"value": round(fl / dt / 1e12, 8), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-            "sample": f"{n} sampled query rows of the LVSA workload (float64 C oracle, "
-                      f"{cores} threads, {dt:.1f} s)", "seconds": round(dt, 2)}
+    call_flop = 4.0 * w.d * w.P * w.P * w.B * counts.astype(np.float64).sum()
+    return {"value": round(fl / dt / 1e12, 8), "unit": "TFLOP/s", "cores": cores, "cpu_model": cpu_model(),
+            "kind": "oracle", "sample": f"{n} sampled query rows of the LVSA workload (float64 C oracle, "
+                                        f"{cores} threads, {dt:.1f} s)", "seconds": round(dt, 2),
+            "rows_per_s": round(n / dt, 1),
+            "extrapolated_ms_per_call": round(call_flop / (fl / dt) * 1e3, 1)}
 
 
 def run_reference(args, rank):
@@ -532,8 +547,8 @@ def run_reference(args, rank):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": WORKLOAD_DESC, "B": w.B, "H": w.H, "T": w.Tq, "P": w.P, "d": w.d,
                    "C": w.C, "W": w.W, "T_per": w.T_per, "step_s": STEP_S},
-        "cpu_baseline": {"value": round(value, 8), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                         "sample": sample},
+        "cpu_baseline": {"value": round(value, 8), "unit": "TFLOP/s", "cores": cores, "cpu_model": cpu_model(),
+                         "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 8), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
