@@ -22,6 +22,7 @@ query rows of the same workload per step; rank 0 alone runs it.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import json
 import math
 import os
@@ -62,10 +63,9 @@ def measured_peaks():
 # traffic is per (head, frame, query tile) unit): 3 x (196.734208 + 52.413696) MB.  Set
 # back to None whenever the forward kernel changes, until it is re-measured.
 NCU_TRAFFIC_BYTES = 747_443_712
-# DRAM bytes read + written by one launch of the gated-delta kernel on the gdn workload,
-# from an ncu capture of that launch: 348.559616 + 97.579264 MB.  None once the kernel
-# changes, until it is re-measured.
-GDN_NCU_TRAFFIC_BYTES = 446_138_880
+# DRAM bytes read + written by the gated-delta kernels of one call on the gdn workload,
+# from an ncu capture.  None once the kernels change, until they are re-measured.
+GDN_NCU_TRAFFIC_BYTES = None
 
 
 def max_over_ranks(x: float, device) -> float:
@@ -418,9 +418,14 @@ def bench_gdn(sfa, dev, stream, flush, reps=20):
     q, k, v, a, b = (x.to(dev) for x in gdn_inputs(w.B, w.H, w.Tq, w.P, w.d, seed=0))
     o = torch.empty_like(q)
     s = torch.empty((w.B, w.H, w.d, w.d), dtype=torch.float32, device=dev)
+    desc = sfa.GdnDesc()
+    desc.B, desc.H, desc.T, desc.P, desc.d = w.B, w.H, w.Tq, w.P, w.d
+    nbytes = ctypes.c_size_t(0)
+    sfa.load().sfa_gdn_workspace(ctypes.byref(desc), ctypes.byref(nbytes))
+    ws = torch.empty(nbytes.value, dtype=torch.uint8, device=dev)
 
     def run():
-        sfa.gdn_forward(q, k, v, a, b, w.P, out=o, state_out=s, stream=stream)
+        sfa.gdn_forward(q, k, v, a, b, w.P, out=o, state_out=s, workspace=ws, stream=stream)
 
     for _ in range(3):
         run()
@@ -449,14 +454,14 @@ def bench_gdn(sfa, dev, stream, flush, reps=20):
             "roofline": {"bound": "tensor", "achieved": round(flop / (ms * 1e-3) / 1e12, 2), "peak": peak,
                          "unit": "TFLOP/s", "frac": round(flop / (ms * 1e-3) / 1e12 / peak, 4),
                          "traffic": GDN_NCU_TRAFFIC_BYTES,
-                         "traffic_note": "DRAM read+write bytes per launch, ncu capture (Q', K', V' read once, O written)"},
+                         "traffic_note": "DRAM read+write bytes of the call's two kernels, ncu capture"},
             "cpu_baseline": {"value": round(flop / w.H / dt / 1e12, 8), "unit": "TFLOP/s",
                              "cores": os.cpu_count() or 1, "kind": "oracle",
                              "sample": f"one head of the workload, all 24 frames (float64 numpy, {dt:.2f} s)"},
             "ms": round(ms, 4), "gflop": round(flop / 1e9, 3), "tflops": round(flop / (ms * 1e-3) / 1e12, 2),
             "frac": round(flop / (ms * 1e-3) / 1e12 / peak, 4),
-            "note": "frames in order per (batch, head); each frame's tiles spread over several CTAs "
-                    "per head that exchange partial state updates (sfa_gdn_forward with a workspace)"}
+            "note": "M_N = K^T diag(beta) K and B_N = K^T diag(beta) V of every frame at once, then the "
+                    "recurrence and O = Q S_{N-1} in several CTAs per head (sfa_gdn_forward: two kernels)"}
 
 
 # ----------------------------------------------------------------------------- oracle timing

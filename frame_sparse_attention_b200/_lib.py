@@ -393,10 +393,10 @@ def forward_dual(q, k, v, frames_local, counts_local, frames_hist, counts_hist, 
 def gdn_forward(q, k, v, alpha, beta, P: int, state_in=None, state_out=None, out=None, update: bool = True,
                 workspace="auto", dev_status=None, stream=None, timeout_us: int = 0):
     """ARL2 inter-frame branch over the T = L / P frames of q, k, v [B, H, L, d]: (O bf16
-    like q, final state fp32 [B, H, d, d]).  alpha fp32 [B, H, T], beta fp32 [B, H, L];
-    state_in fp32 [B, H, d, d] or None (zeros).  workspace: "auto" (allocated here: the
-    frame's tiles spread over several CTAs per head), a uint8 CUDA tensor, or None (one CTA
-    per head)."""
+    like q, final state fp32 [B, H, d, d]).  alpha fp32 [B, H, T], beta fp32 [B, H, L]
+    (>= 0); state_in fp32 [B, H, d, d] or None (zeros).  workspace: "auto" (allocated here),
+    a uint8 CUDA tensor of at least ``sfa_gdn_workspace`` bytes, or None (only for
+    update=False: the update needs it)."""
     B, H, L, d = q.shape
     if L % P:
         raise ValueError(f"sequence length {L} is not a multiple of P = {P}")
@@ -418,9 +418,11 @@ def gdn_forward(q, k, v, alpha, beta, P: int, state_in=None, state_out=None, out
         arr[0], arr[1], arr[2] = t.stride(0), t.stride(1), t.stride(2)
     desc.timeout_us = timeout_us
     if isinstance(workspace, str):
-        nbytes = ctypes.c_size_t(0)
-        _check(load().sfa_gdn_workspace(ctypes.byref(desc), ctypes.byref(nbytes)), "sfa_gdn_workspace")
-        workspace = torch.empty(nbytes.value, dtype=torch.uint8, device=q.device) if nbytes.value else None
+        workspace = None
+        if update:
+            nbytes = ctypes.c_size_t(0)
+            _check(load().sfa_gdn_workspace(ctypes.byref(desc), ctypes.byref(nbytes)), "sfa_gdn_workspace")
+            workspace = torch.empty(nbytes.value, dtype=torch.uint8, device=q.device)
     ws_ptr, ws_bytes = (workspace.data_ptr(), workspace.numel()) if workspace is not None else (None, 0)
     _check(load().sfa_gdn_forward(ctypes.byref(desc), q.data_ptr(), k.data_ptr(), v.data_ptr(), alpha.data_ptr(),
                                   beta.data_ptr(), _ptr(state_in), state_out.data_ptr(), out.data_ptr(),

@@ -357,17 +357,22 @@ sfa_status sfa_forward_blocks_split(const sfa_attn_desc *desc, const void *q, co
  *               aligned bases, strides multiples of 8 elements); q, k, v are the
  *               feature-mapped projections Q', K', V'.
  *   alpha       fp32 [B][H][T] (one forget factor per frame), contiguous.
- *   beta        fp32 [B][H][T*P] (one step size per token), contiguous.
+ *   beta        fp32 [B][H][T*P] (one step size per token, >= 0), contiguous.  A negative
+ *               or NaN beta is reported as SFA_ERR_INVALID_ARG in dev_status and its
+ *               token is left out of the update.
  *   state_in    fp32 [B][H][d][d] (row = key dimension), contiguous, or NULL for zeros.
  *   state_out   fp32 [B][H][d][d]; may be the same buffer as state_in.
- * The tensor cores read S and the per-token corrections as bf16; the state itself is kept
- * and updated in fp32.  Supported: d = 128, any P >= 1, any T >= 1.
- * workspace: with a device workspace of sfa_gdn_workspace bytes (256-byte aligned;
- *   scratch, overwritten) and update != 0, the token tiles of every frame are spread over
- *   several CTAs per (batch, head) that exchange their partial updates through it (one
- *   cooperative launch; every wait is bounded); with NULL, one CTA per (batch, head).
- *   The result is the same up to the order of the fp32 sums.  With update == 0 the
- *   frames are independent and the tiles are always spread; the workspace is not used.
+ * Method: the update is linear in the state, S_N = alpha_N S_{N-1} - M_N S_{N-1} + B_N
+ * with M_N = K'^T diag(beta) K' and B_N = K'^T diag(beta) V' of frame N alone.  A first
+ * kernel forms M_N and B_N of every frame at once on the tensor cores; a second runs the
+ * recurrence (one d x d x d product per frame) in several CTAs per (batch, head), each of
+ * which also computes O for its share of the frame's tokens.  The tensor cores read M_N,
+ * S and sqrt(beta)-scaled K', V' as bf16; M_N S accumulates, B_N and the state are kept
+ * in fp32.  The result does not depend on the launch shape.  Supported: d = 128, any
+ * P >= 1, any T >= 1.
+ * workspace: update != 0 needs a device workspace of sfa_gdn_workspace bytes (256-byte
+ *   aligned; scratch, overwritten; M_N and B_N of every frame), else SFA_ERR_INVALID_ARG.
+ *   With update == 0 it is not used and may be NULL.
  */
 typedef struct {
     int32_t B, H, T, P, d;

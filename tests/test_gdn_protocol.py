@@ -1,21 +1,20 @@
-"""A model of the synchronisation of the gated-delta kernel (csrc/sfa_gdn.cu), run on the CPU.
+"""A model of the synchronisation of the gated-delta kernels (csrc/sfa_gdn.cu), run on the CPU.
 
-The kernel's warps coordinate through mbarriers, a global arrival counter and the
-completion order of the tensor core and the TMA engine.  This model replays the waits the
-kernel's MMA warp and epilogue warps perform, in the same order, with the asynchronous
-engines (MMAs completing in issue order, copies landing and stores reading shared memory
-at random later times) and the head's G CTAs as separate actors, all interleaved at random.
-It checks, at the moment a buffer or TMEM column is overwritten, that every reader of the
-old contents has finished; that no mbarrier wait can alias a parity two phases old; and
-that no interleaving deadlocks.  It is a model: a change to the kernel's waits has to be
-mirrored here.  Planted omissions of single waits must be caught (the model's own check);
-the epilogue's threads are one actor here, so waits among them (the staged barrier) are
-outside the model.
+Each kernel's warps coordinate through mbarriers and the completion order of the tensor
+core and the TMA engine.  This model replays the waits the MMA warp and the element-wise
+warps perform, in the same order, with the asynchronous engines (MMAs completing in issue
+order, copies landing and stores reading shared memory at random later times), all
+interleaved at random.  It checks, at the moment a buffer or TMEM column is overwritten,
+that every reader of the old contents has finished; that no mbarrier wait can alias a
+parity two phases old; and that no interleaving deadlocks.  It is a model: a change to a
+kernel's waits has to be mirrored here.  Planted omissions of single waits must be caught
+(the model's own check).  The element-wise warps are one actor here, so waits among them
+(the staged barrier) are outside the model.
 """
-import itertools
 import random
 
 import pytest
+
 
 class _Fail(AssertionError):
     pass
@@ -26,170 +25,55 @@ def _check(cond, msg):
         raise _Fail(msg)
 
 
-def run_model(n_tiles, G, T, upd, rng, drop=frozenset()):
-    """One kernel launch for one (batch, head): G CTAs, T frames, n_tiles tiles per frame."""
-    spread = upd and G > 1
-    count = [0]
+class _Engines:
+    """Tensor core (in-order completion), copy engine (loads land in any order) and the
+    store engine (stores finish reading shared memory in order), for one CTA."""
 
-    class CTA:
-        pass
+    def __init__(self, rng, done):
+        self.rng, self.done = rng, done
+        self.tc, self.copies, self.stores = [], [], []
+        self.completed = set()      # MMA groups done: (kind, index)
+        self.landed = {}            # buffer -> what landed there
+        self.store_read = -1
 
-    ctas = []
-    for g in range(G):
-        c = CTA()
-        c.g, c.per = g, (n_tiles - g + G - 1) // G
-        c.done = {k: 0 for k in ("full0", "full1", "ks", "o", "u_full", "o_free", "sacc", "s_ready", "sum",
-                                 "staged")}
-        c.slot = [None, None]      # tile whose Q, K, V a slot holds
-        c.stage = [None, None]     # frame whose sums occupy a slot's K and V buffers
-        c.use = {}
-        c.tc = []                  # MMA groups in issue order: (kind, tile, frame, barrier)
-        c.copies = []              # in flight: (barrier, what lands)
-        c.landed = [None, None]    # tile whose copies have landed in a slot
-        c.sum_landed = -1          # frame whose sum has landed
-        c.stores = []
-        c.store_read = -1
-        c.s_frame = 0              # frame whose state the bf16 S buffer holds
-        c.sacc_frame_read = -1     # last frame whose S_acc the epilogue has read out
-        ctas.append(c)
+    def mma(self, kind, idx, bar):
+        self.tc.append((kind, idx, bar))
 
-    def use(c, t):
-        return c.use.setdefault(t, set())
+    def load(self, buf, what, bar):
+        self.landed.pop(buf, None)
+        self.copies.append((buf, what, bar))
 
-    def wait(c, bar, k, name):
-        if name in drop:
+    def actor(self):
+        while True:
+            if self.tc and self.rng.random() < 0.5:
+                kind, idx, bar = self.tc.pop(0)
+                self.completed.add((kind, idx))
+                if bar:
+                    self.done[bar] += 1
+            if self.copies and self.rng.random() < 0.3:
+                buf, what, bar = self.copies.pop(self.rng.randrange(len(self.copies)))
+                self.landed[buf] = what
+                self.done[bar] += 1
+            if self.stores and self.rng.random() < 0.3:
+                self.store_read = max(self.store_read, self.stores.pop(0))
+            yield
+
+
+def _wait(done, bar, k, name, drop):
+    if name in drop:
+        return
+    while True:
+        d = done[bar]
+        _check(d in (k, k + 1), f"parity alias: {bar} phase {k}, {d} completed")
+        if d == k + 1:
             return
-        while True:
-            d = c.done[bar]
-            _check(d in (k, k + 1), f"parity alias: CTA {c.g} {bar} phase {k}, {d} completed")
-            if d == k + 1:
-                return
-            yield
+        yield
 
-    def tensor_core(c):
-        while True:
-            if c.tc and rng.random() < 0.5:
-                kind, t, _, bar = c.tc.pop(0)
-                use(c, t).add(kind)
-                c.done[bar] += 1
-            yield
 
-    def copy_engine(c):
-        while True:
-            if c.copies and rng.random() < 0.3:
-                bar, what = c.copies.pop(rng.randrange(len(c.copies)))
-                if bar == "sum":
-                    c.sum_landed = what
-                else:
-                    c.landed[int(bar[-1])] = what
-                c.done[bar] += 1
-            if c.stores and rng.random() < 0.3:
-                c.store_read = max(c.store_read, c.stores.pop(0))
-            yield
-
-    def mma_warp(c):
-        total, per = c.per * T, c.per
-        last_store = [-1]
-
-        def load(t):
-            s = t & 1
-            prev = c.slot[s]
-            if prev is not None:
-                need = {"qs"} | ({"ks", "sacc", "u"} if upd else set())
-                _check(need <= use(c, prev) and c.store_read >= prev,
-                       f"slot {s} reloaded for tile {t} while tile {prev} still uses it")
-            _check(c.stage[s] is None, f"slot {s} reloaded while it holds the sums of frame {c.stage[s]}")
-            c.slot[s] = t
-            c.landed[s] = None
-            c.copies.append((f"full{s}", t))
-
-        def store(t):
-            _check("ostaged" in use(c, t) and c.slot[t & 1] == t, f"O of tile {t} stored before it was staged")
-            c.stores.append(t)
-            last_store[0] = t
-
-        def issue(kind, t, n, bar):
-            _check(not upd or c.s_frame == n, f"MMA of frame {n} reads the state of frame {c.s_frame}")
-            c.tc.append((kind, t, n, bar))
-
-        if total:
-            load(0)
-        for it in range(total):
-            n, ii = divmod(it, per)
-            s = it & 1
-            if ii == 0 and (upd or n == 0):
-                yield from wait(c, "s_ready", n, "s_ready")
-            yield from wait(c, f"full{s}", it >> 1, "full")
-            _check(c.slot[s] == it and c.landed[s] == it, f"MMA on tile {it} before its copies landed")
-            if upd:
-                _check(it == 0 or "u" in use(c, it - 1), f"KS of tile {it} overwrites an unread KS")
-                issue("ks", it, n, "ks")
-            if it > 0 and ii != 0:
-                yield from wait(c, "o_free", it - 1, "o_free_prev")
-                store(it - 1)
-            _check(it == 0 or "oread" in use(c, it - 1), f"O of tile {it} overwrites an unread O")
-            issue("qs", it, n, "o")
-            if it + 1 < total:
-                if upd and it > 0:
-                    yield from wait(c, "sacc", it - 1, "sacc_prev")
-                if "store_read" not in drop:
-                    while c.store_read < last_store[0]:
-                        yield
-                load(it + 1)
-            if upd:
-                yield from wait(c, "u_full", it, "u_full")
-                _check(ii > 0 or c.sacc_frame_read >= n - 1, f"S_acc of frame {n} restarted before it was read")
-                issue("sacc", it, n, "sacc")
-            if ii + 1 == per:
-                yield from wait(c, "o_free", it, "o_free_last")
-                store(it)
-
-    def epilogue(c):
-        c.done["s_ready"] += 1
-        it = 0
-        for n in range(T):
-            for _ in range(c.per):
-                s = it & 1
-                if upd:
-                    yield from wait(c, "ks", it, "ks_epi")
-                    yield from wait(c, f"full{s}", it >> 1, "full")
-                    _check("ks" in use(c, it) and c.landed[s] == it, f"U of tile {it} formed too early")
-                    use(c, it).add("u")
-                    c.done["u_full"] += 1
-                yield from wait(c, "o", it, "o_epi")
-                _check("qs" in use(c, it) and c.slot[s] == it, f"O of tile {it} staged over a busy Q buffer")
-                use(c, it).update({"oread", "ostaged"})
-                c.done["o_free"] += 1
-                it += 1
-            if not upd:
-                continue
-            yield from wait(c, "sacc", it - 1, "sacc_end")
-            _check(all(x[2] > n for x in c.tc) and "sacc" in use(c, it - 1),
-                   f"frame {n} ends with its MMAs in flight")
-            s = (it - 1) & 1
-            c.sacc_frame_read = n
-            if spread:
-                _check(c.slot[s] == it - 1, "sums staged over a reloaded slot")
-                c.stage[s] = n
-                c.done["staged"] += 1
-                yield from wait(c, "staged", n, "staged")
-                count[0] += 1
-                while count[0] < G * (n + 1):
-                    yield
-                c.copies.append(("sum", n))
-                yield from wait(c, "sum", n, "sum")
-                _check(c.sum_landed == n, f"state of frame {n} updated before the head's sum landed")
-                c.stage[s] = None
-            c.s_frame = n + 1
-            c.done["s_ready"] += 1
-
-    finite, engines = [], []
-    for c in ctas:
-        finite += [mma_warp(c), epilogue(c)]
-        engines += [tensor_core(c), copy_engine(c)]
+def _run(rng, engine, finite):
     live, idle = list(finite), 0
     while live:
-        gen = rng.choice(live + engines)
+        gen = rng.choice(live + [engine])
         try:
             next(gen)
             idle += 1
@@ -200,27 +84,190 @@ def run_model(n_tiles, G, T, upd, rng, drop=frozenset()):
             raise _Fail("deadlock")
 
 
-CASES = [(n, G, T, upd) for n, G, T, upd in itertools.product([1, 2, 3, 5, 13], [1, 2, 3, 7], [1, 2, 4], [True, False])
-         if G <= n]
+def model_main(per, T, upd, rng, drop=frozenset(), NQ=4):
+    """gdn_kernel, one CTA (its CTAs never wait for one another): `per` tiles of T frames."""
+    done = {k: 0 for k in ("q0", "q1", "q2", "q3", "m0", "m1", "d_done", "s_free", "o_done0", "o_done1",
+                           "o_free0", "o_free1", "s_ready")}
+    eng = _Engines(rng, done)
+    st = {"s_frame": 0, "d_read": -1, "staged": set(), "stored": set()}
+    total = per * T
+
+    def wait(bar, k, name):
+        return _wait(done, bar, k, name, drop)
+
+    def mma_warp():
+        last_store = [-1]
+
+        def load_q(t):
+            s = t % NQ
+            if t >= NQ:
+                p = t - NQ
+                _check(("qs", p) in eng.completed and p in st["stored"] and eng.store_read >= p,
+                       f"Q buffer {s} reloaded for tile {t} while tile {p} still uses it")
+            eng.load(f"q{s}", t, f"q{s}")
+
+        def load_m(n):
+            if n >= 2:
+                _check(("d", n - 2) in eng.completed, f"M slot {n & 1} reloaded while its product runs")
+            eng.load(f"m{n & 1}", n, f"m{n & 1}")
+
+        def store(t):
+            _check(t in st["staged"], f"O of tile {t} stored before it was staged")
+            st["stored"].add(t)
+            eng.stores.append(t)
+            last_store[0] = t
+
+        def issue(kind, idx, n, bar):
+            _check(not upd or st["s_frame"] == n, f"MMA of frame {n} reads the state of frame {st['s_frame']}")
+            eng.mma(kind, idx, bar)
+
+        for t in range(min(2, total)):
+            load_q(t)
+        if upd:
+            for n in range(min(2, T)):
+                load_m(n)
+        it = 0
+        for n in range(T):
+            if upd or n == 0:
+                yield from wait("s_ready", n, "s_ready")
+            if upd:
+                if 1 <= n and n + 1 < T:
+                    load_m(n + 1)
+                yield from wait(f"m{n & 1}", n >> 1, "m_full")
+                _check(eng.landed.get(f"m{n & 1}") == n, f"product of frame {n} issued before M landed")
+                _check(st["d_read"] >= n - 1, "M S overwrites an unread product")
+                issue("d", n, n, "d_done")
+            for _ in range(per):
+                s, u = it % NQ, it & 1
+                yield from wait(f"q{s}", it // NQ, "q_full")
+                _check(eng.landed.get(f"q{s}") == it, f"O MMA of tile {it} before its Q landed")
+                if it >= 2:
+                    yield from wait(f"o_free{u}", (it - 2) >> 1, "o_free")
+                    store(it - 2)
+                _check(it < 2 or (it - 2) in st["staged"], f"O of tile {it} overwrites an unread O")
+                issue("qs", it, n, f"o_done{u}")
+                if it + 2 < total:
+                    if it >= 2 and "store_read" not in drop:
+                        while eng.store_read < last_store[0]:
+                            yield
+                    load_q(it + 2)
+                it += 1
+            eng.mma("s_free", n, "s_free")
+        for t in range(max(0, total - 2), total):
+            yield from wait(f"o_free{t & 1}", t >> 1, "o_free")
+            store(t)
+
+    def epilogue():
+        done["s_ready"] += 1
+        it = [0]
+
+        def stage_o():
+            t = it[0]
+            u = t & 1
+            yield from wait(f"o_done{u}", t >> 1, "o_done")
+            _check(("qs", t) in eng.completed and eng.landed.get(f"q{t % NQ}") == t,
+                   f"O of tile {t} staged too early or over a reloaded Q buffer")
+            st["staged"].add(t)
+            done[f"o_free{u}"] += 1
+            it[0] += 1
+
+        for n in range(T):
+            # the frame's O products past its second wait for the first ones' TMEM buffers,
+            # and the frame's MMAs end before the state is rewritten: stage those first
+            early = max(per - 2, 0) if upd else per
+            if upd:
+                yield from wait("d_done", n, "d_done")
+                _check(("d", n) in eng.completed, f"product of frame {n} read before it was done")
+                st["d_read"] = n
+            for _ in range(early):
+                yield from stage_o()
+            if upd:
+                yield from wait("s_free", n, "s_free")
+                _check(not any(x[0] in ("d", "qs") for x in eng.tc), f"state of frame {n} rewritten while read")
+                st["s_frame"] = n + 1
+                done["s_ready"] += 1
+            for _ in range(per - early):
+                yield from stage_o()
+
+    _run(rng, eng.actor(), [mma_warp(), epilogue()])
 
 
-@pytest.mark.parametrize("seed", range(6))
-def test_protocol_has_no_race_or_deadlock(seed):
+def model_prep(nt, rng, drop=frozenset(), S=3):
+    """gdn_prep_kernel, one CTA: nt tiles of one frame through S stages."""
+    done = {k: 0 for k in ("kv0", "kv1", "kv2", "sc0", "sc1", "sc2", "md0", "md1", "md2", "fin")}
+    eng = _Engines(rng, done)
+    scaled = set()
+
+    def wait(bar, k, name):
+        return _wait(done, bar, k, name, drop)
+
+    def mma_warp():
+        def load(t):
+            if t >= S:
+                _check(("mm", t - S) in eng.completed, f"stage {t % S} reloaded while its MMAs run")
+            eng.load(f"kv{t % S}", t, f"kv{t % S}")
+
+        for t in range(min(S, nt)):
+            load(t)
+        for i in range(nt):
+            s = i % S
+            yield from wait(f"sc{s}", i // S, "scaled")
+            _check(i in scaled, f"MMA of tile {i} before its operands were scaled")
+            eng.mma("mm", i, f"md{s}")
+            if i >= 1 and i + 2 < nt:
+                p = i - 1
+                yield from wait(f"md{p % S}", p // S, "mma_done")
+                load(i + 2)
+        eng.mma("fin", 0, "fin")
+
+    def epilogue():
+        for i in range(nt):
+            s = i % S
+            yield from wait(f"kv{s}", i // S, "kv_full")
+            _check(eng.landed.get(f"kv{s}") == i, f"tile {i} scaled before it landed")
+            scaled.add(i)
+            done[f"sc{s}"] += 1
+        yield from wait("fin", 0, "fin")
+        _check(all(("mm", i) in eng.completed for i in range(nt)), "products staged while MMAs run")
+
+    _run(rng, eng.actor(), [mma_warp(), epilogue()])
+
+
+MAIN_CASES = [(per, T, upd) for per in (1, 2, 3, 5) for T in (1, 2, 3, 5) for upd in (True, False)]
+PREP_CASES = [(nt,) for nt in (1, 2, 3, 4, 7, 13)]
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_main_kernel_protocol_has_no_race_or_deadlock(seed):
     rng = random.Random(seed)
-    for case in CASES:
-        run_model(*case, rng)
+    for case in MAIN_CASES:
+        model_main(*case, rng)
 
 
-@pytest.mark.parametrize("dropped", ["s_ready", "full", "sacc_prev", "store_read", "o_free_prev", "sum", "sacc_end",
-                                     "u_full"])
-def test_model_catches_a_missing_wait(dropped):
-    caught = False
-    for seed in range(20):
+@pytest.mark.parametrize("seed", range(8))
+def test_prep_kernel_protocol_has_no_race_or_deadlock(seed):
+    rng = random.Random(seed)
+    for case in PREP_CASES:
+        model_prep(*case, rng)
+
+
+def _caught(fn, cases, dropped):
+    for seed in range(30):
         rng = random.Random(seed)
         try:
-            for case in [(13, 7, 3, True), (3, 1, 4, True), (5, 2, 3, True), (2, 1, 3, False)]:
-                run_model(*case, rng, drop=frozenset({dropped}))
+            for case in cases:
+                fn(*case, rng, drop=frozenset({dropped}))
         except _Fail:
-            caught = True
-            break
-    assert caught, f"dropping the {dropped} wait went unnoticed"
+            return True
+    return False
+
+
+@pytest.mark.parametrize("dropped", ["s_ready", "m_full", "q_full", "o_free", "store_read", "d_done", "s_free",
+                                     "o_done"])
+def test_model_catches_a_missing_wait_in_the_main_kernel(dropped):
+    assert _caught(model_main, [(2, 4, True), (1, 3, True), (3, 3, False)], dropped), dropped
+
+
+@pytest.mark.parametrize("dropped", ["scaled", "mma_done", "kv_full", "fin"])
+def test_model_catches_a_missing_wait_in_the_prep_kernel(dropped):
+    assert _caught(model_prep, [(7,), (13,)], dropped), dropped
