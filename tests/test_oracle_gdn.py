@@ -112,3 +112,26 @@ def test_planted_mistake_is_caught():
     wrong = alpha[0, 0, 0] * s + bb.mean() * kk.T @ (vv - kk @ s)
     _, S1 = gdn.gdn_frames(q, k, v, alpha, beta, 5, S0=S0)
     assert np.abs(S1[0, 0] - wrong).max() > 1e-3
+
+
+def test_linear_form_of_the_update_equals_the_delta_form():
+    # the GPU kernels compute S_N = alpha S - M_N S + B_N with M_N = K^T diag(beta) K and
+    # B_N = K^T diag(beta) V of frame N alone (formed for all frames before the recurrence);
+    # that algebra, run in float64 here, reproduces the oracle's frame-by-frame delta form
+    q, k, v, alpha, beta, S0 = _rand(3, B=2, H=2, T=4, P=6, dk=5, dv=4)
+    P, T = 6, 4
+    o_ref, s_ref = gdn.gdn_frames(q, k, v, alpha, beta, P, S0=S0)
+    for b in range(2):
+        for h in range(2):
+            s = S0[b, h].copy()
+            mats = []
+            for n in range(T):  # independent of the state: all frames first
+                rows = slice(n * P, (n + 1) * P)
+                kb = k[b, h, rows] * beta[b, h, rows][:, None]
+                mats.append((kb.T @ k[b, h, rows], kb.T @ v[b, h, rows]))
+            for n in range(T):
+                rows = slice(n * P, (n + 1) * P)
+                np.testing.assert_allclose(q[b, h, rows] @ s, o_ref[b, h, rows], rtol=0, atol=1e-12)
+                M, Bn = mats[n]
+                s = alpha[b, h, n] * s - M @ s + Bn
+            np.testing.assert_allclose(s, s_ref[b, h], rtol=0, atol=1e-12)
