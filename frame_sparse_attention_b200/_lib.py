@@ -49,12 +49,13 @@ class AttnDesc(ctypes.Structure):
                 ("timeout_us", ctypes.c_uint32), ("debug_flags", ctypes.c_uint32)]
 
 
-_lib = None
 class GdnDesc(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("T", ctypes.c_int32), ("P", ctypes.c_int32),
                 ("d", ctypes.c_int32), ("q_stride", ctypes.c_int64 * 3), ("k_stride", ctypes.c_int64 * 3),
                 ("v_stride", ctypes.c_int64 * 3), ("o_stride", ctypes.c_int64 * 3), ("timeout_us", ctypes.c_uint32)]
 
+
+_lib = None
 
 EXPORTS = ("sfa_error_string", "sfa_version", "sfa_set_max_count", "sfa_build_sets", "sfa_forward",
            "sfa_forward_split_workspace", "sfa_forward_split", "sfa_forward_split_noalloc", "sfa_forward_paged",
@@ -130,6 +131,12 @@ def version() -> int:
     return load().sfa_version()
 
 
+def _require(cond: bool, what: str):
+    """Argument check of the binding (a ValueError, kept under ``python -O``)."""
+    if not cond:
+        raise ValueError(what)
+
+
 def _check(status: int, what: str):
     if status != SFA_OK:
         raise SfaError(status, what)
@@ -176,9 +183,11 @@ def build_sets(params: SetParams, kinds, extra: torch.Tensor | None = None, Amax
     if counts is None:
         counts = torch.empty((H, params.Tq), dtype=torch.int32, device=dev)
     if extra is not None:
-        assert extra.dtype == torch.int32 and extra.is_cuda and extra.is_contiguous()
-        assert extra.shape[0] == H
-    assert frames.is_contiguous() and counts.is_contiguous()
+        _require(extra.dtype == torch.int32 and extra.is_cuda and extra.is_contiguous(),
+                 "expected extra.dtype == torch.int32 and extra.is_cuda and extra.is_contiguous()")
+        _require(extra.shape[0] == H, "expected extra.shape[0] == H")
+    _require(frames.is_contiguous() and counts.is_contiguous(),
+             "expected frames.is_contiguous() and counts.is_contiguous()")
     _check(load().sfa_build_sets(ctypes.byref(params), H, _kinds(kinds), _ptr(extra), n_extra,
                                  frames.data_ptr(), counts.data_ptr(), Amax, _stream(stream)),
            "sfa_build_sets")
@@ -217,11 +226,15 @@ def forward(q, k, v, frames, counts, P: int, scale: float | None = None, out=Non
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, Lq), dtype=torch.float32, device=q.device)
-    assert lse.is_contiguous() and lse.dtype == torch.float32
-    assert frames.dtype == torch.int32 and counts.dtype == torch.int32
-    assert frames.is_contiguous() and counts.is_contiguous()
+    _require(lse.is_contiguous() and lse.dtype == torch.float32,
+             "expected lse.is_contiguous() and lse.dtype == torch.float32")
+    _require(frames.dtype == torch.int32 and counts.dtype == torch.int32,
+             "expected frames.dtype == torch.int32 and counts.dtype == torch.int32")
+    _require(frames.is_contiguous() and counts.is_contiguous(),
+             "expected frames.is_contiguous() and counts.is_contiguous()")
     desc = attn_desc(q, k, v, out, P, frames.shape[2], scale, timeout_us, debug_flags)
-    assert tuple(frames.shape[:2]) == (H, desc.Tq) and tuple(counts.shape) == (H, desc.Tq)
+    _require(tuple(frames.shape[:2]) == (H, desc.Tq) and tuple(counts.shape) == (H, desc.Tq),
+             "expected tuple(frames.shape[:2]) == (H, desc.Tq) and tuple(counts.shape) == (H, desc.Tq)")
     _check(load().sfa_forward(ctypes.byref(desc), q.data_ptr(), k.data_ptr(), v.data_ptr(),
                               frames.data_ptr(), counts.data_ptr(), out.data_ptr(), lse.data_ptr(),
                               _ptr(dev_status), _stream(stream)), "sfa_forward")
@@ -238,9 +251,12 @@ def forward_paged(q, k_cache, v_cache, slots, frames, counts, P: int, T_kv: int,
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, Lq), dtype=torch.float32, device=q.device)
-    assert slots.dtype == torch.int32 and slots.is_contiguous() and tuple(slots.shape) == (H, T_kv)
-    assert frames.dtype == torch.int32 and counts.dtype == torch.int32
-    assert frames.is_contiguous() and counts.is_contiguous() and lse.is_contiguous()
+    _require(slots.dtype == torch.int32 and slots.is_contiguous() and tuple(slots.shape) == (H, T_kv),
+             "expected slots.dtype == torch.int32 and slots.is_contiguous() and tuple(slots.shape) == (H, T_kv)")
+    _require(frames.dtype == torch.int32 and counts.dtype == torch.int32,
+             "expected frames.dtype == torch.int32 and counts.dtype == torch.int32")
+    _require(frames.is_contiguous() and counts.is_contiguous() and lse.is_contiguous(),
+             "expected frames.is_contiguous() and counts.is_contiguous() and lse.is_contiguous()")
     desc = attn_desc(q, k_cache, v_cache, out, P, frames.shape[2], scale, timeout_us)
     desc.T_kv = T_kv
     _check(load().sfa_forward_paged(ctypes.byref(desc), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
@@ -266,8 +282,10 @@ def forward_split(q, k, v, frames, counts, P: int, n_split: int, scale: float | 
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, Lq), dtype=torch.float32, device=q.device)
-    assert frames.dtype == torch.int32 and counts.dtype == torch.int32
-    assert frames.is_contiguous() and counts.is_contiguous() and lse.is_contiguous()
+    _require(frames.dtype == torch.int32 and counts.dtype == torch.int32,
+             "expected frames.dtype == torch.int32 and counts.dtype == torch.int32")
+    _require(frames.is_contiguous() and counts.is_contiguous() and lse.is_contiguous(),
+             "expected frames.is_contiguous() and counts.is_contiguous() and lse.is_contiguous()")
     desc = attn_desc(q, k, v, out, P, frames.shape[2], scale, timeout_us)
     need = split_workspace_bytes(desc, n_split)
     if workspace is None and need:
@@ -285,10 +303,13 @@ def lse_merge(o1, lse1, o2, lse2, out=None, lse=None, stream=None):
     d = o1.shape[-1]
     rows = lse1.numel()
     for t in (o1, o2, lse1, lse2):
-        assert t.is_cuda and t.is_contiguous()
-    assert o1.dtype == torch.bfloat16 and o2.dtype == torch.bfloat16
-    assert lse1.dtype == torch.float32 and lse2.dtype == torch.float32
-    assert o1.numel() == rows * d and o2.shape == o1.shape and lse2.shape == lse1.shape
+        _require(t.is_cuda and t.is_contiguous(), "expected t.is_cuda and t.is_contiguous()")
+    _require(o1.dtype == torch.bfloat16 and o2.dtype == torch.bfloat16,
+             "expected o1.dtype == torch.bfloat16 and o2.dtype == torch.bfloat16")
+    _require(lse1.dtype == torch.float32 and lse2.dtype == torch.float32,
+             "expected lse1.dtype == torch.float32 and lse2.dtype == torch.float32")
+    _require(o1.numel() == rows * d and o2.shape == o1.shape and lse2.shape == lse1.shape,
+             "expected o1.numel() == rows * d and o2.shape == o1.shape and lse2.shape == lse1.shape")
     if out is None:
         out = torch.empty_like(o1)
     if lse is None:
@@ -340,12 +361,16 @@ def forward_blocks(q, k, v, blocks, counts, P: int, scale: float | None = None, 
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, Lq), dtype=torch.float32, device=q.device)
-    assert lse.is_contiguous() and lse.dtype == torch.float32
-    assert blocks.dtype == torch.int32 and counts.dtype == torch.int32
-    assert blocks.is_contiguous() and counts.is_contiguous()
+    _require(lse.is_contiguous() and lse.dtype == torch.float32,
+             "expected lse.is_contiguous() and lse.dtype == torch.float32")
+    _require(blocks.dtype == torch.int32 and counts.dtype == torch.int32,
+             "expected blocks.dtype == torch.int32 and counts.dtype == torch.int32")
+    _require(blocks.is_contiguous() and counts.is_contiguous(),
+             "expected blocks.is_contiguous() and counts.is_contiguous()")
     desc = attn_desc(q, k, v, out, P, blocks.shape[-1], scale, timeout_us)
     nqb = (P + QUERY_BLOCK - 1) // QUERY_BLOCK
-    assert tuple(blocks.shape[:4]) == (B, H, desc.Tq, nqb) and tuple(counts.shape) == (B, H, desc.Tq, nqb)
+    _require(tuple(blocks.shape[:4]) == (B, H, desc.Tq, nqb) and tuple(counts.shape) == (B, H, desc.Tq, nqb),
+             "expected tuple(blocks.shape[:4]) == (B, H, desc.Tq, nqb) and tuple(counts.shape) == (B, H, desc.Tq, nqb)")
     if n_split == 1:
         _check(load().sfa_forward_blocks(ctypes.byref(desc), q.data_ptr(), k.data_ptr(), v.data_ptr(),
                                          blocks.data_ptr(), counts.data_ptr(), out.data_ptr(), lse.data_ptr(),
@@ -373,9 +398,11 @@ def forward_dual(q, k, v, frames_local, counts_local, frames_hist, counts_hist, 
     if lse_full is None:
         lse_full = torch.empty((B, H, Lq), dtype=torch.float32, device=q.device)
     for f, c in ((frames_local, counts_local), (frames_hist, counts_hist)):
-        assert f.dtype == torch.int32 and c.dtype == torch.int32 and f.is_contiguous() and c.is_contiguous()
-    assert frames_local.shape == frames_hist.shape
-    assert tuple(out_local.stride()) == tuple(out_full.stride())
+        _require(f.dtype == torch.int32 and c.dtype == torch.int32 and f.is_contiguous() and c.is_contiguous(),
+                 "expected f.dtype == torch.int32 and c.dtype == torch.int32 and f.is_contiguous() and c.is_contiguous()")
+    _require(frames_local.shape == frames_hist.shape, "expected frames_local.shape == frames_hist.shape")
+    _require(tuple(out_local.stride()) == tuple(out_full.stride()),
+             "expected tuple(out_local.stride()) == tuple(out_full.stride())")
     desc = attn_desc(q, k, v, out_full, P, frames_local.shape[2], scale, timeout_us)
     nbytes = ctypes.c_size_t(0)
     _check(load().sfa_forward_dual_workspace(ctypes.byref(desc), n_split, ctypes.byref(nbytes)),
@@ -407,10 +434,12 @@ def gdn_forward(q, k, v, alpha, beta, P: int, state_in=None, state_out=None, out
     if state_out is None:
         state_out = torch.empty((B, H, d, d), dtype=torch.float32, device=q.device)
     for name, t in (("alpha", alpha), ("beta", beta), ("state_out", state_out)):
-        assert t.dtype == torch.float32 and t.is_contiguous(), name
-    assert tuple(alpha.shape) == (B, H, L // P) and tuple(beta.shape) == (B, H, L)
+        _require(t.dtype == torch.float32 and t.is_contiguous(), f"{name} must be fp32 and contiguous")
+    _require(tuple(alpha.shape) == (B, H, L // P) and tuple(beta.shape) == (B, H, L),
+             "expected tuple(alpha.shape) == (B, H, L // P) and tuple(beta.shape) == (B, H, L)")
     if state_in is not None:
-        assert state_in.dtype == torch.float32 and state_in.is_contiguous() and tuple(state_in.shape) == (B, H, d, d)
+        _require(state_in.dtype == torch.float32 and state_in.is_contiguous() and tuple(state_in.shape) == (B, H, d, d),
+                 "expected state_in.dtype == torch.float32 and state_in.is_contiguous() and tuple(state_in.shape) == (B, H, d, d)")
     desc = GdnDesc()
     desc.B, desc.H, desc.T, desc.P, desc.d = B, H, L // P, P, d
     for field, t in (("q_stride", q), ("k_stride", k), ("v_stride", v), ("o_stride", out)):

@@ -202,3 +202,21 @@ def test_dual_host_checks(sfa):
                                 1, good, 1 << 20, None, None) == 1
     assert lib.sfa_forward_dual(ctypes.byref(d), good, good, good, good, good, good, good, good, good, good, good,
                                 1, good, 1024, None, None) == 1
+
+
+def test_binding_rejects_host_tensors(sfa):
+    # the binding's own argument checks run before any CUDA call: host tensors are refused
+    import torch
+    o = torch.zeros(4, 128, dtype=torch.bfloat16)
+    lse = torch.zeros(4, dtype=torch.float32)
+    with pytest.raises(ValueError):
+        sfa.lse_merge(o, lse, o, lse)
+    q = torch.zeros(1, 1, 128, 128, dtype=torch.bfloat16)
+    a = torch.zeros(1, 1, 1, dtype=torch.float32)
+    b = torch.zeros(1, 1, 128, dtype=torch.float32)
+    with pytest.raises(ValueError):
+        sfa.gdn_forward(q, q, q, a, b, 128)
+    frames = torch.zeros(1, 1, 1, dtype=torch.int32)
+    counts = torch.ones(1, 1, dtype=torch.int32)
+    with pytest.raises(ValueError):
+        sfa.forward(q, q, q, frames, counts, 128)
