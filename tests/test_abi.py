@@ -220,3 +220,33 @@ def test_binding_rejects_host_tensors(sfa):
     counts = torch.ones(1, 1, dtype=torch.int32)
     with pytest.raises(ValueError):
         sfa.forward(q, q, q, frames, counts, 128)
+
+
+def test_gdn_host_checks(sfa):
+    lib = sfa.load()
+    d = sfa.GdnDesc()
+    d.B, d.H, d.T, d.P, d.d = 1, 12, 24, 1560, 128
+    for f in ("q_stride", "k_stride", "v_stride", "o_stride"):
+        arr = getattr(d, f)
+        arr[0], arr[1], arr[2] = 12 * 24 * 1560 * 128, 24 * 1560 * 128, 128
+    ws = ctypes.c_size_t(0)
+    assert lib.sfa_gdn_workspace(ctypes.byref(d), ctypes.byref(ws)) == 0
+    assert ws.value == 12 * 24 * 128 * 128 * (2 + 4)  # M_N bf16 and B_N fp32 per frame and head
+    good = 1 << 20
+
+    def call(w, nbytes, update=1):
+        return lib.sfa_gdn_forward(ctypes.byref(d), good, good, good, good, good, None, good, good, update, w,
+                                   nbytes, None, None)
+
+    # an updating step without, with too small or with a misaligned workspace: refused before any launch
+    assert call(None, 0) == sfa.SFA_ERR_INVALID_ARG
+    assert call(good, ws.value - 1) == sfa.SFA_ERR_INVALID_ARG
+    assert call(good + 16, ws.value) == sfa.SFA_ERR_INVALID_ARG
+    d.q_stride[2] = 100  # token stride below d
+    assert call(good, ws.value) == sfa.SFA_ERR_INVALID_ARG
+    d.q_stride[2] = 128
+    d.d = 64
+    assert lib.sfa_gdn_workspace(ctypes.byref(d), ctypes.byref(ws)) == sfa.SFA_ERR_UNSUPPORTED
+    assert call(good, 1 << 30) == sfa.SFA_ERR_UNSUPPORTED
+    d.d, d.B = 128, 0  # nothing to do
+    assert call(None, 0) == sfa.SFA_OK
