@@ -244,7 +244,9 @@ def run_ours(args, rank, world, local_rank):
     d2h = o_p.numel() * o_p.element_size() + lse_p.numel() * lse_p.element_size()
 
     merge = bench_merge(sfa, dev, stream, flush) if rank == 0 else None
-    hsa_rec = bench_hsa(sfa, dev, stream, flush) if rank == 0 else None
+    workloads = None
+    if rank == 0 and world == 1 and not args.no_workloads:
+        workloads = bench_workloads(sfa, dev, stream, flush, with_cpu=not args.no_cpu_baseline)
 
     if rank != 0:
         return None
@@ -285,22 +287,24 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": 2 * args.steps,
         "clocks": clk,
         "merge": merge,
-        "hsa": hsa_rec,
+        "workloads": workloads,
     }
     if world == 1 and not args.no_cpu_baseline:
         rec["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
     return rec
 
 
-def bench_merge(sfa, dev, stream, flush, reps=20):
-    """LSE merge of the ISPA dual-stream shape (1560 rows x 12 heads, d=128)."""
+def bench_merge(sfa, dev, stream, flush, reps=20, rows=None):
+    """LSE merge of the ISPA dual-stream shape (1560 rows x 12 heads, d=128), or of `rows`
+    rows of d=128 (a size large enough to show the kernel's own HBM rate)."""
     w = WORKLOADS["lsemerge_local"]
-    rows = w.B * w.H * w.Lq
-    g = torch.Generator("cpu").manual_seed(7)
-    o1 = torch.randn(rows, w.d, generator=g).to(torch.bfloat16).to(dev)
-    o2 = torch.randn(rows, w.d, generator=g).to(torch.bfloat16).to(dev)
-    l1 = torch.randn(rows, generator=g).to(dev)
-    l2 = torch.randn(rows, generator=g).to(dev)
+    ispa = rows is None
+    rows = w.B * w.H * w.Lq if ispa else rows
+    g = torch.Generator(dev).manual_seed(7)
+    o1 = torch.randn(rows, w.d, generator=g, device=dev).to(torch.bfloat16)
+    o2 = torch.randn(rows, w.d, generator=g, device=dev).to(torch.bfloat16)
+    l1 = torch.randn(rows, generator=g, device=dev)
+    l2 = torch.randn(rows, generator=g, device=dev)
     o = torch.empty_like(o1)
     lse = torch.empty_like(l1)
     for _ in range(3):
@@ -320,8 +324,37 @@ def bench_merge(sfa, dev, stream, flush, reps=20):
     peaks = measured_peaks()
     gbs = nbytes / (ms * 1e-3) / 1e9
     return {"kernel": "lse_merge_kernel<128>", "rows": rows, "bytes": nbytes, "us": round(ms * 1e3, 2),
+            "workload": "ISPA shape: 1560 rows x 12 heads, d=128" if ispa else f"{rows} rows, d=128",
             "achieved_gbs": round(gbs, 1), "peak_gbs": float(peaks["hbm_gbs"]), "bound": "hbm",
-            "frac": round(gbs / float(peaks["hbm_gbs"]), 4)}
+            "frac": round(gbs / float(peaks["hbm_gbs"]), 4),
+            "note": "launch-latency bound at this size" if ispa else "inputs 1.6 GB, larger than L2"}
+
+
+def bench_sets(sfa, dev, stream, flush, reps=20):
+    """sfa_build_sets of the LVSA (41 and 121 frames) and streaming workloads: device time
+    and bytes written (4 (Amax + 1) per (head, query frame)); launch-bound at these sizes."""
+    out = {}
+    for name in ("lvsa41", "long121", "stream"):
+        w = WORKLOADS[name]
+        kinds = [hs.kind for hs in w.heads]
+        n_extra = max((len(hs.extra) for hs in w.heads), default=0)
+        extra = None
+        if n_extra:
+            ex = torch.full((w.H, n_extra), -1, dtype=torch.int32)
+            for h, hs in enumerate(w.heads):
+                ex[h, :len(hs.extra)] = torch.tensor(hs.extra, dtype=torch.int32)
+            extra = ex.to(dev)
+        params = sfa.set_params(T_kv=w.Tkv, Tq=w.Tq, q_off=w.q_off, C=max(w.C, 1), W=max(w.W, 1), T_per=w.T_per,
+                                step=0, n_sink=w.n_sink, n_prev=w.n_prev, chunk_len=w.chunk_len)
+        Amax = sfa.set_max_count(params, kinds, n_extra)
+        fr = torch.empty((w.H, w.Tq, Amax), dtype=torch.int32, device=dev)
+        cn = torch.empty((w.H, w.Tq), dtype=torch.int32, device=dev)
+        ms = time_device(lambda: sfa.build_sets(params, kinds, extra, Amax, fr, cn, stream=stream), flush, stream,
+                         dev, reps, 3)
+        nbytes = 4 * (Amax + 1) * w.H * w.Tq
+        out[name] = {"us": round(ms * 1e3, 2), "bytes": nbytes, "achieved_gbs": round(nbytes / (ms * 1e-3) / 1e9, 2),
+                     "bound": "launch latency"}
+    return out
 
 
 def block_list_flops(blocks: np.ndarray, counts: np.ndarray, P: int, d: int) -> float:
@@ -451,16 +484,23 @@ def bench_gdn(sfa, dev, stream, flush, reps=20):
     ogdn.gdn_frames(qh[:, :1].float().numpy(), kh[:, :1].float().numpy(), vh[:, :1].float().numpy(),
                     ah[:, :1].numpy(), bh[:, :1].numpy(), w.P)
     dt = time.perf_counter() - t0
+    hbm = float(measured_peaks()["hbm_gbs"])
+    # compulsory bytes: Q', K', V' read and O written (bf16), beta and alpha read, the state written
+    nbytes = 4 * w.B * w.H * w.Tq * w.P * w.d * 2 + w.B * w.H * w.Tq * (w.P + 1) * 4 + w.B * w.H * w.d * w.d * 4
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    tf = flop / (ms * 1e-3) / 1e12
     return {"workload": "gdn: ARL2 inter-frame gated delta rule, 24 frames x 1560 tokens, H=12, d=128",
-            "roofline": {"bound": "tensor", "achieved": round(flop / (ms * 1e-3) / 1e12, 2), "peak": peak,
-                         "unit": "TFLOP/s", "frac": round(flop / (ms * 1e-3) / 1e12 / peak, 4),
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+                         "frac": round(gbs / hbm, 4), "bytes": nbytes,
                          "traffic": GDN_NCU_TRAFFIC_BYTES,
-                         "traffic_note": "DRAM read+write bytes of the call's two kernels, ncu capture"},
+                         "traffic_note": "DRAM read+write bytes of the call's two kernels, ncu capture",
+                         "tensor": {"achieved": round(tf, 2), "peak": peak, "unit": "TFLOP/s",
+                                    "frac": round(tf / peak, 4)}},
             "cpu_baseline": {"value": round(flop / w.H / dt / 1e12, 8), "unit": "TFLOP/s",
                              "cores": os.cpu_count() or 1, "kind": "oracle",
                              "sample": f"one head of the workload, all 24 frames (float64 numpy, {dt:.2f} s)"},
-            "ms": round(ms, 4), "gflop": round(flop / 1e9, 3), "tflops": round(flop / (ms * 1e-3) / 1e12, 2),
-            "frac": round(flop / (ms * 1e-3) / 1e12 / peak, 4),
+            "ms": round(ms, 4), "gflop": round(flop / 1e9, 3), "tflops": round(tf, 2),
+            "frac": round(tf / peak, 4),
             "note": "M_N = K^T diag(beta) K and B_N = K^T diag(beta) V of every frame at once, then the "
                     "recurrence and O = Q S_{N-1} in several CTAs per head (sfa_gdn_forward: two kernels)"}
 
@@ -559,14 +599,12 @@ def run_reference(args, rank):
     }
 
 
-def run_other_workload(args):
-    """Device time of one step of another workload (set build + forward per branch; the
-    LSE-decomposed workload adds the merge of its local and history branches)."""
-    import frame_sparse_attention_b200 as sfa
-    sfa.load()
-    dev = torch.device("cuda", 0)
-    names = {"long121": ["long121"], "stream": ["stream"],
-             "lsemerge": ["lsemerge_local", "lsemerge_hist"]}[args.workload]
+def setup_workload(sfa, dev, stream, name, split=1, dual=False):
+    """Device buffers and one step (set build + forward per branch; the LSE-decomposed
+    workload adds the merge of its local and history branches) of another workload.
+    Returns (step, flops, branches) with flops counted after one step has run."""
+    names = {"long121": ["long121"], "stream": ["stream"], "tiny_dense": ["tiny_dense"],
+             "tiny_sinkwin": ["tiny_sinkwin"], "lsemerge": ["lsemerge_local", "lsemerge_hist"]}[name]
     ws = [WORKLOADS[n] for n in names]
     q_h, k_h, v_h = workload_qkv(ws[0], seed=0)
     q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
@@ -588,26 +626,22 @@ def run_other_workload(args):
         cn = torch.empty((w.H, w.Tq), dtype=torch.int32, device=dev)
         o_b = torch.empty_like(q)
         desc = sfa.attn_desc(q, k, v, o_b, w.P, Amax)
-        ws_bytes = sfa.split_workspace_bytes(desc, args.split)
+        ws_bytes = sfa.split_workspace_bytes(desc, split)
         wsp = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
-        branches.append((w, params, kinds, extra, Amax, fr, cn, o_b,
-                         torch.empty((w.B, w.H, w.Lq), dtype=torch.float32, device=dev), wsp))
+        branches.append([w, params, kinds, extra, Amax, fr, cn, o_b,
+                         torch.empty((w.B, w.H, w.Lq), dtype=torch.float32, device=dev), wsp])
     merged = (torch.empty_like(q), torch.empty((ws[0].B, ws[0].H, ws[0].Lq), dtype=torch.float32, device=dev))
-    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream(dev)
-
-    dual = getattr(args, "dual", False) and len(branches) == 2
+    dual = dual and len(branches) == 2
+    dual_ws = None
     if dual:  # both branches in one launch, local result + their merge (sfa_forward_dual)
         Amax = max(b[4] for b in branches)
-        for i, b in enumerate(branches):
-            w_, p_, k_, e_ = b[0], b[1], b[2], b[3]
-            fr = torch.empty((w_.H, w_.Tq, Amax), dtype=torch.int32, device=dev)
-            branches[i] = (w_, p_, k_, e_, Amax, fr, torch.empty_like(b[6])) + b[7:]
-        import ctypes
+        for b in branches:
+            b[4] = Amax
+            b[5] = torch.empty((b[0].H, b[0].Tq, Amax), dtype=torch.int32, device=dev)
         nbytes = ctypes.c_size_t(0)
         ddesc = sfa.attn_desc(q, k, v, merged[0], branches[0][0].P, Amax)
-        if sfa.load().sfa_forward_dual_workspace(ctypes.byref(ddesc), args.split, ctypes.byref(nbytes)) != 0:
-            raise SystemExit("--dual: bad --split for this head dimension")
+        if sfa.load().sfa_forward_dual_workspace(ctypes.byref(ddesc), split, ctypes.byref(nbytes)) != 0:
+            raise SystemExit("dual launch: bad split for this head dimension")
         dual_ws = torch.empty(max(1, nbytes.value), dtype=torch.uint8, device=dev)
 
     def step():
@@ -615,26 +649,34 @@ def run_other_workload(args):
             (w0, p0, k0, e0, A0, f0, c0, o0, l0, _), (w1, p1, k1, e1, A1, f1, c1, o1, l1, _) = branches
             sfa.build_sets(p0, k0, e0, A0, f0, c0, stream=stream)
             sfa.build_sets(p1, k1, e1, A1, f1, c1, stream=stream)
-            sfa.forward_dual(q, k, v, f0, c0, f1, c1, w0.P, args.split, out_local=o0, lse_local=l0,
+            sfa.forward_dual(q, k, v, f0, c0, f1, c1, w0.P, split, out_local=o0, lse_local=l0,
                              out_full=merged[0], lse_full=merged[1], workspace=dual_ws, stream=stream)
             return
         for (w, params, kinds, extra, Amax, fr, cn, o, lse, wsp) in branches:
             sfa.build_sets(params, kinds, extra, Amax, fr, cn, stream=stream)
-            if args.split > 1:
-                sfa.forward_split(q, k, v, fr, cn, w.P, args.split, out=o, lse=lse, workspace=wsp, stream=stream)
+            if split > 1:
+                sfa.forward_split(q, k, v, fr, cn, w.P, split, out=o, lse=lse, workspace=wsp, stream=stream)
             else:
                 sfa.forward(q, k, v, fr, cn, w.P, out=o, lse=lse, stream=stream)
         if len(branches) == 2:
             sfa.lse_merge(branches[0][7], branches[0][8], branches[1][7], branches[1][8],
                           out=merged[0], lse=merged[1], stream=stream)
 
-    for _ in range(args.warmup):
+    step()
+    torch.cuda.synchronize(dev)
+    flops = sum(attended_flops(b[6].cpu().numpy(), b[0]) for b in branches)
+    return step, flops, branches
+
+
+def time_device(step, flush, stream, dev, steps=20, warmup=5):
+    """Median device time (ms) of `step` over `steps` runs after `warmup`, L2 flushed
+    before every run (outside the events)."""
+    for _ in range(warmup):
         flush.zero_()
         step()
     torch.cuda.synchronize(dev)
-    flops = sum(attended_flops(b[6].cpu().numpy(), b[0]) for b in branches)
     times = []
-    for _ in range(args.steps):
+    for _ in range(steps):
         flush.zero_()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
@@ -643,11 +685,121 @@ def run_other_workload(args):
         e1.record(stream)
         torch.cuda.synchronize(dev)
         times.append(e0.elapsed_time(e1))
-    ms = float(np.median(times))
-    return {"workload": args.workload, "branches": names, "split": args.split, "dual_launch": dual,
-            "attended_tflop_per_step": round(flops / 1e12, 4),
+    return float(np.median(times))
+
+
+def run_other_workload(args):
+    """Device time of one step of another workload (one JSON line, not the bench line)."""
+    import frame_sparse_attention_b200 as sfa
+    sfa.load()
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    step, flops, branches = setup_workload(sfa, dev, stream, args.workload, args.split, getattr(args, "dual", False))
+    ms = time_device(step, flush, stream, dev, args.steps, args.warmup)
+    return {"workload": args.workload, "branches": [b[0].name for b in branches], "split": args.split,
+            "dual_launch": bool(getattr(args, "dual", False)), "attended_tflop_per_step": round(flops / 1e12, 4),
             "ms_per_step": round(ms, 4), "tflops": round(flops / (ms * 1e-3) / 1e12, 1),
             "steps": args.steps, "warmup": args.warmup, "note": "device time, median, L2 flushed between steps"}
+
+
+def oracle_full(name, rows_per_head=None, seed=0):
+    """The float64 oracle on host cores over every query row of a workload (or over
+    rows_per_head sampled rows per head): (seconds, flops done, rows, extra info).
+    The LSE-decomposed workload runs both branches and their merge."""
+    import oracle
+    from oracle import merge as M
+    from oracle import sets as S
+    from sfa_workloads import sample_rows
+    names = {"lsemerge": ["lsemerge_local", "lsemerge_hist"]}.get(name, [name])
+    ws = [WORKLOADS[n] for n in names]
+    q, k, v = workload_qkv(ws[0], seed=seed)
+    cores = os.cpu_count() or 1
+    rows = None
+    if rows_per_head:
+        rows = sample_rows(ws[0], rows_per_head, seed=1)
+    t0 = time.perf_counter()
+    outs, fl = [], 0.0
+    for w in ws:
+        frames, counts = S.workload_sets(w, step=0)
+        outs.append(oracle.attention(q, k, v, frames, counts, w.P, 1.0 / math.sqrt(w.d), rows=rows, n_threads=cores))
+        if rows is None:
+            fl += attended_flops(counts, w)
+        else:
+            h = (rows // w.Lq) % w.H
+            t = (rows % w.Lq) // w.P
+            fl += 4.0 * w.d * w.P * counts[h, t].astype(np.float64).sum()
+    if len(outs) == 2:
+        M.lse_merge(outs[0][0], outs[0][1], outs[1][0], outs[1][1])
+    dt = time.perf_counter() - t0
+    n_rows = ws[0].B * ws[0].H * ws[0].Lq if rows is None else rows.size
+    return dt, fl, n_rows, cores
+
+
+def _cpu_record(name, sample, rows_per_head=None):
+    dt, fl, n_rows, cores = oracle_full(name, rows_per_head)
+    return {"value": round(fl / dt / 1e12, 8), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": sample.format(rows=n_rows, s=dt), "seconds": round(dt, 2)}
+
+
+def bench_workloads(sfa, dev, stream, flush, steps=20, warmup=5, with_cpu=True):
+    """Every other workload's device time, roofline and oracle baseline (rank 0, N = 1)."""
+    peaks = measured_peaks()
+    peak = float(peaks["bf16_tflops"])
+    out = {}
+
+    def entry(name, variants, workload_desc):
+        rec = {"workload": workload_desc, "launches": {}}
+        best = None
+        for label, split, dual in variants:
+            step, flops, _ = setup_workload(sfa, dev, stream, name, split, dual)
+            ms = time_device(step, flush, stream, dev, steps, warmup)
+            tf = flops / (ms * 1e-3) / 1e12
+            rec["launches"][label] = {"ms_per_call": round(ms, 4), "tflops": round(tf, 1),
+                                      "frac": round(tf / peak, 4)}
+            rec["attended_tflop_per_call"] = round(flops / 1e12, 4)
+            if best is None or ms < best[1]:
+                best = (label, ms, tf)
+        rec["ms_per_call"] = round(best[1], 4)
+        rec["tflops"] = round(best[2], 1)
+        rec["best_launch"] = best[0]
+        rec["roofline"] = {"bound": "tensor", "achieved": round(best[2], 1), "peak": peak, "unit": "TFLOP/s",
+                           "frac": round(best[2] / peak, 4), "peak_source": f"{peaks['source']} bf16_tflops (burst)"}
+        return rec
+
+    out["tiny"] = {"workload": "tiny: T=4, P=64, H=2, d=64; dense and sink+window {0, t-1, t}",
+                   "launches": {}}
+    for nm in ("tiny_dense", "tiny_sinkwin"):
+        step, flops, _ = setup_workload(sfa, dev, stream, nm)
+        ms = time_device(step, flush, stream, dev, steps, warmup)
+        out["tiny"]["launches"][nm] = {"ms_per_call": round(ms, 4), "attended_gflop": round(flops / 1e9, 5),
+                                       "note": "launch-latency bound (correctness case)"}
+    out["stream"] = entry("stream", [("sfa_forward", 1, False), ("sfa_forward_split n_split=2", 2, False),
+                                     ("sfa_forward_split n_split=4", 4, False)],
+                          "stream: 3 query frames x 1560 after 21 history frames, H=12, d=128; heads 4 local (6 "
+                          "frames), 4 anchor (7), 4 memory (13)")
+    out["long121"] = entry("long121", [("sfa_forward", 1, False)],
+                           "long121: T=121, P=1560, H=12, d=128, LVSA C=21, W=13, T_per=6, s=0 (|A| = 30-32)")
+    out["lsemerge"] = entry("lsemerge", [("local + history + merge (3 calls)", 1, False),
+                                         ("3 calls, n_split=2", 2, False), ("3 calls, n_split=4", 4, False),
+                                         ("sfa_forward_dual n_split=1", 1, True),
+                                         ("sfa_forward_dual n_split=2", 2, True)],
+                            "lsemerge: query frame 13 (1560 rows), H=12, d=128; local {0, 13} + history {1..12}, "
+                            "LSE-merged")
+    if with_cpu:
+        out["tiny"]["cpu_baseline"] = _cpu_record("tiny_dense", "every row of tiny_dense ({rows} rows, float64 C "
+                                                                "oracle, {s:.2f} s)")
+        out["stream"]["cpu_baseline"] = _cpu_record("stream", "every row of the workload ({rows} rows, float64 C "
+                                                              "oracle, {s:.1f} s)")
+        out["lsemerge"]["cpu_baseline"] = _cpu_record("lsemerge", "every row of both branches and their merge "
+                                                                  "({rows} rows, float64, {s:.1f} s)")
+        out["long121"]["cpu_baseline"] = _cpu_record("long121", "the checked rows: 256 seeded rows per head "
+                                                                "({rows} rows, float64 C oracle, {s:.1f} s)",
+                                                     rows_per_head=256)
+    out["merge_2M"] = bench_merge(sfa, dev, stream, flush, rows=2 * 1024 * 1024)
+    out["hsa"] = bench_hsa(sfa, dev, stream, flush, reps=steps)
+    out["gdn"] = bench_gdn(sfa, dev, stream, flush, reps=steps)
+    return out
 
 
 def main():
@@ -660,9 +812,12 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--heads", type=int, default=0,
                     help="run the workload with this many heads instead of 12 (smaller profiling case)")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="leave out the other workloads (stream, long121, lsemerge, tiny, hsa, gdn, large merge)")
     ap.add_argument("--skip-extras", action="store_true",
                     help="time the device step only: no end-to-end, merge or CPU-baseline legs")
-    ap.add_argument("--workload", choices=["lvsa41", "long121", "stream", "lsemerge", "hsa", "gdn"],
+    ap.add_argument("--workload", choices=["lvsa41", "long121", "stream", "lsemerge", "hsa", "gdn", "merge",
+                                           "tiny_dense", "tiny_sinkwin"],
                     default="lvsa41",
                     help="other workloads are timed on the device only (one JSON line, not the bench line)")
     ap.add_argument("--dual", action="store_true",
@@ -679,13 +834,19 @@ def main():
 
     if args.workload != "lvsa41":
         if rank == 0:
-            if args.workload in ("hsa", "gdn"):
+            if args.workload in ("hsa", "gdn", "merge"):
                 import frame_sparse_attention_b200 as sfa
                 sfa.load()
                 dev = torch.device("cuda", 0)
                 flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
-                fn = bench_hsa if args.workload == "hsa" else bench_gdn
-                rec = fn(sfa, dev, torch.cuda.current_stream(dev), flush, reps=args.steps)
+                st = torch.cuda.current_stream(dev)
+                if args.workload == "merge":  # the ISPA shape, 2M rows, and the set builds
+                    rec = {"merge": bench_merge(sfa, dev, st, flush, reps=args.steps),
+                           "merge_2M": bench_merge(sfa, dev, st, flush, reps=args.steps, rows=2 * 1024 * 1024),
+                           "sets": bench_sets(sfa, dev, st, flush, reps=args.steps)}
+                else:
+                    fn = bench_hsa if args.workload == "hsa" else bench_gdn
+                    rec = fn(sfa, dev, st, flush, reps=args.steps)
             else:
                 rec = run_other_workload(args)
             print(json.dumps(rec), flush=True)

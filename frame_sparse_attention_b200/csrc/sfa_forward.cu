@@ -1127,23 +1127,59 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[SFA_NOALLOC_SCR
 
 constexpr int NOALLOC_MAX_DEVICES = 256;
 std::mutex g_noalloc_mutex;
-void *g_noalloc_ptr[NOALLOC_MAX_DEVICES] = {};
+struct NoallocCache {
+    unsigned long long ctx_id;  // the context the address belongs to (0: none yet)
+    void *ptr;
+};
+NoallocCache g_noalloc[NOALLOC_MAX_DEVICES] = {};
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
+
+// Unique id of the calling thread's current context (CUDA contexts get ids that are never
+// reused within a process), or 0 if it cannot be read.
+unsigned long long current_ctx_id()
+{
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(p);
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
+}
 
 // Device address of the scratch array on the current device.  In host code the array's
-// name only stands for it, so the address is looked up once per device, with that device
-// current, and cached.
+// name only stands for it, so the address is looked up with the device current
+// (cudaGetSymbolAddress) and cached per device together with the id of the context it
+// was found in.  A device reset (cudaDeviceReset) replaces the primary context and may
+// move the array; the next call then sees a new context id and looks the address up again.
 sfa_status noalloc_scratch(void **out)
 {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return SFA_ERR_CUDA;
     if (dev < 0 || dev >= NOALLOC_MAX_DEVICES) return SFA_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (!g_noalloc_ptr[dev]) {
+    NoallocCache &c = g_noalloc[dev];
+    const unsigned long long ctx = current_ctx_id();  // 0 before the runtime has set a context current
+    if (!c.ptr || ctx == 0 || c.ctx_id != ctx) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return SFA_ERR_CUDA;
-        g_noalloc_ptr[dev] = p;
+        c.ptr = p;
+        c.ctx_id = current_ctx_id();  // the lookup has made the device's primary context current
     }
-    *out = g_noalloc_ptr[dev];
+    *out = c.ptr;
     return SFA_OK;
 }
 

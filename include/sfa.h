@@ -19,8 +19,11 @@
  *     (0 <= frame < T_kv).  Frame lists hold absolute key/value frame indices.
  *   - Device pointers are plain CUDA device addresses (cudaMalloc / torch memory).
  *     The library never allocates device memory and keeps no state between calls,
- *     apart from a per-process cache of the CUDA driver entry point it uses to
- *     encode TMA descriptors.
+ *     apart from per-process caches of the CUDA driver entry points it uses (to
+ *     encode TMA descriptors and to read the current context's id) and what
+ *     sfa_forward_split_noalloc needs: a fixed scratch array of device memory on
+ *     every GPU that loads the library, whose contents persist from one call to the
+ *     next, and its cached device address.
  *   - Every call validates its arguments on the host first and returns a status;
  *     nothing is printed and nothing throws across the ABI.  Launch errors come
  *     back as SFA_ERR_CUDA.  Errors that only the GPU can see (a malformed frame
@@ -233,8 +236,10 @@ sfa_status sfa_forward_split(const sfa_attn_desc *desc, const void *q, const voi
  *     process exits.  The call allocates nothing (no cudaMalloc, no cudaFree, no
  *     allocating library routine); the caller still passes inputs and outputs.
  *   - The first call on a device looks up the array's device address with that device
- *     current (cudaGetSymbolAddress) and caches it; make that first call before any
- *     stream capture on the device.
+ *     current (cudaGetSymbolAddress) and caches it with the id of the current context;
+ *     make that first call before any stream capture on the device.  After a device
+ *     reset (cudaDeviceReset) the context id changes and the next call looks the
+ *     address up again, so that call too should come before any stream capture.
  *   - Requests needing more than SFA_NOALLOC_SCRATCH_BYTES of workspace (see
  *     sfa_forward_split_workspace) return SFA_ERR_INVALID_ARG without launching.
  *     n_split == 1 needs no workspace.

@@ -35,8 +35,41 @@ def _kw(w):
                 k_frames=w.k_frames, k_blocks=w.k_blocks)
 
 
+def _valid_top(scores: dict, chosen: set, k: int) -> bool:
+    """chosen is a top-k set of the candidates in scores within SCORE_EPS: it has
+    min(k, n) members and none of the others scores more than SCORE_EPS above any of them."""
+    if len(chosen) != min(k, len(scores)) or not chosen <= set(scores):
+        return False
+    rest = [s for i, s in scores.items() if i not in chosen]
+    return not chosen or not rest or min(scores[i] for i in chosen) >= max(rest) - SCORE_EPS
+
+
+def _frame_sets(fs: dict, n_sel: int, must: set):
+    """Every top-n_sel frame set within SCORE_EPS (fs: frame -> fp64 score) that holds
+    the frames in must.  A frame scoring more than SCORE_EPS above the (n_sel+1)-th score
+    is in every such set, one scoring more than SCORE_EPS below the n_sel-th in none."""
+    from itertools import combinations
+    order = sorted(fs.values(), reverse=True)
+    if n_sel == 0:
+        return [set()]
+    hi = order[n_sel] if n_sel < len(order) else -math.inf
+    lo = order[n_sel - 1]
+    fixed = {f for f, s in fs.items() if s > hi + SCORE_EPS}
+    band = [f for f, s in fs.items() if f not in fixed and s >= lo - SCORE_EPS]
+    out = []
+    for extra in combinations(sorted(band), n_sel - len(fixed)):
+        F = fixed | set(extra)
+        if must <= F and _valid_top(fs, F, n_sel):
+            out.append(F)
+    return out
+
+
 def _check_selection(w, q, k, lists_gpu, counts_gpu):
-    """Exact where the fp64 scores decide clearly; a valid selection elsewhere."""
+    """Lists identical to the oracle's wherever the fp64 scores decide clearly; elsewhere
+    the GPU list must be a valid selection within SCORE_EPS: the always-attended blocks,
+    a top-k_frames set of the history frames, and a top-k_blocks set of those frames'
+    blocks (a near tie at either level is the only way two valid lists can differ).
+    Returns the number of lists that differ."""
     kw = _kw(w)
     Amax = lists_gpu.shape[-1]
     o_lists, o_counts = hsa.build_block_lists(q.float().numpy(), k.float().numpy(), Bmax=Amax, **kw)
@@ -58,15 +91,18 @@ def _check_selection(w, q, k, lists_gpu, counts_gpu):
                     if got == want:
                         continue
                     n_close += 1
-                    # not identical: both selections must be equally good within SCORE_EPS
-                    fs = {f: float(np.dot(qb[b, h, t, i], kf[b, h, f])) for f in hist}
-                    n_sel = min(w.k_frames, len(hist))
-                    kth = sorted(fs.values(), reverse=True)[n_sel - 1] if n_sel else math.inf
                     assert got == sorted(set(got))
                     assert all(f * nb + x in got for f in always for x in range(nb))
                     picked = [g for g in got if g // nb not in always]
-                    assert len(picked) == min(w.k_blocks, n_sel * nb)
-                    assert all(fs[g // nb] >= kth - SCORE_EPS for g in picked)
+                    fs = {f: float(np.dot(qb[b, h, t, i], kf[b, h, f])) for f in hist}
+                    n_sel = min(w.k_frames, len(hist))
+                    ok = False
+                    for F in _frame_sets(fs, n_sel, {g // nb for g in picked}):
+                        bs = {f * nb + x: float(np.dot(qb[b, h, t, i], kb[b, h, f, x])) for f in F for x in range(nb)}
+                        if _valid_top(bs, set(picked), w.k_blocks):
+                            ok = True
+                            break
+                    assert ok, f"list ({b}, {h}, {t}, {i}) is not a valid selection: {got} (oracle {want})"
     return n_close
 
 
@@ -91,6 +127,23 @@ def test_selection_matches_oracle(w):
     torch.cuda.synchronize()
     n_close = _check_selection(w, q, k, blocks.cpu().numpy(), counts.cpu().numpy())
     assert n_close == 0, f"{n_close} lists decided by near-ties"
+
+
+def test_selection_exact_ties_go_to_the_smaller_id():
+    # every history frame a copy of frame 1: all frame scores tie (the first k_frames
+    # history frames win) and every block ties with its copies in the other frames (the
+    # copies in the earliest frames win); pooling is per position inside a frame, so the
+    # GPU's fp32 scores tie exactly too.  The lists must equal the oracle's.
+    w = Workload("hsa_ties", B=1, H=2, Tq=2, Tkv=11, q_off=9, P=300, d=128, n_sink=1, n_prev=1, chunk_len=2,
+                 k_frames=3, k_blocks=4, heads=(SetSpec("hsa"),) * 2)
+    q, k, v = workload_qkv(w, seed=4)
+    k = k.clone()
+    for f in range(2, 8):
+        k[:, :, f * w.P:(f + 1) * w.P] = k[:, :, w.P:2 * w.P]
+    blocks, counts = sfa().hsa_select(q.cuda(), k.cuda(), _params(w), w.k_frames, w.k_blocks)
+    torch.cuda.synchronize()
+    lists, cnts = hsa.build_block_lists(q.float().numpy(), k.float().numpy(), Bmax=blocks.shape[-1], **_kw(w))
+    assert np.array_equal(blocks.cpu().numpy(), lists) and np.array_equal(counts.cpu().numpy(), cnts)
 
 
 @pytest.mark.parametrize("w", SMALL, ids=[w.name for w in SMALL])
@@ -154,7 +207,8 @@ def test_hsa_workload_selection_and_sampled_attention():
     blocks, counts = sfa().hsa_select(q.cuda(), k.cuda(), _params(w), w.k_frames, w.k_blocks)
     torch.cuda.synchronize()
     n_close = _check_selection(w, q, k, blocks.cpu().numpy(), counts.cpu().numpy())
-    assert n_close <= 2, f"{n_close} lists decided by near-ties"
+    print(f"hsa workload: {n_close} of {counts.numel()} lists differ from the oracle's, each a valid "
+          f"selection within a near tie")
     # attention on the oracle's lists, sampled rows (all rows of query frame 0, 256 per head)
     Amax = blocks.shape[-1]
     lists, cnts = hsa.build_block_lists(q.float().numpy(), k.float().numpy(), Bmax=Amax, **_kw(w))
