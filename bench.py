@@ -406,6 +406,11 @@ def bench_hsa(sfa, dev, stream, flush, reps=20):
     split_ws = torch.empty(max(sfa.split_workspace_bytes(desc, 2), 1), dtype=torch.uint8, device=dev)
     fwd2_ms = timed(lambda: sfa.forward_blocks(q, k, v, blocks, counts, w.P, out=o, lse=lse, stream=stream,
                                                n_split=2, workspace=split_ws))
+    nb0 = ctypes.c_size_t(0)
+    sfa.load().sfa_forward_blocks_split_workspace(ctypes.byref(desc), 0, ctypes.byref(nb0))
+    sched_ws = torch.empty(max(nb0.value, 1), dtype=torch.uint8, device=dev)
+    fwd0_ms = timed(lambda: sfa.forward_blocks(q, k, v, blocks, counts, w.P, out=o, lse=lse, stream=stream,
+                                               n_split=0, workspace=sched_ws))
     flops = block_list_flops(blocks.cpu().numpy(), counts.cpu().numpy(), w.P, w.d)
     peak = float(measured_peaks()["bf16_tflops"])
     tf = flops / (fwd_ms * 1e-3) / 1e12
@@ -430,6 +435,8 @@ def bench_hsa(sfa, dev, stream, flush, reps=20):
             "forward_blocks_ms": round(fwd_ms, 4), "attended_tflop": round(flops / 1e12, 4),
             "forward_tflops": round(tf, 1), "forward_frac": round(tf / peak, 4),
             "forward_blocks_split2_ms": round(fwd2_ms, 4),
+            "forward_blocks_scheduled_ms": round(fwd0_ms, 4),
+            "forward_scheduled_tflops": round(flops / (fwd0_ms * 1e-3) / 1e12, 1),
             "forward_split2_tflops": round(flops / (fwd2_ms * 1e-3) / 1e12, 1),
             "step_tflops": round(flops / ((sel_ms + fwd_ms) * 1e-3) / 1e12, 1),
             "mean_blocks_per_list": round(float(counts.float().mean().item()), 2),
@@ -654,7 +661,7 @@ def setup_workload(sfa, dev, stream, name, split=1, dual=False):
             return
         for (w, params, kinds, extra, Amax, fr, cn, o, lse, wsp) in branches:
             sfa.build_sets(params, kinds, extra, Amax, fr, cn, stream=stream)
-            if split > 1:
+            if split != 1:  # 0: scheduled (the library's ranges, longest first)
                 sfa.forward_split(q, k, v, fr, cn, w.P, split, out=o, lse=lse, workspace=wsp, stream=stream)
             else:
                 sfa.forward(q, k, v, fr, cn, w.P, out=o, lse=lse, stream=stream)
@@ -775,15 +782,18 @@ def bench_workloads(sfa, dev, stream, flush, steps=20, warmup=5, with_cpu=True):
         out["tiny"]["launches"][nm] = {"ms_per_call": round(ms, 4), "attended_gflop": round(flops / 1e9, 5),
                                        "note": "launch-latency bound (correctness case)"}
     out["stream"] = entry("stream", [("sfa_forward", 1, False), ("sfa_forward_split n_split=2", 2, False),
-                                     ("sfa_forward_split n_split=4", 4, False)],
+                                     ("sfa_forward_split n_split=4", 4, False),
+                                     ("sfa_forward_split scheduled (n_split=0)", 0, False)],
                           "stream: 3 query frames x 1560 after 21 history frames, H=12, d=128; heads 4 local (6 "
                           "frames), 4 anchor (7), 4 memory (13)")
-    out["long121"] = entry("long121", [("sfa_forward", 1, False)],
+    out["long121"] = entry("long121", [("sfa_forward", 1, False), ("sfa_forward_split scheduled (n_split=0)", 0, False)],
                            "long121: T=121, P=1560, H=12, d=128, LVSA C=21, W=13, T_per=6, s=0 (|A| = 30-32)")
     out["lsemerge"] = entry("lsemerge", [("local + history + merge (3 calls)", 1, False),
                                          ("3 calls, n_split=2", 2, False), ("3 calls, n_split=4", 4, False),
+                                         ("3 calls, scheduled (n_split=0)", 0, False),
                                          ("sfa_forward_dual n_split=1", 1, True),
-                                         ("sfa_forward_dual n_split=2", 2, True)],
+                                         ("sfa_forward_dual n_split=2", 2, True),
+                                         ("sfa_forward_dual scheduled (n_split=0)", 0, True)],
                             "lsemerge: query frame 13 (1560 rows), H=12, d=128; local {0, 13} + history {1..12}, "
                             "LSE-merged")
     if with_cpu:

@@ -7,7 +7,8 @@ Python face of libsfa.so (C ABI in include/sfa.h):
 * ``forward``     - softmax attention over the tokens of A(h, t) only, O bf16 + LSE fp32
 * ``forward_host`` - the same for pinned host tensors, copies pipelined with the attention
 * ``forward_split`` - the same with each unit's key tiles split over several CTAs and the
-                    partials merged by LSE (short or uneven grids)
+                    partials merged by LSE (short or uneven grids); ``n_split=0`` lets the
+                    library choose the split and run the CTAs longest first
 * ``forward_paged`` - the same with K/V read through a per-head frame -> slot table
 * ``forward_dual`` - local and history branches in one launch: the local result and their
                     LSE merge (the full attention)
@@ -25,11 +26,11 @@ from ._lib import (SET_KINDS, SFA_DEBUG_STALL_SOFTMAX, SFA_ERR_BAD_SET, SFA_ERR_
                    forward_host,
                    forward_paged, forward_split, gdn_forward, GdnDesc, hsa_max_count, hsa_select, load, lse_merge,
                    set_max_count,
-                   set_params, split_workspace_bytes, version)
+                   set_params, split_plan, split_workspace_bytes, version)
 
 __all__ = ["SET_KINDS", "SFA_DEBUG_STALL_SOFTMAX", "SFA_ERR_BAD_SET", "SFA_ERR_CUDA",
            "SFA_ERR_INVALID_ARG", "SFA_ERR_TIMEOUT", "SFA_ERR_UNSUPPORTED", "SFA_OK", "AttnDesc",
            "SetParams", "SfaError", "attn_desc", "build_sets", "error_string", "forward", "forward_blocks",
            "forward_dual", "forward_host",
            "forward_paged", "forward_split", "gdn_forward", "GdnDesc", "hsa_max_count", "hsa_select",
-           "load", "lse_merge", "set_max_count", "set_params", "split_workspace_bytes", "version"]
+           "load", "lse_merge", "set_max_count", "set_params", "split_plan", "split_workspace_bytes", "version"]

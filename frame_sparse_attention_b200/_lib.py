@@ -60,7 +60,7 @@ _lib = None
 EXPORTS = ("sfa_error_string", "sfa_version", "sfa_set_max_count", "sfa_build_sets", "sfa_forward",
            "sfa_forward_split_workspace", "sfa_forward_split", "sfa_forward_split_noalloc", "sfa_forward_paged",
            "sfa_lse_merge", "sfa_hsa_max_count", "sfa_hsa_workspace", "sfa_hsa_select", "sfa_forward_blocks",
-           "sfa_forward_blocks_split",
+           "sfa_forward_blocks_split", "sfa_forward_blocks_split_workspace", "sfa_forward_split_plan",
            "sfa_forward_dual_workspace", "sfa_forward_dual", "sfa_gdn_workspace", "sfa_gdn_forward")
 
 
@@ -117,6 +117,10 @@ def load():
     lib.sfa_forward_blocks_split.restype = st
     lib.sfa_forward_blocks_split.argtypes = [ctypes.POINTER(AttnDesc), vp, vp, vp, vp, vp, vp, vp, i32, vp,
                                              ctypes.c_size_t, vp, vp]
+    lib.sfa_forward_blocks_split_workspace.restype = st
+    lib.sfa_forward_blocks_split_workspace.argtypes = [ctypes.POINTER(AttnDesc), i32, ctypes.POINTER(ctypes.c_size_t)]
+    lib.sfa_forward_split_plan.restype = st
+    lib.sfa_forward_split_plan.argtypes = [ctypes.POINTER(AttnDesc), i32, i32, ctypes.POINTER(i32), ctypes.POINTER(i32)]
     lib.sfa_forward_blocks.restype = st
     lib.sfa_forward_blocks.argtypes = [ctypes.POINTER(AttnDesc), vp, vp, vp, vp, vp, vp, vp, vp, vp]
     _lib = lib
@@ -273,10 +277,19 @@ def split_workspace_bytes(desc: AttnDesc, n_split: int) -> int:
     return out.value
 
 
+def split_plan(desc: AttnDesc, n_lists: int = 1, key_blocks: bool = False) -> tuple:
+    """Key-tile ranges per unit that a scheduled call (n_split = 0) uses: (k_first, k_second)."""
+    k0, k1 = ctypes.c_int32(0), ctypes.c_int32(0)
+    _check(load().sfa_forward_split_plan(ctypes.byref(desc), n_lists, 1 if key_blocks else 0, ctypes.byref(k0),
+                                         ctypes.byref(k1)), "sfa_forward_split_plan")
+    return k0.value, k1.value
+
+
 def forward_split(q, k, v, frames, counts, P: int, n_split: int, scale: float | None = None, out=None,
                   lse=None, workspace=None, dev_status=None, stream=None, timeout_us: int = 0):
     """Split-KV frame-sparse attention (same result as forward); workspace is allocated
-    here with torch when not given."""
+    here with torch when not given.  n_split = 0: the library chooses the ranges and runs
+    the CTAs longest range first (a scheduled launch)."""
     B, H, Lq, d = q.shape
     if out is None:
         out = torch.empty_like(q)
@@ -355,7 +368,9 @@ def hsa_select(q, k, params: SetParams, k_frames: int, k_blocks: int, Amax: int 
 
 def forward_blocks(q, k, v, blocks, counts, P: int, scale: float | None = None, out=None, lse=None,
                    dev_status=None, stream=None, timeout_us: int = 0, n_split: int = 1, workspace=None):
-    """Attention of every query block over its key-block list: (O bf16 like q, LSE fp32)."""
+    """Attention of every query block over its key-block list: (O bf16 like q, LSE fp32).
+    n_split > 1 cuts every unit's key tiles into ranges merged by LSE; 0 schedules the
+    launch (the library's choice of ranges, longest first)."""
     B, H, Lq, d = q.shape
     if out is None:
         out = torch.empty_like(q)
@@ -377,7 +392,10 @@ def forward_blocks(q, k, v, blocks, counts, P: int, scale: float | None = None, 
                                          _ptr(dev_status), _stream(stream)), "sfa_forward_blocks")
         return out, lse
     if workspace is None:
-        workspace = torch.empty(max(split_workspace_bytes(desc, n_split), 1), dtype=torch.uint8, device=q.device)
+        nbytes = ctypes.c_size_t(0)
+        _check(load().sfa_forward_blocks_split_workspace(ctypes.byref(desc), n_split, ctypes.byref(nbytes)),
+               "sfa_forward_blocks_split_workspace")
+        workspace = torch.empty(max(nbytes.value, 1), dtype=torch.uint8, device=q.device)
     _check(load().sfa_forward_blocks_split(ctypes.byref(desc), q.data_ptr(), k.data_ptr(), v.data_ptr(),
                                            blocks.data_ptr(), counts.data_ptr(), out.data_ptr(), lse.data_ptr(),
                                            n_split, workspace.data_ptr(), workspace.numel(), _ptr(dev_status),

@@ -114,6 +114,8 @@ struct FwdArgs {
     const int32_t *frames2;  // second list set (two-branch launch: grid y = 2 x splits), or null
     const int32_t *counts2;
     int32_t n_lists;         // 1, or 2 with frames2 / counts2
+    const int2 *items;       // scheduled launch: one work item per CTA (see schedule_kernel), or null
+    int32_t k_first;         // scheduled launch: key-tile ranges of list set 0 (its partial slices)
     float *lse;
     int32_t *status;
     uint64_t timeout_ns;
@@ -822,7 +824,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // work unit: (b, h, t, pair of query tiles), pair fastest so that the tiles sharing
     // one frame's K/V run side by side; the last pair of a frame may hold one tile only
     const int n_pairs = (a.n_qtiles + 1) / 2;
-    int x = blockIdx.x;
+    // work unit and key-tile range: from the CTA's work item (scheduled launch, longest
+    // ranges first), or grid y = list set x split: CTA (unit, y) takes list set y / n_split
+    // and key-tile range y mod n_split of it
+    int x, li, split, n_split, slice;
+    if (a.items) {
+        const int2 w = a.items[blockIdx.x];
+        x = w.x;
+        li = w.y & 1;
+        split = (w.y >> 1) & 255;
+        n_split = w.y >> 9;
+        slice = li ? a.k_first + split : split;
+    } else {
+        x = blockIdx.x;
+        n_split = gridDim.y / a.n_lists;
+        li = blockIdx.y / n_split;
+        split = blockIdx.y - li * n_split;
+        slice = blockIdx.y;
+    }
     const int qt_a = 2 * (x % n_pairs);
     const bool has_b = qt_a + 1 < a.n_qtiles;
     x /= n_pairs;
@@ -830,10 +849,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     x /= a.Tq;
     const int h = x % a.H;
     const int b = x / a.H;
-    // grid y = list set x split: CTA (unit, y) takes list set y / n_split and key-tile range
-    // y mod n_split of it, and with more than one y writes slice y of the partial outputs
-    const int n_split = gridDim.y / a.n_lists;
-    const int li = blockIdx.y / n_split, split = blockIdx.y - li * n_split;
     // the unit's list: frames of (h, t), or key blocks of (b, h, t, query block = pair)
     const int64_t list = a.nblk ? ((((int64_t)b * a.H + h) * a.Tq + t) * n_pairs + qt_a / 2) : (int64_t)h * a.Tq + t;
     const int32_t *fl = (li ? a.frames2 : a.frames) + list * a.Amax;
@@ -844,11 +859,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     : -1;
     const bool bad_set = n_all < 0;
     if (bad_set) n_all = 0;
-    // split-KV: CTA (unit, split) takes the unit's key tiles [t_off, t_off + n_tiles) and
-    // writes a partial result into slice blockIdx.y of the output (batch index b_out)
+    // split-KV: CTA (unit, split) takes the unit's key tiles [t_off, t_off + n_tiles) and,
+    // with more than one slice, writes a partial result into its slice of the output
+    // (batch index b_out)
     const int t_off = (int)(((int64_t)n_all * split) / n_split);
     int n_tiles = (int)(((int64_t)n_all * (split + 1)) / n_split) - t_off;
-    const int b_out = blockIdx.y * a.B + b;
+    const int b_out = slice * a.B + b;
     volatile int32_t *skip = reinterpret_cast<volatile int32_t *>(smem + C::SMEM_BAR + 248);
 
     if (threadIdx.x == 0) {
@@ -902,6 +918,101 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
 }
 
+// ----------------------------------------------------------------- scheduled launches
+// A scheduled launch runs one CTA per work item: (list set, unit, key-tile range), the
+// ranges of list set l being k_l equal parts of the unit's key tiles.  The items are
+// ordered longest range first (a counting sort on the range length, computed from the
+// lists on the device), so that the hardware block scheduler, which hands CTAs to SMs in
+// index order as they free up, runs a longest-processing-time-first schedule: long units
+// start in the first wave and short ones fill the tail.  Items of one list stay together
+// (query-tile pairs fastest), so the CTAs that share the list's keys run side by side.
+constexpr int SCHED_THREADS = 1024;
+constexpr int SCHED_BINS = 2048;  // range lengths (key tiles) at or above the last bin share it
+
+struct SchedArgs {
+    const int32_t *frames[2];
+    const int32_t *counts[2];
+    int32_t k[2];      // key-tile ranges per unit of each list set
+    int32_t n_lists;   // list sets (1 or 2)
+    int32_t B, H, Tq, T_kv, P, Amax, nblk, n_pairs, n_slots;
+    const int32_t *slots;
+    int2 *items;
+};
+
+// Key tiles of entry e of list set li (0 for a malformed list: the forward CTA reports it).
+__device__ int sched_len(const SchedArgs &s, int li, int e)
+{
+    const int32_t *fl = s.frames[li] + (int64_t)e * s.Amax;
+    const int cnt = __ldg(s.counts[li] + e);
+    if (cnt < 0 || cnt > s.Amax) return 0;
+    const int h = s.nblk ? (e / (s.Tq * s.n_pairs)) % s.H : e / s.Tq;
+    const int32_t *srow = s.slots ? s.slots + (int64_t)h * s.T_kv : nullptr;
+    const int n = count_tiles(fl, cnt, s.nblk ? s.T_kv * s.nblk : s.T_kv, s.P, s.nblk, srow, s.n_slots);
+    return n > 0 ? n : 0;
+}
+
+__global__ void __launch_bounds__(SCHED_THREADS) schedule_kernel(const __grid_constant__ SchedArgs s)
+{
+    __shared__ int bins[SCHED_BINS];
+    __shared__ int wsum[SCHED_THREADS / 32];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // entries: frame lists per (h, t), or key-block lists per unit; units per entry
+    const int per_set = s.nblk ? s.B * s.H * s.Tq * s.n_pairs : s.H * s.Tq;
+    const int fan = s.nblk ? 1 : s.B * s.n_pairs;
+    const int n_entries = per_set * s.n_lists;
+    for (int i = tid; i < SCHED_BINS; i += SCHED_THREADS) bins[i] = 0;
+    __syncthreads();
+    for (int e = tid; e < n_entries; e += SCHED_THREADS) {
+        const int li = e / per_set, k = s.k[li];
+        const int key = min(SCHED_BINS - 1, (sched_len(s, li, e - li * per_set) + k - 1) / k);
+        atomicAdd(&bins[key], fan * k);
+    }
+    __syncthreads();
+    // exclusive prefix over the bins in descending length: thread t owns the bins of
+    // lengths SCHED_BINS-1-2t and SCHED_BINS-2-2t
+    static_assert(SCHED_BINS == 2 * SCHED_THREADS, "two bins per thread");
+    const int k0 = SCHED_BINS - 1 - 2 * tid, k1 = k0 - 1;
+    const int v0 = bins[k0], v1 = bins[k1], mine = v0 + v1;
+    int incl = mine;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int w = wsum[lane], wi = w;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, wi, off);
+            if (lane >= off) wi += y;
+        }
+        wsum[lane] = wi - w;  // exclusive
+    }
+    __syncthreads();
+    const int excl = wsum[warp] + incl - mine;
+    bins[k0] = excl;       // now: the next free item index of each length
+    bins[k1] = excl + v0;
+    __syncthreads();
+    for (int e = tid; e < n_entries; e += SCHED_THREADS) {
+        const int li = e / per_set, le = e - li * per_set, k = s.k[li];
+        const int key = min(SCHED_BINS - 1, (sched_len(s, li, le) + k - 1) / k);
+        int off = atomicAdd(&bins[key], fan * k);
+        for (int sp = 0; sp < k; ++sp) {
+            const int tag = li | (sp << 1) | (k << 9);
+            if (s.nblk) {
+                s.items[off++] = make_int2(le, tag);
+            } else {
+                const int h = le / s.Tq, t = le - h * s.Tq;
+                for (int b = 0; b < s.B; ++b)
+                    for (int pr = 0; pr < s.n_pairs; ++pr)
+                        s.items[off++] = make_int2(((b * s.H + h) * s.Tq + t) * s.n_pairs + pr, tag);
+            }
+        }
+    }
+}
+
 // ----------------------------------------------------------------- host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
@@ -946,20 +1057,29 @@ bool stride_ok(const int64_t *s, int d)
     return s[2] >= d;
 }
 
+// Scheduled launch: key-tile ranges per unit of each list set, and room for the work items.
+struct Schedule {
+    int k0, k1;
+    int2 *items;
+};
+
 // Forward launch.  n_split == 1: O and LSE go to the caller's buffers.  n_split > 1:
 // every unit's key tiles are split into n_split ranges, CTA (unit, split) writes its
 // partial O / LSE into the workspace slices [split][B][H][Tq*P][d] (bf16, contiguous) and
-// [split][B][H][Tq*P] (fp32), and a k-way LSE merge writes the caller's O and LSE.
+// [split][B][H][Tq*P] (fp32), and a k-way LSE merge writes the caller's O and LSE.  With a
+// schedule the list sets take k0 and k1 ranges, one CTA per work item, longest first.
 template <int D>
 sfa_status launch(const sfa_attn_desc *d, const void *q, const void *k, const void *v, const int32_t *frames,
                   const int32_t *counts, void *o, float *lse, int32_t *dev_status, cudaStream_t stream,
                   int n_split = 1, void *ws_o = nullptr, float *ws_lse = nullptr, const int32_t *slots = nullptr,
                   int n_slots = 0, int nblk = 0, const int32_t *frames2 = nullptr, const int32_t *counts2 = nullptr,
-                  void *o_first = nullptr, float *lse_first = nullptr)
+                  void *o_first = nullptr, float *lse_first = nullptr, const Schedule *sched = nullptr)
 {
     using C = Cfg<D>;
     const int n_lists = frames2 ? 2 : 1;
-    const int slices = n_lists * n_split;  // partial outputs (1: straight to o / lse)
+    // partial outputs (1: straight to o / lse)
+    const int slices = sched ? sched->k0 + (n_lists == 2 ? sched->k1 : 0) : n_lists * n_split;
+    const int k_first = sched ? sched->k0 : n_split;
     CUtensorMap tq, tk, tv, to;
     const int kv_frames = slots ? n_slots : d->T_kv;  // frames held by the K/V buffers
     const uint64_t P = d->P, Tq = d->Tq, Lkv = (uint64_t)kv_frames * d->P;
@@ -1006,6 +1126,8 @@ sfa_status launch(const sfa_attn_desc *d, const void *q, const void *k, const vo
     a.frames2 = frames2;
     a.counts2 = counts2;
     a.n_lists = n_lists;
+    a.items = sched ? sched->items : nullptr;
+    a.k_first = k_first;
     a.status = dev_status;
     a.timeout_ns = (uint64_t)(d->timeout_us ? d->timeout_us : DEFAULT_TIMEOUT_US) * 1000;
     a.debug_flags = d->debug_flags;
@@ -1014,13 +1136,40 @@ sfa_status launch(const sfa_attn_desc *d, const void *q, const void *k, const vo
     if (cudaFuncSetAttribute(sfa_forward_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
         cudaSuccess)
         return SFA_ERR_CUDA;
-    sfa_forward_kernel<D><<<dim3((unsigned)grid, (unsigned)slices), NUM_THREADS, C::SMEM_BYTES, stream>>>(
-        tq, tk, tv, to, a);
+    if (sched) {
+        SchedArgs sa;
+        sa.frames[0] = frames;
+        sa.counts[0] = counts;
+        sa.frames[1] = frames2 ? frames2 : frames;
+        sa.counts[1] = counts2 ? counts2 : counts;
+        sa.k[0] = sched->k0;
+        sa.k[1] = n_lists == 2 ? sched->k1 : 0;
+        sa.n_lists = n_lists;
+        sa.B = d->B;
+        sa.H = d->H;
+        sa.Tq = d->Tq;
+        sa.T_kv = d->T_kv;
+        sa.P = d->P;
+        sa.Amax = d->Amax;
+        sa.nblk = nblk;
+        sa.n_pairs = (a.n_qtiles + 1) / 2;
+        sa.n_slots = kv_frames;
+        sa.slots = slots;
+        sa.items = sched->items;
+        schedule_kernel<<<1, SCHED_THREADS, 0, stream>>>(sa);
+        sfa_status st0 = launch_status();
+        if (st0 != SFA_OK) return st0;
+        const int64_t n_items = grid * (sched->k0 + (n_lists == 2 ? sched->k1 : 0));
+        sfa_forward_kernel<D><<<dim3((unsigned)n_items, 1), NUM_THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, to, a);
+    } else {
+        sfa_forward_kernel<D><<<dim3((unsigned)grid, (unsigned)slices), NUM_THREADS, C::SMEM_BYTES, stream>>>(
+            tq, tk, tv, to, a);
+    }
     sfa_status st = launch_status();
     if (st != SFA_OK || slices == 1) return st;
     const int64_t Lq = (int64_t)d->Tq * d->P;
     return launch_lse_combine((int64_t)d->B * d->H * Lq, slices, D, d->H, Lq, ws_o, ws_lse, o, d->o_stride, lse,
-                              stream, n_lists == 2 ? n_split : 0, o_first, lse_first);
+                              stream, n_lists == 2 ? k_first : 0, o_first, lse_first);
 }
 
 size_t split_ws_o_bytes(const sfa_attn_desc *d, int n_split)
@@ -1033,6 +1182,79 @@ size_t split_ws_bytes(const sfa_attn_desc *d, int n_split)
 {
     const size_t rows = (size_t)d->B * d->H * d->Tq * d->P;
     return split_ws_o_bytes(d, n_split) + ((size_t)n_split * rows * 4 + 255) / 256 * 256;
+}
+
+// ----------------------------------------------------------------- automatic split
+// n_split = 0 asks for a scheduled launch with the key-tile ranges per unit chosen here.
+// The host does not see the lists (they live on the device), so the choice uses Amax as
+// every unit's length (an upper bound) and models the launch as waves of equal pieces,
+// each a range plus a fixed prologue / epilogue cost, plus the merge of the partials;
+// the schedule kernel then orders the real ranges longest first.
+constexpr double SCHED_OVERHEAD_TILES = 3.0;  // Q load, pipeline fill, epilogue of one CTA, in key tiles
+constexpr double STEP_US = 2.4;               // one key tile of a CTA (both query tiles), measured
+constexpr double HBM_BYTES_PER_US = 6.5e6;
+
+int sm_count()
+{
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return sms > 0 ? sms : 148;
+}
+
+// Ranges per unit (k0 for the first list set, k1 for the second) of a scheduled launch.
+void auto_splits(const sfa_attn_desc *d, int n_lists, int nblk, int &k0, int &k1)
+{
+    const int sms = sm_count();
+    const int n_qt = (d->P + BM - 1) / BM;
+    const double units = (double)d->B * d->H * d->Tq * ((n_qt + 1) / 2);
+    const double len = nblk ? (double)d->Amax : (double)d->Amax * n_qt;  // key tiles per unit, at most
+    const int cap = d->d / 8;                                           // partial slices the merge takes
+    const double slice_bytes = (double)d->B * d->H * d->Tq * d->P * (2.0 * d->d + 4.0);
+    auto cost = [&](int pieces_per_unit, int longest_k, int slices) {
+        const double piece = std::ceil(len / longest_k) + SCHED_OVERHEAD_TILES;
+        const double waves = std::ceil(units * pieces_per_unit / sms);
+        const double merge = slices > 1 ? (slices + 1) * slice_bytes / HBM_BYTES_PER_US : 0.0;
+        return waves * piece * STEP_US + merge;
+    };
+    k1 = 0;
+    if (n_lists == 1) {
+        k0 = 1;
+        if (units >= 8.0 * sms) return;  // many full waves: splitting only adds merge traffic
+        double best = cost(1, 1, 1);
+        for (int k = 2; k <= cap; ++k) {
+            const double c = cost(k, k, k);
+            if (c < best) {
+                best = c;
+                k0 = k;
+            }
+        }
+        return;
+    }
+    // two list sets sharing Amax: the first (local) branch is the short one and keeps one
+    // range per unit; the second (history) branch is split
+    k0 = 1;
+    k1 = 1;
+    double best = cost(2, 1, 2);
+    for (int k = 2; k + 1 <= cap; ++k) {
+        const double c = cost(1 + k, k, 1 + k);
+        if (c < best) {
+            best = c;
+            k1 = k;
+        }
+    }
+}
+
+size_t sched_items_bytes(const sfa_attn_desc *d, int pieces_per_unit)
+{
+    const size_t grid = (size_t)d->B * d->H * d->Tq * (((d->P + BM - 1) / BM + 1) / 2);
+    return (grid * pieces_per_unit * sizeof(int2) + 255) / 256 * 256;
+}
+
+// Workspace of a scheduled launch: the partial slices (when there are several), then the items.
+size_t sched_ws_bytes(const sfa_attn_desc *d, int k0, int k1)
+{
+    const int slices = k0 + k1;
+    return (slices > 1 ? split_ws_bytes(d, slices) : 0) + sched_items_bytes(d, slices);
 }
 
 sfa_status check_desc(const sfa_attn_desc *d)
@@ -1083,8 +1305,27 @@ extern "C" sfa_status sfa_forward_split_workspace(const sfa_attn_desc *d, int32_
 {
     sfa_status st = check_desc(d);
     if (st != SFA_OK) return st;
-    if (!bytes || n_split < 1 || n_split > d->d / 8) return SFA_ERR_INVALID_ARG;
+    if (!bytes || n_split < 0 || n_split > d->d / 8) return SFA_ERR_INVALID_ARG;
+    if (n_split == 0) {
+        int k0, k1;
+        auto_splits(d, 1, 0, k0, k1);
+        *bytes = sched_ws_bytes(d, k0, 0);
+        return SFA_OK;
+    }
     *bytes = n_split == 1 ? 0 : split_ws_bytes(d, n_split);
+    return SFA_OK;
+}
+
+extern "C" sfa_status sfa_forward_split_plan(const sfa_attn_desc *d, int32_t n_lists, int32_t key_blocks,
+                                             int32_t *k_first, int32_t *k_second)
+{
+    sfa_status st = check_desc(d);
+    if (st != SFA_OK) return st;
+    if (!k_first || (n_lists != 1 && n_lists != 2) || (key_blocks && n_lists != 1)) return SFA_ERR_INVALID_ARG;
+    int k0, k1;
+    auto_splits(d, n_lists, key_blocks ? (d->P + KEY_BLOCK - 1) / KEY_BLOCK : 0, k0, k1);
+    *k_first = k0;
+    if (k_second) *k_second = k1;
     return SFA_OK;
 }
 
@@ -1095,11 +1336,26 @@ extern "C" sfa_status sfa_forward_split(const sfa_attn_desc *d, const void *q, c
 {
     sfa_status st = check_desc(d);
     if (st != SFA_OK) return st;
-    if (n_split < 1 || n_split > d->d / 8) return SFA_ERR_INVALID_ARG;
+    if (n_split < 0 || n_split > d->d / 8) return SFA_ERR_INVALID_ARG;
     if (d->B == 0) return SFA_OK;
     st = check_buffers(d, q, k, v, frames, counts, o, lse);
     if (st != SFA_OK) return st;
     cudaStream_t s = as_cuda(stream);
+    if (n_split == 0) {  // scheduled: ranges chosen here, longest first
+        Schedule sc;
+        auto_splits(d, 1, 0, sc.k0, sc.k1);
+        if (!workspace || reinterpret_cast<uintptr_t>(workspace) % 256 || workspace_bytes < sched_ws_bytes(d, sc.k0, 0))
+            return SFA_ERR_INVALID_ARG;
+        uint8_t *ws = static_cast<uint8_t *>(workspace);
+        sc.items = reinterpret_cast<int2 *>(ws + (sc.k0 > 1 ? split_ws_bytes(d, sc.k0) : 0));
+        float *ws_lse = reinterpret_cast<float *>(ws + split_ws_o_bytes(d, sc.k0));
+        void *ws_o = sc.k0 > 1 ? workspace : nullptr;
+        if (sc.k0 == 1) ws_lse = nullptr;
+        return d->d == 128 ? launch<128>(d, q, k, v, frames, counts, o, lse, dev_status, s, sc.k0, ws_o, ws_lse,
+                                         nullptr, 0, 0, nullptr, nullptr, nullptr, nullptr, &sc)
+                           : launch<64>(d, q, k, v, frames, counts, o, lse, dev_status, s, sc.k0, ws_o, ws_lse,
+                                        nullptr, 0, 0, nullptr, nullptr, nullptr, nullptr, &sc);
+    }
     if (n_split == 1)
         return d->d == 128 ? launch<128>(d, q, k, v, frames, counts, o, lse, dev_status, s)
                            : launch<64>(d, q, k, v, frames, counts, o, lse, dev_status, s);
@@ -1220,7 +1476,13 @@ extern "C" sfa_status sfa_forward_dual_workspace(const sfa_attn_desc *d, int32_t
 {
     sfa_status st = check_desc(d);
     if (st != SFA_OK) return st;
-    if (!bytes || n_split < 1 || 2 * n_split > d->d / 8) return SFA_ERR_INVALID_ARG;
+    if (!bytes || n_split < 0 || 2 * n_split > d->d / 8) return SFA_ERR_INVALID_ARG;
+    if (n_split == 0) {
+        int k0, k1;
+        auto_splits(d, 2, 0, k0, k1);
+        *bytes = sched_ws_bytes(d, k0, k1);
+        return SFA_OK;
+    }
     *bytes = split_ws_bytes(d, 2 * n_split);
     return SFA_OK;
 }
@@ -1234,12 +1496,30 @@ extern "C" sfa_status sfa_forward_dual(const sfa_attn_desc *d, const void *q, co
 {
     sfa_status st = check_desc(d);
     if (st != SFA_OK) return st;
-    if (n_split < 1 || 2 * n_split > d->d / 8) return SFA_ERR_INVALID_ARG;
+    if (n_split < 0 || 2 * n_split > d->d / 8) return SFA_ERR_INVALID_ARG;
     if (d->B == 0) return SFA_OK;
     st = check_buffers(d, q, k, v, frames_local, counts_local, o_full, lse_full);
     if (st != SFA_OK) return st;
     if (!frames_hist || !counts_hist || !o_local || !lse_local || reinterpret_cast<uintptr_t>(o_local) % 16)
         return SFA_ERR_INVALID_ARG;
+    if (n_split == 0) {  // scheduled: the local branch one range per unit, the history branch split
+        Schedule sc;
+        auto_splits(d, 2, 0, sc.k0, sc.k1);
+        const int slices = sc.k0 + sc.k1;
+        if (!workspace || workspace_bytes < sched_ws_bytes(d, sc.k0, sc.k1) ||
+            reinterpret_cast<uintptr_t>(workspace) % 256)
+            return SFA_ERR_INVALID_ARG;
+        uint8_t *ws = static_cast<uint8_t *>(workspace);
+        sc.items = reinterpret_cast<int2 *>(ws + split_ws_bytes(d, slices));
+        float *ws_lse = reinterpret_cast<float *>(ws + split_ws_o_bytes(d, slices));
+        cudaStream_t s = as_cuda(stream);
+        return d->d == 128 ? launch<128>(d, q, k, v, frames_local, counts_local, o_full, lse_full, dev_status, s,
+                                         sc.k0, workspace, ws_lse, nullptr, 0, 0, frames_hist, counts_hist, o_local,
+                                         lse_local, &sc)
+                           : launch<64>(d, q, k, v, frames_local, counts_local, o_full, lse_full, dev_status, s,
+                                        sc.k0, workspace, ws_lse, nullptr, 0, 0, frames_hist, counts_hist, o_local,
+                                        lse_local, &sc);
+    }
     const size_t need = split_ws_bytes(d, 2 * n_split);
     if (!workspace || workspace_bytes < need || reinterpret_cast<uintptr_t>(workspace) % 256)
         return SFA_ERR_INVALID_ARG;
@@ -1255,6 +1535,21 @@ extern "C" sfa_status sfa_forward_dual(const sfa_attn_desc *d, const void *q, co
 // Key-block lists (hierarchical selection): each (b, h, t, query block of 256 rows) has
 // its own sorted list of 128-token key blocks.
 // ------------------------------------------------------------------------------------
+extern "C" sfa_status sfa_forward_blocks_split_workspace(const sfa_attn_desc *d, int32_t n_split, size_t *bytes)
+{
+    sfa_status st = check_desc(d);
+    if (st != SFA_OK) return st;
+    if (!bytes || n_split < 0 || n_split > d->d / 8) return SFA_ERR_INVALID_ARG;
+    if (n_split == 0) {
+        int k0, k1;
+        auto_splits(d, 1, (d->P + KEY_BLOCK - 1) / KEY_BLOCK, k0, k1);
+        *bytes = sched_ws_bytes(d, k0, 0);
+        return SFA_OK;
+    }
+    *bytes = n_split == 1 ? 0 : split_ws_bytes(d, n_split);
+    return SFA_OK;
+}
+
 extern "C" sfa_status sfa_forward_blocks_split(const sfa_attn_desc *d, const void *q, const void *k, const void *v,
                                                const int32_t *blocks, const int32_t *counts, void *o, float *lse,
                                                int32_t n_split, void *workspace, size_t workspace_bytes,
@@ -1263,12 +1558,26 @@ extern "C" sfa_status sfa_forward_blocks_split(const sfa_attn_desc *d, const voi
     sfa_status st = check_desc(d);
     if (st != SFA_OK) return st;
     if ((int64_t)d->T_kv * ((d->P + KEY_BLOCK - 1) / KEY_BLOCK) >= ((int64_t)1 << 31)) return SFA_ERR_INVALID_ARG;
-    if (n_split < 1 || n_split > d->d / 8) return SFA_ERR_INVALID_ARG;
+    if (n_split < 0 || n_split > d->d / 8) return SFA_ERR_INVALID_ARG;
     if (d->B == 0) return SFA_OK;
     st = check_buffers(d, q, k, v, blocks, counts, o, lse);
     if (st != SFA_OK) return st;
     cudaStream_t s = as_cuda(stream);
     const int nblk = (d->P + KEY_BLOCK - 1) / KEY_BLOCK;
+    if (n_split == 0) {  // scheduled: ranges chosen here, longest first
+        Schedule sc;
+        auto_splits(d, 1, nblk, sc.k0, sc.k1);
+        if (!workspace || reinterpret_cast<uintptr_t>(workspace) % 256 || workspace_bytes < sched_ws_bytes(d, sc.k0, 0))
+            return SFA_ERR_INVALID_ARG;
+        uint8_t *ws = static_cast<uint8_t *>(workspace);
+        sc.items = reinterpret_cast<int2 *>(ws + (sc.k0 > 1 ? split_ws_bytes(d, sc.k0) : 0));
+        void *ws_o = sc.k0 > 1 ? workspace : nullptr;
+        float *ws_lse = sc.k0 > 1 ? reinterpret_cast<float *>(ws + split_ws_o_bytes(d, sc.k0)) : nullptr;
+        return d->d == 128 ? launch<128>(d, q, k, v, blocks, counts, o, lse, dev_status, s, sc.k0, ws_o, ws_lse,
+                                         nullptr, 0, nblk, nullptr, nullptr, nullptr, nullptr, &sc)
+                           : launch<64>(d, q, k, v, blocks, counts, o, lse, dev_status, s, sc.k0, ws_o, ws_lse, nullptr,
+                                        0, nblk, nullptr, nullptr, nullptr, nullptr, &sc);
+    }
     if (n_split == 1)
         return d->d == 128 ? launch<128>(d, q, k, v, blocks, counts, o, lse, dev_status, s, 1, nullptr, nullptr, nullptr,
                                          0, nblk)

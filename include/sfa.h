@@ -212,14 +212,29 @@ sfa_status sfa_forward_paged(const sfa_attn_desc *desc, const void *q, const voi
  * sfa_lse_merge's rule over n_split branches).  Use it when B*H*Tq*ceil(P/128) is small
  * next to the number of SMs or the sets differ a lot in size between heads.
  *
+ * n_split = 0 (scheduled): the library chooses the number of ranges (Amax taken as every
+ * unit's length, the launch modelled as waves of equal pieces plus the merge; with many
+ * full waves it keeps one range and writes O directly), and a one-CTA kernel first
+ * counts every list's key tiles on the device and orders the CTAs longest range first,
+ * so that the block scheduler runs a longest-first schedule over the SMs.  The result is
+ * the same attention; the order of the partial merge is fixed by the ranges, so a call
+ * is deterministic.  sfa_forward_split_plan reports the choice.
+ *
  * sfa_forward_split_workspace: bytes of device workspace for this descriptor and
- *   n_split (0 when n_split == 1).  1 <= n_split <= d/8, else SFA_ERR_INVALID_ARG.
+ *   n_split (0 when n_split == 1).  0 <= n_split <= d/8, else SFA_ERR_INVALID_ARG.
  * sfa_forward_split: arguments as sfa_forward, plus n_split and a caller-owned device
  *   workspace of at least that many bytes, 256-byte aligned (unused when n_split == 1;
  *   its contents are scratch and are overwritten).  Partial O is rounded to bf16 before
  *   the merge, in fp32, rounds it once more.
  */
 sfa_status sfa_forward_split_workspace(const sfa_attn_desc *desc, int32_t n_split, size_t *bytes);
+
+/* The key-tile ranges per unit a scheduled call (n_split = 0) uses for this descriptor:
+ * n_lists = 1 for sfa_forward_split (key_blocks = 0) or sfa_forward_blocks_split
+ * (key_blocks = 1), 2 for sfa_forward_dual (k_first for the local lists, k_second for
+ * the history lists).  k_second may be NULL. */
+sfa_status sfa_forward_split_plan(const sfa_attn_desc *desc, int32_t n_lists, int32_t key_blocks, int32_t *k_first,
+                                  int32_t *k_second);
 
 sfa_status sfa_forward_split(const sfa_attn_desc *desc, const void *q, const void *k, const void *v,
                              const int32_t *frames, const int32_t *counts, void *o, float *lse,
@@ -268,6 +283,9 @@ sfa_status sfa_forward_split_noalloc(const sfa_attn_desc *desc, const void *q, c
  * frames_local / counts_local and frames_hist / counts_hist: [H][Tq][Amax] / [H][Tq] as
  * sfa_build_sets writes them (the same Amax).  o_local and o_full use desc->o_stride.
  * sfa_forward_dual_workspace: bytes of workspace for n_split (1 <= 2 n_split <= d/8).
+ * n_split = 0 schedules the launch as sfa_forward_split does: the local lists keep one
+ * key-tile range per unit, the history lists get the number of ranges the library
+ * chooses (sfa_forward_split_plan with n_lists = 2), and the CTAs run longest range first.
  * The workspace must be 256-byte aligned; partial O is rounded to bf16 before the merge.
  */
 sfa_status sfa_forward_dual_workspace(const sfa_attn_desc *desc, int32_t n_split, size_t *bytes);
@@ -340,8 +358,11 @@ sfa_status sfa_forward_blocks(const sfa_attn_desc *desc, const void *q, const vo
                               int32_t *dev_status, sfa_stream_t stream);
 
 /* sfa_forward_blocks with the key tiles of every unit cut into n_split ranges and merged
- * by LSE, as sfa_forward_split does for frame lists (workspace: the size
- * sfa_forward_split_workspace gives for the same descriptor and n_split). */
+ * by LSE, as sfa_forward_split does for frame lists; n_split = 0 schedules the launch
+ * (the library's choice of ranges, longest first).  Workspace: the size
+ * sfa_forward_blocks_split_workspace gives for the same descriptor and n_split. */
+sfa_status sfa_forward_blocks_split_workspace(const sfa_attn_desc *desc, int32_t n_split, size_t *bytes);
+
 sfa_status sfa_forward_blocks_split(const sfa_attn_desc *desc, const void *q, const void *k, const void *v,
                                     const int32_t *blocks, const int32_t *counts, void *o, float *lse,
                                     int32_t n_split, void *workspace, size_t workspace_bytes,

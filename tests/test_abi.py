@@ -136,6 +136,10 @@ def test_no_oracle_in_product_path():
                 assert "oracle" not in text.lower(), f"{fn} mentions the oracle"
 
 
+def _round256(n):
+    return (n + 255) // 256 * 256
+
+
 def test_split_workspace_and_arguments(sfa):
     lib = sfa.load()
     d = _desc(sfa)  # B=1, H=2, Tq=4, P=64, d=64: 512 query rows
@@ -144,7 +148,14 @@ def test_split_workspace_and_arguments(sfa):
     assert lib.sfa_forward_split_workspace(ctypes.byref(d), 2, ctypes.byref(out)) == 0
     assert out.value == 2 * 512 * 64 * 2 + 2 * 512 * 4
     assert lib.sfa_forward_split_workspace(ctypes.byref(d), 9, ctypes.byref(out)) == 1   # > d/8
-    assert lib.sfa_forward_split_workspace(ctypes.byref(d), 0, ctypes.byref(out)) == 1
+    assert lib.sfa_forward_split_workspace(ctypes.byref(d), -1, ctypes.byref(out)) == 1
+    # n_split = 0: a scheduled launch; its workspace holds the partials (more than one
+    # range) and one 8-byte work item per CTA, each part rounded up to 256 bytes
+    k0, _ = sfa.split_plan(d)
+    assert 1 <= k0 <= 8
+    part = 0 if k0 == 1 else _round256(k0 * 512 * 64 * 2) + _round256(k0 * 512 * 4)
+    assert lib.sfa_forward_split_workspace(ctypes.byref(d), 0, ctypes.byref(out)) == 0
+    assert out.value == part + _round256(8 * k0 * 1 * 2 * 4 * 1)
     good = 1 << 20
     # workspace missing, too small or misaligned: refused before any launch
     assert lib.sfa_forward_split(ctypes.byref(d), good, good, good, good, good, good, good, 2, None, 0,
@@ -250,3 +261,30 @@ def test_gdn_host_checks(sfa):
     assert call(good, 1 << 30) == sfa.SFA_ERR_UNSUPPORTED
     d.d, d.B = 128, 0  # nothing to do
     assert call(None, 0) == sfa.SFA_OK
+
+
+def test_scheduled_split_plan(sfa):
+    # the choice of key-tile ranges of a scheduled launch (n_split = 0), on the host; with
+    # no GPU visible the SM count defaults to the B200's 148
+    lib = sfa.load()
+    # a launch of many full waves (the 41-frame LVSA shape: 3444 units) keeps one range
+    d = _desc(sfa, B=1, H=12, Tq=41, T_kv=41, P=1560, d=128, Amax=21)
+    assert sfa.split_plan(d) == (1, 0)
+    out = ctypes.c_size_t(0)
+    assert lib.sfa_forward_split_workspace(ctypes.byref(d), 0, ctypes.byref(out)) == 0
+    assert out.value == _round256(8 * 12 * 41 * 7)          # the work items only
+    # one query frame over 12 history frames (84 units of up to 156 key tiles): split
+    d = _desc(sfa, B=1, H=12, Tq=1, T_kv=14, P=1560, d=128, Amax=12)
+    k0, _ = sfa.split_plan(d)
+    assert 2 <= k0 <= 16
+    # two branches: the local lists keep one range, the history lists are split
+    k_local, k_hist = sfa.split_plan(d, n_lists=2)
+    assert k_local == 1 and 2 <= k_hist <= 15
+    assert lib.sfa_forward_dual_workspace(ctypes.byref(d), 0, ctypes.byref(out)) == 0
+    rows = 12 * 1560
+    slices = k_local + k_hist
+    assert out.value == _round256(slices * rows * 128 * 2) + _round256(slices * rows * 4) + _round256(8 * 84 * slices)
+    k_blocks, _ = sfa.split_plan(d, key_blocks=True)
+    assert 1 <= k_blocks <= 16
+    with pytest.raises(sfa.SfaError):
+        sfa.split_plan(d, n_lists=3)

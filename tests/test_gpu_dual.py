@@ -51,7 +51,8 @@ def _run(local, hist_w, full, n_split, seed, rows=None):
     return q, k, v, (fl, cl, fh, ch), (ol, ll, of, lf)
 
 
-@pytest.mark.parametrize("P,d,n_split", [(200, 128, 1), (200, 128, 2), (136, 64, 4), (1, 128, 1), (300, 64, 2)])
+@pytest.mark.parametrize("P,d,n_split", [(200, 128, 1), (200, 128, 2), (136, 64, 4), (1, 128, 1), (300, 64, 2),
+                                         (200, 128, 0), (136, 64, 0), (1, 128, 0)])
 def test_dual_matches_oracle_full_rows(P, d, n_split):
     local, hist_w, full = _branches(P, d, B=2)
     _run(local, hist_w, full, n_split, seed=P + d)
@@ -105,3 +106,11 @@ def test_dual_argument_checks():
     with pytest.raises(m.SfaError):
         m.forward_dual(q, k, v, fl, cl, fh, ch, local.P, 1, workspace=torch.empty(16, dtype=torch.uint8,
                                                                                      device="cuda"))
+
+
+def test_dual_scheduled_ispa_workload_sampled():
+    # n_split = 0 on the ISPA shape: the local lists one range per unit, the history lists
+    # split as planned, longest ranges first
+    local, hist_w = WORKLOADS["lsemerge_local"], WORKLOADS["lsemerge_hist"]
+    full = WORKLOADS["lsemerge_full"]
+    _run(local, hist_w, full, 0, seed=0, rows=sample_rows(local, 256, seed=3))

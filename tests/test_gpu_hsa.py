@@ -221,7 +221,7 @@ def test_hsa_workload_selection_and_sampled_attention():
     compare(o.float().cpu().reshape(-1, w.d).numpy()[rows], lse.cpu().reshape(-1).numpy()[rows], o_ref, l_ref)
 
 
-@pytest.mark.parametrize("n_split", [2, 4])
+@pytest.mark.parametrize("n_split", [2, 4, 0])
 def test_forward_blocks_split_matches_oracle(n_split):
     w = SMALL[0]
     q, k, v = workload_qkv(w, seed=5)
@@ -234,3 +234,20 @@ def test_forward_blocks_split_matches_oracle(n_split):
                                         w.P, 1 / math.sqrt(w.d))
     compare(o.float().cpu().reshape(-1, w.d).numpy(), lse.cpu().reshape(-1).numpy(), o_ref.reshape(-1, w.d),
             l_ref.reshape(-1))
+
+
+def test_forward_blocks_scheduled_workload_sampled():
+    # n_split = 0 on the hsa workload (252 units of uneven block lists)
+    w = WORKLOADS["hsa"]
+    q, k, v = workload_qkv(w, seed=0)
+    Amax = sfa().hsa_max_count(_params(w), w.P, w.k_frames, w.k_blocks)
+    lists, cnts = hsa.build_block_lists(q.float().numpy(), k.float().numpy(), Bmax=Amax, **_kw(w))
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o, lse = sfa().forward_blocks(q.cuda(), k.cuda(), v.cuda(), torch.from_numpy(lists).cuda(),
+                                  torch.from_numpy(cnts).cuda(), w.P, n_split=0, dev_status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    rows = sample_rows(w, 256, seed=4, frames=(2,))
+    o_ref, l_ref = hsa.attention_blocks(q.float().numpy(), k.float().numpy(), v.float().numpy(), lists, cnts,
+                                        w.P, 1 / math.sqrt(w.d), rows=rows)
+    compare(o.float().cpu().reshape(-1, w.d).numpy()[rows], lse.cpu().reshape(-1).numpy()[rows], o_ref, l_ref)

@@ -77,3 +77,70 @@ def test_split_matches_unsplit():
 def test_split_full_size_sampled(name, n_split):
     w = WORKLOADS[name]
     _run(w, n_split, seed=0, rows=sample_rows(w, 256, seed=1))
+
+
+# ---------------------------------------------------------------------------- scheduled
+# n_split = 0: the library picks the number of ranges and a one-CTA kernel orders the
+# CTAs longest range first.  The result must equal forward_split with the planned number
+# of ranges bit for bit (same ranges, same merge order), which also shows that every
+# (unit, range) ran exactly once, and meet the oracle bar.
+
+def _planned(w, q, k, v, fr, cn):
+    m = sfa()
+    desc = m.attn_desc(q, k, v, torch.empty_like(q), w.P, fr.shape[2])
+    return m.split_plan(desc)[0]
+
+
+@pytest.mark.parametrize("name", ["lvsa_p200", "stream_small", "lvsa_d64", "tiny_sinkwin"])
+def test_scheduled_small_full(name):
+    w = SMALL[name]
+    _run(w, 0)
+    q, k, v = (x.cuda() for x in workload_qkv(w, seed=1))
+    fr, cn = __import__("gpu_helpers").gpu_sets(w)
+    kp = _planned(w, q, k, v, fr, cn)
+    o0, l0 = sfa().forward_split(q, k, v, fr, cn, w.P, 0)
+    ok, lk = sfa().forward_split(q, k, v, fr, cn, w.P, kp)
+    torch.cuda.synchronize()
+    assert torch.equal(o0, ok) and torch.equal(l0, lk)
+
+
+@pytest.mark.parametrize("name", ["stream", "lsemerge_hist"])
+def test_scheduled_full_size(name):
+    w = WORKLOADS[name]
+    _run(w, 0, seed=0, rows=sample_rows(w, 256, seed=2, frames=(0,)))
+    q, k, v = (x.cuda() for x in workload_qkv(w, seed=0))
+    fr, cn = __import__("gpu_helpers").gpu_sets(w)
+    kp = _planned(w, q, k, v, fr, cn)
+    assert kp > 1  # a sub-wave grid is split
+    o0, l0 = sfa().forward_split(q, k, v, fr, cn, w.P, 0)
+    ok, lk = sfa().forward_split(q, k, v, fr, cn, w.P, kp)
+    torch.cuda.synchronize()
+    assert torch.equal(o0, ok) and torch.equal(l0, lk)
+
+
+def test_scheduled_many_waves_keeps_one_range():
+    # 1280 units (more than 8 waves of 148 SMs): one range per unit, the output written
+    # directly; identical to the plain forward
+    w = Workload("waves", B=2, H=8, Tq=40, Tkv=40, q_off=0, P=512, d=128, C=5, W=3, T_per=4,
+                 heads=(SetSpec("lvsa"),) * 8)
+    q, k, v = (x.cuda() for x in workload_qkv(w, seed=3))
+    fr, cn = __import__("gpu_helpers").gpu_sets(w)
+    assert _planned(w, q, k, v, fr, cn) == 1
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o1, l1 = sfa().forward(q, k, v, fr, cn, w.P)
+    o0, l0 = sfa().forward_split(q, k, v, fr, cn, w.P, 0, dev_status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    assert torch.equal(o0, o1) and torch.equal(l0, l1)
+
+
+def test_scheduled_bad_list_is_reported():
+    w = SMALL["stream_small"]
+    q, k, v = (x.cuda() for x in workload_qkv(w, seed=1))
+    fr, cn = __import__("gpu_helpers").gpu_sets(w)
+    bad = fr.clone()
+    bad[1, 0, 0] = w.Tkv  # out of range
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sfa().forward_split(q, k, v, bad, cn, w.P, 0, dev_status=status)
+    torch.cuda.synchronize()
+    assert status.item() == sfa().SFA_ERR_BAD_SET
