@@ -213,19 +213,20 @@ def run_ours(args, rank, world, local_rank):
             "ms_per_step": round(total_ms / args.steps, 4), "heads": w.H,
             "forward_ms": round(float(np.mean(fwd_ms)), 4), "note": "device step only (--skip-extras)"}
 
-    # end to end through the public API with host buffers: H2D of Q, K, V from pinned
-    # memory, sets + attention, D2H of O and LSE into pinned memory, every step
-    # (sfa.forward_host overlaps the copies of one head group with the attention of another)
+    # end to end through the C ABI with host buffers: H2D of Q, K, V from pinned memory,
+    # sets + attention, D2H of O and LSE into pinned memory, every step (sfa_forward_host
+    # pipelines the copies of one head group with the attention of another in the library)
     q_p, k_p, v_p = (x.pin_memory() for x in (q_h, k_h, v_h))
     o_p = torch.empty(q_h.shape, dtype=torch.bfloat16).pin_memory()
     lse_p = torch.empty((w.B, w.H, w.Lq), dtype=torch.float32).pin_memory()
+    host_ws = torch.empty(sfa.host_workspace_bytes(q_p, k_p, w.P, Amax), dtype=torch.uint8, device=dev)
 
     def e2e_step():
         # sets on the device, then the host-to-host forward: per (batch, head-group) chunk,
-        # the copy in, the attention and the copy out run on three streams as a pipeline
+        # the copy in, the attention and the copy out run on their own streams as a pipeline
         sfa.build_sets(params, kinds, None, Amax, frames, counts, stream=stream)
-        sfa.forward_host(q_p, k_p, v_p, frames, counts, w.P, out_host=o_p, lse_host=lse_p,
-                         buffers=(q, k, v, out, lse), dev_status=status, stream=stream)
+        sfa.forward_host(q_p, k_p, v_p, frames, counts, w.P, out_host=o_p, lse_host=lse_p, workspace=host_ws,
+                         dev_status=status, stream=stream)
 
     e2e_step()
     torch.cuda.synchronize(dev)
@@ -283,7 +284,8 @@ def run_ours(args, rank, world, local_rank):
                      "traffic_note": "DRAM read+write bytes per launch, ncu capture of the 4-head case x 3",
                      "forward_ms": round(fwd_avg, 4), "set_build_ms": round(float(np.mean(sets_ms)), 4)},
         "e2e": {"value": round(job_rate_tflops(flops, world, e2e_ms), 2), "unit": "TFLOP/s",
-                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "api": "sfa_build_sets + sfa_forward_host (C ABI, host buffers)"},
         "gpu_launches": 2 * args.steps,
         "clocks": clk,
         "merge": merge,

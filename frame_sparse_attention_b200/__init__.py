@@ -5,7 +5,8 @@ Python face of libsfa.so (C ABI in include/sfa.h):
 * ``build_sets``  - attended frame sets A(h, t) (LVSA anchors + window, sink/local/memory
                     caches, explicit lists), built on the GPU
 * ``forward``     - softmax attention over the tokens of A(h, t) only, O bf16 + LSE fp32
-* ``forward_host`` - the same for pinned host tensors, copies pipelined with the attention
+* ``forward_host`` - the same for pinned host tensors (sfa_forward_host: the copies and the
+                    attention pipelined inside the library)
 * ``forward_split`` - the same with each unit's key tiles split over several CTAs and the
                     partials merged by LSE (short or uneven grids); ``n_split=0`` lets the
                     library choose the split and run the CTAs longest first
@@ -23,7 +24,7 @@ Tensors are PyTorch CUDA tensors; calls run on the current CUDA stream.
 from ._lib import (SET_KINDS, SFA_DEBUG_STALL_SOFTMAX, SFA_ERR_BAD_SET, SFA_ERR_CUDA,
                    SFA_ERR_INVALID_ARG, SFA_ERR_TIMEOUT, SFA_ERR_UNSUPPORTED, SFA_OK, AttnDesc,
                    SetParams, SfaError, attn_desc, build_sets, error_string, forward, forward_blocks, forward_dual,
-                   forward_host,
+                   forward_host, host_workspace_bytes,
                    forward_paged, forward_split, gdn_forward, GdnDesc, hsa_max_count, hsa_select, load, lse_merge,
                    set_max_count,
                    set_params, split_plan, split_workspace_bytes, version)
@@ -31,6 +32,6 @@ from ._lib import (SET_KINDS, SFA_DEBUG_STALL_SOFTMAX, SFA_ERR_BAD_SET, SFA_ERR_
 __all__ = ["SET_KINDS", "SFA_DEBUG_STALL_SOFTMAX", "SFA_ERR_BAD_SET", "SFA_ERR_CUDA",
            "SFA_ERR_INVALID_ARG", "SFA_ERR_TIMEOUT", "SFA_ERR_UNSUPPORTED", "SFA_OK", "AttnDesc",
            "SetParams", "SfaError", "attn_desc", "build_sets", "error_string", "forward", "forward_blocks",
-           "forward_dual", "forward_host",
+           "forward_dual", "forward_host", "host_workspace_bytes",
            "forward_paged", "forward_split", "gdn_forward", "GdnDesc", "hsa_max_count", "hsa_select",
            "load", "lse_merge", "set_max_count", "set_params", "split_plan", "split_workspace_bytes", "version"]

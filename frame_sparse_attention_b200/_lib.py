@@ -61,6 +61,7 @@ EXPORTS = ("sfa_error_string", "sfa_version", "sfa_set_max_count", "sfa_build_se
            "sfa_forward_split_workspace", "sfa_forward_split", "sfa_forward_split_noalloc", "sfa_forward_paged",
            "sfa_lse_merge", "sfa_hsa_max_count", "sfa_hsa_workspace", "sfa_hsa_select", "sfa_forward_blocks",
            "sfa_forward_blocks_split", "sfa_forward_blocks_split_workspace", "sfa_forward_split_plan",
+           "sfa_forward_host_workspace", "sfa_forward_host",
            "sfa_forward_dual_workspace", "sfa_forward_dual", "sfa_gdn_workspace", "sfa_gdn_forward")
 
 
@@ -121,6 +122,11 @@ def load():
     lib.sfa_forward_blocks_split_workspace.argtypes = [ctypes.POINTER(AttnDesc), i32, ctypes.POINTER(ctypes.c_size_t)]
     lib.sfa_forward_split_plan.restype = st
     lib.sfa_forward_split_plan.argtypes = [ctypes.POINTER(AttnDesc), i32, i32, ctypes.POINTER(i32), ctypes.POINTER(i32)]
+    lib.sfa_forward_host_workspace.restype = st
+    lib.sfa_forward_host_workspace.argtypes = [ctypes.POINTER(AttnDesc), ctypes.POINTER(ctypes.c_size_t)]
+    lib.sfa_forward_host.restype = st
+    lib.sfa_forward_host.argtypes = [ctypes.POINTER(AttnDesc), vp, vp, vp, vp, vp, vp, vp, i32, vp, ctypes.c_size_t,
+                                     vp, vp]
     lib.sfa_forward_blocks.restype = st
     lib.sfa_forward_blocks.argtypes = [ctypes.POINTER(AttnDesc), vp, vp, vp, vp, vp, vp, vp, vp, vp]
     _lib = lib
@@ -199,14 +205,14 @@ def build_sets(params: SetParams, kinds, extra: torch.Tensor | None = None, Amax
 
 
 def attn_desc(q, k, v, o, P: int, Amax: int, scale: float | None = None, timeout_us: int = 0,
-              debug_flags: int = 0) -> AttnDesc:
+              debug_flags: int = 0, on_host: bool = False) -> AttnDesc:
     B, H, Lq, d = q.shape
     Lkv = k.shape[2]
     if Lq % P or Lkv % P:
         raise ValueError(f"sequence lengths {Lq}, {Lkv} are not multiples of P = {P}")
     for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
-        if t.dtype != torch.bfloat16 or not t.is_cuda:
-            raise ValueError(f"{name} must be a bf16 CUDA tensor")
+        if t.dtype != torch.bfloat16 or t.is_cuda == on_host:
+            raise ValueError(f"{name} must be a bf16 {'CPU' if on_host else 'CUDA'} tensor")
         if t.dim() != 4 or t.stride(3) != 1:
             raise ValueError(f"{name} must be [B, H, L, d] with d contiguous")
     if scale is None:
@@ -478,64 +484,43 @@ def gdn_forward(q, k, v, alpha, beta, P: int, state_in=None, state_out=None, out
     return out, state_out
 
 
-def forward_host(q_host, k_host, v_host, frames, counts, P: int, out_host=None, lse_host=None, n_chunks: int = 12,
-                 scale: float | None = None, device=None, buffers=None, dev_status=None, stream=None,
-                 compute_streams: int = 2):
-    """Frame-sparse attention of host tensors: (O, LSE) back in pinned host memory.
+def host_workspace_bytes(q_host, k_host, P: int, Amax: int) -> int:
+    """Device workspace bytes of forward_host for these shapes."""
+    desc = attn_desc(q_host, k_host, k_host, q_host, P, Amax, on_host=True)
+    out = ctypes.c_size_t(0)
+    _check(load().sfa_forward_host_workspace(ctypes.byref(desc), ctypes.byref(out)), "sfa_forward_host_workspace")
+    return out.value
 
-    q_host, k_host, v_host: pinned bf16 CPU tensors [B, H, L, d]; frames / counts as for
-    ``forward`` (device).  The (batch, head-group) chunks run as a pipeline: the copy of
-    chunk i+1 to the GPU and of chunk i-1 back overlap the attention of chunk i, and the
-    attention of consecutive chunks alternates between ``compute_streams`` streams so
-    that the last wave of one kernel overlaps the first of the next.  The whole call is ordered after the work already queued on ``stream``
-    and ``stream`` waits for it to finish, like a single kernel on that stream.
-    ``buffers``: optional device tensors (q, k, v, out, lse) to reuse between calls."""
+
+def forward_host(q_host, k_host, v_host, frames, counts, P: int, out_host=None, lse_host=None, n_chunks: int = 12,
+                 scale: float | None = None, workspace=None, dev_status=None, stream=None, timeout_us: int = 0):
+    """Frame-sparse attention of host tensors (sfa_forward_host): (O, LSE) in pinned host
+    memory.  q_host, k_host, v_host: pinned, contiguous bf16 CPU tensors [B, H, L, d];
+    frames / counts as for ``forward`` (device).  The copies in, the attention and the
+    copies out run inside the library as a pipeline over (batch, head-group) chunks.  The
+    call is asynchronous on ``stream`` like a kernel: synchronise before reading the
+    results.  ``workspace``: a uint8 CUDA tensor of at least ``host_workspace_bytes``
+    (allocated here when not given)."""
     B, H, Lq, d = q_host.shape
-    device = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    for name, t in (("q_host", q_host), ("k_host", k_host), ("v_host", v_host)):
+        if t.dtype != torch.bfloat16 or t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 CPU tensor [B, H, L, d]")
+    _require(frames.dtype == torch.int32 and counts.dtype == torch.int32 and frames.is_cuda,
+             "expected frames.dtype == torch.int32 and counts.dtype == torch.int32 and frames.is_cuda")
     if out_host is None:
         out_host = torch.empty(q_host.shape, dtype=torch.bfloat16).pin_memory()
     if lse_host is None:
         lse_host = torch.empty((B, H, Lq), dtype=torch.float32).pin_memory()
-    own = buffers is None
-    if own:
-        buffers = (torch.empty(q_host.shape, dtype=torch.bfloat16, device=device),
-                   torch.empty(k_host.shape, dtype=torch.bfloat16, device=device),
-                   torch.empty(v_host.shape, dtype=torch.bfloat16, device=device),
-                   torch.empty(q_host.shape, dtype=torch.bfloat16, device=device),
-                   torch.empty((B, H, Lq), dtype=torch.float32, device=device))
-    q, k, v, out, lse = buffers
-    main = torch.cuda.current_stream(device) if stream is None else stream
-    per_b = max(1, min(H, n_chunks // B if n_chunks >= B else 1))
-    bounds = [(b, (H * i) // per_b, (H * (i + 1)) // per_b) for b in range(B) for i in range(per_b)]
-    s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
-    s_runs = [torch.cuda.Stream(device) for _ in range(max(1, compute_streams))]
-    start = torch.cuda.Event()
-    start.record(main)
-    for s in [s_in, s_out] + s_runs:
-        s.wait_event(start)
-    if own:  # the side streams use these buffers after this call returns
-        for t in buffers:
-            for s in [s_in, s_out] + s_runs:
-                t.record_stream(s)
-    for c, (b, h0, h1) in enumerate(bounds):
-        s_run = s_runs[c % len(s_runs)]
-        sl = (slice(b, b + 1), slice(h0, h1))
-        with torch.cuda.stream(s_in):
-            for dst, src in ((q, q_host), (k, k_host), (v, v_host)):
-                dst[sl].copy_(src[sl], non_blocking=True)
-            e_in = torch.cuda.Event()
-            e_in.record(s_in)
-        s_run.wait_event(e_in)
-        forward(q[sl], k[sl], v[sl], frames[h0:h1], counts[h0:h1], P, scale=scale, out=out[sl], lse=lse[sl],
-                dev_status=dev_status, stream=s_run)
-        e_run = torch.cuda.Event()
-        e_run.record(s_run)
-        s_out.wait_event(e_run)
-        with torch.cuda.stream(s_out):
-            out_host[sl].copy_(out[sl], non_blocking=True)
-            lse_host[sl].copy_(lse[sl], non_blocking=True)
-    for s in [s_in, s_out] + s_runs:
-        end = torch.cuda.Event()
-        end.record(s)
-        main.wait_event(end)
+    _require(out_host.is_contiguous() and lse_host.is_contiguous() and not out_host.is_cuda,
+             "expected contiguous host out_host and lse_host")
+    desc = attn_desc(q_host, k_host, v_host, out_host, P, frames.shape[2], scale, timeout_us, on_host=True)
+    if workspace is None:
+        nbytes = ctypes.c_size_t(0)
+        _check(load().sfa_forward_host_workspace(ctypes.byref(desc), ctypes.byref(nbytes)),
+               "sfa_forward_host_workspace")
+        workspace = torch.empty(nbytes.value, dtype=torch.uint8, device=frames.device)
+    _check(load().sfa_forward_host(ctypes.byref(desc), q_host.data_ptr(), k_host.data_ptr(), v_host.data_ptr(),
+                                   frames.data_ptr(), counts.data_ptr(), out_host.data_ptr(), lse_host.data_ptr(),
+                                   n_chunks, workspace.data_ptr(), workspace.numel(), _ptr(dev_status),
+                                   _stream(stream)), "sfa_forward_host")
     return out_host, lse_host

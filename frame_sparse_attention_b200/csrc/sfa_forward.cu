@@ -33,6 +33,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <mutex>
@@ -921,13 +922,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // ----------------------------------------------------------------- scheduled launches
 // A scheduled launch runs one CTA per work item: (list set, unit, key-tile range), the
 // ranges of list set l being k_l equal parts of the unit's key tiles.  The items are
-// ordered longest range first (a counting sort on the range length, computed from the
-// lists on the device), so that the hardware block scheduler, which hands CTAs to SMs in
-// index order as they free up, runs a longest-processing-time-first schedule: long units
-// start in the first wave and short ones fill the tail.  Items of one list stay together
-// (query-tile pairs fastest), so the CTAs that share the list's keys run side by side.
+// ordered longest range first, so that the hardware block scheduler, which hands CTAs to
+// SMs in index order as they free up, runs a longest-processing-time-first schedule: long
+// units start in the first wave and short ones fill the tail.  Ranges are ranked by a
+// coarse length class (a quarter octave), and inside a class the natural order is kept
+// (a stable counting sort): units of similar length stay in (batch, head, frame) order,
+// so the CTAs that read the same keys (the pairs of one list, the frames of one head) run
+// side by side and find them in L2.
 constexpr int SCHED_THREADS = 1024;
-constexpr int SCHED_BINS = 2048;  // range lengths (key tiles) at or above the last bin share it
+constexpr int SCHED_BINS = 64;  // length classes: floor(4 log2(range)), the last holding the rest
 
 struct SchedArgs {
     const int32_t *frames[2];
@@ -951,65 +954,90 @@ __device__ int sched_len(const SchedArgs &s, int li, int e)
     return n > 0 ? n : 0;
 }
 
+// Length class of a range of `len` key tiles: higher runs first.
+__device__ __forceinline__ int sched_bin(int len)
+{
+    if (len <= 1) return 0;
+    const float c = 4.f * __log2f((float)len);
+    return min(SCHED_BINS - 1, (int)c);
+}
+
 __global__ void __launch_bounds__(SCHED_THREADS) schedule_kernel(const __grid_constant__ SchedArgs s)
 {
-    __shared__ int bins[SCHED_BINS];
-    __shared__ int wsum[SCHED_THREADS / 32];
+    constexpr int NW = SCHED_THREADS / 32;
+    __shared__ int bin_start[SCHED_BINS];     // first item of each class (descending class order)
+    __shared__ int carry[SCHED_BINS];         // items of each class placed by earlier chunks
+    __shared__ int wcount[NW][SCHED_BINS];    // items of each class per warp, this chunk
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     // entries: frame lists per (h, t), or key-block lists per unit; units per entry
     const int per_set = s.nblk ? s.B * s.H * s.Tq * s.n_pairs : s.H * s.Tq;
     const int fan = s.nblk ? 1 : s.B * s.n_pairs;
     const int n_entries = per_set * s.n_lists;
-    for (int i = tid; i < SCHED_BINS; i += SCHED_THREADS) bins[i] = 0;
+    if (tid < SCHED_BINS) {
+        bin_start[tid] = 0;
+        carry[tid] = 0;
+    }
     __syncthreads();
     for (int e = tid; e < n_entries; e += SCHED_THREADS) {
         const int li = e / per_set, k = s.k[li];
-        const int key = min(SCHED_BINS - 1, (sched_len(s, li, e - li * per_set) + k - 1) / k);
-        atomicAdd(&bins[key], fan * k);
+        atomicAdd(&bin_start[sched_bin((sched_len(s, li, e - li * per_set) + k - 1) / k)], fan * k);
     }
     __syncthreads();
-    // exclusive prefix over the bins in descending length: thread t owns the bins of
-    // lengths SCHED_BINS-1-2t and SCHED_BINS-2-2t
-    static_assert(SCHED_BINS == 2 * SCHED_THREADS, "two bins per thread");
-    const int k0 = SCHED_BINS - 1 - 2 * tid, k1 = k0 - 1;
-    const int v0 = bins[k0], v1 = bins[k1], mine = v0 + v1;
-    int incl = mine;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += y;
-    }
-    if (lane == 31) wsum[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-        int w = wsum[lane], wi = w;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, wi, off);
-            if (lane >= off) wi += y;
+    if (tid == 0) {  // exclusive prefix in descending class order (64 classes)
+        int acc = 0;
+        for (int b = SCHED_BINS - 1; b >= 0; --b) {
+            const int v = bin_start[b];
+            bin_start[b] = acc;
+            acc += v;
         }
-        wsum[lane] = wi - w;  // exclusive
     }
     __syncthreads();
-    const int excl = wsum[warp] + incl - mine;
-    bins[k0] = excl;       // now: the next free item index of each length
-    bins[k1] = excl + v0;
-    __syncthreads();
-    for (int e = tid; e < n_entries; e += SCHED_THREADS) {
-        const int li = e / per_set, le = e - li * per_set, k = s.k[li];
-        const int key = min(SCHED_BINS - 1, (sched_len(s, li, le) + k - 1) / k);
-        int off = atomicAdd(&bins[key], fan * k);
-        for (int sp = 0; sp < k; ++sp) {
-            const int tag = li | (sp << 1) | (k << 9);
-            if (s.nblk) {
-                s.items[off++] = make_int2(le, tag);
-            } else {
-                const int h = le / s.Tq, t = le - h * s.Tq;
-                for (int b = 0; b < s.B; ++b)
-                    for (int pr = 0; pr < s.n_pairs; ++pr)
-                        s.items[off++] = make_int2(((b * s.H + h) * s.Tq + t) * s.n_pairs + pr, tag);
+    // stable placement, SCHED_THREADS entries per chunk in entry order: an entry's items go
+    // after those of every earlier entry of its class
+    for (int c0 = 0; c0 < n_entries; c0 += SCHED_THREADS) {
+        const int e = c0 + tid;
+        const bool on = e < n_entries;
+        int li = 0, le = 0, k = 1, bin = -1;
+        if (on) {
+            li = e / per_set;
+            le = e - li * per_set;
+            k = s.k[li];
+            bin = sched_bin((sched_len(s, li, le) + k - 1) / k);
+        }
+        for (int i = tid; i < NW * SCHED_BINS; i += SCHED_THREADS) (&wcount[0][0])[i] = 0;
+        __syncthreads();
+        // lanes of this warp in the same class, before this lane: their items come first
+        // (an entry of list set l has fan * k_l items)
+        const unsigned same = __match_any_sync(0xffffffffu, bin);
+        const unsigned in_set1 = __ballot_sync(0xffffffffu, on && li == 1);
+        const unsigned lt = (1u << lane) - 1u;
+        const int k0 = s.k[0], k1 = s.n_lists == 2 ? s.k[1] : 0;
+        const int before = fan * (k0 * __popc(same & lt & ~in_set1) + k1 * __popc(same & lt & in_set1));
+        if (on && __popc(same & lt) == 0)  // the class's first lane in this warp
+            wcount[warp][bin] = fan * (k0 * __popc(same & ~in_set1) + k1 * __popc(same & in_set1));
+        __syncthreads();
+        if (on) {
+            int off = bin_start[bin] + carry[bin] + before;
+            for (int w = 0; w < warp; ++w) off += wcount[w][bin];
+            for (int sp = 0; sp < k; ++sp) {
+                const int tag = li | (sp << 1) | (k << 9);
+                if (s.nblk) {
+                    s.items[off++] = make_int2(le, tag);
+                } else {
+                    const int h = le / s.Tq, t = le - h * s.Tq;
+                    for (int b = 0; b < s.B; ++b)
+                        for (int pr = 0; pr < s.n_pairs; ++pr)
+                            s.items[off++] = make_int2(((b * s.H + h) * s.Tq + t) * s.n_pairs + pr, tag);
+                }
             }
         }
+        __syncthreads();
+        if (tid < SCHED_BINS) {
+            int add = 0;
+            for (int w = 0; w < NW; ++w) add += wcount[w][tid];
+            carry[tid] += add;
+        }
+        __syncthreads();
     }
 }
 
@@ -1220,6 +1248,10 @@ void auto_splits(const sfa_attn_desc *d, int n_lists, int nblk, int &k0, int &k1
     if (n_lists == 1) {
         k0 = 1;
         if (units >= 8.0 * sms) return;  // many full waves: splitting only adds merge traffic
+        // key-block lists: measured on the hsa workload, their ranges cost more than they
+        // recover (0.67 ms at 2 ranges, 1.20 at 4, 0.56 unsplit), so they keep one range
+        // unless the grid fills less than half the SMs
+        if (nblk && units >= 0.5 * sms) return;
         double best = cost(1, 1, 1);
         for (int k = 2; k <= cap; ++k) {
             const double c = cost(k, k, k);
@@ -1364,6 +1396,150 @@ extern "C" sfa_status sfa_forward_split(const sfa_attn_desc *d, const void *q, c
     float *ws_lse = reinterpret_cast<float *>(static_cast<char *>(workspace) + split_ws_o_bytes(d, n_split));
     return d->d == 128 ? launch<128>(d, q, k, v, frames, counts, o, lse, dev_status, s, n_split, workspace, ws_lse)
                        : launch<64>(d, q, k, v, frames, counts, o, lse, dev_status, s, n_split, workspace, ws_lse);
+}
+
+// ------------------------------------------------------------------------------------
+// Host buffers in, host buffers out: the copies and the attention as one pipeline.
+// The (batch, head-group) chunks run in order: the copy of chunk i+1 to the device (one
+// stream), the attention of chunk i (two streams in turn, so the last wave of one kernel
+// overlaps the first of the next) and the copy of chunk i-1 back (a third stream) overlap.
+// ------------------------------------------------------------------------------------
+namespace sfa {
+namespace {
+
+struct HostLayout {
+    size_t q, k, v, o, lse, total;
+};
+
+HostLayout host_layout(const sfa_attn_desc *d)
+{
+    auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+    const size_t bh = (size_t)d->B * d->H, lq = (size_t)d->Tq * d->P, lk = (size_t)d->T_kv * d->P;
+    HostLayout w;
+    w.q = 0;
+    w.k = up(bh * lq * d->d * 2);
+    w.v = w.k + up(bh * lk * d->d * 2);
+    w.o = w.v + up(bh * lk * d->d * 2);
+    w.lse = w.o + up(bh * lq * d->d * 2);
+    w.total = w.lse + up(bh * lq * 4);
+    return w;
+}
+
+// RAII set of the call's streams and events (released when the call returns; work still
+// queued on a destroyed stream completes normally)
+struct HostPipe {
+    cudaStream_t in = nullptr, out = nullptr, run[2] = {nullptr, nullptr};
+    cudaEvent_t start = nullptr, e_in = nullptr, e_run[2] = {nullptr, nullptr}, end[4] = {};
+    bool ok = true;
+    HostPipe()
+    {
+        for (cudaStream_t *st : {&in, &out, &run[0], &run[1]})
+            ok = ok && cudaStreamCreateWithFlags(st, cudaStreamNonBlocking) == cudaSuccess;
+        for (cudaEvent_t *ev : {&start, &e_in, &e_run[0], &e_run[1], &end[0], &end[1], &end[2], &end[3]})
+            ok = ok && cudaEventCreateWithFlags(ev, cudaEventDisableTiming) == cudaSuccess;
+    }
+    ~HostPipe()
+    {
+        for (cudaEvent_t ev : {start, e_in, e_run[0], e_run[1], end[0], end[1], end[2], end[3]})
+            if (ev) cudaEventDestroy(ev);
+        for (cudaStream_t st : {in, out, run[0], run[1]})
+            if (st) cudaStreamDestroy(st);
+    }
+};
+
+}  // namespace
+}  // namespace sfa
+
+extern "C" sfa_status sfa_forward_host_workspace(const sfa_attn_desc *d, size_t *bytes)
+{
+    sfa_status st = check_desc(d);
+    if (st != SFA_OK) return st;
+    if (!bytes) return SFA_ERR_INVALID_ARG;
+    *bytes = host_layout(d).total;
+    return SFA_OK;
+}
+
+extern "C" sfa_status sfa_forward_host(const sfa_attn_desc *d, const void *q_host, const void *k_host,
+                                       const void *v_host, const int32_t *frames, const int32_t *counts,
+                                       void *o_host, float *lse_host, int32_t n_chunks, void *workspace,
+                                       size_t workspace_bytes, int32_t *dev_status, sfa_stream_t stream)
+{
+    sfa_status st = check_desc(d);
+    if (st != SFA_OK) return st;
+    if (n_chunks < 1) return SFA_ERR_INVALID_ARG;
+    if (d->B == 0) return SFA_OK;
+    if (!q_host || !k_host || !v_host || !o_host || !lse_host || !frames || !counts) return SFA_ERR_INVALID_ARG;
+    const HostLayout w = host_layout(d);
+    if (!workspace || reinterpret_cast<uintptr_t>(workspace) % 256 || workspace_bytes < w.total)
+        return SFA_ERR_INVALID_ARG;
+    const int64_t lq = (int64_t)d->Tq * d->P, lk = (int64_t)d->T_kv * d->P, D = d->d;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    uint8_t *q = ws + w.q, *k = ws + w.k, *v = ws + w.v, *o = ws + w.o;
+    float *lse = reinterpret_cast<float *>(ws + w.lse);
+    const uint8_t *qh = static_cast<const uint8_t *>(q_host), *kh = static_cast<const uint8_t *>(k_host),
+                  *vh = static_cast<const uint8_t *>(v_host);
+    uint8_t *oh = static_cast<uint8_t *>(o_host);
+    cudaStream_t main = as_cuda(stream);
+    HostPipe pp;
+    if (!pp.ok) return SFA_ERR_CUDA;
+    // every side stream starts after the work already queued on the caller's stream
+    if (cudaEventRecord(pp.start, main) != cudaSuccess) return SFA_ERR_CUDA;
+    for (cudaStream_t sx : {pp.in, pp.out, pp.run[0], pp.run[1]})
+        if (cudaStreamWaitEvent(sx, pp.start, 0) != cudaSuccess) return SFA_ERR_CUDA;
+    // chunks: per batch entry, groups of heads (contiguous in the [B][H][L][d] layout)
+    auto enqueue = [&]() -> sfa_status {
+        const int per_b = std::max(1, std::min<int>(d->H, n_chunks >= d->B ? n_chunks / d->B : 1));
+        int c = 0;
+        for (int b = 0; b < d->B; ++b) {
+            for (int g = 0; g < per_b; ++g, ++c) {
+                const int h0 = (int)((int64_t)d->H * g / per_b), h1 = (int)((int64_t)d->H * (g + 1) / per_b);
+                if (h1 == h0) continue;
+                const int64_t hq = ((int64_t)b * d->H + h0) * lq, hk = ((int64_t)b * d->H + h0) * lk;
+                const int64_t nq = (int64_t)(h1 - h0) * lq, nk = (int64_t)(h1 - h0) * lk;
+                const size_t bq = (size_t)nq * D * 2, bk = (size_t)nk * D * 2;
+                if (cudaMemcpyAsync(q + hq * D * 2, qh + hq * D * 2, bq, cudaMemcpyHostToDevice, pp.in) != cudaSuccess ||
+                    cudaMemcpyAsync(k + hk * D * 2, kh + hk * D * 2, bk, cudaMemcpyHostToDevice, pp.in) != cudaSuccess ||
+                    cudaMemcpyAsync(v + hk * D * 2, vh + hk * D * 2, bk, cudaMemcpyHostToDevice, pp.in) != cudaSuccess ||
+                    cudaEventRecord(pp.e_in, pp.in) != cudaSuccess)
+                    return SFA_ERR_CUDA;
+                cudaStream_t run = pp.run[c & 1];
+                if (cudaStreamWaitEvent(run, pp.e_in, 0) != cudaSuccess) return SFA_ERR_CUDA;
+                sfa_attn_desc cd = *d;
+                cd.B = 1;
+                cd.H = h1 - h0;
+                cd.q_stride[0] = cd.o_stride[0] = (int64_t)cd.H * lq * D;
+                cd.q_stride[1] = cd.o_stride[1] = lq * D;
+                cd.q_stride[2] = cd.o_stride[2] = D;
+                cd.k_stride[0] = cd.v_stride[0] = (int64_t)cd.H * lk * D;
+                cd.k_stride[1] = cd.v_stride[1] = lk * D;
+                cd.k_stride[2] = cd.v_stride[2] = D;
+                const int32_t *fr = frames + (int64_t)h0 * d->Tq * d->Amax, *cn = counts + (int64_t)h0 * d->Tq;
+                st = D == 128 ? launch<128>(&cd, q + hq * D * 2, k + hk * D * 2, v + hk * D * 2, fr, cn, o + hq * D * 2,
+                                            lse + hq, dev_status, run)
+                              : launch<64>(&cd, q + hq * D * 2, k + hk * D * 2, v + hk * D * 2, fr, cn, o + hq * D * 2,
+                                           lse + hq, dev_status, run);
+                if (st != SFA_OK) return st;
+                if (cudaEventRecord(pp.e_run[c & 1], run) != cudaSuccess ||
+                    cudaStreamWaitEvent(pp.out, pp.e_run[c & 1], 0) != cudaSuccess ||
+                    cudaMemcpyAsync(oh + hq * D * 2, o + hq * D * 2, bq, cudaMemcpyDeviceToHost, pp.out) != cudaSuccess ||
+                    cudaMemcpyAsync(lse_host + hq, lse + hq, (size_t)nq * 4, cudaMemcpyDeviceToHost, pp.out) !=
+                        cudaSuccess)
+                    return SFA_ERR_CUDA;
+            }
+        }
+        return SFA_OK;
+    };
+    const sfa_status queued = enqueue();
+    // the caller's stream waits for the whole pipeline, like a single kernel on it (also
+    // after an error, for whatever was queued)
+    int i = 0;
+    sfa_status joined = SFA_OK;
+    for (cudaStream_t sx : {pp.in, pp.out, pp.run[0], pp.run[1]}) {
+        if (cudaEventRecord(pp.end[i], sx) != cudaSuccess || cudaStreamWaitEvent(main, pp.end[i], 0) != cudaSuccess)
+            joined = SFA_ERR_CUDA;
+        ++i;
+    }
+    return queued != SFA_OK ? queued : joined;
 }
 
 // ------------------------------------------------------------------------------------

@@ -9,7 +9,8 @@
 //
 // Two kernels:
 //   * hsa_pool_kernel: one CTA per segment (128-token key block or 256-row query block)
-//     of keys or queries; 16-byte loads, fp32 sums per column, one mean per segment.
+//     of keys or queries, both in one launch; 16-byte loads, four rows of them in flight
+//     per thread, fp32 sums per column, one mean per segment.
 //     HBM-bound: every K and Q element is read once.  hsa_frame_mean_kernel then forms
 //     each frame's mean as the token-weighted average of its block means.
 //   * hsa_select_kernel: one CTA per (b, h, t, query block): scores of the history
@@ -38,35 +39,58 @@ constexpr int MAX_ENTRIES = 65536;  // T_kv * nblk bound (the block flags live i
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
-// Mean of one segment of `seg` rows of one frame of x (P rows of D bf16, row stride
-// s_row elements), written to out[((b*H + h)*n_frames + f)*nseg + sg][D]; the last
-// segment of a frame holds the remaining rows.  One CTA per (segment, frame, b*H + h):
-// D/8 threads per row (8 columns, one 16-byte load each), POOL_THREADS / (D/8) rows at a
-// time, then a shared-memory pass adds the row groups.
+// Mean of one segment of rows of one frame: the segments of the keys (KEY_BLOCK rows) and
+// of the queries (QUERY_BLOCK rows) in one launch.  CTA x of grid row bh = b*H + h takes
+// key segment x (x < nk = nblk * T_kv: segment x % nblk of frame x / nblk) or query
+// segment x - nk; it writes the mean to out[((bh * n_frames + f) * nseg + sg)][D] of its
+// tensor; the last segment of a frame holds the remaining rows.  D/8 threads per row (8
+// columns, one 16-byte load each), POOL_THREADS / (D/8) rows at a time and four of those
+// in flight per thread, then a shared-memory pass adds the row groups.
+struct PoolArgs {
+    const uint16_t *k, *q;
+    int64_t k_sb, k_sh, k_sr, q_sb, q_sh, q_sr;  // strides in elements
+    int H, P, T_kv, Tq, nblk, nqb;
+    float *kb, *qb;
+};
+
 template <int D>
-__global__ void __launch_bounds__(POOL_THREADS) hsa_pool_kernel(const uint16_t *x, int64_t s_b, int64_t s_h,
-                                                                  int64_t s_row, int H, int P, int seg,
-                                                                  int n_frames, float *out)
+__global__ void __launch_bounds__(POOL_THREADS) hsa_pool_kernel(const __grid_constant__ PoolArgs a)
 {
     constexpr int TPR = D / 8;                 // threads per row
-    constexpr int RG = POOL_THREADS / TPR;     // rows in flight
+    constexpr int RG = POOL_THREADS / TPR;     // rows per load round
+    constexpr int UNROLL = 4;                  // load rounds in flight
     __shared__ float part[RG][D];
-    const int sg = blockIdx.x, f = blockIdx.y, bh = blockIdx.z;
-    const int nseg = gridDim.x;
+    const int bh = blockIdx.y;
+    const int nk = a.nblk * a.T_kv;
+    const bool is_k = (int)blockIdx.x < nk;
+    const int x = is_k ? blockIdx.x : blockIdx.x - nk;
+    const int nseg = is_k ? a.nblk : a.nqb, seg = is_k ? KEY_BLOCK : QUERY_BLOCK;
+    const int sg = x % nseg, f = x / nseg;
+    const int n_frames = is_k ? a.T_kv : a.Tq;
     const int cg = threadIdx.x % TPR, rg = threadIdx.x / TPR;
-    const int r0 = sg * seg, r1 = min(r0 + seg, P);
-    const uint16_t *base = x + (int64_t)(bh / H) * s_b + (int64_t)(bh % H) * s_h + (int64_t)f * P * s_row + cg * 8;
+    const int r0 = sg * seg, r1 = min(r0 + seg, a.P);
+    const int64_t s_b = is_k ? a.k_sb : a.q_sb, s_h = is_k ? a.k_sh : a.q_sh, s_row = is_k ? a.k_sr : a.q_sr;
+    const uint16_t *base = (is_k ? a.k : a.q) + (int64_t)(bh / a.H) * s_b + (int64_t)(bh % a.H) * s_h +
+                           (int64_t)f * a.P * s_row + cg * 8;
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int r = r0 + rg; r < r1; r += RG) {
-        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(base + (int64_t)r * s_row));
-        acc[0] += bf16_lo(v.x);
-        acc[1] += bf16_hi(v.x);
-        acc[2] += bf16_lo(v.y);
-        acc[3] += bf16_hi(v.y);
-        acc[4] += bf16_lo(v.z);
-        acc[5] += bf16_hi(v.z);
-        acc[6] += bf16_lo(v.w);
-        acc[7] += bf16_hi(v.w);
+    for (int r = r0 + rg; r < r1; r += UNROLL * RG) {
+        uint4 v[UNROLL];
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u)
+            if (r + u * RG < r1) v[u] = __ldg(reinterpret_cast<const uint4 *>(base + (int64_t)(r + u * RG) * s_row));
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u) {
+            if (r + u * RG < r1) {
+                acc[0] += bf16_lo(v[u].x);
+                acc[1] += bf16_hi(v[u].x);
+                acc[2] += bf16_lo(v[u].y);
+                acc[3] += bf16_hi(v[u].y);
+                acc[4] += bf16_lo(v[u].z);
+                acc[5] += bf16_hi(v[u].z);
+                acc[6] += bf16_lo(v[u].w);
+                acc[7] += bf16_hi(v[u].w);
+            }
+        }
     }
 #pragma unroll
     for (int i = 0; i < 8; ++i) part[rg][cg * 8 + i] = acc[i];
@@ -74,6 +98,7 @@ __global__ void __launch_bounds__(POOL_THREADS) hsa_pool_kernel(const uint16_t *
     if (threadIdx.x < D) {
         float sum = 0.f;
         for (int g = 0; g < RG; ++g) sum += part[g][threadIdx.x];
+        float *out = is_k ? a.kb : a.qb;
         out[(((int64_t)bh * n_frames + f) * nseg + sg) * D + threadIdx.x] = sum / (float)(r1 - r0);
     }
 }
@@ -273,7 +298,7 @@ bool desc_ok(const sfa_attn_desc *d)
 {
     if (!d || d->B < 0 || d->H < 1 || d->Tq < 1 || d->T_kv < 1 || d->P < 1 || d->Amax < 1) return false;
     if ((int64_t)d->Tq * d->P >= ((int64_t)1 << 31) || (int64_t)d->T_kv * d->P >= ((int64_t)1 << 31)) return false;
-    if ((int64_t)d->B * d->H > 65535 || d->T_kv > 65535) return false;  // grid z / y of the pooling launch
+    if ((int64_t)d->B * d->H > 65535 || d->T_kv > 65535) return false;  // grid y of the pooling launch; frame ids
     return true;
 }
 
@@ -291,12 +316,24 @@ sfa_status run_select(const sfa_attn_desc *d, const sfa_set_params *p, int k_fra
     float *qb = reinterpret_cast<float *>(ws + w.qb);
     const int nblk = (d->P + KEY_BLOCK - 1) / KEY_BLOCK, nqb = (d->P + QUERY_BLOCK - 1) / QUERY_BLOCK;
     const unsigned bh = (unsigned)d->B * d->H;
-    hsa_pool_kernel<D><<<dim3(nblk, d->T_kv, bh), POOL_THREADS, 0, s>>>(
-        static_cast<const uint16_t *>(k), d->k_stride[0], d->k_stride[1], d->k_stride[2], d->H, d->P, KEY_BLOCK,
-        d->T_kv, kb);
-    hsa_pool_kernel<D><<<dim3(nqb, d->Tq, bh), POOL_THREADS, 0, s>>>(
-        static_cast<const uint16_t *>(q), d->q_stride[0], d->q_stride[1], d->q_stride[2], d->H, d->P, QUERY_BLOCK,
-        d->Tq, qb);
+    PoolArgs pa;
+    pa.k = static_cast<const uint16_t *>(k);
+    pa.q = static_cast<const uint16_t *>(q);
+    pa.k_sb = d->k_stride[0];
+    pa.k_sh = d->k_stride[1];
+    pa.k_sr = d->k_stride[2];
+    pa.q_sb = d->q_stride[0];
+    pa.q_sh = d->q_stride[1];
+    pa.q_sr = d->q_stride[2];
+    pa.H = d->H;
+    pa.P = d->P;
+    pa.T_kv = d->T_kv;
+    pa.Tq = d->Tq;
+    pa.nblk = nblk;
+    pa.nqb = nqb;
+    pa.kb = kb;
+    pa.qb = qb;
+    hsa_pool_kernel<D><<<dim3((unsigned)(nblk * d->T_kv + nqb * d->Tq), bh), POOL_THREADS, 0, s>>>(pa);
     const int64_t n_kf = (int64_t)bh * d->T_kv * D;
     hsa_frame_mean_kernel<D><<<(unsigned)((n_kf + 255) / 256), 256, 0, s>>>(kb, n_kf, d->P, nblk, kf);
     SelectArgs a;

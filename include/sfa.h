@@ -9,9 +9,9 @@
  *                   only, writing O (bf16) and the per-row log-sum-exp (fp32)
  *   sfa_lse_merge   merge of two partial attentions (e.g. local + history branch)
  *
- * plus variants of the forward (paged caches, split-KV, two branches in one launch), the
- * hierarchical block selection of Light Forcing (sfa_hsa_select + sfa_forward_blocks) and
- * ARL2's inter-frame gated-delta branch (sfa_gdn_forward).
+ * plus variants of the forward (host buffers, paged caches, split-KV, two branches in one
+ * launch), the hierarchical block selection of Light Forcing (sfa_hsa_select +
+ * sfa_forward_blocks) and ARL2's inter-frame gated-delta branch (sfa_gdn_forward).
  *
  * Conventions
  *   - A video has T latent frames of P tokens each; token i belongs to frame i / P.
@@ -181,6 +181,38 @@ typedef struct {
 sfa_status sfa_forward(const sfa_attn_desc *desc, const void *q, const void *k, const void *v,
                        const int32_t *frames, const int32_t *counts, void *o, float *lse,
                        int32_t *dev_status, sfa_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
+ * Host buffers in and out
+ * ------------------------------------------------------------------------------------
+ * sfa_forward ("LVSA", §2 Mecanismo Central: attention of every query frame over A(t)
+ * only) for Q, K, V in host memory, with O and LSE written back to host memory, the
+ * copies and the attention run as one pipeline on the device: the (batch, head-group)
+ * chunks go in order, and the copy of chunk i+1 to the device, the attention of chunk i
+ * (two streams in turn, so that one kernel's last wave overlaps the next one's first)
+ * and the copy of chunk i-1 back overlap.
+ *   q_host, k_host, v_host  bf16 [B][H][Tq*P][d] and [B][H][T_kv*P][d], contiguous (the
+ *                      descriptor's strides are not used); page-locked (cudaHostAlloc /
+ *                      pinned torch memory) for the copies to overlap, else the copies
+ *                      run synchronously and the result is the same.
+ *   frames, counts     device lists as for sfa_forward.
+ *   o_host             bf16 [B][H][Tq*P][d], lse_host fp32 [B][H][Tq*P], host, written.
+ *   n_chunks           chunks per call (>= 1): min(H, n_chunks / B) head groups per batch
+ *                      entry (at least one).
+ *   workspace          caller-owned device memory of sfa_forward_host_workspace bytes,
+ *                      256-byte aligned: the device copies of Q, K, V, O and LSE.
+ * The call creates its own streams and events and destroys them before it returns (work
+ * queued on them completes normally); all its work is ordered after the work already on
+ * `stream`, and `stream` waits for all of it, like a single kernel: synchronise `stream`
+ * before reading o_host / lse_host.  On an error the work already queued still joins
+ * `stream`.  Argument errors are returned before anything is queued.
+ */
+sfa_status sfa_forward_host_workspace(const sfa_attn_desc *desc, size_t *bytes);
+
+sfa_status sfa_forward_host(const sfa_attn_desc *desc, const void *q_host, const void *k_host, const void *v_host,
+                            const int32_t *frames, const int32_t *counts, void *o_host, float *lse_host,
+                            int32_t n_chunks, void *workspace, size_t workspace_bytes, int32_t *dev_status,
+                            sfa_stream_t stream);
 
 /* ------------------------------------------------------------------------------------
  * Paged key/value caches

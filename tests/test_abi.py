@@ -288,3 +288,27 @@ def test_scheduled_split_plan(sfa):
     assert 1 <= k_blocks <= 16
     with pytest.raises(sfa.SfaError):
         sfa.split_plan(d, n_lists=3)
+
+
+def test_forward_host_host_checks(sfa):
+    # sfa_forward_host: workspace size (device copies of Q, K, V, O, LSE, each rounded up to
+    # 256 bytes) and refusals before anything is queued
+    lib = sfa.load()
+    d = _desc(sfa)  # B=1, H=2, Tq=4, T_kv=4, P=64, d=64
+    out = ctypes.c_size_t(0)
+    assert lib.sfa_forward_host_workspace(ctypes.byref(d), ctypes.byref(out)) == 0
+    q = _round256(2 * 256 * 64 * 2)
+    assert out.value == 4 * q + _round256(2 * 256 * 4)
+    good = 1 << 20
+    args = [good] * 7
+    # n_chunks < 1
+    assert lib.sfa_forward_host(ctypes.byref(d), *args, 0, good, out.value, None, None) == 1
+    # no workspace, a short one, a misaligned one
+    assert lib.sfa_forward_host(ctypes.byref(d), *args, 4, None, out.value, None, None) == 1
+    assert lib.sfa_forward_host(ctypes.byref(d), *args, 4, good, out.value - 1, None, None) == 1
+    assert lib.sfa_forward_host(ctypes.byref(d), *args, 4, good + 16, out.value, None, None) == 1
+    # a missing host pointer
+    assert lib.sfa_forward_host(ctypes.byref(d), None, *args[1:], 4, good, out.value, None, None) == 1
+    # B = 0 is a no-op
+    d0 = _desc(sfa, B=0)
+    assert lib.sfa_forward_host(ctypes.byref(d0), *args, 4, None, 0, None, None) == 0

@@ -186,7 +186,21 @@ def test_forward_host_pipeline_equals_device_forward():
     fr, cn = gpu_sets(w)
     o_ref, l_ref = sfa().forward(q.cuda(), k.cuda(), v.cuda(), fr, cn, w.P)
     qp, kp, vp = (x.pin_memory() for x in (q, k, v))
-    for n_chunks in (1, 3, 7):
+    for n_chunks in (1, 3, 7, 100):
         o, l = sfa().forward_host(qp, kp, vp, fr, cn, w.P, n_chunks=n_chunks)
         torch.cuda.synchronize()
         assert torch.equal(o, o_ref.cpu()) and torch.equal(l, l_ref.cpu())
+
+
+def test_forward_host_d64_and_pageable_memory():
+    # sfa_forward_host at d = 64 with a ragged frame (P = 136), from pageable host memory
+    # (the copies then run synchronously): the device call's result exactly
+    w = Workload("host64", B=1, H=3, Tq=4, Tkv=4, q_off=0, P=136, d=64, C=3, W=3, T_per=2,
+                 heads=(SetSpec("lvsa"),) * 3)
+    q, k, v = workload_qkv(w, seed=13)
+    fr, cn = gpu_sets(w)
+    o_ref, l_ref = sfa().forward(q.cuda(), k.cuda(), v.cuda(), fr, cn, w.P)
+    o, l = sfa().forward_host(q, k, v, fr, cn, w.P, out_host=torch.empty(q.shape, dtype=torch.bfloat16),
+                              lse_host=torch.empty(w.B, w.H, w.Lq), n_chunks=2)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o_ref.cpu()) and torch.equal(l, l_ref.cpu())
