@@ -403,6 +403,11 @@ def bench_hsa(sfa, dev, stream, flush, reps=20):
         return float(np.median(ts))
 
     sel_ms = timed(lambda: sfa.hsa_select(q, k, params, w.k_frames, w.k_blocks, workspace=wsp, stream=stream))
+    # steady state of an autoregressive cache: the history keys' means pooled once, then
+    # every call pools the queries and selects (sfa_hsa_select_pooled)
+    sfa.hsa_pool_keys(k, q, w.P, wsp, blocks.shape[-1], stream=stream)
+    selp_ms = timed(lambda: sfa.hsa_select_pooled(q, k, params, w.k_frames, w.k_blocks, wsp, Amax=blocks.shape[-1],
+                                                  stream=stream))
     fwd_ms = timed(lambda: sfa.forward_blocks(q, k, v, blocks, counts, w.P, out=o, lse=lse, stream=stream))
     # 252 CTAs are 1.7 waves of 148 SMs: the split form balances them
     split_ws = torch.empty(max(sfa.split_workspace_bytes(desc, 2), 1), dtype=torch.uint8, device=dev)
@@ -434,6 +439,9 @@ def bench_hsa(sfa, dev, stream, flush, reps=20):
     return {"workload": "hsa: 3 query frames after 21 history frames, P=1560, H=12, d=128; sink 1 + "
                         "local 6 frames always, 24 blocks of the 4 best history frames per 256-row query block",
             "select_ms": round(sel_ms, 4), "select_pool_bytes": pool_bytes,
+            "select_pooled_keys_ms": round(selp_ms, 4),
+            "select_share_of_attention": round(sel_ms / fwd_ms, 4),
+            "select_pooled_keys_share_of_attention": round(selp_ms / fwd_ms, 4),
             "forward_blocks_ms": round(fwd_ms, 4), "attended_tflop": round(flops / 1e12, 4),
             "forward_tflops": round(tf, 1), "forward_frac": round(tf / peak, 4),
             "forward_blocks_split2_ms": round(fwd2_ms, 4),

@@ -25,7 +25,8 @@ from ._lib import (SET_KINDS, SFA_DEBUG_STALL_SOFTMAX, SFA_ERR_BAD_SET, SFA_ERR_
                    SFA_ERR_INVALID_ARG, SFA_ERR_TIMEOUT, SFA_ERR_UNSUPPORTED, SFA_OK, AttnDesc,
                    SetParams, SfaError, attn_desc, build_sets, error_string, forward, forward_blocks, forward_dual,
                    forward_host, host_workspace_bytes,
-                   forward_paged, forward_split, gdn_forward, GdnDesc, hsa_max_count, hsa_select, load, lse_merge,
+                   forward_paged, forward_split, gdn_forward, GdnDesc, hsa_max_count, hsa_pool_keys, hsa_select, hsa_select_pooled,
+                   hsa_workspace_bytes, load, lse_merge,
                    set_max_count,
                    set_params, split_plan, split_workspace_bytes, version)
 
@@ -33,5 +34,6 @@ __all__ = ["SET_KINDS", "SFA_DEBUG_STALL_SOFTMAX", "SFA_ERR_BAD_SET", "SFA_ERR_C
            "SFA_ERR_INVALID_ARG", "SFA_ERR_TIMEOUT", "SFA_ERR_UNSUPPORTED", "SFA_OK", "AttnDesc",
            "SetParams", "SfaError", "attn_desc", "build_sets", "error_string", "forward", "forward_blocks",
            "forward_dual", "forward_host", "host_workspace_bytes",
-           "forward_paged", "forward_split", "gdn_forward", "GdnDesc", "hsa_max_count", "hsa_select",
+           "forward_paged", "forward_split", "gdn_forward", "GdnDesc", "hsa_max_count", "hsa_pool_keys", "hsa_select",
+           "hsa_select_pooled", "hsa_workspace_bytes",
            "load", "lse_merge", "set_max_count", "set_params", "split_plan", "split_workspace_bytes", "version"]

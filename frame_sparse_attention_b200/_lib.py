@@ -61,7 +61,7 @@ EXPORTS = ("sfa_error_string", "sfa_version", "sfa_set_max_count", "sfa_build_se
            "sfa_forward_split_workspace", "sfa_forward_split", "sfa_forward_split_noalloc", "sfa_forward_paged",
            "sfa_lse_merge", "sfa_hsa_max_count", "sfa_hsa_workspace", "sfa_hsa_select", "sfa_forward_blocks",
            "sfa_forward_blocks_split", "sfa_forward_blocks_split_workspace", "sfa_forward_split_plan",
-           "sfa_forward_host_workspace", "sfa_forward_host",
+           "sfa_forward_host_workspace", "sfa_forward_host", "sfa_hsa_pool_keys", "sfa_hsa_select_pooled",
            "sfa_forward_dual_workspace", "sfa_forward_dual", "sfa_gdn_workspace", "sfa_gdn_forward")
 
 
@@ -105,6 +105,11 @@ def load():
     lib.sfa_hsa_select.restype = st
     lib.sfa_hsa_select.argtypes = [ctypes.POINTER(AttnDesc), ctypes.POINTER(SetParams), i32, i32, vp, vp, vp,
                                    ctypes.c_size_t, vp, vp, vp]
+    lib.sfa_hsa_pool_keys.restype = st
+    lib.sfa_hsa_pool_keys.argtypes = [ctypes.POINTER(AttnDesc), vp, vp, ctypes.c_size_t, vp]
+    lib.sfa_hsa_select_pooled.restype = st
+    lib.sfa_hsa_select_pooled.argtypes = [ctypes.POINTER(AttnDesc), ctypes.POINTER(SetParams), i32, i32, vp, vp,
+                                          ctypes.c_size_t, vp, vp, vp]
     lib.sfa_forward_dual_workspace.restype = st
     lib.sfa_forward_dual_workspace.argtypes = [ctypes.POINTER(AttnDesc), i32, ctypes.POINTER(ctypes.c_size_t)]
     lib.sfa_forward_dual.restype = st
@@ -370,6 +375,41 @@ def hsa_select(q, k, params: SetParams, k_frames: int, k_blocks: int, Amax: int 
                                  k.data_ptr(), workspace.data_ptr(), workspace.numel(), blocks.data_ptr(),
                                  counts.data_ptr(), _stream(stream)), "sfa_hsa_select")
     return blocks, counts
+
+
+def hsa_pool_keys(k, q_like, P: int, workspace, Amax: int = 1, stream=None):
+    """Pool the keys' frame and block means into ``workspace`` (a uint8 CUDA tensor of
+    ``sfa_hsa_workspace`` bytes for the descriptor of (q_like, k)), for later
+    ``hsa_select_pooled`` calls over the same keys."""
+    desc = attn_desc(q_like, k, k, q_like, P, Amax)
+    _check(load().sfa_hsa_pool_keys(ctypes.byref(desc), k.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                                    _stream(stream)), "sfa_hsa_pool_keys")
+    return workspace
+
+
+def hsa_select_pooled(q, k_like, params: SetParams, k_frames: int, k_blocks: int, workspace, Amax: int | None = None,
+                      stream=None):
+    """hsa_select from the pooled keys already in ``workspace`` (``hsa_pool_keys``): pools
+    the queries only.  ``k_like`` gives the key shape (its data is not read)."""
+    B, H, Lq, d = q.shape
+    P = Lq // params.Tq
+    if Amax is None:
+        Amax = hsa_max_count(params, P, k_frames, k_blocks)
+    nqb = (P + QUERY_BLOCK - 1) // QUERY_BLOCK
+    desc = attn_desc(q, k_like, k_like, q, P, Amax)
+    blocks = torch.empty((B, H, params.Tq, nqb, Amax), dtype=torch.int32, device=q.device)
+    counts = torch.empty((B, H, params.Tq, nqb), dtype=torch.int32, device=q.device)
+    _check(load().sfa_hsa_select_pooled(ctypes.byref(desc), ctypes.byref(params), k_frames, k_blocks, q.data_ptr(),
+                                        workspace.data_ptr(), workspace.numel(), blocks.data_ptr(), counts.data_ptr(),
+                                        _stream(stream)), "sfa_hsa_select_pooled")
+    return blocks, counts
+
+
+def hsa_workspace_bytes(q, k, P: int, Amax: int = 1) -> int:
+    desc = attn_desc(q, k, k, q, P, Amax)
+    nbytes = ctypes.c_size_t(0)
+    _check(load().sfa_hsa_workspace(ctypes.byref(desc), ctypes.byref(nbytes)), "sfa_hsa_workspace")
+    return nbytes.value
 
 
 def forward_blocks(q, k, v, blocks, counts, P: int, scale: float | None = None, out=None, lse=None,

@@ -50,6 +50,7 @@ struct PoolArgs {
     const uint16_t *k, *q;
     int64_t k_sb, k_sh, k_sr, q_sb, q_sh, q_sr;  // strides in elements
     int H, P, T_kv, Tq, nblk, nqb;
+    int k_on;  // 1: the launch pools the keys (the first nblk * T_kv CTAs of a row), 0: queries only
     float *kb, *qb;
 };
 
@@ -61,7 +62,7 @@ __global__ void __launch_bounds__(POOL_THREADS) hsa_pool_kernel(const __grid_con
     constexpr int UNROLL = 4;                  // load rounds in flight
     __shared__ float part[RG][D];
     const int bh = blockIdx.y;
-    const int nk = a.nblk * a.T_kv;
+    const int nk = a.k_on ? a.nblk * a.T_kv : 0;
     const bool is_k = (int)blockIdx.x < nk;
     const int x = is_k ? blockIdx.x : blockIdx.x - nk;
     const int nseg = is_k ? a.nblk : a.nqb, seg = is_k ? KEY_BLOCK : QUERY_BLOCK;
@@ -142,17 +143,30 @@ __device__ __forceinline__ int rank_of(const float *scores, const int *ids, int 
     return r;
 }
 
-// dot(q, key) of D floats by one warp
-template <int D>
-__device__ __forceinline__ float warp_dot(const float *q, const float *key)
+// dot(q, key_b) of D floats for NB keys by one warp: the loads of all NB keys are issued
+// before any sum, so the warp waits for L2 once per NB dots.  Each lane adds its D / 32
+// products in order, then a butterfly adds the lanes: equal inputs give equal scores.
+template <int D, int NB>
+__device__ __forceinline__ void warp_dots(const float *q, const float *const (&key)[NB], const bool (&on)[NB],
+                                          float (&res)[NB])
 {
     const int lane = threadIdx.x & 31;
-    float s = 0.f;
+    float kv[NB][D / 32];
 #pragma unroll
-    for (int i = lane; i < D; i += 32) s = fmaf(q[i], __ldg(key + i), s);
+    for (int b = 0; b < NB; ++b)
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-    return s;
+        for (int i = 0; i < D / 32; ++i) kv[b][i] = on[b] ? __ldg(key[b] + lane + 32 * i) : 0.f;
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+        float s = 0.f;
+#pragma unroll
+        for (int i = 0; i < D / 32; ++i) s = fmaf(q[lane + 32 * i], kv[b][i], s);
+        res[b] = s;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+        for (int b = 0; b < NB; ++b) res[b] += __shfl_xor_sync(0xffffffffu, res[b], off);
 }
 
 // Dynamic shared memory: frame scores/ids [T_kv], block scores/ids [k_frames' * nblk],
@@ -199,11 +213,21 @@ __global__ void __launch_bounds__(SELECT_THREADS) hsa_select_kernel(const __grid
     }
     __syncthreads();
     const int n_hist = n_hist_s;
-    // frame scores
-    for (int i = warp; i < n_hist; i += nwarps) {
-        const float s = warp_dot<D>(qv, a.kf + (bh * a.T_kv + f_id[i]) * D);
+    // frame scores, four per warp at a time
+    for (int i0 = 4 * warp; i0 < n_hist; i0 += 4 * nwarps) {
+        const float *key[4];
+        bool on[4];
+        float sc[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            on[u] = i0 + u < n_hist;
+            key[u] = a.kf + (bh * a.T_kv + (on[u] ? f_id[i0 + u] : 0)) * D;
+        }
+        warp_dots<D, 4>(qv, key, on, sc);
         if (lane == 0) {
-            f_score[i] = s;
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (on[u]) f_score[i0 + u] = sc[u];
         }
     }
     __syncthreads();
@@ -220,13 +244,28 @@ __global__ void __launch_bounds__(SELECT_THREADS) hsa_select_kernel(const __grid
     __syncthreads();
     const int n_sel = n_sel_s;
     const int n_bc = n_sel * a.nblk;
-    // block scores of the selected frames
-    for (int i = warp; i < n_bc; i += nwarps) {
-        const int f = sel[i / a.nblk], bb = i % a.nblk;
-        const float s = warp_dot<D>(qv, a.kb + ((bh * a.T_kv + f) * a.nblk + bb) * D);
+    // block scores of the selected frames, four per warp at a time
+    for (int i0 = 4 * warp; i0 < n_bc; i0 += 4 * nwarps) {
+        const float *key[4];
+        bool on[4];
+        float sc[4];
+        int ids[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = i0 + u;
+            on[u] = i < n_bc;
+            const int f = on[u] ? sel[i / a.nblk] : 0, bb = on[u] ? i % a.nblk : 0;
+            ids[u] = f * a.nblk + bb;
+            key[u] = a.kb + ((bh * a.T_kv + f) * a.nblk + bb) * D;
+        }
+        warp_dots<D, 4>(qv, key, on, sc);
         if (lane == 0) {
-            b_score[i] = s;
-            b_id[i] = f * a.nblk + bb;
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (on[u]) {
+                    b_score[i0 + u] = sc[u];
+                    b_id[i0 + u] = ids[u];
+                }
         }
     }
     __syncthreads();
@@ -307,9 +346,10 @@ bool stride_ok(const int64_t *s, int d)
     return s[2] >= d && s[0] >= 0 && s[1] >= 0 && s[0] % 8 == 0 && s[1] % 8 == 0 && s[2] % 8 == 0;
 }
 
+// Pooling launch: the keys (with their frame means) and/or the queries of a descriptor.
 template <int D>
-sfa_status run_select(const sfa_attn_desc *d, const sfa_set_params *p, int k_frames, int k_blocks, const void *q,
-                      const void *k, uint8_t *ws, int32_t *blocks, int32_t *counts, cudaStream_t s)
+sfa_status run_pool(const sfa_attn_desc *d, const void *q, const void *k, uint8_t *ws, bool keys, bool queries,
+                    cudaStream_t s)
 {
     const WsLayout w = ws_layout(d);
     float *kf = reinterpret_cast<float *>(ws + w.kf), *kb = reinterpret_cast<float *>(ws + w.kb);
@@ -331,11 +371,24 @@ sfa_status run_select(const sfa_attn_desc *d, const sfa_set_params *p, int k_fra
     pa.Tq = d->Tq;
     pa.nblk = nblk;
     pa.nqb = nqb;
+    pa.k_on = keys ? 1 : 0;
     pa.kb = kb;
     pa.qb = qb;
-    hsa_pool_kernel<D><<<dim3((unsigned)(nblk * d->T_kv + nqb * d->Tq), bh), POOL_THREADS, 0, s>>>(pa);
-    const int64_t n_kf = (int64_t)bh * d->T_kv * D;
-    hsa_frame_mean_kernel<D><<<(unsigned)((n_kf + 255) / 256), 256, 0, s>>>(kb, n_kf, d->P, nblk, kf);
+    const unsigned grid_x = (unsigned)((keys ? nblk * d->T_kv : 0) + (queries ? nqb * d->Tq : 0));
+    hsa_pool_kernel<D><<<dim3(grid_x, bh), POOL_THREADS, 0, s>>>(pa);
+    if (keys) {
+        const int64_t n_kf = (int64_t)bh * d->T_kv * D;
+        hsa_frame_mean_kernel<D><<<(unsigned)((n_kf + 255) / 256), 256, 0, s>>>(kb, n_kf, d->P, nblk, kf);
+    }
+    return launch_status();
+}
+
+// Selection from the pooled keys and queries in the workspace.
+template <int D>
+sfa_status run_select(const sfa_attn_desc *d, const sfa_set_params *p, int k_frames, int k_blocks, uint8_t *ws,
+                      int32_t *blocks, int32_t *counts, cudaStream_t s)
+{
+    const WsLayout w = ws_layout(d);
     SelectArgs a;
     a.B = d->B;
     a.H = d->H;
@@ -351,9 +404,9 @@ sfa_status run_select(const sfa_attn_desc *d, const sfa_set_params *p, int k_fra
     a.chunk_len = p->chunk_len;
     a.k_frames = k_frames;
     a.k_blocks = k_blocks;
-    a.kf = kf;
-    a.kb = kb;
-    a.qb = qb;
+    a.kf = reinterpret_cast<const float *>(ws + w.kf);
+    a.kb = reinterpret_cast<const float *>(ws + w.kb);
+    a.qb = reinterpret_cast<const float *>(ws + w.qb);
     a.blocks = blocks;
     a.counts = counts;
     const int n_sel_max = std::min(k_frames, d->T_kv);
@@ -367,6 +420,25 @@ sfa_status run_select(const sfa_attn_desc *d, const sfa_set_params *p, int k_fra
     const int64_t grid = (int64_t)d->B * d->H * d->Tq * a.nqb;
     hsa_select_kernel<D><<<(unsigned)grid, SELECT_THREADS, smem, s>>>(a);
     return launch_status();
+}
+
+// Common host checks of the selection entry points (the tensors present are checked).
+sfa_status select_checks(const sfa_attn_desc *d, const sfa_set_params *p, int k_frames, int k_blocks, const void *q,
+                         const void *k, void *workspace, size_t workspace_bytes, const int32_t *blocks,
+                         const int32_t *counts, bool need_k)
+{
+    if (!desc_ok(d) || !params_ok(p, d ? d->P : 0, k_frames, k_blocks)) return SFA_ERR_INVALID_ARG;
+    if (d->d != 64 && d->d != 128) return SFA_ERR_UNSUPPORTED;
+    if (p->T_kv != d->T_kv || p->Tq != d->Tq) return SFA_ERR_INVALID_ARG;
+    if (max_count(p, d->P, k_frames, k_blocks) > d->Amax) return SFA_ERR_INVALID_ARG;
+    if (d->B == 0) return SFA_OK;
+    if (!q || (need_k && !k) || !workspace || !blocks || !counts) return SFA_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(q) % 16 || (need_k && reinterpret_cast<uintptr_t>(k) % 16) ||
+        reinterpret_cast<uintptr_t>(workspace) % 256)
+        return SFA_ERR_INVALID_ARG;
+    if (!stride_ok(d->q_stride, d->d) || (need_k && !stride_ok(d->k_stride, d->d))) return SFA_ERR_INVALID_ARG;
+    if (workspace_bytes < ws_layout(d).total) return SFA_ERR_INVALID_ARG;
+    return SFA_OK;
 }
 
 }  // namespace
@@ -396,19 +468,43 @@ extern "C" sfa_status sfa_hsa_select(const sfa_attn_desc *d, const sfa_set_param
                                      int32_t k_blocks, const void *q, const void *k, void *workspace,
                                      size_t workspace_bytes, int32_t *blocks, int32_t *counts, sfa_stream_t stream)
 {
-    if (!desc_ok(d) || !params_ok(p, d ? d->P : 0, k_frames, k_blocks)) return SFA_ERR_INVALID_ARG;
-    if (d->d != 64 && d->d != 128) return SFA_ERR_UNSUPPORTED;
-    if (p->T_kv != d->T_kv || p->Tq != d->Tq) return SFA_ERR_INVALID_ARG;
-    if (max_count(p, d->P, k_frames, k_blocks) > d->Amax) return SFA_ERR_INVALID_ARG;
-    if (d->B == 0) return SFA_OK;
-    if (!q || !k || !workspace || !blocks || !counts) return SFA_ERR_INVALID_ARG;
-    if (reinterpret_cast<uintptr_t>(q) % 16 || reinterpret_cast<uintptr_t>(k) % 16 ||
-        reinterpret_cast<uintptr_t>(workspace) % 256)
-        return SFA_ERR_INVALID_ARG;
-    if (!stride_ok(d->q_stride, d->d) || !stride_ok(d->k_stride, d->d)) return SFA_ERR_INVALID_ARG;
-    if (workspace_bytes < ws_layout(d).total) return SFA_ERR_INVALID_ARG;
+    sfa_status st = select_checks(d, p, k_frames, k_blocks, q, k, workspace, workspace_bytes, blocks, counts, true);
+    if (st != SFA_OK || d->B == 0) return st;
     cudaStream_t s = as_cuda(stream);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
-    return d->d == 128 ? run_select<128>(d, p, k_frames, k_blocks, q, k, ws, blocks, counts, s)
-                       : run_select<64>(d, p, k_frames, k_blocks, q, k, ws, blocks, counts, s);
+    st = d->d == 128 ? run_pool<128>(d, q, k, ws, true, true, s) : run_pool<64>(d, q, k, ws, true, true, s);
+    if (st != SFA_OK) return st;
+    return d->d == 128 ? run_select<128>(d, p, k_frames, k_blocks, ws, blocks, counts, s)
+                       : run_select<64>(d, p, k_frames, k_blocks, ws, blocks, counts, s);
+}
+
+extern "C" sfa_status sfa_hsa_pool_keys(const sfa_attn_desc *d, const void *k, void *workspace,
+                                        size_t workspace_bytes, sfa_stream_t stream)
+{
+    if (!desc_ok(d)) return SFA_ERR_INVALID_ARG;
+    if (d->d != 64 && d->d != 128) return SFA_ERR_UNSUPPORTED;
+    if ((int64_t)d->T_kv * ((d->P + KEY_BLOCK - 1) / KEY_BLOCK) > MAX_ENTRIES) return SFA_ERR_INVALID_ARG;
+    if (d->B == 0) return SFA_OK;
+    if (!k || !workspace || reinterpret_cast<uintptr_t>(k) % 16 || reinterpret_cast<uintptr_t>(workspace) % 256)
+        return SFA_ERR_INVALID_ARG;
+    if (!stride_ok(d->k_stride, d->d) || workspace_bytes < ws_layout(d).total) return SFA_ERR_INVALID_ARG;
+    cudaStream_t s = as_cuda(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    return d->d == 128 ? run_pool<128>(d, nullptr, k, ws, true, false, s)
+                       : run_pool<64>(d, nullptr, k, ws, true, false, s);
+}
+
+extern "C" sfa_status sfa_hsa_select_pooled(const sfa_attn_desc *d, const sfa_set_params *p, int32_t k_frames,
+                                            int32_t k_blocks, const void *q, void *workspace, size_t workspace_bytes,
+                                            int32_t *blocks, int32_t *counts, sfa_stream_t stream)
+{
+    sfa_status st =
+        select_checks(d, p, k_frames, k_blocks, q, nullptr, workspace, workspace_bytes, blocks, counts, false);
+    if (st != SFA_OK || d->B == 0) return st;
+    cudaStream_t s = as_cuda(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    st = d->d == 128 ? run_pool<128>(d, q, nullptr, ws, false, true, s) : run_pool<64>(d, q, nullptr, ws, false, true, s);
+    if (st != SFA_OK) return st;
+    return d->d == 128 ? run_select<128>(d, p, k_frames, k_blocks, ws, blocks, counts, s)
+                       : run_select<64>(d, p, k_frames, k_blocks, ws, blocks, counts, s);
 }

@@ -385,6 +385,22 @@ sfa_status sfa_hsa_select(const sfa_attn_desc *desc, const sfa_set_params *p, in
                           int32_t k_blocks, const void *q, const void *k, void *workspace,
                           size_t workspace_bytes, int32_t *blocks, int32_t *counts, sfa_stream_t stream);
 
+/* Selection with the pooled keys kept from an earlier call.  The history frames of an
+ * autoregressive cache do not change while later chunks attend them, so their frame and
+ * block means ("LIGHT FORCING", §2.2: token compression of the keys) need computing once:
+ * sfa_hsa_pool_keys writes them into the workspace (the part sfa_hsa_select also fills),
+ * and sfa_hsa_select_pooled pools the queries only and selects from the keys' means
+ * already there.  sfa_hsa_pool_keys followed by sfa_hsa_select_pooled gives the lists
+ * sfa_hsa_select gives for the same q and k, bit for bit.  Arguments as sfa_hsa_select;
+ * the workspace must be the one the keys were pooled into, for the same descriptor
+ * (B, H, T_kv, P, d); its other parts are overwritten. */
+sfa_status sfa_hsa_pool_keys(const sfa_attn_desc *desc, const void *k, void *workspace, size_t workspace_bytes,
+                             sfa_stream_t stream);
+
+sfa_status sfa_hsa_select_pooled(const sfa_attn_desc *desc, const sfa_set_params *p, int32_t k_frames,
+                                 int32_t k_blocks, const void *q, void *workspace, size_t workspace_bytes,
+                                 int32_t *blocks, int32_t *counts, sfa_stream_t stream);
+
 sfa_status sfa_forward_blocks(const sfa_attn_desc *desc, const void *q, const void *k, const void *v,
                               const int32_t *blocks, const int32_t *counts, void *o, float *lse,
                               int32_t *dev_status, sfa_stream_t stream);

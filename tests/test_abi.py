@@ -312,3 +312,19 @@ def test_forward_host_host_checks(sfa):
     # B = 0 is a no-op
     d0 = _desc(sfa, B=0)
     assert lib.sfa_forward_host(ctypes.byref(d0), *args, 4, None, 0, None, None) == 0
+
+
+def test_hsa_pooled_host_checks(sfa):
+    lib = sfa.load()
+    d = _desc(sfa, Tq=3, T_kv=24, P=1560, d=128, Amax=7 * 13 + 24)
+    need = ctypes.c_size_t(0)
+    assert lib.sfa_hsa_workspace(ctypes.byref(d), ctypes.byref(need)) == 0
+    good = 1 << 20
+    assert lib.sfa_hsa_pool_keys(ctypes.byref(d), None, good, need.value, None) == 1          # no keys
+    assert lib.sfa_hsa_pool_keys(ctypes.byref(d), good, good + 16, need.value, None) == 1     # misaligned
+    assert lib.sfa_hsa_pool_keys(ctypes.byref(d), good, good, need.value - 1, None) == 1      # short
+    p = sfa.set_params(T_kv=24, Tq=3, q_off=21, n_sink=1, n_prev=3, chunk_len=3)
+    assert lib.sfa_hsa_select_pooled(ctypes.byref(d), ctypes.byref(p), 4, 24, good, good, need.value - 256,
+                                     good, good, None) == 1
+    assert lib.sfa_hsa_select_pooled(ctypes.byref(d), ctypes.byref(p), 4, 24, None, good, need.value,
+                                     good, good, None) == 1

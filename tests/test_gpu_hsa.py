@@ -251,3 +251,20 @@ def test_forward_blocks_scheduled_workload_sampled():
     o_ref, l_ref = hsa.attention_blocks(q.float().numpy(), k.float().numpy(), v.float().numpy(), lists, cnts,
                                         w.P, 1 / math.sqrt(w.d), rows=rows)
     compare(o.float().cpu().reshape(-1, w.d).numpy()[rows], lse.cpu().reshape(-1).numpy()[rows], o_ref, l_ref)
+
+
+@pytest.mark.parametrize("w", SMALL + [WORKLOADS["hsa"]], ids=[w.name for w in SMALL] + ["hsa"])
+def test_pooled_keys_reused_equal_full_selection(w):
+    # keys pooled once (sfa_hsa_pool_keys), then two selections with different queries
+    # (sfa_hsa_select_pooled) give the lists of full selections, bit for bit
+    m = sfa()
+    q, k, _ = (x.cuda() for x in workload_qkv(w, seed=8))
+    q2 = torch.flip(q, dims=[2]).contiguous()
+    Amax = m.hsa_max_count(_params(w), w.P, w.k_frames, w.k_blocks)
+    ws = torch.empty(m.hsa_workspace_bytes(q, k, w.P, Amax), dtype=torch.uint8, device="cuda")
+    m.hsa_pool_keys(k, q, w.P, ws, Amax)
+    for qq in (q, q2):
+        b1, c1 = m.hsa_select_pooled(qq, k, _params(w), w.k_frames, w.k_blocks, ws, Amax=Amax)
+        b0, c0 = m.hsa_select(qq, k, _params(w), w.k_frames, w.k_blocks, Amax=Amax)
+        torch.cuda.synchronize()
+        assert torch.equal(b0, b1) and torch.equal(c0, c1)
