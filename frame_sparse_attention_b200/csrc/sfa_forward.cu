@@ -1375,6 +1375,9 @@ extern "C" sfa_status sfa_forward_split(const sfa_attn_desc *d, const void *q, c
         auto_splits(d, 1, 0, sc.k0, sc.k1);
         if (!workspace || reinterpret_cast<uintptr_t>(workspace) % 256 || workspace_bytes < sched_ws_bytes(d, sc.k0, 0))
             return SFA_ERR_INVALID_ARG;
+        if (sc.k0 == 1)  // one range per unit: the plain launch (ordering alone measured no gain)
+            return d->d == 128 ? launch<128>(d, q, k, v, frames, counts, o, lse, dev_status, s)
+                               : launch<64>(d, q, k, v, frames, counts, o, lse, dev_status, s);
         uint8_t *ws = static_cast<uint8_t *>(workspace);
         sc.items = reinterpret_cast<int2 *>(ws + (sc.k0 > 1 ? split_ws_bytes(d, sc.k0) : 0));
         float *ws_lse = reinterpret_cast<float *>(ws + split_ws_o_bytes(d, sc.k0));
@@ -1742,6 +1745,11 @@ extern "C" sfa_status sfa_forward_blocks_split(const sfa_attn_desc *d, const voi
         auto_splits(d, 1, nblk, sc.k0, sc.k1);
         if (!workspace || reinterpret_cast<uintptr_t>(workspace) % 256 || workspace_bytes < sched_ws_bytes(d, sc.k0, 0))
             return SFA_ERR_INVALID_ARG;
+        if (sc.k0 == 1)  // one range per unit: the plain launch
+            return d->d == 128 ? launch<128>(d, q, k, v, blocks, counts, o, lse, dev_status, s, 1, nullptr, nullptr,
+                                             nullptr, 0, nblk)
+                               : launch<64>(d, q, k, v, blocks, counts, o, lse, dev_status, s, 1, nullptr, nullptr,
+                                            nullptr, 0, nblk);
         uint8_t *ws = static_cast<uint8_t *>(workspace);
         sc.items = reinterpret_cast<int2 *>(ws + (sc.k0 > 1 ? split_ws_bytes(d, sc.k0) : 0));
         void *ws_o = sc.k0 > 1 ? workspace : nullptr;

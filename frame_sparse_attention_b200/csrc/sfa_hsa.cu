@@ -8,12 +8,12 @@
 // (sfa_forward_blocks, in sfa_forward.cu).
 //
 // Two kernels:
-//   * hsa_pool_kernel: one CTA per segment (128-token key block or 256-row query block)
-//     of keys or queries, both in one launch; 16-byte loads, four rows of them in flight
-//     per thread, fp32 sums per column, one mean per segment.
+//   * hsa_pool_kernel: one CTA per 128-token key block; 16-byte loads, four rows of them
+//     in flight per thread, fp32 sums per column, one mean per block.
 //     HBM-bound: every K and Q element is read once.  hsa_frame_mean_kernel then forms
 //     each frame's mean as the token-weighted average of its block means.
-//   * hsa_select_kernel: one CTA per (b, h, t, query block): scores of the history
+//   * hsa_select_kernel: one CTA per (b, h, t, query block): the mean of its query rows
+//     (the same pooling code), scores of the history
 //     frames, top k_frames, scores of their blocks, top k_blocks (a candidate is kept
 //     when fewer than k candidates rank before it: one pass, no serial rounds), then the
 //     sorted union with the always-attended blocks, compacted with a block-wide prefix
@@ -39,40 +39,19 @@ constexpr int MAX_ENTRIES = 65536;  // T_kv * nblk bound (the block flags live i
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
-// Mean of one segment of rows of one frame: the segments of the keys (KEY_BLOCK rows) and
-// of the queries (QUERY_BLOCK rows) in one launch.  CTA x of grid row bh = b*H + h takes
-// key segment x (x < nk = nblk * T_kv: segment x % nblk of frame x / nblk) or query
-// segment x - nk; it writes the mean to out[((bh * n_frames + f) * nseg + sg)][D] of its
-// tensor; the last segment of a frame holds the remaining rows.  D/8 threads per row (8
-// columns, one 16-byte load each), POOL_THREADS / (D/8) rows at a time and four of those
-// in flight per thread, then a shared-memory pass adds the row groups.
-struct PoolArgs {
-    const uint16_t *k, *q;
-    int64_t k_sb, k_sh, k_sr, q_sb, q_sh, q_sr;  // strides in elements
-    int H, P, T_kv, Tq, nblk, nqb;
-    int k_on;  // 1: the launch pools the keys (the first nblk * T_kv CTAs of a row), 0: queries only
-    float *kb, *qb;
-};
-
+// Mean of rows [r0, r1) of one frame, per column: `frame` points at the frame's first row
+// (row stride s_row elements).  POOL_THREADS threads: D/8 per row (8 columns, one 16-byte
+// load each), POOL_THREADS / (D/8) rows per round and UNROLL rounds of loads in flight, then
+// the row groups are added in order through `part`; threads < D write out[column].
 template <int D>
-__global__ void __launch_bounds__(POOL_THREADS) hsa_pool_kernel(const __grid_constant__ PoolArgs a)
+__device__ __forceinline__ void pool_segment(const uint16_t *frame, int64_t s_row, int r0, int r1,
+                                             float (*part)[D], float *out)
 {
     constexpr int TPR = D / 8;                 // threads per row
     constexpr int RG = POOL_THREADS / TPR;     // rows per load round
     constexpr int UNROLL = 4;                  // load rounds in flight
-    __shared__ float part[RG][D];
-    const int bh = blockIdx.y;
-    const int nk = a.k_on ? a.nblk * a.T_kv : 0;
-    const bool is_k = (int)blockIdx.x < nk;
-    const int x = is_k ? blockIdx.x : blockIdx.x - nk;
-    const int nseg = is_k ? a.nblk : a.nqb, seg = is_k ? KEY_BLOCK : QUERY_BLOCK;
-    const int sg = x % nseg, f = x / nseg;
-    const int n_frames = is_k ? a.T_kv : a.Tq;
     const int cg = threadIdx.x % TPR, rg = threadIdx.x / TPR;
-    const int r0 = sg * seg, r1 = min(r0 + seg, a.P);
-    const int64_t s_b = is_k ? a.k_sb : a.q_sb, s_h = is_k ? a.k_sh : a.q_sh, s_row = is_k ? a.k_sr : a.q_sr;
-    const uint16_t *base = (is_k ? a.k : a.q) + (int64_t)(bh / a.H) * s_b + (int64_t)(bh % a.H) * s_h +
-                           (int64_t)f * a.P * s_row + cg * 8;
+    const uint16_t *base = frame + cg * 8;
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     for (int r = r0 + rg; r < r1; r += UNROLL * RG) {
         uint4 v[UNROLL];
@@ -99,9 +78,41 @@ __global__ void __launch_bounds__(POOL_THREADS) hsa_pool_kernel(const __grid_con
     if (threadIdx.x < D) {
         float sum = 0.f;
         for (int g = 0; g < RG; ++g) sum += part[g][threadIdx.x];
-        float *out = is_k ? a.kb : a.qb;
-        out[(((int64_t)bh * n_frames + f) * nseg + sg) * D + threadIdx.x] = sum / (float)(r1 - r0);
+        out[threadIdx.x] = sum / (float)(r1 - r0);
     }
+    __syncthreads();
+}
+
+// Pooling launch: segment means of the keys (KEY_BLOCK rows) and/or the queries
+// (QUERY_BLOCK rows).  CTA x of grid row bh = b*H + h takes key segment x (x < nk =
+// nblk * T_kv when the keys are pooled: segment x % nblk of frame x / nblk) or query
+// segment x - nk, and writes its mean to out[((bh * n_frames + f) * nseg + sg)][D] of its
+// tensor; the last segment of a frame holds the remaining rows.
+struct PoolArgs {
+    const uint16_t *k, *q;
+    int64_t k_sb, k_sh, k_sr, q_sb, q_sh, q_sr;  // strides in elements
+    int H, P, T_kv, Tq, nblk, nqb;
+    int k_on;  // 1: the launch pools the keys (the first nblk * T_kv CTAs of a row), 0: queries only
+    float *kb, *qb;
+};
+
+template <int D>
+__global__ void __launch_bounds__(POOL_THREADS) hsa_pool_kernel(const __grid_constant__ PoolArgs a)
+{
+    __shared__ float part[POOL_THREADS / (D / 8)][D];
+    const int bh = blockIdx.y;
+    const int nk = a.k_on ? a.nblk * a.T_kv : 0;
+    const bool is_k = (int)blockIdx.x < nk;
+    const int x = is_k ? blockIdx.x : blockIdx.x - nk;
+    const int nseg = is_k ? a.nblk : a.nqb, seg = is_k ? KEY_BLOCK : QUERY_BLOCK;
+    const int sg = x % nseg, f = x / nseg;
+    const int n_frames = is_k ? a.T_kv : a.Tq;
+    const int r0 = sg * seg, r1 = min(r0 + seg, a.P);
+    const int64_t s_b = is_k ? a.k_sb : a.q_sb, s_h = is_k ? a.k_sh : a.q_sh, s_row = is_k ? a.k_sr : a.q_sr;
+    const uint16_t *frame = (is_k ? a.k : a.q) + (int64_t)(bh / a.H) * s_b + (int64_t)(bh % a.H) * s_h +
+                            (int64_t)f * a.P * s_row;
+    float *out = (is_k ? a.kb : a.qb) + (((int64_t)bh * n_frames + f) * nseg + sg) * D;
+    pool_segment<D>(frame, s_row, r0, r1, part, out);
 }
 
 // Frame means from the block means: the token-weighted average of a frame's blocks.
@@ -123,7 +134,8 @@ struct SelectArgs {
     int q_off, n_sink, n_prev, chunk_len, k_frames, k_blocks;
     const float *kf;  // [B][H][T_kv][D]
     const float *kb;  // [B][H][T_kv][nblk][D]
-    const float *qb;  // [B][H][Tq][nqb][D]
+    const uint16_t *q;         // bf16 queries: the CTA pools its own query block
+    int64_t q_sb, q_sh, q_sr;  // strides in elements
     int32_t *blocks;  // [B][H][Tq][nqb][Amax]
     int32_t *counts;  // [B][H][Tq][nqb]
 };
@@ -201,8 +213,11 @@ __global__ void __launch_bounds__(SELECT_THREADS) hsa_select_kernel(const __grid
     const int c0 = c - c % a.chunk_len;
     const int w_lo = c0 - a.n_prev, w_hi = c0 + a.chunk_len;  // local window [w_lo, w_hi)
     const int64_t bh = (int64_t)b * a.H + h;
-    for (int i = threadIdx.x; i < D; i += SELECT_THREADS)
-        qv[i] = a.qb[(((bh * a.Tq + t) * a.nqb) + qi) * D + i];
+    {  // the pooled (mean) query of this query block
+        __shared__ float part[SELECT_THREADS / (D / 8)][D];
+        const uint16_t *frame = a.q + (int64_t)b * a.q_sb + (int64_t)h * a.q_sh + (int64_t)t * a.P * a.q_sr;
+        pool_segment<D>(frame, a.q_sr, qi * QUERY_BLOCK, min(qi * QUERY_BLOCK + QUERY_BLOCK, a.P), part, qv);
+    }
     for (int i = threadIdx.x; i < n_entries; i += SELECT_THREADS) flag[i] = 0;
     if (threadIdx.x == 0) {
         // history candidates in ascending order
@@ -385,8 +400,8 @@ sfa_status run_pool(const sfa_attn_desc *d, const void *q, const void *k, uint8_
 
 // Selection from the pooled keys and queries in the workspace.
 template <int D>
-sfa_status run_select(const sfa_attn_desc *d, const sfa_set_params *p, int k_frames, int k_blocks, uint8_t *ws,
-                      int32_t *blocks, int32_t *counts, cudaStream_t s)
+sfa_status run_select(const sfa_attn_desc *d, const sfa_set_params *p, int k_frames, int k_blocks, const void *q,
+                      uint8_t *ws, int32_t *blocks, int32_t *counts, cudaStream_t s)
 {
     const WsLayout w = ws_layout(d);
     SelectArgs a;
@@ -406,7 +421,10 @@ sfa_status run_select(const sfa_attn_desc *d, const sfa_set_params *p, int k_fra
     a.k_blocks = k_blocks;
     a.kf = reinterpret_cast<const float *>(ws + w.kf);
     a.kb = reinterpret_cast<const float *>(ws + w.kb);
-    a.qb = reinterpret_cast<const float *>(ws + w.qb);
+    a.q = static_cast<const uint16_t *>(q);
+    a.q_sb = d->q_stride[0];
+    a.q_sh = d->q_stride[1];
+    a.q_sr = d->q_stride[2];
     a.blocks = blocks;
     a.counts = counts;
     const int n_sel_max = std::min(k_frames, d->T_kv);
@@ -472,10 +490,10 @@ extern "C" sfa_status sfa_hsa_select(const sfa_attn_desc *d, const sfa_set_param
     if (st != SFA_OK || d->B == 0) return st;
     cudaStream_t s = as_cuda(stream);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
-    st = d->d == 128 ? run_pool<128>(d, q, k, ws, true, true, s) : run_pool<64>(d, q, k, ws, true, true, s);
+    st = d->d == 128 ? run_pool<128>(d, q, k, ws, true, false, s) : run_pool<64>(d, q, k, ws, true, false, s);
     if (st != SFA_OK) return st;
-    return d->d == 128 ? run_select<128>(d, p, k_frames, k_blocks, ws, blocks, counts, s)
-                       : run_select<64>(d, p, k_frames, k_blocks, ws, blocks, counts, s);
+    return d->d == 128 ? run_select<128>(d, p, k_frames, k_blocks, q, ws, blocks, counts, s)
+                       : run_select<64>(d, p, k_frames, k_blocks, q, ws, blocks, counts, s);
 }
 
 extern "C" sfa_status sfa_hsa_pool_keys(const sfa_attn_desc *d, const void *k, void *workspace,
@@ -503,8 +521,6 @@ extern "C" sfa_status sfa_hsa_select_pooled(const sfa_attn_desc *d, const sfa_se
     if (st != SFA_OK || d->B == 0) return st;
     cudaStream_t s = as_cuda(stream);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
-    st = d->d == 128 ? run_pool<128>(d, q, nullptr, ws, false, true, s) : run_pool<64>(d, q, nullptr, ws, false, true, s);
-    if (st != SFA_OK) return st;
-    return d->d == 128 ? run_select<128>(d, p, k_frames, k_blocks, ws, blocks, counts, s)
-                       : run_select<64>(d, p, k_frames, k_blocks, ws, blocks, counts, s);
+    return d->d == 128 ? run_select<128>(d, p, k_frames, k_blocks, q, ws, blocks, counts, s)
+                       : run_select<64>(d, p, k_frames, k_blocks, q, ws, blocks, counts, s);
 }

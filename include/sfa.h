@@ -245,10 +245,10 @@ sfa_status sfa_forward_paged(const sfa_attn_desc *desc, const void *q, const voi
  * next to the number of SMs or the sets differ a lot in size between heads.
  *
  * n_split = 0 (scheduled): the library chooses the number of ranges (Amax taken as every
- * unit's length, the launch modelled as waves of equal pieces plus the merge; with many
- * full waves it keeps one range and writes O directly), and a one-CTA kernel first
- * counts every list's key tiles on the device and orders the CTAs longest range first,
- * so that the block scheduler runs a longest-first schedule over the SMs.  The result is
+ * unit's length, the launch modelled as waves of equal pieces plus the merge); with one
+ * range per unit (many full waves) the call is sfa_forward's launch.  With several, a
+ * one-CTA kernel first counts every list's key tiles on the device and orders the CTAs
+ * longest range first, so that the block scheduler runs a longest-first schedule.  The result is
  * the same attention; the order of the partial merge is fixed by the ranges, so a call
  * is deterministic.  sfa_forward_split_plan reports the choice.
  *
