@@ -122,12 +122,14 @@ def test_repeat_runs_identical_and_correct(name):
         assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
-@pytest.mark.parametrize("d", [64, 128])
-def test_running_max_rescale_path(d):
+@pytest.mark.parametrize("d,P", [(64, 192), (128, 192), (128, 320)])
+def test_running_max_rescale_path(d, P):
     # Keys of frame f are scaled by 2^(f // 2) (exact in bf16), so a row's running max grows
     # by far more than 2^8 from tile to tile and O is rescaled in flight many times.  The
-    # softmax ends up sharp, so the bound is the bf16-P one: |dO| <= 2^-7 max|v|.
-    T, P, H = 8, 192, 2
+    # softmax ends up sharp, so the bound is the bf16-P one: |dO| <= 2^-7 max|v|.  P = 320
+    # gives every frame a CTA with one query tile, whose two warpgroups take alternate key
+    # tiles and rescale their own partial results.
+    T, H = 8, 2
     w = Workload("rescale", B=1, H=H, Tq=T, Tkv=T, q_off=0, P=P, d=d, heads=(SetSpec("dense"),) * H)
     q, k, v = workload_qkv(w, seed=6)
     factor = (2.0 ** (torch.arange(T * P) // P // 2)).to(torch.float32)
@@ -135,7 +137,7 @@ def test_running_max_rescale_path(d):
     assert torch.isfinite(k.float()).all()
     bound = 2.0 ** -7 * float(v.float().abs().max()) + 1e-5
     o_err, l_err = run_and_check(w, q, k, v, o_tol=bound)
-    print(f"rescale path, d = {d}: O max-abs error {o_err:.2e} (bound {bound:.2e}), LSE {l_err:.2e}")
+    print(f"rescale path, d = {d}, P = {P}: O max-abs error {o_err:.2e} (bound {bound:.2e}), LSE {l_err:.2e}")
 
 
 # ------------------------------------------------------------------ full-size workloads, sampled rows
