@@ -81,7 +81,7 @@ struct Cfg {
     static constexpr int SMEM_V = SMEM_K + NSK * TILE_BYTES;
     static constexpr int SMEM_BAR = SMEM_V + NSV * TILE_BYTES;
     static constexpr int SMEM_BYTES = SMEM_BAR + 256 + 1024;  // + barriers, + alignment slack
-    static_assert(2 * NSK + 2 * NSV + 8 <= 20, "mbarriers must fit in 160 bytes");
+    static_assert(2 * NSK + 2 * NSV + 10 <= 20, "mbarriers must fit in 160 bytes");
     static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 };
 
@@ -99,7 +99,8 @@ struct Bars {
     __device__ uint32_t o_final() const { return q_full() + 40; }              // after the last P V
     __device__ uint32_t drain() const { return q_full() + 48; }
     __device__ uint32_t pv_done() const { return q_full() + 56; }  // one-tile CTAs: a P V complete
-    static constexpr int COUNT = 2 * Cfg<D>::NSK + 2 * Cfg<D>::NSV + 8;
+    __device__ uint32_t pv_x(int x) const { return q_full() + 64 + 8 * x; }  // P V of query tile x complete
+    static constexpr int COUNT = 2 * Cfg<D>::NSK + 2 * Cfg<D>::NSV + 10;
 };
 
 struct FwdArgs {
@@ -386,11 +387,11 @@ __device__ __forceinline__ void commit_one(uint32_t bar)
 }
 
 // One warp issues all tensor-core work, in the order
-//   S_A(0) S_B(0) | P V_A(j) S_A(j+1) P V_B(j) S_B(j+1) | ...
+//   S_A(0) S_B(0) | S_A(j+1) P V_A(j) S_B(j+1) P V_B(j) | ...
 // While one softmax warpgroup works on its tile, the tensor cores run the other tile's
-// P V and next S.  Because one thread issues everything and a commit tracks every MMA it
-// issued before, the completion of S_x(j+1) implies P V_x(j) is done: the softmax can
-// then overwrite P_x and rescale O_x without further waits.
+// next S and P V.  Once the softmax of tile x has handed over P_x(j) it has read S_x(j)
+// out, so S_x(j+1) is issued first: the softmax of the next tile starts while P V_x(j)
+// still runs, and waits for it (pv_x) only before it overwrites P_x or rescales O_x.
 template <int D>
 __device__ void mma_role(const FwdArgs &a, uint32_t sbase, uint32_t tmem, int h, bool has_b, const int32_t *fl,
                          int cnt, int t_off, int n_tiles, const Ctl &ctl)
@@ -423,6 +424,15 @@ __device__ void mma_role(const FwdArgs &a, uint32_t sbase, uint32_t tmem, int h,
         const int sv = j % C::NSV, sk = (j + 1) % C::NSK;
         for (int x = 0; x < nx; ++x) {
             if (!__all_sync(0xffffffffu, wait_bar(bar.p_full(x), j & 1, ctl))) goto done;
+            if (j + 1 < n_tiles) {
+                if (x == 0 && !__all_sync(0xffffffffu, wait_bar(bar.k_full(sk), ((j + 1) / C::NSK) & 1, ctl)))
+                    goto done;
+                tc_fence_after();
+                issue_s<D>(tmem + tcol_s(x), desc_add(dq, x * C::TILE_BYTES), desc_add(dk, sk * C::TILE_BYTES),
+                           idesc_bf16_f32(BM, mma_n(nv_next), false));
+                commit_one(bar.s_full(x));
+                if (x == nx - 1) commit_one(bar.k_free(sk));  // both tiles' S have read this K slot
+            }
             if (x == 0) {
                 if (!__all_sync(0xffffffffu, wait_bar(bar.v_full(sv), (j / C::NSV) & 1, ctl))) goto done;
                 if (nv_cur & 15) {
@@ -444,19 +454,11 @@ __device__ void mma_role(const FwdArgs &a, uint32_t sbase, uint32_t tmem, int h,
             tc_fence_after();
             issue_pv<D>(tmem + tcol_o(x), desc_add(dp, x * C::P_BYTES), desc_add(dv, sv * C::TILE_BYTES),
                         mma_n(nv_cur), j > 0);
+            commit_one(bar.pv_x(x));
             if (x == nx - 1) {
                 commit_one(bar.v_free(sv));  // both tiles' P V have read this V slot
                 // single-phase signal for the epilogues: O of both tiles is complete
                 if (j == n_tiles - 1) commit_one(bar.o_final());
-            }
-            if (j + 1 < n_tiles) {
-                if (x == 0 && !__all_sync(0xffffffffu, wait_bar(bar.k_full(sk), ((j + 1) / C::NSK) & 1, ctl)))
-                    goto done;
-                tc_fence_after();
-                issue_s<D>(tmem + tcol_s(x), desc_add(dq, x * C::TILE_BYTES), desc_add(dk, sk * C::TILE_BYTES),
-                           idesc_bf16_f32(BM, mma_n(nv_next), false));
-                commit_one(bar.s_full(x));
-                if (x == nx - 1) commit_one(bar.k_free(sk));  // both tiles' S have read this K slot
             }
         }
         nv_cur = nv_next;
@@ -611,6 +613,31 @@ __device__ __forceinline__ void exp_store_chunk(const uint32_t (&r)[32], float s
     }
 }
 
+// exp_store_chunk in two halves: the 16 bf16 pairs of the chunk are formed first and
+// stored later, so a wait can sit between them
+__device__ __forceinline__ void exp_chunk(const uint32_t (&r)[32], float sl2, float neg_m, uint32_t (&pk)[16],
+                                          float (&acc)[8])
+{
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float p0 = ex2_approx(fmaf(__uint_as_float(r[2 * i]), sl2, neg_m));
+        const float p1 = ex2_approx(fmaf(__uint_as_float(r[2 * i + 1]), sl2, neg_m));
+        acc[(2 * i) & 7] += p0;
+        acc[(2 * i + 1) & 7] += p1;
+        pk[i] = pack_bf16x2(p0, p1);
+    }
+}
+
+__device__ __forceinline__ void store_chunk(const uint32_t (&pk)[16], uint32_t p_row, int row, int c)
+{
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const uint32_t v[4] = {pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]};
+        const uint32_t chunk = (uint32_t)((c & 1) * 4 + q);
+        st_shared_v4(p_row + (c >> 1) * 16384 + ((chunk ^ (uint32_t)(row & 7)) << 4), v);
+    }
+}
+
 __device__ __forceinline__ float sum8(const float (&acc)[8])
 {
     return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
@@ -623,9 +650,12 @@ __device__ __forceinline__ float sum8(const float (&acc)[8])
 // max.  The first tile, and a tile on which any lane of the warp finds a larger max,
 // take the exact two-pass path: row max first, then P (S is re-read from TMEM; P lives
 // in shared memory), and O is rescaled in place.  FULL: all 128 keys valid.
+// pv_first (two-tile CTAs, j > 0): P V of the previous tile may still read P and write O;
+// its completion is waited for after the first chunk's exponentials, before any store.
 template <int D, bool FULL>
 __device__ __forceinline__ bool softmax_tile(uint32_t t_s, uint32_t p_row, int row, uint32_t t_o, int nv, float sl2,
-                                             float &m_used, float &l, int j, uint32_t pv_done, const Ctl &ctl)
+                                             float &m_used, float &l, int j, uint32_t pv_done, uint32_t pv_first,
+                                             const Ctl &ctl)
 {
     const int nch = FULL ? 4 : (nv + 31) >> 5;
     if (j > 0) {  // streaming pass against the current max
@@ -644,7 +674,15 @@ __device__ __forceinline__ bool softmax_tile(uint32_t t_s, uint32_t p_row, int r
                 if (c + 1 < 4 && (FULL || c + 1 < nch)) tmem_ld32(t_s + (c + 1) * 32, nxt);
                 mask_chunk<FULL>(c, nv, cur);
                 grow |= max32(cur) * sl2 > m_used + RESCALE_LOG2;
-                exp_store_chunk(cur, sl2, neg_m, p_row, row, c, acc);
+                if (c == 0 && pv_first) {
+                    uint32_t pk[16];
+                    exp_chunk(cur, sl2, neg_m, pk, acc);
+                    if (!__all_sync(0xffffffffu, wait_bar(pv_first, (j - 1) & 1, ctl))) return false;
+                    tc_fence_after();
+                    store_chunk(pk, p_row, row, 0);
+                } else {
+                    exp_store_chunk(cur, sl2, neg_m, p_row, row, c, acc);
+                }
             }
         }
         if (!__any_sync(0xffffffffu, grow)) {
@@ -676,8 +714,8 @@ __device__ __forceinline__ bool softmax_tile(uint32_t t_s, uint32_t p_row, int r
         }
     }
     // O must be rescaled before P V of this tile accumulates into it; the warp does it
-    // together (tcgen05.ld/st are warp-wide).  P V of the previous tile is already done:
-    // S of this tile was issued after it, and its completion was waited for.
+    // together (tcgen05.ld/st are warp-wide).  In a two-tile CTA P V of the previous tile
+    // is already done: the streaming pass waited for it (pv_first).
     if (j > 0 && __any_sync(0xffffffffu, resc)) {
         // (one-tile CTAs run S two tiles ahead: P V of the previous tile may still run)
         if (pv_done) {
@@ -708,7 +746,7 @@ __device__ void softmax_role(const CUtensorMap *tm_o, const FwdArgs &a, uint8_t 
 {
     using C = Cfg<D>;
     const Bars<D> bar{sbase + C::SMEM_BAR};
-    // 8 flags after the mbarriers (at most 15 x 8 bytes) and before the words at +240
+    // 8 flags after the mbarriers (at most 20 x 8 bytes) and before the words at +240
     volatile int32_t *epi_ok = reinterpret_cast<volatile int32_t *>(smem + C::SMEM_BAR + 160) + 4 * x;
     const int row = threadIdx.x & 127;  // query row inside the tile == TMEM lane
     const int warp = (threadIdx.x >> 5) & 3;
@@ -738,8 +776,9 @@ __device__ void softmax_role(const CUtensorMap *tm_o, const FwdArgs &a, uint8_t 
         }
         tc_fence_after();
         const uint32_t pvw = one_tile ? bar.pv_done() : 0u;
-        const bool ok = nv >= BN ? softmax_tile<D, true>(t_s, p_row, row, t_o, nv, sl2, m_used, l, j, pvw, ctl)
-                                 : softmax_tile<D, false>(t_s, p_row, row, t_o, nv, sl2, m_used, l, j, pvw, ctl);
+        const uint32_t pvf = (!one_tile && j > 0) ? bar.pv_x(x) : 0u;
+        const bool ok = nv >= BN ? softmax_tile<D, true>(t_s, p_row, row, t_o, nv, sl2, m_used, l, j, pvw, pvf, ctl)
+                                 : softmax_tile<D, false>(t_s, p_row, row, t_o, nv, sl2, m_used, l, j, pvw, pvf, ctl);
         if (!ok) {
             alive = false;
             break;
@@ -747,7 +786,9 @@ __device__ void softmax_role(const CUtensorMap *tm_o, const FwdArgs &a, uint8_t 
         tmem_wait_st();            // O rescale stores, if any
         fence_proxy_async_smem();  // P written with st.shared is read by the tensor cores
         tc_fence_before();
-        if (!((a.debug_flags & SFA_DEBUG_STALL_SOFTMAX) && j == 0)) mbar_arrive(bar.p_full(xb));
+        __syncwarp();              // one arrival per warp, after all its lanes' writes and fences
+        if ((threadIdx.x & 31) == 0 && !((a.debug_flags & SFA_DEBUG_STALL_SOFTMAX) && j == 0))
+            mbar_arrive(bar.p_full(xb));
     }
 
     // ---- epilogue: O / l -> bf16 -> swizzled smem (this tile's Q space) -> TMA store
@@ -871,8 +912,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (threadIdx.x == 0) {
         const Bars<D> bar{bars};
         for (int i = 0; i < Bars<D>::COUNT; ++i) mbar_init(bars + 8 * i, 1);
-        mbar_init(bar.p_full(0), BM);    // P full: every softmax thread of the tile arrives
-        mbar_init(bar.p_full(1), BM);
+        mbar_init(bar.p_full(0), BM / 32);  // P full: every softmax warp of the tile arrives
+        mbar_init(bar.p_full(1), BM / 32);
         *abort_flag = 0;
         // once a CTA has timed out, the ones that start later skip their work
         *skip = (a.status && *reinterpret_cast<volatile int32_t *>(a.status) == SFA_ERR_TIMEOUT) ? 1 : 0;
