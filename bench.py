@@ -60,9 +60,9 @@ def measured_peaks():
 
 # DRAM bytes (read + write) of one forward launch on this workload, from one ncu capture
 # of the same kernel on the 4-head version of the workload scaled by 3 to 12 heads (the
-# traffic is per (head, frame, query tile) unit): 3 x (197.301760 + 54.478592) MB.  Set
+# traffic is per (head, frame, query tile) unit): 3 x (197.425664 + 52.770560) MB.  Set
 # back to None whenever the forward kernel changes, until it is re-measured.
-NCU_TRAFFIC_BYTES = 755_341_056
+NCU_TRAFFIC_BYTES = 750_588_672
 # DRAM bytes read + written by the gated-delta kernels of one call on the gdn workload,
 # from an ncu capture: prep 232.055040 + 14.310912 MB, recurrence 143.407104 + 67.331584 MB.
 # None once the kernels change, until they are re-measured.
