@@ -44,7 +44,6 @@ constexpr int GW_MMA = 8;        // warp 8: TMA copies and MMAs
 constexpr int GTHREADS = GEPI + 32;
 constexpr int G_BOX = 128 * 128; // one 128-row x 64-column bf16 box (128-byte swizzle)
 constexpr int G_TILE = 2 * G_BOX;
-constexpr int F_BOX = 128 * 128; // one 128-row x 32-column fp32 box (128-byte swizzle)
 
 // gdn_prep_kernel shared memory: three stages of K, V tiles (scaled in place)
 constexpr int PR_STAGES = 3, PR_SLOT = 2 * G_TILE;
@@ -67,7 +66,9 @@ struct GdnArgs {
     const float *beta;   // [B][H][T*P]
     const float *s_in;   // [B][H][d][d] or null (zeros)
     float *s_out;        // [B][H][d][d]
-    const float *bws;    // [B*H*T][d][d] fp32 B_N, written by gdn_prep_kernel
+    const float *bws;    // fp32 B_N, written by gdn_prep_kernel: per (b, h, frame) [32][d][4], element
+                         // (row r, column 4 cg + i) at cg * 4 d + 4 r + i, so that the 16-byte
+                         // pieces of 32 consecutive rows lie side by side
     int32_t *status;
     uint64_t timeout_ns;
 };
@@ -116,10 +117,6 @@ __device__ __forceinline__ uint32_t swz(int row, int col)  // byte offset of bf1
     return (uint32_t)(box * G_BOX + row * 128 + ((chunk ^ (row & 7)) << 4) + (col & 7) * 2);
 }
 
-// byte offset of fp32 columns 4 j .. + 3 of row r in a swizzled 32-column box (the layout
-// a 128-byte-swizzle TMA copy of a 32 x 128 fp32 box uses)
-__device__ __forceinline__ uint32_t fswz(int r, int j) { return (uint32_t)(r * 128 + ((j ^ (r & 7)) << 4)); }
-
 __device__ __forceinline__ float bf16f(uint16_t x) { return __uint_as_float((uint32_t)x << 16); }
 
 // x * s for the 8 bf16 of a 16-byte chunk, rounded back to bf16
@@ -142,8 +139,7 @@ __device__ __forceinline__ uint4 scale_bf16x8(uint4 v, float s)
 // ------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(GTHREADS, 1)
     gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                    const __grid_constant__ CUtensorMap tm_mw, const __grid_constant__ CUtensorMap tm_bw,
-                    const __grid_constant__ GdnArgs a)
+                    const __grid_constant__ CUtensorMap tm_mw, const __grid_constant__ GdnArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -176,7 +172,6 @@ __global__ void __launch_bounds__(GTHREADS, 1)
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
             tma_prefetch_desc(&tm_mw);
-            tma_prefetch_desc(&tm_bw);
         }
         tmem_alloc(smem_u32(tmem_slot), 256);
         tmem_relinquish();
@@ -280,8 +275,9 @@ __global__ void __launch_bounds__(GTHREADS, 1)
         }
         if (ok && nt > 0 && (ok = __all_sync(0xffffffffu, gwait(fin, 0, abort, a.status, a.timeout_ns)))) {
             tc_fence_after();
-            // M_N row r as bf16 into stage 0 (the layout of the bf16 map's two boxes), B_N row
-            // r as fp32 into stage 1 (four swizzled 32-column boxes); every stage is free now
+            // M_N row r as bf16 into stage 0 (the layout of the bf16 map's two boxes; every
+            // stage is free now); B_N row r straight to global memory, 16 bytes per store, the
+            // lanes of a warp (32 consecutive rows) writing 512 contiguous bytes
 #pragma unroll
             for (int cc = 0; cc < 2; ++cc) {
                 const int c = c0 + cc;
@@ -298,11 +294,11 @@ __global__ void __launch_bounds__(GTHREADS, 1)
                         w[j] = pack_bf16x2(__uint_as_float(m[8 * q + 2 * j]), __uint_as_float(m[8 * q + 2 * j + 1]));
                     st_shared_v4(sbase + swz(r, c * 32 + q * 8), w);
                 }
+                float4 *bo = reinterpret_cast<float4 *>(const_cast<float *>(a.bws)) + ((int64_t)fr * 32 + c * 8) * GD + r;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const uint32_t w[4] = {bv[4 * j], bv[4 * j + 1], bv[4 * j + 2], bv[4 * j + 3]};
-                    st_shared_v4(sbase + PR_SLOT + c * F_BOX + fswz(r, j), w);
-                }
+                for (int j = 0; j < 8; ++j)
+                    __stcg(bo + j * GD, make_float4(__uint_as_float(bv[4 * j]), __uint_as_float(bv[4 * j + 1]),
+                                                    __uint_as_float(bv[4 * j + 2]), __uint_as_float(bv[4 * j + 3])));
             }
             fence_proxy_async_smem();
             mbar_arrive(staged);
@@ -310,8 +306,6 @@ __global__ void __launch_bounds__(GTHREADS, 1)
                 const int y = fr * GD;
 #pragma unroll
                 for (int kb = 0; kb < 2; ++kb) tma_store_2d(&tm_mw, sbase + kb * G_BOX, kb * 64, y);
-#pragma unroll
-                for (int c = 0; c < 4; ++c) tma_store_2d(&tm_bw, sbase + PR_SLOT + c * F_BOX, c * 32, y);
                 bulk_commit_and_wait_all();
             }
         }
@@ -576,11 +570,12 @@ __global__ void __launch_bounds__(GTHREADS, 1)
             const int early = upd ? (per > 2 ? per - 2 : 0) : per;
             uint32_t pk[32];  // bf16 pairs of the new state row (this half)
             if (upd) {
-                // B_N row r (this half), in flight while M_N S is computed
-                const float4 *bp = reinterpret_cast<const float4 *>(a.bws + ((bhi * a.T + n) * GD + r) * GD + hc * 64);
+                // B_N row r (this half), in flight while M_N S is computed: column groups
+                // 16 hc .. 16 hc + 15, each load of the warp 512 contiguous bytes
+                const float4 *bp = reinterpret_cast<const float4 *>(a.bws) + ((bhi * a.T + n) * 32 + hc * 16) * GD + r;
                 float4 bn[16];
 #pragma unroll
-                for (int j = 0; j < 16; ++j) bn[j] = __ldcg(bp + j);
+                for (int j = 0; j < 16; ++j) bn[j] = __ldg(bp + j * GD);
                 const float al = a.alpha[bhi * a.T + n];
                 if (!(ok = __all_sync(0xffffffffu, gwait(d_done, n & 1, abort, a.status, a.timeout_ns)))) break;
                 tc_fence_after();
@@ -685,17 +680,16 @@ bool encode_frames(CUtensorMap *m, const void *base, int B, int H, int T, int P,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// [rows][d] row-major as a 2-D map with a 128-byte-swizzled box of 128 rows: 64 columns
-// for bf16 (M_N), 32 for fp32 (B_N)
-bool encode_rows(CUtensorMap *m, void *base, int64_t rows, bool fp32)
+// bf16 [rows][d] row-major (M_N) as a 2-D map with a 128-byte-swizzled box of 128 rows x
+// 64 columns
+bool encode_rows(CUtensorMap *m, void *base, int64_t rows)
 {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
-    const int es_bytes = fp32 ? 4 : 2;
     const cuuint64_t gd[2] = {(cuuint64_t)GD, (cuuint64_t)rows};
-    const cuuint64_t gs[1] = {(cuuint64_t)GD * es_bytes};
-    const cuuint32_t box[2] = {(cuuint32_t)(128 / es_bytes), 128}, es[2] = {1, 1};
-    return fn(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, gd, gs, box, es,
+    const cuuint64_t gs[1] = {(cuuint64_t)GD * 2};
+    const cuuint32_t box[2] = {64, 128}, es[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, gd, gs, box, es,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -715,7 +709,7 @@ int gdn_split(const sfa_gdn_desc *d)
     return (int)std::max<int64_t>(1, std::min<int64_t>(n_tiles, sms / heads));
 }
 
-// workspace: M_N bf16 [B*H*T][d][d], then B_N fp32 [B*H*T][d][d]
+// workspace: M_N bf16 [B*H*T][d][d], then B_N fp32 [B*H*T][32][d][4] (see GdnArgs::bws)
 size_t gdn_m_bytes(const sfa_gdn_desc *d) { return (size_t)d->B * d->H * d->T * GD * GD * 2; }
 size_t gdn_ws_bytes(const sfa_gdn_desc *d) { return gdn_m_bytes(d) * 3; }
 
@@ -776,16 +770,15 @@ extern "C" sfa_status sfa_gdn_forward(const sfa_gdn_desc *d, const void *q, cons
     if (update) {
         const int64_t rows = (int64_t)d->B * d->H * d->T * GD;
         uint8_t *ws = static_cast<uint8_t *>(workspace);
-        CUtensorMap tk, tv, tb;
+        CUtensorMap tk, tv;
         if (!encode_frames(&tk, k, d->B, d->H, d->T, d->P, d->k_stride) ||
-            !encode_frames(&tv, v, d->B, d->H, d->T, d->P, d->v_stride) || !encode_rows(&tm, ws, rows, false) ||
-            !encode_rows(&tb, ws + gdn_m_bytes(d), rows, true))
+            !encode_frames(&tv, v, d->B, d->H, d->T, d->P, d->v_stride) || !encode_rows(&tm, ws, rows))
             return SFA_ERR_UNSUPPORTED;
         a.bws = reinterpret_cast<const float *>(ws + gdn_m_bytes(d));
         if (cudaFuncSetAttribute(gdn_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PR_SMEM) !=
             cudaSuccess)
             return SFA_ERR_CUDA;
-        gdn_prep_kernel<<<(unsigned)(d->B * d->H * d->T), GTHREADS, PR_SMEM, s>>>(tk, tv, tm, tb, a);
+        gdn_prep_kernel<<<(unsigned)(d->B * d->H * d->T), GTHREADS, PR_SMEM, s>>>(tk, tv, tm, a);
         if (cudaGetLastError() != cudaSuccess) return SFA_ERR_CUDA;
     }
     if (cudaFuncSetAttribute(gdn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, MS_SMEM) != cudaSuccess)
