@@ -430,9 +430,6 @@ __global__ void __launch_bounds__(GTHREADS, 1)
                 !(ok = __all_sync(0xffffffffu, gwait(s_ready, n & 1, abort, a.status, a.timeout_ns))))
                 break;
             if (upd) {
-                // M_{n+1} takes the slot of M_{n-1}: the product of frame n - 1 was read out
-                // before the state was ready
-                if (n >= 1 && n + 1 < a.T) load_m(n + 1);
                 if (!(ok = __all_sync(0xffffffffu, gwait(m_full(n & 1), (n >> 1) & 1, abort, a.status, a.timeout_ns))))
                     break;
                 m_landed = n + 1;
@@ -448,6 +445,9 @@ __global__ void __launch_bounds__(GTHREADS, 1)
                 }
                 __syncwarp();
                 issued = true;
+                // M_{n+1} takes the slot of M_{n-1}: the product of frame n - 1 was read out
+                // before the state was ready
+                if (n >= 1 && n + 1 < a.T) load_m(n + 1);
             }
             for (int ii = 0; ii < per && ok; ++ii, ++it) {
                 const int s = it % NQ, u = it & 1;
@@ -469,6 +469,9 @@ __global__ void __launch_bounds__(GTHREADS, 1)
                         mma_ss(tmem + T_O0 + u * 128, dq + (ka >> 4), ds + ((kk * 2048) >> 4), id_qs, kk > 0);
                     }
                     tc_commit(o_done(u));
+                    // after the frame's last MMA that reads S: the state may be rewritten
+                    // while this warp waits for the O store below
+                    if (ii == per - 1) tc_commit(s_free);
                 }
                 __syncwarp();
                 issued = true;
@@ -479,8 +482,6 @@ __global__ void __launch_bounds__(GTHREADS, 1)
                 }
             }
             if (!ok) break;
-            if (elect_one()) tc_commit(s_free);  // after every MMA of frame n that reads S
-            __syncwarp();
         }
         for (int t = total >= 2 ? total - 2 : 0; t < total && ok; ++t) {  // the last two tiles' O
             if (!(ok = __all_sync(0xffffffffu, gwait(o_free(t & 1), (t >> 1) & 1, abort, a.status, a.timeout_ns))))
