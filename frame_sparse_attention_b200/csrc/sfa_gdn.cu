@@ -45,10 +45,15 @@ constexpr int GTHREADS = GEPI + 32;
 constexpr int G_BOX = 128 * 128; // one 128-row x 64-column bf16 box (128-byte swizzle)
 constexpr int G_TILE = 2 * G_BOX;
 
-// gdn_prep_kernel shared memory: three stages of K, V tiles (scaled in place)
-constexpr int PR_STAGES = 3, PR_SLOT = 2 * G_TILE;
+// gdn_prep_kernel shared memory: three stages of 64-token K, V tiles (scaled in place);
+// two CTAs share an SM, so one streams its tiles while the other starts or ends a frame
+constexpr int PBM = 64;                  // tokens per prep tile
+constexpr int P_BOX = PBM * 128;         // one 64-row x 64-column bf16 box (128-byte swizzle)
+constexpr int P_TILE = 2 * P_BOX;        // one K or V tile
+constexpr int PR_STAGES = 3, PR_SLOT = 2 * P_TILE;
 constexpr int PR_BAR = PR_STAGES * PR_SLOT;
-constexpr int PR_SMEM = PR_BAR + 128 + 1024;
+constexpr int PR_SMEM = PR_BAR + 256 + 1024;
+static_assert(PR_STAGES * PR_SLOT >= G_TILE, "the stages hold the bf16 M_N tile for its store");
 constexpr uint32_t PT_M = 0, PT_B = 128;  // tensor-memory columns (256 allocated)
 
 // gdn_kernel shared memory: the bf16 state (B operand), two M_N tiles, a ring of Q tiles
@@ -117,6 +122,13 @@ __device__ __forceinline__ uint32_t swz(int row, int col)  // byte offset of bf1
     return (uint32_t)(box * G_BOX + row * 128 + ((chunk ^ (row & 7)) << 4) + (col & 7) * 2);
 }
 
+// byte offset of 16-byte chunk `chunk` (0-7) of row `row` of box `box` in a swizzled
+// 64-row prep tile
+__device__ __forceinline__ uint32_t pswz(int box, int row, int chunk)
+{
+    return (uint32_t)(box * P_BOX + row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
 __device__ __forceinline__ float bf16f(uint16_t x) { return __uint_as_float((uint32_t)x << 16); }
 
 // x * s for the 8 bf16 of a 16-byte chunk, rounded back to bf16
@@ -133,11 +145,11 @@ __device__ __forceinline__ uint4 scale_bf16x8(uint4 v, float s)
 // ------------------------------------------------------------------------------------
 // M_N = K^T diag(beta) K (bf16, the A operand of the recurrence) and B_N = K^T diag(beta) V
 // (fp32) of one frame: K~ = sqrt(beta) K and V~ = sqrt(beta) V are formed in place, then
-// M_N = K~^T K~ and B_N = K~^T V~ accumulate over the frame's tiles (M = N = d, K = 128
+// M_N = K~^T K~ and B_N = K~^T V~ accumulate over the frame's tiles (M = N = d, K = 64
 // tokens per tile; both operands MN-major).  beta must be >= 0 (a step size); a negative or
 // NaN beta stores SFA_ERR_INVALID_ARG and its token is left out.
 // ------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(GTHREADS, 1)
+__global__ void __launch_bounds__(GTHREADS, 2)
     gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_mw, const __grid_constant__ GdnArgs a)
 {
@@ -145,15 +157,15 @@ __global__ void __launch_bounds__(GTHREADS, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem), bb = sbase + PR_BAR;
     auto kv_full = [&](int s) { return bb + 8 * s; };        // K, V of stage s landed
-    auto scaled = [&](int s) { return bb + 24 + 8 * s; };    // K~, V~ of stage s formed (all threads)
-    auto mma_done = [&](int s) { return bb + 48 + 8 * s; };  // the MMAs reading stage s are done
-    const uint32_t fin = bb + 72, staged = bb + 80, drain = bb + 88;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + PR_BAR + 96);
-    volatile int32_t *abort = reinterpret_cast<volatile int32_t *>(smem + PR_BAR + 100);
+    auto scaled = [&](int s) { return bb + 48 + 8 * s; };    // K~, V~ of stage s formed (all threads)
+    auto mma_done = [&](int s) { return bb + 96 + 8 * s; };  // the MMAs reading stage s are done
+    const uint32_t fin = bb + 144, staged = bb + 152, drain = bb + 160;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + PR_BAR + 176);
+    volatile int32_t *abort = reinterpret_cast<volatile int32_t *>(smem + PR_BAR + 180);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int fr = blockIdx.x;  // (b * H + h) * T + n
     const int bhi = fr / a.T, n = fr % a.T, b = bhi / a.H, h = bhi % a.H;
-    const int nt = a.n_tiles;
+    const int nt = (a.P + PBM - 1) / PBM;  // 64-token tiles of the frame
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < PR_STAGES; ++s) {
@@ -189,11 +201,11 @@ __global__ void __launch_bounds__(GTHREADS, 1)
             const int s = t % PR_STAGES;
             const uint32_t dst = sbase + s * PR_SLOT;
             if (elect_one()) {
-                mbar_arrive_expect_tx(kv_full(s), 2 * G_TILE);
+                mbar_arrive_expect_tx(kv_full(s), 2 * P_TILE);
 #pragma unroll
                 for (int kb = 0; kb < 2; ++kb) {
-                    tma_load_5d(dst + kb * G_BOX, &tm_k, kv_full(s), kb * 64, t * GBM, n, h, b);
-                    tma_load_5d(dst + G_TILE + kb * G_BOX, &tm_v, kv_full(s), kb * 64, t * GBM, n, h, b);
+                    tma_load_5d(dst + kb * P_BOX, &tm_k, kv_full(s), kb * 64, t * PBM, n, h, b);
+                    tma_load_5d(dst + P_TILE + kb * P_BOX, &tm_v, kv_full(s), kb * 64, t * PBM, n, h, b);
                 }
             }
             __syncwarp();
@@ -206,11 +218,11 @@ __global__ void __launch_bounds__(GTHREADS, 1)
                 break;
             n_seen = i + 1;
             tc_fence_after();
-            const uint64_t dk = sdesc_sw128(sbase + s * PR_SLOT, G_BOX, 1024);           // K~ [tokens][d]
-            const uint64_t dv = sdesc_sw128(sbase + s * PR_SLOT + G_TILE, G_BOX, 1024);  // V~ [tokens][d]
+            const uint64_t dk = sdesc_sw128(sbase + s * PR_SLOT, P_BOX, 1024);           // K~ [tokens][d]
+            const uint64_t dv = sdesc_sw128(sbase + s * PR_SLOT + P_TILE, P_BOX, 1024);  // V~ [tokens][d]
             if (elect_one()) {
 #pragma unroll
-                for (uint32_t kk = 0; kk < GBM / 16; ++kk) {
+                for (uint32_t kk = 0; kk < PBM / 16; ++kk) {
                     const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
                     mma_ss(tmem + PT_M, dk + ((kk * 2048) >> 4), dk + ((kk * 2048) >> 4), id_mm, acc);
                     mma_ss(tmem + PT_B, dk + ((kk * 2048) >> 4), dv + ((kk * 2048) >> 4), id_mm, acc);
@@ -219,13 +231,13 @@ __global__ void __launch_bounds__(GTHREADS, 1)
             }
             __syncwarp();
             issued = true;
-            // tile i + 2 takes the stage of tile i - 1 once that tile's MMAs are done
-            if (i >= 1 && i + 2 < nt) {
+            // tile i + PR_STAGES - 1 takes the stage of tile i - 1 once that tile's MMAs are done
+            if (i >= 1 && i + PR_STAGES - 1 < nt) {
                 const int p = i - 1;
                 if (!(ok = __all_sync(0xffffffffu, gwait(mma_done(p % PR_STAGES), (p / PR_STAGES) & 1, abort,
                                                           a.status, a.timeout_ns))))
                     break;
-                load(i + 2);
+                load(i + PR_STAGES - 1);
             }
         }
         if (ok && nt > 0) {
@@ -242,17 +254,18 @@ __global__ void __launch_bounds__(GTHREADS, 1)
         }
         __syncwarp();
     } else {
-        // ---------------------------------------------------------------- row r, half hc
+        // ------------------------------------------------- tile row tr, columns 32 cq .. + 31
         const int e = threadIdx.x, qd = warp & 3, hc = warp >> 2;
-        const int r = qd * 32 + lane, c0 = hc * 2;
+        const int r = qd * 32 + lane, c0 = hc * 2;  // TMEM lane and column half of the epilogue
+        const int tr = (warp & 1) * 32 + lane, cq = warp >> 1;
         const uint32_t lane_base = tmem + ((uint32_t)(qd * 32) << 16);
         const float *beta = a.beta + (int64_t)fr * a.P;
         bool ok = true;
-        float bt_next = r < a.P ? beta[r] : 0.f;
+        float bt_next = tr < a.P ? beta[tr] : 0.f;
         for (int i = 0; i < nt; ++i) {
-            const int s = i % PR_STAGES, row = i * GBM + r;
+            const int s = i % PR_STAGES, row = i * PBM + tr;
             const float bt = bt_next;
-            bt_next = (i + 1 < nt && row + GBM < a.P) ? beta[row + GBM] : 0.f;
+            bt_next = (i + 1 < nt && row + PBM < a.P) ? beta[row + PBM] : 0.f;
             if (!(ok = __all_sync(0xffffffffu, gwait(kv_full(s), (i / PR_STAGES) & 1, abort, a.status, a.timeout_ns))))
                 break;
             float sb = 0.f;
@@ -262,11 +275,11 @@ __global__ void __launch_bounds__(GTHREADS, 1)
                 else if (a.status)
                     atomicCAS(a.status, 0, SFA_ERR_INVALID_ARG);
             }
-            // K~ and V~ rows (this half), in place
+            // K~ and V~ of tile row tr, columns 32 cq .. 32 cq + 31, in place
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const uint32_t off = s * PR_SLOT + swz(r, hc * 64 + q * 8);
-                uint4 *pk = reinterpret_cast<uint4 *>(smem + off), *pv = reinterpret_cast<uint4 *>(smem + off + G_TILE);
+            for (int q = 0; q < 4; ++q) {
+                const uint32_t off = s * PR_SLOT + pswz(cq >> 1, tr, (cq & 1) * 4 + q);
+                uint4 *pk = reinterpret_cast<uint4 *>(smem + off), *pv = reinterpret_cast<uint4 *>(smem + off + P_TILE);
                 *pk = scale_bf16x8(*pk, sb);
                 *pv = scale_bf16x8(*pv, sb);
             }
@@ -665,17 +678,18 @@ EncodeTiledFn encode_fn()
     return fn;
 }
 
-// bf16 [B][H][T*P][d] as a 5-D map (d, P, T, H, B), box 64 x 128 x 1 x 1 x 1, 128-byte
+// bf16 [B][H][T*P][d] as a 5-D map (d, P, T, H, B), box 64 x rows x 1 x 1 x 1, 128-byte
 // swizzle: a tile never crosses its frame; rows past the frame read as zero and are not
 // written by a store
-bool encode_frames(CUtensorMap *m, const void *base, int B, int H, int T, int P, const int64_t *stride)
+bool encode_frames(CUtensorMap *m, const void *base, int B, int H, int T, int P, const int64_t *stride,
+                   int rows = GBM)
 {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t gd[5] = {(cuuint64_t)GD, (cuuint64_t)P, (cuuint64_t)T, (cuuint64_t)H, (cuuint64_t)B};
     const cuuint64_t gs[4] = {(cuuint64_t)stride[2] * 2, (cuuint64_t)P * stride[2] * 2, (cuuint64_t)stride[1] * 2,
                               (cuuint64_t)stride[0] * 2};
-    const cuuint32_t box[5] = {64, (cuuint32_t)GBM, 1, 1, 1}, es[5] = {1, 1, 1, 1, 1};
+    const cuuint32_t box[5] = {64, (cuuint32_t)rows, 1, 1, 1}, es[5] = {1, 1, 1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), gd, gs, box, es,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -772,8 +786,8 @@ extern "C" sfa_status sfa_gdn_forward(const sfa_gdn_desc *d, const void *q, cons
         const int64_t rows = (int64_t)d->B * d->H * d->T * GD;
         uint8_t *ws = static_cast<uint8_t *>(workspace);
         CUtensorMap tk, tv;
-        if (!encode_frames(&tk, k, d->B, d->H, d->T, d->P, d->k_stride) ||
-            !encode_frames(&tv, v, d->B, d->H, d->T, d->P, d->v_stride) || !encode_rows(&tm, ws, rows))
+        if (!encode_frames(&tk, k, d->B, d->H, d->T, d->P, d->k_stride, PBM) ||
+            !encode_frames(&tv, v, d->B, d->H, d->T, d->P, d->v_stride, PBM) || !encode_rows(&tm, ws, rows))
             return SFA_ERR_UNSUPPORTED;
         a.bws = reinterpret_cast<const float *>(ws + gdn_m_bytes(d));
         if (cudaFuncSetAttribute(gdn_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PR_SMEM) !=
