@@ -314,6 +314,7 @@ def bench_merge(sfa, dev, stream, flush, reps=20, rows=None):
     times = []
     for _ in range(reps):
         flush.zero_()
+        gpu_lead(stream)
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
         a.record(stream)
@@ -393,6 +394,7 @@ def bench_hsa(sfa, dev, stream, flush, reps=20):
         ts = []
         for _ in range(reps):
             flush.zero_()
+            gpu_lead(stream)
             a = torch.cuda.Event(enable_timing=True)
             b = torch.cuda.Event(enable_timing=True)
             a.record(stream)
@@ -483,6 +485,7 @@ def bench_gdn(sfa, dev, stream, flush, reps=20):
     ts = []
     for _ in range(reps):
         flush.zero_()
+        gpu_lead(stream)
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
@@ -685,6 +688,15 @@ def setup_workload(sfa, dev, stream, name, split=1, dual=False):
     return step, flops, branches
 
 
+def gpu_lead(stream):
+    """Keep the GPU busy for about 50 us (a spin of 10^5 cycles) right before a start
+    event: the host then enqueues the timed launches before the GPU reaches the event, so
+    that the events bracket device work only, not the host's launch overhead (which the
+    e2e figure includes).  Matters for calls of a few microseconds."""
+    with torch.cuda.stream(stream):
+        torch.cuda._sleep(100_000)
+
+
 def time_device(step, flush, stream, dev, steps=20, warmup=5):
     """Median device time (ms) of `step` over `steps` runs after `warmup`, L2 flushed
     before every run (outside the events)."""
@@ -695,6 +707,7 @@ def time_device(step, flush, stream, dev, steps=20, warmup=5):
     times = []
     for _ in range(steps):
         flush.zero_()
+        gpu_lead(stream)
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)

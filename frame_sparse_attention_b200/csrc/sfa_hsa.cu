@@ -42,14 +42,14 @@ __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w 
 // Mean of rows [r0, r1) of one frame, per column: `frame` points at the frame's first row
 // (row stride s_row elements).  POOL_THREADS threads: D/8 per row (8 columns, one 16-byte
 // load each), POOL_THREADS / (D/8) rows per round and UNROLL rounds of loads in flight, then
-// the row groups are added in order through `part`; threads < D write out[column].
-template <int D>
+// the row groups are added in order through `part`; threads < D write out[column].  Each
+// thread adds its rows in row order whatever UNROLL is, so every UNROLL gives the same means.
+template <int D, int UNROLL>
 __device__ __forceinline__ void pool_segment(const uint16_t *frame, int64_t s_row, int r0, int r1,
                                              float (*part)[D], float *out)
 {
     constexpr int TPR = D / 8;                 // threads per row
     constexpr int RG = POOL_THREADS / TPR;     // rows per load round
-    constexpr int UNROLL = 4;                  // load rounds in flight
     const int cg = threadIdx.x % TPR, rg = threadIdx.x / TPR;
     const uint16_t *base = frame + cg * 8;
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -112,7 +112,7 @@ __global__ void __launch_bounds__(POOL_THREADS) hsa_pool_kernel(const __grid_con
     const uint16_t *frame = (is_k ? a.k : a.q) + (int64_t)(bh / a.H) * s_b + (int64_t)(bh % a.H) * s_h +
                             (int64_t)f * a.P * s_row;
     float *out = (is_k ? a.kb : a.qb) + (((int64_t)bh * n_frames + f) * nseg + sg) * D;
-    pool_segment<D>(frame, s_row, r0, r1, part, out);
+    pool_segment<D, 4>(frame, s_row, r0, r1, part, out);
 }
 
 // Frame means from the block means: the token-weighted average of a frame's blocks.
@@ -184,7 +184,7 @@ __device__ __forceinline__ void warp_dots(const float *q, const float *const (&k
 // Dynamic shared memory: frame scores/ids [T_kv], block scores/ids [k_frames' * nblk],
 // selected frames, frame flags [T_kv], entry flags [T_kv * nblk].
 template <int D>
-__global__ void __launch_bounds__(SELECT_THREADS) hsa_select_kernel(const __grid_constant__ SelectArgs a)
+__global__ void __launch_bounds__(SELECT_THREADS, 2) hsa_select_kernel(const __grid_constant__ SelectArgs a)
 {
     extern __shared__ __align__(16) uint8_t sm[];
     __shared__ float qv[D];
@@ -216,7 +216,9 @@ __global__ void __launch_bounds__(SELECT_THREADS) hsa_select_kernel(const __grid
     {  // the pooled (mean) query of this query block
         __shared__ float part[SELECT_THREADS / (D / 8)][D];
         const uint16_t *frame = a.q + (int64_t)b * a.q_sb + (int64_t)h * a.q_sh + (int64_t)t * a.P * a.q_sr;
-        pool_segment<D>(frame, a.q_sr, qi * QUERY_BLOCK, min(qi * QUERY_BLOCK + QUERY_BLOCK, a.P), part, qv);
+        // every row of the query block in one round of loads
+        constexpr int UNROLL = QUERY_BLOCK / (SELECT_THREADS / (D / 8));
+        pool_segment<D, UNROLL>(frame, a.q_sr, qi * QUERY_BLOCK, min(qi * QUERY_BLOCK + QUERY_BLOCK, a.P), part, qv);
     }
     for (int i = threadIdx.x; i < n_entries; i += SELECT_THREADS) flag[i] = 0;
     if (threadIdx.x == 0) {
