@@ -55,7 +55,8 @@ constexpr int NUM_THREADS = 352;
 constexpr int K_LOAD_WARP = 8;
 constexpr int MMA_WARP = 9;
 constexpr int V_LOAD_WARP = 10;
-constexpr float RESCALE_LOG2 = 8.0f;    // keep a stale row max while the new one is < 2^8 above
+constexpr float RESCALE_LOG2 = 8.0f;    // keep a stale row max while the tile's row sum against it stays < 2^8
+constexpr float RESCALE_LIMIT = 256.0f;  // 2^RESCALE_LOG2
 constexpr uint32_t DEFAULT_TIMEOUT_US = 2000000;  // 2 s; a healthy wait lasts microseconds
 constexpr uint32_t DRAIN_TIMEOUT_US = 2000000;
 constexpr uint32_t MAX_SPINS = 1u << 30;           // backstop should the timer not advance
@@ -645,11 +646,12 @@ __device__ __forceinline__ float sum8(const float (&acc)[8])
 
 // One K/V tile of the online softmax for this thread's query row (thread = TMEM lane):
 // S (fp32, TMEM) -> P = exp2(S * scale * log2e - m) as bf16 into shared memory, running
-// max m and sum l.  A row keeps a stale max m until a tile's max exceeds it by 2^RESCALE_LOG2, so
-// the common case streams S through registers 32 columns at a time against the current
-// max.  The first tile, and a tile on which any lane of the warp finds a larger max,
-// take the exact two-pass path: row max first, then P (S is re-read from TMEM; P lives
-// in shared memory), and O is rescaled in place.  FULL: all 128 keys valid.
+// max m and sum l.  A row keeps a stale max m while a tile's row sum against it stays at
+// most 2^RESCALE_LOG2 (every probability is then at most that), so the common case
+// streams S through registers 32 columns at a time against the current max.  The first
+// tile, and a tile on which any lane of the warp exceeds that sum, take the exact
+// two-pass path: row max first, then P against the larger max (S is re-read from TMEM; P
+// lives in shared memory), and O is rescaled in place.  FULL: all 128 keys valid.
 // pv_first (two-tile CTAs, j > 0): P V of the previous tile may still read P and write O;
 // its completion is waited for after the first chunk's exponentials, before any store.
 template <int D, bool FULL>
@@ -660,7 +662,6 @@ __device__ __forceinline__ bool softmax_tile(uint32_t t_s, uint32_t p_row, int r
     const int nch = FULL ? 4 : (nv + 31) >> 5;
     if (j > 0) {  // streaming pass against the current max
         float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        bool grow = false;
         const float neg_m = -m_used;
         // two register buffers: the load of chunk c+1 is in flight while chunk c is used
         uint32_t ra[32], rb[32];
@@ -673,7 +674,6 @@ __device__ __forceinline__ bool softmax_tile(uint32_t t_s, uint32_t p_row, int r
                 tmem_wait_ld_regs(cur);
                 if (c + 1 < 4 && (FULL || c + 1 < nch)) tmem_ld32(t_s + (c + 1) * 32, nxt);
                 mask_chunk<FULL>(c, nv, cur);
-                grow |= max32(cur) * sl2 > m_used + RESCALE_LOG2;
                 if (c == 0 && pv_first) {
                     uint32_t pk[16];
                     exp_chunk(cur, sl2, neg_m, pk, acc);
@@ -685,8 +685,12 @@ __device__ __forceinline__ bool softmax_tile(uint32_t t_s, uint32_t p_row, int r
                 }
             }
         }
-        if (!__any_sync(0xffffffffu, grow)) {
-            l += sum8(acc);
+        // a probability above 2^RESCALE_LOG2 (a row max that grew past the stale one by
+        // more than that) makes the tile's row sum exceed it too; a sum above it without
+        // such a probability only sends the row through the exact pass a little early
+        const float lt = sum8(acc);
+        if (!__any_sync(0xffffffffu, lt > RESCALE_LIMIT)) {
+            l += lt;
             return true;
         }
     }
@@ -701,7 +705,8 @@ __device__ __forceinline__ bool softmax_tile(uint32_t t_s, uint32_t p_row, int r
         }
     }
     const float m_cand = mx * sl2;
-    const bool resc = m_cand > m_used + RESCALE_LOG2;
+    // (after the streaming pass some probability exceeded 2, so the max has grown)
+    const bool resc = m_cand > m_used;
     const float m_new = resc ? m_cand : m_used;
     const float alpha = ex2_approx(m_used - m_new);  // 0 on the first tile, 1 if unchanged
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
