@@ -591,11 +591,28 @@ __device__ __forceinline__ void load_s_chunk(uint32_t taddr, int c, int nv, uint
     }
 }
 
+// Eight fp32 partial row sums kept as four pairs, each pair added with one two-lane
+// instruction (every lane rounds like a scalar fp32 add, so the sums are those of eight
+// scalar accumulators).
+struct Acc8 {
+    uint64_t v[4] = {0, 0, 0, 0};
+    __device__ __forceinline__ void add(int k, float a, float b)
+    {
+        asm("{\n\t.reg .b64 t;\n\tmov.b64 t, {%1, %2};\n\tadd.rn.f32x2 %0, %0, t;\n\t}"
+            : "+l"(v[k])
+            : "f"(a), "f"(b));
+    }
+    __device__ __forceinline__ float get(int i) const
+    {
+        return __uint_as_float((uint32_t)(v[i >> 1] >> ((i & 1) * 32)));
+    }
+};
+
 // exp2(s * sl2 - m) of columns 32c..32c+31 -> bf16, stored into this thread's row of the
 // P tile in shared memory (K-major, 128-byte swizzle: 64 keys per 16 KB box, 16-byte
 // chunk k of row r at chunk position k ^ (r & 7)); row sum into acc
 __device__ __forceinline__ void exp_store_chunk(const uint32_t (&r)[32], float sl2, float neg_m, uint32_t p_row,
-                                                int row, int c, float (&acc)[8])
+                                                int row, int c, Acc8 &acc)
 {
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -605,8 +622,7 @@ __device__ __forceinline__ void exp_store_chunk(const uint32_t (&r)[32], float s
             const int e = q * 8 + 2 * i;
             const float p0 = ex2_approx(fmaf(__uint_as_float(r[e]), sl2, neg_m));
             const float p1 = ex2_approx(fmaf(__uint_as_float(r[e + 1]), sl2, neg_m));
-            acc[(2 * i) & 7] += p0;
-            acc[(2 * i + 1) & 7] += p1;
+            acc.add(i & 3, p0, p1);
             pk[i] = pack_bf16x2(p0, p1);
         }
         const uint32_t chunk = (uint32_t)((c & 1) * 4 + q);
@@ -617,14 +633,13 @@ __device__ __forceinline__ void exp_store_chunk(const uint32_t (&r)[32], float s
 // exp_store_chunk in two halves: the 16 bf16 pairs of the chunk are formed first and
 // stored later, so a wait can sit between them
 __device__ __forceinline__ void exp_chunk(const uint32_t (&r)[32], float sl2, float neg_m, uint32_t (&pk)[16],
-                                          float (&acc)[8])
+                                          Acc8 &acc)
 {
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
         const float p0 = ex2_approx(fmaf(__uint_as_float(r[2 * i]), sl2, neg_m));
         const float p1 = ex2_approx(fmaf(__uint_as_float(r[2 * i + 1]), sl2, neg_m));
-        acc[(2 * i) & 7] += p0;
-        acc[(2 * i + 1) & 7] += p1;
+        acc.add(i & 3, p0, p1);
         pk[i] = pack_bf16x2(p0, p1);
     }
 }
@@ -639,9 +654,10 @@ __device__ __forceinline__ void store_chunk(const uint32_t (&pk)[16], uint32_t p
     }
 }
 
-__device__ __forceinline__ float sum8(const float (&acc)[8])
+__device__ __forceinline__ float sum8(const Acc8 &acc)
 {
-    return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+    return ((acc.get(0) + acc.get(1)) + (acc.get(2) + acc.get(3))) +
+           ((acc.get(4) + acc.get(5)) + (acc.get(6) + acc.get(7)));
 }
 
 // One K/V tile of the online softmax for this thread's query row (thread = TMEM lane):
@@ -661,7 +677,7 @@ __device__ __forceinline__ bool softmax_tile(uint32_t t_s, uint32_t p_row, int r
 {
     const int nch = FULL ? 4 : (nv + 31) >> 5;
     if (j > 0) {  // streaming pass against the current max
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        Acc8 acc;
         const float neg_m = -m_used;
         // two register buffers: the load of chunk c+1 is in flight while chunk c is used
         uint32_t ra[32], rb[32];
@@ -709,7 +725,7 @@ __device__ __forceinline__ bool softmax_tile(uint32_t t_s, uint32_t p_row, int r
     const bool resc = m_cand > m_used;
     const float m_new = resc ? m_cand : m_used;
     const float alpha = ex2_approx(m_used - m_new);  // 0 on the first tile, 1 if unchanged
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    Acc8 acc;
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
         if (FULL || c < nch) {
