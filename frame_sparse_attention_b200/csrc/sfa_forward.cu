@@ -55,8 +55,7 @@ constexpr int NUM_THREADS = 352;
 constexpr int K_LOAD_WARP = 8;
 constexpr int MMA_WARP = 9;
 constexpr int V_LOAD_WARP = 10;
-constexpr float RESCALE_LOG2 = 8.0f;    // keep a stale row max while the tile's row sum against it stays < 2^8
-constexpr float RESCALE_LIMIT = 256.0f;  // 2^RESCALE_LOG2
+constexpr float RESCALE_LIMIT = 256.0f;  // keep a stale row max while the tile's row sum against it stays <= 2^8
 constexpr uint32_t DEFAULT_TIMEOUT_US = 2000000;  // 2 s; a healthy wait lasts microseconds
 constexpr uint32_t DRAIN_TIMEOUT_US = 2000000;
 constexpr uint32_t MAX_SPINS = 1u << 30;           // backstop should the timer not advance
@@ -663,7 +662,7 @@ __device__ __forceinline__ float sum8(const Acc8 &acc)
 // One K/V tile of the online softmax for this thread's query row (thread = TMEM lane):
 // S (fp32, TMEM) -> P = exp2(S * scale * log2e - m) as bf16 into shared memory, running
 // max m and sum l.  A row keeps a stale max m while a tile's row sum against it stays at
-// most 2^RESCALE_LOG2 (every probability is then at most that), so the common case
+// most RESCALE_LIMIT (every probability is then at most that), so the common case
 // streams S through registers 32 columns at a time against the current max.  The first
 // tile, and a tile on which any lane of the warp exceeds that sum, take the exact
 // two-pass path: row max first, then P against the larger max (S is re-read from TMEM; P
@@ -701,9 +700,9 @@ __device__ __forceinline__ bool softmax_tile(uint32_t t_s, uint32_t p_row, int r
                 }
             }
         }
-        // a probability above 2^RESCALE_LOG2 (a row max that grew past the stale one by
-        // more than that) makes the tile's row sum exceed it too; a sum above it without
-        // such a probability only sends the row through the exact pass a little early
+        // a probability above RESCALE_LIMIT (a row max that grew past the stale one by
+        // more than 8 in log2 units) makes the tile's row sum exceed it too; a sum above it
+        // without such a probability only sends the row through the exact pass a little early
         const float lt = sum8(acc);
         if (!__any_sync(0xffffffffu, lt > RESCALE_LIMIT)) {
             l += lt;
