@@ -6,7 +6,8 @@
 // M = max(L1, L2):  L = M + ln(e^{L1-M} + e^{L2-M}),  O = e^{L1-L} O1 + e^{L2-L} O2.
 //
 // Memory-bound: each row reads 2 x (d bf16 + 1 fp32) and writes d bf16 + 1 fp32.
-// A group of d/8 threads owns a row, every thread moves 16 bytes of each O.
+// A group of d/8 threads owns a row, every thread moves 16 bytes of each O; each thread
+// takes RPT rows, all their loads issued before any arithmetic.
 #include <cstdint>
 
 #include "sfa.h"
@@ -32,43 +33,56 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(int64_t rows, const uint
                                                         const float *__restrict__ lse2, uint4 *o, float *lse)
 {
     constexpr int G = D / 8;  // threads per row
+    constexpr int RPT = 2;  // rows per thread (measured: 2 beat 1 and 4 on 2M rows)
     const int64_t gtid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int sub = threadIdx.x % G;
     const int64_t row_stride = (int64_t)gridDim.x * blockDim.x / G;
-    for (int64_t r = gtid / G; r < rows; r += row_stride) {
-        // the row's first lane reads both LSEs and hands them to its group, so an
-        // in-place lse write below cannot overtake another lane's read
-        const unsigned group = ((1u << G) - 1u) << ((threadIdx.x % 32) & ~(G - 1));
-        const uint4 a = o1[r * G + sub];  // issued first: independent of the LSEs
-        const uint4 b = o2[r * G + sub];
-        float l1 = 0.f, l2 = 0.f;
-        if (sub == 0) {
-            l1 = lse1[r];
-            l2 = lse2[r];
-        }
-        l1 = __shfl_sync(group, l1, 0, G);
-        l2 = __shfl_sync(group, l2, 0, G);
-        const float m = fmaxf(l1, l2);
-        float w1 = 0.f, w2 = 0.f, L = -INFINITY;
-        if (m != -INFINITY) {
-            const float e1 = l1 == -INFINITY ? 0.f : expf(l1 - m);
-            const float e2 = l2 == -INFINITY ? 0.f : expf(l2 - m);
-            const float s = e1 + e2;
-            L = m + logf(s);
-            w1 = e1 / s;
-            w2 = e2 / s;
-        }
-        const uint32_t av[4] = {a.x, a.y, a.z, a.w};
-        const uint32_t bv[4] = {b.x, b.y, b.z, b.w};
-        uint32_t ov[4];
+    const unsigned group = ((1u << G) - 1u) << ((threadIdx.x % 32) & ~(G - 1));
+    for (int64_t r0 = gtid / G; r0 < rows; r0 += row_stride * RPT) {
+        uint4 a[RPT], b[RPT];
+        float l1[RPT], l2[RPT];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float lo = w1 * bf16_lo(av[i]) + w2 * bf16_lo(bv[i]);
-            const float hi = w1 * bf16_hi(av[i]) + w2 * bf16_hi(bv[i]);
-            ov[i] = to_bf16x2(lo, hi);
+        for (int k = 0; k < RPT; ++k) {
+            const int64_t r = r0 + k * row_stride;
+            l1[k] = 0.f;
+            l2[k] = 0.f;
+            if (r < rows) {
+                a[k] = o1[r * G + sub];
+                b[k] = o2[r * G + sub];
+                if (sub == 0) {
+                    l1[k] = lse1[r];
+                    l2[k] = lse2[r];
+                }
+            }
         }
-        o[r * G + sub] = make_uint4(ov[0], ov[1], ov[2], ov[3]);
-        if (sub == 0) lse[r] = L;
+#pragma unroll
+        for (int k = 0; k < RPT; ++k) {
+            const int64_t r = r0 + k * row_stride;
+            if (r >= rows) break;
+            const float x1 = __shfl_sync(group, l1[k], 0, G);
+            const float x2 = __shfl_sync(group, l2[k], 0, G);
+            const float m = fmaxf(x1, x2);
+            float w1 = 0.f, w2 = 0.f, L = -INFINITY;
+            if (m != -INFINITY) {
+                const float e1 = x1 == -INFINITY ? 0.f : expf(x1 - m);
+                const float e2 = x2 == -INFINITY ? 0.f : expf(x2 - m);
+                const float sm = e1 + e2;
+                L = m + logf(sm);
+                w1 = e1 / sm;
+                w2 = e2 / sm;
+            }
+            const uint32_t av[4] = {a[k].x, a[k].y, a[k].z, a[k].w};
+            const uint32_t bv[4] = {b[k].x, b[k].y, b[k].z, b[k].w};
+            uint32_t ov[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float lo = w1 * bf16_lo(av[i]) + w2 * bf16_lo(bv[i]);
+                const float hi = w1 * bf16_hi(av[i]) + w2 * bf16_hi(bv[i]);
+                ov[i] = to_bf16x2(lo, hi);
+            }
+            o[r * G + sub] = make_uint4(ov[0], ov[1], ov[2], ov[3]);
+            if (sub == 0) lse[r] = L;
+        }
     }
 }
 
@@ -193,7 +207,7 @@ extern "C" sfa_status sfa_lse_merge(int64_t rows, int32_t d, const void *o1, con
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int threads = 256;
-    const int64_t need = (rows * (d / 8) + threads - 1) / threads;
+    const int64_t need = (rows * (d / 8) + threads * 2 - 1) / (threads * 2);  // two rows per thread
     const int64_t cap = (int64_t)sms * 8;  // 8 resident blocks of 256 threads per SM
     const int blocks = (int)(need < cap ? need : cap);
     cudaStream_t s = as_cuda(stream);
