@@ -127,8 +127,8 @@ def test_running_max_rescale_path(d, P):
     # Keys of frame f are scaled by 2^(f // 2) (exact in bf16), so a row's running max grows
     # by far more than 2^8 from tile to tile and O is rescaled in flight many times.  The
     # softmax ends up sharp, so the bound is the bf16-P one: |dO| <= 2^-7 max|v|.  P = 320
-    # gives every frame a CTA with one query tile, whose two warpgroups take alternate key
-    # tiles and rescale their own partial results.
+    # gives every frame a CTA with one query tile (S two key tiles ahead of its softmax),
+    # whose rescales first wait for the previous tile's P V.
     T, H = 8, 2
     w = Workload("rescale", B=1, H=H, Tq=T, Tkv=T, q_off=0, P=P, d=d, heads=(SetSpec("dense"),) * H)
     q, k, v = workload_qkv(w, seed=6)
@@ -138,6 +138,28 @@ def test_running_max_rescale_path(d, P):
     bound = 2.0 ** -7 * float(v.float().abs().max()) + 1e-5
     o_err, l_err = run_and_check(w, q, k, v, o_tol=bound)
     print(f"rescale path, d = {d}, P = {P}: O max-abs error {o_err:.2e} (bound {bound:.2e}), LSE {l_err:.2e}")
+
+
+@pytest.mark.parametrize("d,P", [(64, 192), (128, 192), (128, 320)])
+def test_moderate_max_growth_path(d, P):
+    # One query row repeated; every key of frame f is that row scaled so that it scores
+    # 1.5 f in log2 units after the softmax scale.  The first key tile of each new frame
+    # lifts the row max by 1.5, far below 2^8, but its row sum against the stale max
+    # (128 x 2^1.5) exceeds the limit of 256, so that tile takes the exact pass and adopts
+    # the larger max; the frame's second tile (64 keys at P = 192) stays on the streaming
+    # pass.  Bound as in the rescale test: bf16 P, |dO| <= 2^-7 max|v|.
+    T, H = 8, 2
+    w = Workload("growth", B=1, H=H, Tq=T, Tkv=T, q_off=0, P=P, d=d, heads=(SetSpec("dense"),) * H)
+    q, _, v = workload_qkv(w, seed=7)
+    q0 = q[:, :, :1, :].float()                              # [B, H, 1, d]
+    q = q0.expand(-1, -1, T * P, -1).to(torch.bfloat16).contiguous()
+    sl2 = (1.0 / math.sqrt(d)) / math.log(2.0)               # softmax scale in log2 units
+    beta = 1.5 * (torch.arange(T * P) // P).to(torch.float32) / sl2
+    k = (beta[None, None, :, None] * q0 / (q0 * q0).sum(-1, keepdim=True)).to(torch.bfloat16)
+    assert torch.isfinite(k.float()).all()
+    bound = 2.0 ** -7 * float(v.float().abs().max()) + 1e-5
+    o_err, l_err = run_and_check(w, q, k, v, o_tol=bound)
+    print(f"moderate growth, d = {d}, P = {P}: O max-abs error {o_err:.2e} (bound {bound:.2e}), LSE {l_err:.2e}")
 
 
 # ------------------------------------------------------------------ full-size workloads, sampled rows
