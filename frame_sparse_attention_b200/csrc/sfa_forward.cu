@@ -994,6 +994,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // each head's keys were then read twice from HBM, and the launch took 1.0 ms against 0.56.
 constexpr int SCHED_THREADS = 1024;
 constexpr int SCHED_BINS = 32;  // length classes: floor(log2(range))
+constexpr int SCHED_CACHE = 8192;  // entries whose class the first pass keeps for the second
 
 struct SchedArgs {
     const int32_t *frames[2];
@@ -1026,6 +1027,7 @@ __global__ void __launch_bounds__(SCHED_THREADS) schedule_kernel(const __grid_co
     __shared__ int bin_start[SCHED_BINS];     // first item of each class (descending class order)
     __shared__ int carry[SCHED_BINS];         // items of each class placed by earlier chunks
     __shared__ int wcount[NW][SCHED_BINS];    // items of each class per warp, this chunk
+    __shared__ uint8_t cls[SCHED_CACHE];      // class of the first SCHED_CACHE entries
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     // entries: frame lists per (h, t), or key-block lists per unit; units per entry
     const int per_set = s.nblk ? s.B * s.H * s.Tq * s.n_pairs : s.H * s.Tq;
@@ -1038,7 +1040,9 @@ __global__ void __launch_bounds__(SCHED_THREADS) schedule_kernel(const __grid_co
     __syncthreads();
     for (int e = tid; e < n_entries; e += SCHED_THREADS) {
         const int li = e / per_set, k = s.k[li];
-        atomicAdd(&bin_start[sched_bin((sched_len(s, li, e - li * per_set) + k - 1) / k)], fan * k);
+        const int bin = sched_bin((sched_len(s, li, e - li * per_set) + k - 1) / k);
+        if (e < SCHED_CACHE) cls[e] = (uint8_t)bin;
+        atomicAdd(&bin_start[bin], fan * k);
     }
     __syncthreads();
     if (tid == 0) {  // exclusive prefix in descending class order
@@ -1060,7 +1064,7 @@ __global__ void __launch_bounds__(SCHED_THREADS) schedule_kernel(const __grid_co
             li = e / per_set;
             le = e - li * per_set;
             k = s.k[li];
-            bin = sched_bin((sched_len(s, li, le) + k - 1) / k);
+            bin = e < SCHED_CACHE ? cls[e] : sched_bin((sched_len(s, li, le) + k - 1) / k);
         }
         for (int i = tid; i < NW * SCHED_BINS; i += SCHED_THREADS) (&wcount[0][0])[i] = 0;
         __syncthreads();
