@@ -17,7 +17,8 @@ data-path collective); timing is the max over ranks.
 
 --impl reference times the CPU oracle (float64, the repository's plain reference
 implementation of the same computation) on the host cores, on a bounded sample of
-query rows of the same workload per step; rank 0 alone runs it.
+query rows of the same workload per step, sized so that the warm-up and timed steps
+take about --reference-seconds (120 s by default) of oracle time; rank 0 alone runs it.
 """
 from __future__ import annotations
 
@@ -588,7 +589,7 @@ def run_reference(args, rank):
     t0 = time.perf_counter()
     oracle.attention(q, k, v, frames, counts, w.P, scale, rows=probe, n_threads=cores)
     per_row = (time.perf_counter() - t0) / probe.size
-    budget_s = 120.0 / max(1, args.steps + args.warmup)
+    budget_s = args.reference_seconds / max(1, args.steps + args.warmup)
     n_per_head = max(1, int(budget_s / per_row / w.H))
     step_times, step_flops = [], []
     for i in range(args.warmup + args.steps):
@@ -845,6 +846,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--reference-seconds", type=float, default=120.0,
+                    help="oracle time of the reference arm's warm-up and timed steps together")
     ap.add_argument("--heads", type=int, default=0,
                     help="run the workload with this many heads instead of 12 (smaller profiling case)")
     ap.add_argument("--no-workloads", action="store_true",
