@@ -359,7 +359,13 @@ __global__ void __launch_bounds__(GTHREADS, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int bh = blockIdx.x / a.G, g = blockIdx.x % a.G, b = bh / a.H, h = bh % a.H;
     const bool upd = a.update != 0;
-    const int per = (a.n_tiles - g + a.G - 1) / a.G;  // tiles of a frame this CTA takes: g, g + G, ...
+    // Tiles of frame n that this CTA takes: first(n), first(n) + G, ...  The assignment
+    // rotates by one CTA per frame, so that when the tiles of a frame do not divide evenly
+    // among the G CTAs the extra ones fall on a different CTA in every frame: each CTA then
+    // carries its share of them instead of CTA 0 carrying all of them in every frame (every
+    // CTA runs the whole recurrence, so the slowest one sets the call's time).
+    auto first_tile = [&](int n) { return (g - n % a.G + a.G) % a.G; };
+    auto tiles_in = [&](int n) { return (a.n_tiles - first_tile(n) + a.G - 1) / a.G; };
 
     if (threadIdx.x == 0) {
         const uint32_t single[10] = {q_full(0), q_full(1), q_full(2), q_full(3), m_full(0),
@@ -390,16 +396,27 @@ __global__ void __launch_bounds__(GTHREADS, 1)
         // ---------------------------------------------------------------- TMA + MMA
         const uint64_t ds = sdesc_sw128(sbase + MS_S, G_BOX, 1024);  // S: [d_k rows][d_v], MN-major B
         constexpr uint32_t id_qs = idesc_bf16_f32(GBM, GD, true);
-        const int total = per * a.T;
+        int total = 0;
+        for (int n = 0; n < a.T; ++n) total += tiles_in(n);
         int q_loaded = 0, q_landed = 0, m_loaded = 0, m_landed = 0;
         bool ok = true, issued = false;
-        auto tile_of = [&](int t, int &n, int &i) {
-            n = t / per;
-            i = g + (t % per) * a.G;
+        // the CTA's tiles in order (frame n, j-th tile of the frame), one cursor for the Q
+        // loads and one for the O stores, each visiting them once in that order
+        struct Cursor {
+            int n, j;
         };
-        auto load_q = [&](int t) {
+        Cursor lc = {0, 0}, sc = {0, 0};
+        auto next_tile = [&](Cursor &c, int &n, int &i) {
+            n = c.n;
+            i = first_tile(c.n) + c.j * a.G;
+            if (++c.j == tiles_in(c.n)) {
+                c.j = 0;
+                ++c.n;
+            }
+        };
+        auto load_q = [&](int t) {  // tile t of the CTA's sequence, the next one the cursor gives
             int n, i;
-            tile_of(t, n, i);
+            next_tile(lc, n, i);
             const int s = t % NQ;
             if (elect_one()) {
                 mbar_arrive_expect_tx(q_full(s), G_TILE);
@@ -423,9 +440,9 @@ __global__ void __launch_bounds__(GTHREADS, 1)
         };
         // O of tile t (staged by the epilogue in its Q buffer) -> global; lane 0 owns the
         // bulk groups
-        auto store_o = [&](int t) {
+        auto store_o = [&](int t) {  // tile t of the CTA's sequence, the next one the cursor gives
             int n, i;
-            tile_of(t, n, i);
+            next_tile(sc, n, i);
             const uint32_t src = sbase + MS_Q + (t % NQ) * G_TILE;
             if (lane == 0) {
 #pragma unroll
@@ -462,6 +479,7 @@ __global__ void __launch_bounds__(GTHREADS, 1)
                 // before the state was ready
                 if (n >= 1 && n + 1 < a.T) load_m(n + 1);
             }
+            const int per = tiles_in(n);
             for (int ii = 0; ii < per && ok; ++ii, ++it) {
                 const int s = it % NQ, u = it & 1;
                 if (!(ok = __all_sync(0xffffffffu, gwait(q_full(s), (it / NQ) & 1, abort, a.status, a.timeout_ns))))
@@ -581,6 +599,7 @@ __global__ void __launch_bounds__(GTHREADS, 1)
             // the frame's O products past its second wait for the TMEM buffers of its first
             // ones, and the frame's MMAs end before the state is rewritten: those first ones
             // are staged before the state
+            const int per = tiles_in(n);
             const int early = upd ? (per > 2 ? per - 2 : 0) : per;
             uint32_t pk[32];  // bf16 pairs of the new state row (this half)
             if (upd) {

@@ -85,12 +85,16 @@ def _run(rng, engine, finite):
 
 
 def model_main(per, T, upd, rng, drop=frozenset(), NQ=4):
-    """gdn_kernel, one CTA (its CTAs never wait for one another): `per` tiles of T frames."""
+    """gdn_kernel, one CTA (its CTAs never wait for one another): T frames of `per` tiles each,
+    or per[n] tiles in frame n (the kernel rotates the tiles of a frame over the CTAs, so a
+    CTA's count changes from frame to frame when they do not divide evenly)."""
+    pers = [per] * T if isinstance(per, int) else list(per)
+    assert len(pers) == T
     done = {k: 0 for k in ("q0", "q1", "q2", "q3", "m0", "m1", "d_done", "s_free", "o_done0", "o_done1",
                            "o_free0", "o_free1", "s_ready")}
     eng = _Engines(rng, done)
     st = {"s_frame": 0, "d_read": -1, "staged": set(), "stored": set()}
-    total = per * T
+    total = sum(pers)
 
     def wait(bar, k, name):
         return _wait(done, bar, k, name, drop)
@@ -137,7 +141,7 @@ def model_main(per, T, upd, rng, drop=frozenset(), NQ=4):
                 _check(eng.landed.get(f"m{n & 1}") == n, f"product of frame {n} issued before M landed")
                 _check(st["d_read"] >= n - 1, "M S overwrites an unread product")
                 issue("d", n, n, "d_done")
-            for _ in range(per):
+            for _ in range(pers[n]):
                 s, u = it % NQ, it & 1
                 yield from wait(f"q{s}", it // NQ, "q_full")
                 _check(eng.landed.get(f"q{s}") == it, f"O MMA of tile {it} before its Q landed")
@@ -174,7 +178,7 @@ def model_main(per, T, upd, rng, drop=frozenset(), NQ=4):
         for n in range(T):
             # the frame's O products past its second wait for the first ones' TMEM buffers,
             # and the frame's MMAs end before the state is rewritten: stage those first
-            early = max(per - 2, 0) if upd else per
+            early = max(pers[n] - 2, 0) if upd else pers[n]
             if upd:
                 yield from wait("d_done", n, "d_done")
                 _check(("d", n) in eng.completed, f"product of frame {n} read before it was done")
@@ -186,7 +190,7 @@ def model_main(per, T, upd, rng, drop=frozenset(), NQ=4):
                 _check(not any(x[0] in ("d", "qs") for x in eng.tc), f"state of frame {n} rewritten while read")
                 st["s_frame"] = n + 1
                 done["s_ready"] += 1
-            for _ in range(per - early):
+            for _ in range(pers[n] - early):
                 yield from stage_o()
 
     _run(rng, eng.actor(), [mma_warp(), epilogue()])
@@ -233,7 +237,12 @@ def model_prep(nt, rng, drop=frozenset(), S=3):
     _run(rng, eng.actor(), [mma_warp(), epilogue()])
 
 
-MAIN_CASES = [(per, T, upd) for per in (1, 2, 3, 5) for T in (1, 2, 3, 5) for upd in (True, False)]
+# per-frame tile counts that change from frame to frame, as the rotating assignment gives
+# them (13 tiles over 12 CTAs: a CTA takes two tiles in one frame of every 12; 8 tiles over
+# 3 CTAs: 3, 3, 2, 3, 3, 2, ...), in denser patterns than those
+ROTATED = [[1, 2, 1, 1, 2], [2, 1, 1, 2, 1], [3, 2, 2, 3, 2], [1, 1, 2, 1, 1, 1]]
+MAIN_CASES = ([(per, T, upd) for per in (1, 2, 3, 5) for T in (1, 2, 3, 5) for upd in (True, False)] +
+              [(pers, len(pers), upd) for pers in ROTATED for upd in (True, False)])
 PREP_CASES = [(nt,) for nt in (1, 2, 3, 4, 7, 13)]
 
 
@@ -265,7 +274,8 @@ def _caught(fn, cases, dropped):
 @pytest.mark.parametrize("dropped", ["s_ready", "m_full", "q_full", "o_free", "store_read", "d_done", "s_free",
                                      "o_done"])
 def test_model_catches_a_missing_wait_in_the_main_kernel(dropped):
-    assert _caught(model_main, [(2, 4, True), (1, 3, True), (3, 3, False)], dropped), dropped
+    assert _caught(model_main, [(2, 4, True), (1, 3, True), (3, 3, False), ([1, 2, 1, 2], 4, True)],
+                   dropped), dropped
 
 
 @pytest.mark.parametrize("dropped", ["scaled", "mma_done", "kv_full", "fin"])
