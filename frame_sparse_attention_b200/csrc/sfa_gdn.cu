@@ -15,12 +15,15 @@
 //     formed in shared memory, then M_N = K~^T K~ and B_N = K~^T V~);
 //   gdn_kernel: G CTAs per (batch, head) each run the recurrence over the frames (one
 //     128 x 128 x 128 product M_N S_{N-1} per frame, the rest in fp32), and each computes
-//     O = Q S_{N-1} for its own token tiles of every frame (CTA g: tiles g, g + G, ...).
-//     The G CTAs of a head repeat the same small recurrence and never wait for one another.
+//     O = Q S_{N-1} for its own token tiles of every frame (in frame n, CTA g takes the
+//     tiles i with (i + n) mod G = g).  The G CTAs of a head repeat the same small
+//     recurrence and never wait for one another.
 // Read-only steps (update = 0) run only the O contraction with the input state.
 // In both kernels warps 0-7 (two threads per TMEM lane, 64 columns each) do the
-// element-wise work and warp 8 issues the TMA copies and the MMAs.  Every wait is bounded;
-// a wait that runs out stores SFA_ERR_TIMEOUT and the CTA drains and exits.
+// element-wise work.  In gdn_prep_kernel warp 8 issues the TMA copies and the MMAs; in
+// gdn_kernel warp 8 issues the MMAs and warp 9 the TMA copies, so that no copy waits in
+// the issue stream of the frame's recurrence.  Every wait is bounded; a wait that runs
+// out stores SFA_ERR_TIMEOUT and the CTA drains and exits.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -40,8 +43,10 @@ namespace {
 constexpr int GD = 128;          // d_k = d_v
 constexpr int GBM = 128;         // tokens per tile
 constexpr int GEPI = 256;        // warps 0-7: element-wise work (two threads per TMEM lane)
-constexpr int GW_MMA = 8;        // warp 8: TMA copies and MMAs
-constexpr int GTHREADS = GEPI + 32;
+constexpr int GW_MMA = 8;        // warp 8: TMA copies and MMAs (gdn_prep_kernel), MMAs (gdn_kernel)
+constexpr int GW_TMA = 9;        // warp 9 of gdn_kernel: its TMA copies
+constexpr int GTHREADS = GEPI + 32;       // gdn_prep_kernel
+constexpr int GTHREADS_REC = GEPI + 64;   // gdn_kernel
 constexpr int G_BOX = 128 * 128; // one 128-row x 64-column bf16 box (128-byte swizzle)
 constexpr int G_TILE = 2 * G_BOX;
 
@@ -337,9 +342,10 @@ __global__ void __launch_bounds__(GTHREADS, 2)
 // frame by frame (M_N S as one 128 x 128 x 128 MMA), and the O MMAs of its tiles of frame N
 // read the same bf16(S_{N-1}) in shared memory; the state buffer is rewritten once they are
 // done.  Tiles of consecutive frames stream through a ring of NQ Q buffers; O is read out
-// of one of two TMEM buffers, staged in the tile's Q buffer and written by a TMA store.
+// of one of two TMEM buffers, staged in the tile's Q buffer and written by a TMA store
+// that warp 9 issues, which then refills the buffer with the tile NQ places further on.
 // ------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(GTHREADS, 1)
+__global__ void __launch_bounds__(GTHREADS_REC, 1)
     gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o,
                const __grid_constant__ CUtensorMap tm_mw, const __grid_constant__ GdnArgs a)
 {
@@ -351,11 +357,17 @@ __global__ void __launch_bounds__(GTHREADS, 1)
     const uint32_t d_done = bb + 48;                         // M_N S in TMEM
     const uint32_t s_free = bb + 56;                         // the frame's MMAs no longer read S
     auto o_done = [&](int u) { return bb + 64 + 8 * u; };    // O of a tile in TMEM buffer u
-    auto o_free = [&](int u) { return bb + 80 + 8 * u; };    // O buffer u read out and staged (all)
+    // O of the tile in Q buffer s read out of TMEM and staged in that buffer (all).  One
+    // barrier per Q buffer rather than per TMEM buffer: the TMA warp waits for the tiles in
+    // order to send them, and the next completion of a Q buffer's barrier needs the copy the
+    // TMA warp makes only after that wait (no phase can be skipped unseen)
+    auto o_staged = [&](int s) { return bb + 112 + 8 * s; };
+    auto m_free = [&](int s) { return bb + 144 + 8 * s; };  // the product reading M slot s is done
     const uint32_t s_ready = bb + 96;                        // state of the next frame written (all)
     const uint32_t drain = bb + 104;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + MS_BAR + 128);
-    volatile int32_t *abort = reinterpret_cast<volatile int32_t *>(smem + MS_BAR + 132);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + MS_BAR + 160);
+    volatile int32_t *abort = reinterpret_cast<volatile int32_t *>(smem + MS_BAR + 164);
+    int32_t *landed = reinterpret_cast<int32_t *>(smem + MS_BAR + 168);  // Q tiles, M frames the MMA warp saw land
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int bh = blockIdx.x / a.G, g = blockIdx.x % a.G, b = bh / a.H, h = bh % a.H;
     const bool upd = a.update != 0;
@@ -372,8 +384,9 @@ __global__ void __launch_bounds__(GTHREADS, 1)
                                      m_full(1), d_done,    s_free,    o_done(0), o_done(1)};
         for (uint32_t x : single) mbar_init(x, 1);
         mbar_init(drain, 1);
-        mbar_init(o_free(0), GEPI);
-        mbar_init(o_free(1), GEPI);
+        for (int x = 0; x < NQ; ++x) mbar_init(o_staged(x), GEPI);
+        mbar_init(m_free(0), 1);
+        mbar_init(m_free(1), 1);
         mbar_init(s_ready, GEPI);
         *abort = 0;
         fence_mbar_init();
@@ -391,15 +404,78 @@ __global__ void __launch_bounds__(GTHREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    int q_loaded = 0, m_loaded = 0;  // copies the TMA warp issued
 
     if (warp == GW_MMA) {
-        // ---------------------------------------------------------------- TMA + MMA
+        // ---------------------------------------------------------------- MMA
         const uint64_t ds = sdesc_sw128(sbase + MS_S, G_BOX, 1024);  // S: [d_k rows][d_v], MN-major B
         constexpr uint32_t id_qs = idesc_bf16_f32(GBM, GD, true);
+        int q_landed = 0, m_landed = 0;
+        bool ok = true, issued = false;
+        int it = 0;
+        for (int n = 0; n < a.T && ok; ++n) {
+            if ((upd || n == 0) &&
+                !(ok = __all_sync(0xffffffffu, gwait(s_ready, n & 1, abort, a.status, a.timeout_ns))))
+                break;
+            if (upd) {
+                if (!(ok = __all_sync(0xffffffffu, gwait(m_full(n & 1), (n >> 1) & 1, abort, a.status, a.timeout_ns))))
+                    break;
+                m_landed = n + 1;
+                tc_fence_after();
+                const uint64_t dm = sdesc_sw128(sbase + MS_M + (n & 1) * G_TILE, 16, 1024);  // M_N, K-major A
+                if (elect_one()) {
+#pragma unroll
+                    for (uint32_t kk = 0; kk < GD / 16; ++kk) {
+                        const uint32_t ka = (kk >> 2) * G_BOX + (kk & 3) * 32;
+                        mma_ss(tmem + T_D, dm + (ka >> 4), ds + ((kk * 2048) >> 4), id_qs, kk > 0);
+                    }
+                    tc_commit(d_done);
+                    tc_commit(m_free(n & 1));
+                }
+                __syncwarp();
+                issued = true;
+            }
+            const int per = tiles_in(n);
+            for (int ii = 0; ii < per && ok; ++ii, ++it) {
+                const int s = it % NQ, u = it & 1;
+                if (!(ok = __all_sync(0xffffffffu, gwait(q_full(s), (it / NQ) & 1, abort, a.status, a.timeout_ns))))
+                    break;
+                q_landed = it + 1;
+                // TMEM buffer u last held tile it - 2: read out and staged
+                if (it >= 2 && !(ok = __all_sync(0xffffffffu, gwait(o_staged((it - 2) % NQ), ((it - 2) / NQ) & 1, abort,
+                                                                      a.status, a.timeout_ns))))
+                    break;
+                tc_fence_after();
+                const uint64_t dq = sdesc_sw128(sbase + MS_Q + s * G_TILE, 16, 1024);  // Q tile, K-major A
+                if (elect_one()) {
+#pragma unroll
+                    for (uint32_t kk = 0; kk < GD / 16; ++kk) {
+                        const uint32_t ka = (kk >> 2) * G_BOX + (kk & 3) * 32;
+                        mma_ss(tmem + T_O0 + u * 128, dq + (ka >> 4), ds + ((kk * 2048) >> 4), id_qs, kk > 0);
+                    }
+                    tc_commit(o_done(u));
+                    // after the frame's last MMA that reads S: the state may be rewritten
+                    if (ii == per - 1) tc_commit(s_free);
+                }
+                __syncwarp();
+                issued = true;
+            }
+        }
+        if (__any_sync(0xffffffffu, *abort != 0) && issued) {  // tensor cores idle before TMEM is freed
+            if (elect_one()) tc_commit(drain);
+            __syncwarp();
+            gdrain(drain, 0);
+        }
+        if (lane == 0) {
+            landed[0] = q_landed;
+            landed[1] = m_landed;
+        }
+        __syncwarp();
+    } else if (warp == GW_TMA) {
+        // ---------------------------------------------------------------- TMA: Q, M_N in, O out
         int total = 0;
         for (int n = 0; n < a.T; ++n) total += tiles_in(n);
-        int q_loaded = 0, q_landed = 0, m_loaded = 0, m_landed = 0;
-        bool ok = true, issued = false;
+        bool ok = true;
         // the CTA's tiles in order (frame n, j-th tile of the frame), one cursor for the Q
         // loads and one for the O stores, each visiting them once in that order
         struct Cursor {
@@ -425,7 +501,6 @@ __global__ void __launch_bounds__(GTHREADS, 1)
                     tma_load_5d(sbase + MS_Q + s * G_TILE + kb * G_BOX, &tm_q, q_full(s), kb * 64, i * GBM, n, h, b);
             }
             __syncwarp();
-            q_loaded = t + 1;
         };
         auto load_m = [&](int n) {
             const int s = n & 1, y = (bh * a.T + n) * GD;
@@ -436,11 +511,10 @@ __global__ void __launch_bounds__(GTHREADS, 1)
                     tma_load_2d(sbase + MS_M + s * G_TILE + kb * G_BOX, &tm_mw, m_full(s), kb * 64, y);
             }
             __syncwarp();
-            m_loaded = n + 1;
         };
         // O of tile t (staged by the epilogue in its Q buffer) -> global; lane 0 owns the
         // bulk groups
-        auto store_o = [&](int t) {  // tile t of the CTA's sequence, the next one the cursor gives
+        auto store_o = [&](int t) {
             int n, i;
             next_tile(sc, n, i);
             const uint32_t src = sbase + MS_Q + (t % NQ) * G_TILE;
@@ -451,86 +525,40 @@ __global__ void __launch_bounds__(GTHREADS, 1)
             }
             __syncwarp();
         };
-        for (int t = 0; t < 2 && t < total; ++t) load_q(t);
+        for (; q_loaded < NQ && q_loaded < total; ++q_loaded) load_q(q_loaded);
         if (upd)
-            for (int n = 0; n < 2 && n < a.T; ++n) load_m(n);
-        int it = 0;
+            for (; m_loaded < 2 && m_loaded < a.T; ++m_loaded) load_m(m_loaded);
+        int t = 0;
         for (int n = 0; n < a.T && ok; ++n) {
-            if ((upd || n == 0) &&
-                !(ok = __all_sync(0xffffffffu, gwait(s_ready, n & 1, abort, a.status, a.timeout_ns))))
-                break;
-            if (upd) {
-                if (!(ok = __all_sync(0xffffffffu, gwait(m_full(n & 1), (n >> 1) & 1, abort, a.status, a.timeout_ns))))
+            if (upd && n + 2 < a.T) {  // M_{n+2} takes the slot of M_n once the product of frame n is done
+                if (!(ok = __all_sync(0xffffffffu, gwait(m_free(n & 1), (n >> 1) & 1, abort, a.status, a.timeout_ns))))
                     break;
-                m_landed = n + 1;
-                tc_fence_after();
-                const uint64_t dm = sdesc_sw128(sbase + MS_M + (n & 1) * G_TILE, 16, 1024);  // M_N, K-major A
-                if (elect_one()) {
-#pragma unroll
-                    for (uint32_t kk = 0; kk < GD / 16; ++kk) {
-                        const uint32_t ka = (kk >> 2) * G_BOX + (kk & 3) * 32;
-                        mma_ss(tmem + T_D, dm + (ka >> 4), ds + ((kk * 2048) >> 4), id_qs, kk > 0);
-                    }
-                    tc_commit(d_done);
-                }
-                __syncwarp();
-                issued = true;
-                // M_{n+1} takes the slot of M_{n-1}: the product of frame n - 1 was read out
-                // before the state was ready
-                if (n >= 1 && n + 1 < a.T) load_m(n + 1);
+                load_m(n + 2);
+                m_loaded = n + 3;
             }
             const int per = tiles_in(n);
-            for (int ii = 0; ii < per && ok; ++ii, ++it) {
-                const int s = it % NQ, u = it & 1;
-                if (!(ok = __all_sync(0xffffffffu, gwait(q_full(s), (it / NQ) & 1, abort, a.status, a.timeout_ns))))
+            // the O stores of frame n wait for the product of frame n + 1 to be done, so that
+            // their shared-memory reads do not slow it down (it sets the pace of the frames);
+            // not when a Q buffer must be refilled within the frame (the frame's products
+            // would wait for a store that waits for the next frame)
+            if (upd && n + 1 < a.T && per <= NQ &&
+                !(ok = __all_sync(0xffffffffu, gwait(m_free((n + 1) & 1), ((n + 1) >> 1) & 1, abort, a.status,
+                                                     a.timeout_ns))))
+                break;
+            for (int ii = 0; ii < per && ok; ++ii, ++t) {
+                // tile t's O staged in its Q buffer: send it; the buffer then takes tile t + NQ
+                if (!(ok = __all_sync(0xffffffffu, gwait(o_staged(t % NQ), (t / NQ) & 1, abort, a.status, a.timeout_ns))))
                     break;
-                q_landed = it + 1;
-                if (it >= 2) {  // TMEM buffer u last held tile it - 2: read out, staged, sent
-                    if (!(ok = __all_sync(0xffffffffu,
-                                          gwait(o_free(u), ((it - 2) >> 1) & 1, abort, a.status, a.timeout_ns))))
-                        break;
-                    store_o(it - 2);
-                }
-                tc_fence_after();
-                const uint64_t dq = sdesc_sw128(sbase + MS_Q + s * G_TILE, 16, 1024);  // Q tile, K-major A
-                if (elect_one()) {
-#pragma unroll
-                    for (uint32_t kk = 0; kk < GD / 16; ++kk) {
-                        const uint32_t ka = (kk >> 2) * G_BOX + (kk & 3) * 32;
-                        mma_ss(tmem + T_O0 + u * 128, dq + (ka >> 4), ds + ((kk * 2048) >> 4), id_qs, kk > 0);
-                    }
-                    tc_commit(o_done(u));
-                    // after the frame's last MMA that reads S: the state may be rewritten
-                    // while this warp waits for the O store below
-                    if (ii == per - 1) tc_commit(s_free);
-                }
-                __syncwarp();
-                issued = true;
-                if (it + 2 < total) {  // tile it + 2 takes the Q buffer of tile it - 2 once its O is out
-                    if (it >= 2 && lane == 0) tma_store_wait_read_all();
+                store_o(t);
+                if (t + NQ < total) {
+                    if (lane == 0) tma_store_wait_read_all();
                     __syncwarp();
-                    load_q(it + 2);
+                    load_q(t + NQ);
+                    q_loaded = t + NQ + 1;
                 }
             }
-            if (!ok) break;
-        }
-        for (int t = total >= 2 ? total - 2 : 0; t < total && ok; ++t) {  // the last two tiles' O
-            if (!(ok = __all_sync(0xffffffffu, gwait(o_free(t & 1), (t >> 1) & 1, abort, a.status, a.timeout_ns))))
-                break;
-            store_o(t);
         }
         if (lane == 0) bulk_commit_and_wait_all();  // every O store complete
-        __syncwarp();
-        if (__any_sync(0xffffffffu, *abort != 0)) {
-            if (issued) {  // tensor cores idle before TMEM is freed
-                if (elect_one()) tc_commit(drain);
-                __syncwarp();
-                gdrain(drain, 0);
-            }
-            // copies still in flight land before the CTA exits
-            for (int t = q_landed; t < q_loaded; ++t) gdrain(q_full(t % NQ), (t / NQ) & 1);
-            for (int t = m_landed; t < m_loaded; ++t) gdrain(m_full(t & 1), (t >> 1) & 1);
-        }
         __syncwarp();
     } else {
         // ---------------------------------------------------------------- row r, half hc
@@ -567,7 +595,7 @@ __global__ void __launch_bounds__(GTHREADS, 1)
         mbar_arrive(s_ready);
         bool ok = true;
         int it = 0;
-        // O of tile it -> bf16 into its Q buffer, for the MMA warp's store
+        // O of tile it -> bf16 into its Q buffer, for the TMA warp's store
         auto stage_o = [&]() -> bool {
             const int u = it & 1;
             if (!__all_sync(0xffffffffu, gwait(o_done(u), (it >> 1) & 1, abort, a.status, a.timeout_ns)))
@@ -591,7 +619,7 @@ __global__ void __launch_bounds__(GTHREADS, 1)
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(o_free(u));
+            mbar_arrive(o_staged(it % NQ));
             ++it;
             return true;
         };
@@ -675,6 +703,11 @@ __global__ void __launch_bounds__(GTHREADS, 1)
     if (warp == GW_MMA) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
+    } else if (warp == GW_TMA && *abort) {
+        // copies still in flight (issued, never seen landing by the MMA warp) land before
+        // the CTA exits
+        for (int x = landed[0]; x < q_loaded; ++x) gdrain(q_full(x % NQ), (x / NQ) & 1);
+        for (int x = landed[1]; x < m_loaded; ++x) gdrain(m_full(x & 1), (x >> 1) & 1);
     }
 }
 
@@ -817,6 +850,6 @@ extern "C" sfa_status sfa_gdn_forward(const sfa_gdn_desc *d, const void *q, cons
     }
     if (cudaFuncSetAttribute(gdn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, MS_SMEM) != cudaSuccess)
         return SFA_ERR_CUDA;
-    gdn_kernel<<<(unsigned)(d->B * d->H * a.G), GTHREADS, MS_SMEM, s>>>(tq, to, tm, a);
+    gdn_kernel<<<(unsigned)(d->B * d->H * a.G), GTHREADS_REC, MS_SMEM, s>>>(tq, to, tm, a);
     return launch_status();
 }

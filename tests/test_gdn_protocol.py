@@ -1,8 +1,8 @@
 """A model of the synchronisation of the gated-delta kernels (csrc/sfa_gdn.cu), run on the CPU.
 
 Each kernel's warps coordinate through mbarriers and the completion order of the tensor
-core and the TMA engine.  This model replays the waits the MMA warp and the element-wise
-warps perform, in the same order, with the asynchronous engines (MMAs completing in issue
+core and the TMA engine.  This model replays the waits the MMA warp, the TMA warp (the
+recurrence kernel's copies) and the element-wise warps perform, in the same order, with the asynchronous engines (MMAs completing in issue
 order, copies landing and stores reading shared memory at random later times), all
 interleaved at random.  It checks, at the moment a buffer or TMEM column is overwritten,
 that every reader of the old contents has finished; that no mbarrier wait can alias a
@@ -91,7 +91,9 @@ def model_main(per, T, upd, rng, drop=frozenset(), NQ=4):
     pers = [per] * T if isinstance(per, int) else list(per)
     assert len(pers) == T
     done = {k: 0 for k in ("q0", "q1", "q2", "q3", "m0", "m1", "d_done", "s_free", "o_done0", "o_done1",
-                           "o_free0", "o_free1", "s_ready")}
+                           "s_ready")}
+    done.update({f"o_staged{x}": 0 for x in range(NQ)})
+    done.update({"m_free0": 0, "m_free1": 0})
     eng = _Engines(rng, done)
     st = {"s_frame": 0, "d_read": -1, "staged": set(), "stored": set()}
     total = sum(pers)
@@ -100,6 +102,32 @@ def model_main(per, T, upd, rng, drop=frozenset(), NQ=4):
         return _wait(done, bar, k, name, drop)
 
     def mma_warp():
+        def issue(kind, idx, n, bar):
+            _check(not upd or st["s_frame"] == n, f"MMA of frame {n} reads the state of frame {st['s_frame']}")
+            eng.mma(kind, idx, bar)
+
+        it = 0
+        for n in range(T):
+            if upd or n == 0:
+                yield from wait("s_ready", n, "s_ready")
+            if upd:
+                yield from wait(f"m{n & 1}", n >> 1, "m_full")
+                _check(eng.landed.get(f"m{n & 1}") == n, f"product of frame {n} issued before M landed")
+                _check(st["d_read"] >= n - 1, "M S overwrites an unread product")
+                issue("d", n, n, "d_done")
+                eng.mma("m_free", n, f"m_free{n & 1}")
+            for _ in range(pers[n]):
+                s, u = it % NQ, it & 1
+                yield from wait(f"q{s}", it // NQ, "q_full")
+                _check(eng.landed.get(f"q{s}") == it, f"O MMA of tile {it} before its Q landed")
+                if it >= 2:
+                    yield from wait(f"o_staged{(it - 2) % NQ}", (it - 2) // NQ, "o_free")
+                _check(it < 2 or (it - 2) in st["staged"], f"O of tile {it} overwrites an unread O")
+                issue("qs", it, n, f"o_done{u}")
+                it += 1
+            eng.mma("s_free", n, "s_free")
+
+    def tma_warp():
         last_store = [-1]
 
         def load_q(t):
@@ -121,45 +149,29 @@ def model_main(per, T, upd, rng, drop=frozenset(), NQ=4):
             eng.stores.append(t)
             last_store[0] = t
 
-        def issue(kind, idx, n, bar):
-            _check(not upd or st["s_frame"] == n, f"MMA of frame {n} reads the state of frame {st['s_frame']}")
-            eng.mma(kind, idx, bar)
-
-        for t in range(min(2, total)):
+        for t in range(min(NQ, total)):
             load_q(t)
         if upd:
             for n in range(min(2, T)):
                 load_m(n)
-        it = 0
+        t = 0
         for n in range(T):
-            if upd or n == 0:
-                yield from wait("s_ready", n, "s_ready")
-            if upd:
-                if 1 <= n and n + 1 < T:
-                    load_m(n + 1)
-                yield from wait(f"m{n & 1}", n >> 1, "m_full")
-                _check(eng.landed.get(f"m{n & 1}") == n, f"product of frame {n} issued before M landed")
-                _check(st["d_read"] >= n - 1, "M S overwrites an unread product")
-                issue("d", n, n, "d_done")
+            if upd and n + 2 < T:
+                yield from wait(f"m_free{n & 1}", n >> 1, "m_slot")
+                load_m(n + 2)
+            # the frame's stores wait for the next frame's product (not when a Q buffer is
+            # refilled within the frame)
+            if upd and n + 1 < T and pers[n] <= NQ:
+                yield from wait(f"m_free{(n + 1) & 1}", (n + 1) >> 1, "store_after_product")
             for _ in range(pers[n]):
-                s, u = it % NQ, it & 1
-                yield from wait(f"q{s}", it // NQ, "q_full")
-                _check(eng.landed.get(f"q{s}") == it, f"O MMA of tile {it} before its Q landed")
-                if it >= 2:
-                    yield from wait(f"o_free{u}", (it - 2) >> 1, "o_free")
-                    store(it - 2)
-                _check(it < 2 or (it - 2) in st["staged"], f"O of tile {it} overwrites an unread O")
-                issue("qs", it, n, f"o_done{u}")
-                if it + 2 < total:
-                    if it >= 2 and "store_read" not in drop:
+                yield from wait(f"o_staged{t % NQ}", t // NQ, "o_staged")
+                store(t)
+                if t + NQ < total:
+                    if "store_read" not in drop:
                         while eng.store_read < last_store[0]:
                             yield
-                    load_q(it + 2)
-                it += 1
-            eng.mma("s_free", n, "s_free")
-        for t in range(max(0, total - 2), total):
-            yield from wait(f"o_free{t & 1}", t >> 1, "o_free")
-            store(t)
+                    load_q(t + NQ)
+                t += 1
 
     def epilogue():
         done["s_ready"] += 1
@@ -172,7 +184,7 @@ def model_main(per, T, upd, rng, drop=frozenset(), NQ=4):
             _check(("qs", t) in eng.completed and eng.landed.get(f"q{t % NQ}") == t,
                    f"O of tile {t} staged too early or over a reloaded Q buffer")
             st["staged"].add(t)
-            done[f"o_free{u}"] += 1
+            done[f"o_staged{t % NQ}"] += 1
             it[0] += 1
 
         for n in range(T):
@@ -193,7 +205,7 @@ def model_main(per, T, upd, rng, drop=frozenset(), NQ=4):
             for _ in range(pers[n] - early):
                 yield from stage_o()
 
-    _run(rng, eng.actor(), [mma_warp(), epilogue()])
+    _run(rng, eng.actor(), [mma_warp(), tma_warp(), epilogue()])
 
 
 def model_prep(nt, rng, drop=frozenset(), S=3):
@@ -240,7 +252,7 @@ def model_prep(nt, rng, drop=frozenset(), S=3):
 # per-frame tile counts that change from frame to frame, as the rotating assignment gives
 # them (13 tiles over 12 CTAs: a CTA takes two tiles in one frame of every 12; 8 tiles over
 # 3 CTAs: 3, 3, 2, 3, 3, 2, ...), in denser patterns than those
-ROTATED = [[1, 2, 1, 1, 2], [2, 1, 1, 2, 1], [3, 2, 2, 3, 2], [1, 1, 2, 1, 1, 1]]
+ROTATED = [[1, 2, 1, 1, 2], [2, 1, 1, 2, 1], [3, 2, 2, 3, 2], [1, 1, 2, 1, 1, 1], [1, 1, 1, 1, 1, 1, 1, 2, 1]]
 MAIN_CASES = ([(per, T, upd) for per in (1, 2, 3, 5) for T in (1, 2, 3, 5) for upd in (True, False)] +
               [(pers, len(pers), upd) for pers in ROTATED for upd in (True, False)])
 PREP_CASES = [(nt,) for nt in (1, 2, 3, 4, 7, 13)]
@@ -271,8 +283,8 @@ def _caught(fn, cases, dropped):
     return False
 
 
-@pytest.mark.parametrize("dropped", ["s_ready", "m_full", "q_full", "o_free", "store_read", "d_done", "s_free",
-                                     "o_done"])
+@pytest.mark.parametrize("dropped", ["s_ready", "m_full", "q_full", "o_free", "o_staged", "m_slot", "store_read",
+                                     "d_done", "s_free", "o_done"])
 def test_model_catches_a_missing_wait_in_the_main_kernel(dropped):
     assert _caught(model_main, [(2, 4, True), (1, 3, True), (3, 3, False), ([1, 2, 1, 2], 4, True)],
                    dropped), dropped
