@@ -197,6 +197,9 @@ __global__ void __launch_bounds__(GTHREADS, 2)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // the recurrence kernel may take the SMs this grid leaves free and set itself up; it
+    // waits for this grid's results before it reads them
+    pdl_launch_dependents();
 
     if (warp == GW_MMA) {
         constexpr uint32_t id_mm = idesc_bf16_f32(GD, GD, true) | (1u << 15);  // A and B MN-major
@@ -526,6 +529,7 @@ __global__ void __launch_bounds__(GTHREADS_REC, 1)
             __syncwarp();
         };
         for (; q_loaded < NQ && q_loaded < total; ++q_loaded) load_q(q_loaded);
+        pdl_wait();  // M_N comes from the preparation kernel
         if (upd)
             for (; m_loaded < 2 && m_loaded < a.T; ++m_loaded) load_m(m_loaded);
         int t = 0;
@@ -593,6 +597,7 @@ __global__ void __launch_bounds__(GTHREADS_REC, 1)
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(s_ready);
+        pdl_wait();  // B_N comes from the preparation kernel
         bool ok = true;
         int it = 0;
         // O of tile it -> bf16 into its Q buffer, for the TMA warp's store
@@ -850,6 +855,19 @@ extern "C" sfa_status sfa_gdn_forward(const sfa_gdn_desc *d, const void *q, cons
     }
     if (cudaFuncSetAttribute(gdn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, MS_SMEM) != cudaSuccess)
         return SFA_ERR_CUDA;
-    gdn_kernel<<<(unsigned)(d->B * d->H * a.G), GTHREADS_REC, MS_SMEM, s>>>(tq, to, tm, a);
+    // after the preparation kernel: a programmatic dependent launch, so that the recurrence
+    // kernel's set-up (barriers, tensor memory, its first Q tiles, the input state) overlaps
+    // the preparation's last CTAs
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(d->B * d->H * a.G));
+    cfg.blockDim = dim3(GTHREADS_REC);
+    cfg.dynamicSmemBytes = MS_SMEM;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = update ? 1 : 0;
+    if (cudaLaunchKernelEx(&cfg, gdn_kernel, tq, to, tm, a) != cudaSuccess) return SFA_ERR_CUDA;
     return launch_status();
 }

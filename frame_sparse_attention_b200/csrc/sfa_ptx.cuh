@@ -23,6 +23,15 @@ __device__ __forceinline__ bool elect_one()
     return pred != 0;
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// The kernel launched after this one on the stream (with the programmatic-serialisation
+// launch attribute) may start once every CTA of this grid has executed this or exited.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Waits until the grids this one depends on have completed and their writes are visible;
+// returns at once in a kernel launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
 {
