@@ -882,6 +882,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     volatile int32_t *abort_flag = reinterpret_cast<volatile int32_t *>(smem + C::SMEM_BAR + 244);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    // a scheduled launch is a programmatic dependent of the schedule kernel: its items (and
+    // all that the kernels before that one wrote) are visible after this wait; with partial
+    // results, the kernel that merges them may start once every CTA of this grid runs
+    if (a.items) pdl_wait();
+    if (a.items || gridDim.y > 1) pdl_launch_dependents();
 
     // work unit: (b, h, t, pair of query tiles), pair fastest so that the tiles sharing
     // one frame's K/V run side by side; the last pair of a frame may hold one tile only
@@ -1023,6 +1028,7 @@ __device__ __forceinline__ int sched_bin(int len) { return len <= 1 ? 0 : 31 - _
 
 __global__ void __launch_bounds__(SCHED_THREADS) schedule_kernel(const __grid_constant__ SchedArgs s)
 {
+    pdl_launch_dependents();  // the forward kernel's CTAs may take their SMs and wait for the items
     constexpr int NW = SCHED_THREADS / 32;
     __shared__ int bin_start[SCHED_BINS];     // first item of each class (descending class order)
     __shared__ int carry[SCHED_BINS];         // items of each class placed by earlier chunks
@@ -1250,7 +1256,17 @@ sfa_status launch(const sfa_attn_desc *d, const void *q, const void *k, const vo
         sfa_status st0 = launch_status();
         if (st0 != SFA_OK) return st0;
         const int64_t n_items = grid * (sched->k0 + (n_lists == 2 ? sched->k1 : 0));
-        sfa_forward_kernel<D><<<dim3((unsigned)n_items, 1), NUM_THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, to, a);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)n_items, 1);
+        cfg.blockDim = dim3(NUM_THREADS);
+        cfg.dynamicSmemBytes = C::SMEM_BYTES;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, sfa_forward_kernel<D>, tq, tk, tv, to, a) != cudaSuccess) return SFA_ERR_CUDA;
     } else {
         sfa_forward_kernel<D><<<dim3((unsigned)grid, (unsigned)slices), NUM_THREADS, C::SMEM_BYTES, stream>>>(
             tq, tk, tv, to, a);

@@ -12,6 +12,7 @@
 
 #include "sfa.h"
 #include "sfa_internal.h"
+#include "sfa_ptx.cuh"
 
 namespace sfa {
 namespace {
@@ -97,6 +98,7 @@ __global__ void __launch_bounds__(256) lse_combine_kernel(int64_t rows, int S, i
                                                           int64_t os0, int64_t os1, int64_t os2, float *lse,
                                                           uint16_t *o1, float *lse1)
 {
+    pdl_wait();  // launched as a dependent of the forward kernel that writes the partials
     // Merges slices [0, S) of the partials into (o, lse) and, when o1 is set, slices
     // [0, S1) into (o1, lse1) (same strides): one group of D/8 threads per row, lane `sub`
     // of the group holds slice `sub`'s LSE.
@@ -179,14 +181,23 @@ sfa_status launch_lse_combine(int64_t rows, int S, int d, int H, int64_t Lq, con
     const int64_t need = (rows * (d / 8) + threads - 1) / threads;
     const int64_t cap = (int64_t)sms * 8;
     const int blocks = (int)(need < cap ? need : cap);
-    if (d == 128)
-        lse_combine_kernel<128><<<blocks, threads, 0, s>>>(rows, S, S1, H, Lq, (const uint4 *)o_part, lse_part,
-                                                           (uint16_t *)o, o_stride[0], o_stride[1], o_stride[2], lse,
-                                                           (uint16_t *)o1, lse1);
-    else
-        lse_combine_kernel<64><<<blocks, threads, 0, s>>>(rows, S, S1, H, Lq, (const uint4 *)o_part, lse_part,
-                                                          (uint16_t *)o, o_stride[0], o_stride[1], o_stride[2], lse,
-                                                          (uint16_t *)o1, lse1);
+    // a programmatic dependent of the forward kernel before it on the stream: its CTAs take
+    // the SMs that kernel leaves and wait there for its partials
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)blocks);
+    cfg.blockDim = dim3(threads);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e =
+        d == 128 ? cudaLaunchKernelEx(&cfg, lse_combine_kernel<128>, rows, S, S1, H, Lq, (const uint4 *)o_part, lse_part,
+                                      (uint16_t *)o, o_stride[0], o_stride[1], o_stride[2], lse, (uint16_t *)o1, lse1)
+                 : cudaLaunchKernelEx(&cfg, lse_combine_kernel<64>, rows, S, S1, H, Lq, (const uint4 *)o_part, lse_part,
+                                      (uint16_t *)o, o_stride[0], o_stride[1], o_stride[2], lse, (uint16_t *)o1, lse1);
+    if (e != cudaSuccess) return SFA_ERR_CUDA;
     return launch_status();
 }
 
