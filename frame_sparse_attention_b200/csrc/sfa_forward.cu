@@ -1297,6 +1297,11 @@ size_t split_ws_bytes(const sfa_attn_desc *d, int n_split)
 // each a range plus a fixed prologue / epilogue cost, plus the merge of the partials;
 // the schedule kernel then orders the real ranges longest first.
 constexpr double SCHED_OVERHEAD_TILES = 3.0;  // Q load, pipeline fill, epilogue of one CTA, in key tiles
+// the same for the ranges of a two-list launch: fitted to a sweep of the history branch's
+// range count on the LSE-merge workload (12 heads x 7 query-tile pairs, lists of 2 and 12
+// frames; 4, 5, 6, 7, 8, 10 ranges measured 0.263, 0.290, 0.271, 0.286, 0.294, 0.300 ms),
+// whose order the 3-tile figure does not reproduce (it picked 6)
+constexpr double DUAL_OVERHEAD_TILES = 16.0;
 constexpr double STEP_US = 2.4;               // one key tile of a CTA (both query tiles), measured
 constexpr double HBM_BYTES_PER_US = 6.5e6;
 
@@ -1316,8 +1321,8 @@ void auto_splits(const sfa_attn_desc *d, int n_lists, int nblk, int &k0, int &k1
     const double len = nblk ? (double)d->Amax : (double)d->Amax * n_qt;  // key tiles per unit, at most
     const int cap = d->d / 8;                                           // partial slices the merge takes
     const double slice_bytes = (double)d->B * d->H * d->Tq * d->P * (2.0 * d->d + 4.0);
-    auto cost = [&](int pieces_per_unit, int longest_k, int slices) {
-        const double piece = std::ceil(len / longest_k) + SCHED_OVERHEAD_TILES;
+    auto cost = [&](int pieces_per_unit, int longest_k, int slices, double overhead = SCHED_OVERHEAD_TILES) {
+        const double piece = std::ceil(len / longest_k) + overhead;
         const double waves = std::ceil(units * pieces_per_unit / sms);
         const double merge = slices > 1 ? (slices + 1) * slice_bytes / HBM_BYTES_PER_US : 0.0;
         return waves * piece * STEP_US + merge;
@@ -1344,9 +1349,9 @@ void auto_splits(const sfa_attn_desc *d, int n_lists, int nblk, int &k0, int &k1
     // range per unit; the second (history) branch is split
     k0 = 1;
     k1 = 1;
-    double best = cost(2, 1, 2);
+    double best = cost(2, 1, 2, DUAL_OVERHEAD_TILES);
     for (int k = 2; k + 1 <= cap; ++k) {
-        const double c = cost(1 + k, k, 1 + k);
+        const double c = cost(1 + k, k, 1 + k, DUAL_OVERHEAD_TILES);
         if (c < best) {
             best = c;
             k1 = k;
