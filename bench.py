@@ -61,13 +61,13 @@ def measured_peaks():
 
 # DRAM bytes (read + write) of one forward launch on this workload, from one ncu capture
 # of the same kernel on the 4-head version of the workload scaled by 3 to 12 heads (the
-# traffic is per (head, frame, query tile) unit): 3 x (197.054208 + 52.115712) MB.  Set
+# traffic is per (head, frame, query tile) unit): 3 x (196.842496 + 51.089408) MB.  Set
 # back to None whenever the forward kernel changes, until it is re-measured.
-NCU_TRAFFIC_BYTES = 747_509_760
+NCU_TRAFFIC_BYTES = 743_795_712
 # DRAM bytes read + written by the gated-delta kernels of one call on the gdn workload,
-# from an ncu capture: prep 231.950592 + 0.430080 MB, recurrence 145.723904 + 69.110272 MB.
+# from an ncu capture: prep 231.952896 + 3.159552 MB, recurrence 143.392256 + 67.441664 MB.
 # None once the kernels change, until they are re-measured.
-GDN_NCU_TRAFFIC_BYTES = 447_214_848
+GDN_NCU_TRAFFIC_BYTES = 445_946_368
 
 
 def max_over_ranks(x: float, device) -> float:
