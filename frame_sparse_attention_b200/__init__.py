@@ -21,7 +21,7 @@ Python face of libsfa.so (C ABI in include/sfa.h):
 
 Tensors are PyTorch CUDA tensors; calls run on the current CUDA stream.
 """
-from ._lib import (SET_KINDS, SFA_DEBUG_STALL_SOFTMAX, SFA_ERR_BAD_SET, SFA_ERR_CUDA,
+from ._lib import (SET_KINDS, SFA_DEBUG_STALL_GDN_STATE, SFA_DEBUG_STALL_SOFTMAX, SFA_ERR_BAD_SET, SFA_ERR_CUDA,
                    SFA_ERR_INVALID_ARG, SFA_ERR_TIMEOUT, SFA_ERR_UNSUPPORTED, SFA_OK, AttnDesc,
                    SetParams, SfaError, attn_desc, build_sets, error_string, forward, forward_blocks, forward_dual,
                    forward_host, host_workspace_bytes,
@@ -30,7 +30,7 @@ from ._lib import (SET_KINDS, SFA_DEBUG_STALL_SOFTMAX, SFA_ERR_BAD_SET, SFA_ERR_
                    set_max_count,
                    set_params, split_plan, split_workspace_bytes, version)
 
-__all__ = ["SET_KINDS", "SFA_DEBUG_STALL_SOFTMAX", "SFA_ERR_BAD_SET", "SFA_ERR_CUDA",
+__all__ = ["SET_KINDS", "SFA_DEBUG_STALL_GDN_STATE", "SFA_DEBUG_STALL_SOFTMAX", "SFA_ERR_BAD_SET", "SFA_ERR_CUDA",
            "SFA_ERR_INVALID_ARG", "SFA_ERR_TIMEOUT", "SFA_ERR_UNSUPPORTED", "SFA_OK", "AttnDesc",
            "SetParams", "SfaError", "attn_desc", "build_sets", "error_string", "forward", "forward_blocks",
            "forward_dual", "forward_host", "host_workspace_bytes",

@@ -27,6 +27,7 @@ SFA_ERR_BAD_SET = 5
 SET_KINDS = {"dense": 0, "lvsa": 1, "local": 2, "anchor": 3, "memory": 4, "explicit": 5}
 SFA_MAX_HEADS = 1024
 SFA_DEBUG_STALL_SOFTMAX = 1
+SFA_DEBUG_STALL_GDN_STATE = 2
 
 
 class SfaError(RuntimeError):
@@ -52,7 +53,8 @@ class AttnDesc(ctypes.Structure):
 class GdnDesc(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("T", ctypes.c_int32), ("P", ctypes.c_int32),
                 ("d", ctypes.c_int32), ("q_stride", ctypes.c_int64 * 3), ("k_stride", ctypes.c_int64 * 3),
-                ("v_stride", ctypes.c_int64 * 3), ("o_stride", ctypes.c_int64 * 3), ("timeout_us", ctypes.c_uint32)]
+                ("v_stride", ctypes.c_int64 * 3), ("o_stride", ctypes.c_int64 * 3), ("timeout_us", ctypes.c_uint32),
+                ("debug_flags", ctypes.c_uint32)]
 
 
 _lib = None
@@ -482,7 +484,7 @@ def forward_dual(q, k, v, frames_local, counts_local, frames_hist, counts_hist, 
 
 
 def gdn_forward(q, k, v, alpha, beta, P: int, state_in=None, state_out=None, out=None, update: bool = True,
-                workspace="auto", dev_status=None, stream=None, timeout_us: int = 0):
+                workspace="auto", dev_status=None, stream=None, timeout_us: int = 0, debug_flags: int = 0):
     """ARL2 inter-frame branch over the T = L / P frames of q, k, v [B, H, L, d]: (O bf16
     like q, final state fp32 [B, H, d, d]).  alpha fp32 [B, H, T], beta fp32 [B, H, L]
     (>= 0); state_in fp32 [B, H, d, d] or None (zeros).  workspace: "auto" (allocated here),
@@ -510,6 +512,7 @@ def gdn_forward(q, k, v, alpha, beta, P: int, state_in=None, state_out=None, out
         arr = getattr(desc, field)
         arr[0], arr[1], arr[2] = t.stride(0), t.stride(1), t.stride(2)
     desc.timeout_us = timeout_us
+    desc.debug_flags = debug_flags
     if isinstance(workspace, str):
         workspace = None
         if update:

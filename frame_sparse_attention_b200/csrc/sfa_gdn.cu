@@ -81,6 +81,7 @@ struct GdnArgs {
                          // pieces of 32 consecutive rows lie side by side
     int32_t *status;
     uint64_t timeout_ns;
+    uint32_t debug_flags;  // SFA_DEBUG_STALL_GDN_STATE: the input state is never signalled ready
 };
 
 __device__ __forceinline__ uint64_t gns()
@@ -596,7 +597,7 @@ __global__ void __launch_bounds__(GTHREADS_REC, 1)
         tmem_wait_st();
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(s_ready);
+        if (!(a.debug_flags & SFA_DEBUG_STALL_GDN_STATE)) mbar_arrive(s_ready);
         pdl_wait();  // B_N comes from the preparation kernel
         bool ok = true;
         int it = 0;
@@ -838,6 +839,7 @@ extern "C" sfa_status sfa_gdn_forward(const sfa_gdn_desc *d, const void *q, cons
     a.bws = nullptr;
     a.status = dev_status;
     a.timeout_ns = (uint64_t)(d->timeout_us ? d->timeout_us : 2000000u) * 1000;
+    a.debug_flags = d->debug_flags;
     cudaStream_t s = as_cuda(stream);
     if (update) {
         const int64_t rows = (int64_t)d->B * d->H * d->T * GD;

@@ -454,8 +454,15 @@ typedef struct {
     int64_t k_stride[3];
     int64_t v_stride[3];
     int64_t o_stride[3];
-    uint32_t timeout_us; /* limit of every wait inside the kernel; 0 = 2 s */
+    uint32_t timeout_us;  /* limit of every wait inside the kernel; 0 = 2 s */
+    uint32_t debug_flags; /* SFA_DEBUG_* below; 0 in normal use */
 } sfa_gdn_desc;
+
+/* Test hook: the element-wise warps of the recurrence kernel never signal the input state
+ * ready, so its tensor-core warp's first wait runs out; the call must then report
+ * SFA_ERR_TIMEOUT through dev_status, its copies in flight must land, and it must return
+ * cleanly. */
+#define SFA_DEBUG_STALL_GDN_STATE 2u
 
 sfa_status sfa_gdn_workspace(const sfa_gdn_desc *desc, size_t *bytes);
 

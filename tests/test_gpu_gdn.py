@@ -280,3 +280,24 @@ def test_gdn_negative_step_size_is_reported():
     sfa().gdn_forward(q, k, v, a, b, P, state_in=s0, dev_status=status)
     torch.cuda.synchronize()
     assert status.item() == sfa().SFA_ERR_INVALID_ARG
+
+
+def test_gdn_stalled_recurrence_times_out_and_context_survives():
+    # the test hook keeps the recurrence kernel's input state from being signalled ready:
+    # its tensor-core warp's first wait runs out after 20 ms, the other roles stop at their
+    # next wait, the copy warp lets its copies in flight land, and the call reports
+    # SFA_ERR_TIMEOUT; the next call on the same context is correct
+    B, H, T, P = 1, 2, 3, 300
+    q, k, v, a, b, s0 = _inputs(B, H, T, P, seed=31)
+    qc, kc, vc, ac, bc, sc = (x.cuda() for x in (q, k, v, a, b, s0))
+    m = sfa()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    m.gdn_forward(qc, kc, vc, ac, bc, P, state_in=sc, dev_status=status, timeout_us=20000,
+                  debug_flags=m.SFA_DEBUG_STALL_GDN_STATE)
+    torch.cuda.synchronize()
+    assert status.item() == m.SFA_ERR_TIMEOUT
+    status.zero_()
+    o, s = m.gdn_forward(qc, kc, vc, ac, bc, P, state_in=sc, dev_status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    check_elementwise(q, k, v, a, b, P, s0, o, s)
