@@ -489,7 +489,8 @@ def gdn_forward(q, k, v, alpha, beta, P: int, state_in=None, state_out=None, out
     like q, final state fp32 [B, H, d, d]).  alpha fp32 [B, H, T], beta fp32 [B, H, L]
     (>= 0); state_in fp32 [B, H, d, d] or None (zeros).  workspace: "auto" (allocated here),
     a uint8 CUDA tensor of at least ``sfa_gdn_workspace`` bytes, or None (only for
-    update=False: the update needs it)."""
+    update=False: the update needs it).  debug_flags: SFA_DEBUG_* test hooks, 0 in normal
+    use."""
     B, H, L, d = q.shape
     if L % P:
         raise ValueError(f"sequence length {L} is not a multiple of P = {P}")
