@@ -277,9 +277,11 @@ def test_scheduled_split_plan(sfa):
     d = _desc(sfa, B=1, H=12, Tq=1, T_kv=14, P=1560, d=128, Amax=12)
     k0, _ = sfa.split_plan(d)
     assert 2 <= k0 <= 16
-    # two branches: the local lists keep one range, the history lists are split
+    # two branches: the local lists keep one range, the history lists are split; on this
+    # shape (the ISPA step: lists of 2 and 12 frames) into 4 ranges, the fastest of a
+    # measured sweep of 4 to 10 ranges
     k_local, k_hist = sfa.split_plan(d, n_lists=2)
-    assert k_local == 1 and 2 <= k_hist <= 15
+    assert k_local == 1 and k_hist == 4
     assert lib.sfa_forward_dual_workspace(ctypes.byref(d), 0, ctypes.byref(out)) == 0
     rows = 12 * 1560
     slices = k_local + k_hist
