@@ -290,6 +290,12 @@ def test_scheduled_split_plan(sfa):
     assert 1 <= k_blocks <= 16
     with pytest.raises(sfa.SfaError):
         sfa.split_plan(d, n_lists=3)
+    # the plans the measurements were taken with: one history call of the ISPA step in 7
+    # ranges, the streaming chunk (3 query frames, lists of up to 13 frames) in 4, the
+    # hsa block lists (3 query frames, up to 115 key blocks) whole
+    assert sfa.split_plan(d) == (7, 0)
+    assert sfa.split_plan(_desc(sfa, B=1, H=12, Tq=3, T_kv=24, P=1560, d=128, Amax=13)) == (4, 0)
+    assert sfa.split_plan(_desc(sfa, B=1, H=12, Tq=3, T_kv=24, P=1560, d=128, Amax=115), key_blocks=True) == (1, 0)
 
 
 def test_forward_host_host_checks(sfa):
